@@ -1,0 +1,155 @@
+"""ctypes marshalling for the CPU oracle in ``oracle/dfx_oracle.c``.
+
+TEST INFRASTRUCTURE ONLY.  The oracle is the plain single-threaded CPU
+statement of the DFX1 codec that the CUDA library is checked against.  Only
+the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+may import this module; the product path (``lossless_entropy_coded_exponent_b200``)
+never does, and the two share no code.  Every function here only moves
+arguments across the C boundary: the arithmetic lives in the C file.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dfx_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+OK, ERR_ARG, ERR_CAPACITY, ERR_CORRUPT = 0, 1, 2, 3
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"oracle {what} failed with code {code}")
+        self.code = code
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/liboracle.so`` (gcc, -O2, plain C11)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-shared", "-fPIC", "-o", tmp, _SRC]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        u64p = ctypes.POINTER(ctypes.c_uint64)
+        L.dfxo_exponent.argtypes = [ctypes.c_uint16]
+        L.dfxo_exponent.restype = ctypes.c_uint8
+        L.dfxo_sign_mantissa.argtypes = [ctypes.c_uint16]
+        L.dfxo_sign_mantissa.restype = ctypes.c_uint8
+        L.dfxo_merge.argtypes = [ctypes.c_uint8, ctypes.c_uint8]
+        L.dfxo_merge.restype = ctypes.c_uint16
+        L.dfxo_histogram.argtypes = [u16p, ctypes.c_uint64, u64p]
+        L.dfxo_code_lengths.argtypes = [u64p, ctypes.c_uint32, u8p]
+        L.dfxo_canonical_codes.argtypes = [u8p, u32p]
+        L.dfxo_container_bytes.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint64]
+        L.dfxo_container_bytes.restype = ctypes.c_uint64
+        L.dfxo_max_container_bytes.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32]
+        L.dfxo_max_container_bytes.restype = ctypes.c_uint64
+        L.dfxo_encode.argtypes = [u16p, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint32,
+                                  u8p, ctypes.c_uint64, u64p]
+        L.dfxo_decode.argtypes = [u8p, ctypes.c_uint64, u16p, ctypes.c_uint64, u64p]
+        for f in ("dfxo_histogram", "dfxo_code_lengths", "dfxo_canonical_codes", "dfxo_encode", "dfxo_decode"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def exponent(w: int) -> int:
+    return int(lib().dfxo_exponent(w))
+
+
+def sign_mantissa(w: int) -> int:
+    return int(lib().dfxo_sign_mantissa(w))
+
+
+def merge(e: int, m: int) -> int:
+    return int(lib().dfxo_merge(e, m))
+
+
+def histogram(w: np.ndarray) -> np.ndarray:
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    counts = np.zeros(256, dtype=np.uint64)
+    rc = lib().dfxo_histogram(_ptr(w, ctypes.c_uint16), w.size, _ptr(counts, ctypes.c_uint64))
+    if rc:
+        raise OracleError(rc, "histogram")
+    return counts
+
+
+def code_lengths(counts, max_len: int = 24) -> np.ndarray:
+    c = np.zeros(256, dtype=np.uint64)
+    src = np.asarray(counts, dtype=np.uint64)
+    c[: src.size] = src
+    out = np.zeros(256, dtype=np.uint8)
+    rc = lib().dfxo_code_lengths(_ptr(c, ctypes.c_uint64), max_len, _ptr(out, ctypes.c_uint8))
+    if rc:
+        raise OracleError(rc, "code_lengths")
+    return out
+
+
+def canonical_codes(lengths) -> np.ndarray:
+    ln = np.zeros(256, dtype=np.uint8)
+    src = np.asarray(lengths, dtype=np.uint8)
+    ln[: src.size] = src
+    code = np.zeros(256, dtype=np.uint32)
+    rc = lib().dfxo_canonical_codes(_ptr(ln, ctypes.c_uint8), _ptr(code, ctypes.c_uint32))
+    if rc:
+        raise OracleError(rc, "canonical_codes")
+    return code
+
+
+def container_bytes(n: int, K: int, G: int, total_bits: int) -> int:
+    return int(lib().dfxo_container_bytes(n, K, G, total_bits))
+
+
+def max_container_bytes(n: int, K: int, G: int) -> int:
+    return int(lib().dfxo_max_container_bytes(n, K, G))
+
+
+def encode(w: np.ndarray, K: int = 64, G: int = 32, max_len: int = 24) -> np.ndarray:
+    """Whole-tensor encode into a fresh uint8 array holding exactly the container."""
+    w = np.ascontiguousarray(w, dtype=np.uint16).reshape(-1)
+    cap = max_container_bytes(w.size, K, G)
+    out = np.empty(cap, dtype=np.uint8)
+    used = np.zeros(1, dtype=np.uint64)
+    rc = lib().dfxo_encode(_ptr(w, ctypes.c_uint16), w.size, K, G, max_len,
+                           _ptr(out, ctypes.c_uint8), cap, _ptr(used, ctypes.c_uint64))
+    if rc:
+        raise OracleError(rc, "encode")
+    return out[: int(used[0])].copy()
+
+
+def decode(c: np.ndarray, n_cap: int | None = None) -> np.ndarray:
+    """Decode a container; raises OracleError(ERR_CORRUPT) on any malformed byte."""
+    c = np.ascontiguousarray(c, dtype=np.uint8).reshape(-1)
+    if n_cap is None:
+        n_cap = int(c[8:16].view(np.uint64)[0]) if c.size >= 16 else 0
+        n_cap = min(n_cap, 1 << 32)
+    out = np.empty(max(n_cap, 1), dtype=np.uint16)
+    n_out = np.zeros(1, dtype=np.uint64)
+    rc = lib().dfxo_decode(_ptr(c, ctypes.c_uint8), c.size, _ptr(out, ctypes.c_uint16), n_cap,
+                           _ptr(n_out, ctypes.c_uint64))
+    if rc:
+        raise OracleError(rc, "decode")
+    return out[: int(n_out[0])]

@@ -1,0 +1,444 @@
+/*
+ * dfx_oracle.c -- plain, slow, single-threaded CPU oracle for the DFX1 codec.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file exists to check the CUDA codec.  Only the
+ * test-suite, the package smoke check and the benchmark's CPU-baseline leg may
+ * load it.  It shares no source, header, table or helper with the CUDA library
+ * (lossless_entropy_coded_exponent_b200/csrc), and the CUDA library never calls it.
+ *
+ * What it computes.  The method is lossless entropy coding of BF16 weights:
+ * weights of trained networks have a low-entropy value distribution, so a
+ * variable-length code that gives frequent values short codes shrinks them
+ * with bit-for-bit identical reconstruction
+ *   ("DFloat11: lossless LLM compression for GPU", aikraft.ru blog, section 02
+ *    "How DFloat11 works: entropy coding of the weights"; the ~1.5:1 figure of
+ *    "From a Lossless (~1.5:1) Compression Algorithm for Llama2 7B Weights to
+ *    Variable Precision, Variable Range, Compressed Numeric Data Types for CNNs
+ *    and LLMs", abstract).
+ * The pages leave the concrete code open.  This codec's reading, written out
+ * step by step below, is:
+ *   1. split every BF16 word into its 8-bit exponent and an 8-bit
+ *      sign+mantissa byte;
+ *   2. histogram the exponents;
+ *   3. length-limited (max_len, default 24) Huffman code lengths by
+ *      package-merge, ties broken by symbol value;
+ *   4. canonical codes from the lengths;
+ *   5. concatenate the codes MSB-first into 32-bit words;
+ *   6. index: per chunk of K symbols its bit length, per group of G chunks its
+ *      start bit (the "lightweight auxiliary variables" that let GPU threads
+ *      find their read positions, DFloat11 blog section 03, item 2);
+ *   7. serialise the DFX1 container;
+ *   8. decode bit by bit (canonical first-code/count walk), check the index
+ *      against the walk, merge the two bytes back.
+ * No step is blocked, fused or reordered beyond that list.
+ *
+ * The container layout (all integers little-endian, every section starts at a
+ * 16-byte boundary, every padding byte is zero):
+ *   0   "DFX1"                                  magic
+ *   4   u16 version = 1, u16 header_bytes = 64
+ *   8   u64 n              number of BF16 elements
+ *   16  u64 total_bits     length of the code stream in bits
+ *   24  u64 total_bytes    size of the whole container
+ *   32  u32 K              symbols per chunk
+ *   36  u32 G              chunks per group
+ *   40  u32 n_chunk = ceil(n / K)
+ *   44  u32 n_group = ceil(n_chunk / G)
+ *   48  u64 off_m          byte offset of the sign+mantissa plane
+ *   56  u32 max_len        code-length limit used by the encoder
+ *   60  u32 reserved = 0
+ *   64  u8  len[256]       code length of every exponent value (0 = unused)
+ *   320 u64 gbase[n_group + 1]  start bit of each group, gbase[n_group] = total_bits
+ *   .   u16 clen[n_chunk]       bit length of each chunk
+ *   .   u8  m[n]                sign+mantissa bytes, element order
+ *   .   u32 stream[...]         codes, bit k of the stream = bit (31 - k % 32)
+ *                               of word k / 32; 4*ceil(total_bits/32) bytes
+ *                               rounded up to 16, then 16 zero bytes of slack
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define DFXO_OK 0
+#define DFXO_ERR_ARG 1
+#define DFXO_ERR_CAPACITY 2
+#define DFXO_ERR_CORRUPT 3
+
+#define DFXO_HEADER_BYTES 64u
+#define DFXO_LEN_OFFSET 64u
+#define DFXO_GBASE_OFFSET 320u
+
+/* ------------------------------------------------------------------ */
+/* little-endian helpers (the container is little-endian by definition) */
+
+static void put_u16(uint8_t *p, uint16_t v) { p[0] = (uint8_t)v; p[1] = (uint8_t)(v >> 8); }
+static void put_u32(uint8_t *p, uint32_t v) { for (int i = 0; i < 4; i++) p[i] = (uint8_t)(v >> (8 * i)); }
+static void put_u64(uint8_t *p, uint64_t v) { for (int i = 0; i < 8; i++) p[i] = (uint8_t)(v >> (8 * i)); }
+static uint16_t get_u16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+static uint32_t get_u32(const uint8_t *p) {
+    uint32_t v = 0;
+    for (int i = 3; i >= 0; i--) v = (v << 8) | p[i];
+    return v;
+}
+static uint64_t get_u64(const uint8_t *p) {
+    uint64_t v = 0;
+    for (int i = 7; i >= 0; i--) v = (v << 8) | p[i];
+    return v;
+}
+static uint64_t align16(uint64_t x) { return (x + 15u) & ~(uint64_t)15u; }
+
+/* ------------------------------------------------------------------ */
+/* Step 1: the split.  BF16 = sign(1) | exponent(8) | mantissa(7).      */
+
+uint8_t dfxo_exponent(uint16_t w) { return (uint8_t)((w >> 7) & 0xFF); }
+uint8_t dfxo_sign_mantissa(uint16_t w) { return (uint8_t)(((w >> 8) & 0x80) | (w & 0x7F)); }
+uint16_t dfxo_merge(uint8_t e, uint8_t m) {
+    return (uint16_t)(((uint16_t)(m & 0x80) << 8) | ((uint16_t)e << 7) | (m & 0x7F));
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 2: histogram of the exponents ("frequent values get short codes",
+ * DFloat11 blog, section 02).                                           */
+
+int dfxo_histogram(const uint16_t *w, uint64_t n, uint64_t counts[256]) {
+    for (int s = 0; s < 256; s++) counts[s] = 0;
+    for (uint64_t i = 0; i < n; i++) counts[dfxo_exponent(w[i])]++;
+    return DFXO_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 3: length-limited code lengths by package-merge.
+ *
+ * The coin-collector formulation: every used symbol is a coin of weight
+ * count[s] at each of max_len denominations.  Start from the leaves sorted by
+ * (count, symbol); max_len - 1 times, pair consecutive items of the current
+ * list into packages (a trailing odd item is dropped) and merge the packages
+ * with the leaves by weight, a leaf ahead of a package of equal weight.  The
+ * first 2m - 2 items of the last list are selected; the length of a symbol is
+ * the number of times its leaf occurs inside the selected items, packages
+ * expanded down to their leaves.
+ * One used symbol (m = 1): that symbol and a phantom partner (symbol 1 if the
+ * used one is 0, else symbol 0) both get length 1; the phantom never occurs. */
+
+typedef struct {
+    uint64_t w;   /* weight */
+    int sym;      /* leaf: symbol value; package: -1 */
+    int a, b;     /* package: indices of its two children in the previous list */
+} pm_item;
+
+static int leaf_before(const pm_item *x, const pm_item *y) {
+    /* leaf order: count ascending, then symbol ascending */
+    if (x->w != y->w) return x->w < y->w;
+    return x->sym < y->sym;
+}
+
+static void pm_expand(pm_item **lists, int level, int idx, uint8_t len[256]) {
+    const pm_item *it = &lists[level][idx];
+    if (it->sym >= 0) {
+        len[it->sym]++;
+        return;
+    }
+    pm_expand(lists, level - 1, it->a, len);
+    pm_expand(lists, level - 1, it->b, len);
+}
+
+int dfxo_code_lengths(const uint64_t counts[256], uint32_t max_len, uint8_t len[256]) {
+    pm_item leaves[256];
+    int m = 0;
+    for (int s = 0; s < 256; s++) len[s] = 0;
+    for (int s = 0; s < 256; s++)
+        if (counts[s] > 0) {
+            leaves[m].w = counts[s];
+            leaves[m].sym = s;
+            leaves[m].a = leaves[m].b = -1;
+            m++;
+        }
+    if (m == 0) return DFXO_OK;
+    if (m == 1) {
+        int s0 = leaves[0].sym;
+        len[s0] = 1;
+        len[s0 == 0 ? 1 : 0] = 1;
+        return DFXO_OK;
+    }
+    if (max_len < 1 || max_len > 32) return DFXO_ERR_ARG;
+    if (max_len < 9 && (1u << max_len) < (uint32_t)m) return DFXO_ERR_ARG; /* no prefix code exists */
+
+    /* insertion sort of the leaves by (count, symbol) */
+    for (int i = 1; i < m; i++) {
+        pm_item x = leaves[i];
+        int j = i - 1;
+        while (j >= 0 && leaf_before(&x, &leaves[j])) {
+            leaves[j + 1] = leaves[j];
+            j--;
+        }
+        leaves[j + 1] = x;
+    }
+
+    int L = (int)max_len;
+    pm_item **lists = (pm_item **)calloc((size_t)L, sizeof(pm_item *));
+    int *sizes = (int *)calloc((size_t)L, sizeof(int));
+    if (!lists || !sizes) { free(lists); free(sizes); return DFXO_ERR_ARG; }
+    lists[0] = (pm_item *)malloc(sizeof(pm_item) * (size_t)m);
+    memcpy(lists[0], leaves, sizeof(pm_item) * (size_t)m);
+    sizes[0] = m;
+    for (int j = 1; j < L; j++) {
+        int np = sizes[j - 1] / 2;
+        pm_item *pk = (pm_item *)malloc(sizeof(pm_item) * (size_t)(np > 0 ? np : 1));
+        for (int k = 0; k < np; k++) {
+            pk[k].w = lists[j - 1][2 * k].w + lists[j - 1][2 * k + 1].w;
+            pk[k].sym = -1;
+            pk[k].a = 2 * k;
+            pk[k].b = 2 * k + 1;
+        }
+        lists[j] = (pm_item *)malloc(sizeof(pm_item) * (size_t)(m + np));
+        int i = 0, k = 0, o = 0;
+        while (i < m || k < np) {
+            if (k >= np || (i < m && leaves[i].w <= pk[k].w))
+                lists[j][o++] = leaves[i++];
+            else
+                lists[j][o++] = pk[k++];
+        }
+        sizes[j] = o;
+        free(pk);
+    }
+    int take = 2 * m - 2;
+    int rc = DFXO_OK;
+    if (sizes[L - 1] < take) rc = DFXO_ERR_ARG;
+    else
+        for (int t = 0; t < take; t++) pm_expand(lists, L - 1, t, len);
+    for (int j = 0; j < L; j++) free(lists[j]);
+    free(lists);
+    free(sizes);
+    return rc;
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 4: canonical codes.  Walk the used symbols in (length, symbol)
+ * order; the first gets code 0, each next one the previous code plus one,
+ * shifted left by the growth in length.                                 */
+
+int dfxo_canonical_codes(const uint8_t len[256], uint32_t code[256]) {
+    uint32_t c = 0;
+    int prev = -1;
+    for (int s = 0; s < 256; s++) code[s] = 0;
+    for (int l = 1; l <= 32; l++)
+        for (int s = 0; s < 256; s++) {
+            if (len[s] != l) continue;
+            if (prev < 0) c = 0;
+            else c = (c + 1) << (l - prev);
+            code[s] = c;
+            prev = l;
+        }
+    return DFXO_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Layout rules.                                                        */
+
+static int params_ok(uint64_t n, uint32_t K, uint32_t G, uint32_t max_len) {
+    if (n >= ((uint64_t)1 << 32)) return 0;
+    if (max_len < 1 || max_len > 24) return 0;
+    if (K < 1 || G < 1) return 0;
+    if ((uint64_t)K * max_len > 65535u) return 0; /* a chunk length must fit in u16 */
+    return 1;
+}
+
+static uint64_t n_chunks(uint64_t n, uint32_t K) { return (n + K - 1) / K; }
+static uint64_t n_groups(uint64_t nc, uint32_t G) { return (nc + G - 1) / G; }
+static uint64_t off_clen_of(uint64_t ng) { return align16(DFXO_GBASE_OFFSET + 8 * (ng + 1)); }
+static uint64_t off_m_of(uint64_t nc, uint64_t ng) { return align16(off_clen_of(ng) + 2 * nc); }
+static uint64_t off_stream_of(uint64_t n, uint64_t nc, uint64_t ng) { return align16(off_m_of(nc, ng) + n); }
+static uint64_t stream_bytes_of(uint64_t total_bits) { return align16(4 * ((total_bits + 31) / 32)) + 16; }
+
+uint64_t dfxo_container_bytes(uint64_t n, uint32_t K, uint32_t G, uint64_t total_bits) {
+    uint64_t nc = n_chunks(n, K), ng = n_groups(nc, G);
+    return off_stream_of(n, nc, ng) + stream_bytes_of(total_bits);
+}
+
+/* ------------------------------------------------------------------ */
+/* Steps 5-7: stream, index, container.                                 */
+
+static void put_bits(uint8_t *stream, uint64_t pos, uint32_t code, uint32_t l) {
+    /* bit k of the stream is bit (31 - k % 32) of little-endian word k / 32 */
+    for (uint32_t b = 0; b < l; b++) {
+        uint32_t bit = (code >> (l - 1 - b)) & 1u;
+        uint64_t k = pos + b;
+        uint64_t word = k / 32;
+        uint32_t within = 31u - (uint32_t)(k % 32);
+        uint8_t *byte = stream + 4 * word + within / 8; /* little-endian word: byte i holds bits 8i..8i+7 */
+        if (bit) *byte |= (uint8_t)(1u << (within % 8));
+    }
+}
+
+static uint32_t get_bit(const uint8_t *stream, uint64_t k) {
+    uint64_t word = k / 32;
+    uint32_t within = 31u - (uint32_t)(k % 32);
+    return (stream[4 * word + within / 8] >> (within % 8)) & 1u;
+}
+
+int dfxo_encode(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t max_len,
+                uint8_t *out, uint64_t cap, uint64_t *out_bytes) {
+    if (!params_ok(n, K, G, max_len) || max_len < 8) return DFXO_ERR_ARG;
+    uint64_t counts[256];
+    uint8_t len[256];
+    uint32_t code[256];
+    dfxo_histogram(w, n, counts);
+    int rc = dfxo_code_lengths(counts, max_len, len);
+    if (rc) return rc;
+    dfxo_canonical_codes(len, code);
+
+    uint64_t total_bits = 0;
+    for (uint64_t i = 0; i < n; i++) total_bits += len[dfxo_exponent(w[i])];
+    uint64_t nc = n_chunks(n, K), ng = n_groups(nc, G);
+    uint64_t total = dfxo_container_bytes(n, K, G, total_bits);
+    if (out_bytes) *out_bytes = total;
+    if (cap < total) return DFXO_ERR_CAPACITY;
+    memset(out, 0, (size_t)total);
+
+    memcpy(out, "DFX1", 4);
+    put_u16(out + 4, 1);
+    put_u16(out + 6, DFXO_HEADER_BYTES);
+    put_u64(out + 8, n);
+    put_u64(out + 16, total_bits);
+    put_u64(out + 24, total);
+    put_u32(out + 32, K);
+    put_u32(out + 36, G);
+    put_u32(out + 40, (uint32_t)nc);
+    put_u32(out + 44, (uint32_t)ng);
+    put_u64(out + 48, off_m_of(nc, ng));
+    put_u32(out + 56, max_len);
+    put_u32(out + 60, 0);
+    memcpy(out + DFXO_LEN_OFFSET, len, 256);
+
+    /* index: chunk bit lengths and group start bits, from the prefix of code lengths */
+    uint8_t *gbase = out + DFXO_GBASE_OFFSET;
+    uint8_t *clen = out + off_clen_of(ng);
+    uint64_t pos = 0;
+    for (uint64_t c = 0; c < nc; c++) {
+        if (c % G == 0) put_u64(gbase + 8 * (c / G), pos);
+        uint64_t start = pos;
+        uint64_t end_i = (c + 1) * K < n ? (c + 1) * K : n;
+        for (uint64_t i = c * K; i < end_i; i++) pos += len[dfxo_exponent(w[i])];
+        put_u16(clen + 2 * c, (uint16_t)(pos - start));
+    }
+    put_u64(gbase + 8 * ng, pos);
+
+    uint8_t *mplane = out + off_m_of(nc, ng);
+    uint8_t *stream = out + off_stream_of(n, nc, ng);
+    pos = 0;
+    for (uint64_t i = 0; i < n; i++) {
+        uint8_t e = dfxo_exponent(w[i]);
+        mplane[i] = dfxo_sign_mantissa(w[i]);
+        put_bits(stream, pos, code[e], len[e]);
+        pos += len[e];
+    }
+    return DFXO_OK;
+}
+
+uint64_t dfxo_max_container_bytes(uint64_t n, uint32_t K, uint32_t G) {
+    /* An optimal length-limited code never costs more than the 8-bit
+     * fixed-length code (feasible because max_len >= 8); the one-symbol
+     * phantom code costs 1 bit per element. */
+    return dfxo_container_bytes(n, K, G, 8 * n);
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 8: decode.  Validate everything, then walk the stream one bit at a
+ * time: a code of length l is complete when its value minus the first
+ * canonical code of length l is below the number of codes of length l.    */
+
+int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, uint64_t *n_out) {
+    if (bytes < DFXO_GBASE_OFFSET + 8) return DFXO_ERR_CORRUPT;
+    if (memcmp(c, "DFX1", 4) != 0) return DFXO_ERR_CORRUPT;
+    if (get_u16(c + 4) != 1 || get_u16(c + 6) != DFXO_HEADER_BYTES) return DFXO_ERR_CORRUPT;
+    uint64_t n = get_u64(c + 8);
+    uint64_t total_bits = get_u64(c + 16);
+    uint64_t total = get_u64(c + 24);
+    uint32_t K = get_u32(c + 32), G = get_u32(c + 36);
+    uint32_t max_len = get_u32(c + 56);
+    if (!params_ok(n, K, G, max_len)) return DFXO_ERR_CORRUPT;
+    if (get_u32(c + 60) != 0) return DFXO_ERR_CORRUPT;
+    uint64_t nc = n_chunks(n, K), ng = n_groups(nc, G);
+    if (get_u32(c + 40) != nc || get_u32(c + 44) != ng) return DFXO_ERR_CORRUPT;
+    if (get_u64(c + 48) != off_m_of(nc, ng)) return DFXO_ERR_CORRUPT;
+    if (total_bits > (uint64_t)max_len * n) return DFXO_ERR_CORRUPT;
+    if (total != dfxo_container_bytes(n, K, G, total_bits) || total > bytes) return DFXO_ERR_CORRUPT;
+    if (n_out) *n_out = n;
+    if (n > n_cap) return DFXO_ERR_CAPACITY;
+
+    /* code lengths: at most max_len; Kraft sum exactly 1 when n > 0, no code when n = 0 */
+    const uint8_t *len = c + DFXO_LEN_OFFSET;
+    uint64_t kraft = 0;
+    for (int s = 0; s < 256; s++) {
+        if (len[s] > max_len) return DFXO_ERR_CORRUPT;
+        if (len[s]) kraft += (uint64_t)1 << (24 - len[s]);
+    }
+    if (n > 0 && kraft != ((uint64_t)1 << 24)) return DFXO_ERR_CORRUPT;
+    if (n == 0 && kraft != 0) return DFXO_ERR_CORRUPT;
+
+    /* canonical decoding tables: count and first code per length, symbols in (length, symbol) order */
+    uint32_t count[33] = {0}, first[33] = {0}, index_of_first[33] = {0};
+    uint8_t sorted[256];
+    int ns = 0;
+    for (int l = 1; l <= 24; l++)
+        for (int s = 0; s < 256; s++)
+            if (len[s] == l) {
+                if (count[l] == 0) index_of_first[l] = (uint32_t)ns;
+                count[l]++;
+                sorted[ns++] = (uint8_t)s;
+            }
+    {
+        uint32_t code = 0;
+        int prev = -1;
+        for (int l = 1; l <= 24; l++) {
+            if (count[l] == 0) continue;
+            if (prev < 0) code = 0;
+            else code = (code + 1) << (l - prev);   /* code held the last code of length prev */
+            first[l] = code;
+            code += count[l] - 1;
+            prev = l;
+        }
+    }
+
+    const uint8_t *gbase = c + DFXO_GBASE_OFFSET;
+    const uint8_t *clen = c + off_clen_of(ng);
+    const uint8_t *mplane = c + off_m_of(nc, ng);
+    const uint8_t *stream = c + off_stream_of(n, nc, ng);
+
+    /* every padding byte must be zero */
+    for (uint64_t b = DFXO_GBASE_OFFSET + 8 * (ng + 1); b < off_clen_of(ng); b++) if (c[b]) return DFXO_ERR_CORRUPT;
+    for (uint64_t b = off_clen_of(ng) + 2 * nc; b < off_m_of(nc, ng); b++) if (c[b]) return DFXO_ERR_CORRUPT;
+    for (uint64_t b = off_m_of(nc, ng) + n; b < off_stream_of(n, nc, ng); b++) if (c[b]) return DFXO_ERR_CORRUPT;
+    if (get_u64(gbase) != 0 || get_u64(gbase + 8 * ng) != total_bits) return DFXO_ERR_CORRUPT;
+
+    uint64_t pos = 0;
+    uint64_t chunk_start = 0;
+    for (uint64_t i = 0; i < n; i++) {
+        if (i % K == 0) {
+            uint64_t ci = i / K;
+            chunk_start = pos;
+            if (ci % G == 0 && get_u64(gbase + 8 * (ci / G)) != pos) return DFXO_ERR_CORRUPT;
+        }
+        uint32_t code = 0;
+        int l = 0, found = -1;
+        while (l < 24) {
+            if (pos >= total_bits) return DFXO_ERR_CORRUPT;
+            code = (code << 1) | get_bit(stream, pos);
+            pos++;
+            l++;
+            if (count[l] && code >= first[l] && code - first[l] < count[l]) {
+                found = sorted[index_of_first[l] + (code - first[l])];
+                break;
+            }
+        }
+        if (found < 0) return DFXO_ERR_CORRUPT;
+        w[i] = dfxo_merge((uint8_t)found, mplane[i]);
+        if ((i + 1) % K == 0 || i + 1 == n) {
+            if (get_u16(clen + 2 * (i / K)) != pos - chunk_start) return DFXO_ERR_CORRUPT;
+        }
+    }
+    if (pos != total_bits) return DFXO_ERR_CORRUPT;
+    /* stream bits after total_bits, the rounding words and the slack are zero */
+    for (uint64_t k = total_bits; k < 32 * ((total_bits + 31) / 32); k++) if (get_bit(stream, k)) return DFXO_ERR_CORRUPT;
+    for (uint64_t b = 4 * ((total_bits + 31) / 32); b < stream_bytes_of(total_bits); b++) if (stream[b]) return DFXO_ERR_CORRUPT;
+    return DFXO_OK;
+}

@@ -1,0 +1,338 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+* the BF16 field split, against the IEEE value of every one of the 65 536 patterns;
+* hand-worked containers and tie-rule vectors (tests/golden, derived by hand);
+* brute-force optimality of the code lengths on tiny alphabets;
+* equality with the textbook (heap) Huffman cost when the tree fits the limit;
+* an independent dynamic program for the length-limited optimum (Fibonacci clamp);
+* Kraft equality, the entropy bound, canonical-code prefix-freedom;
+* exhaustive and edge-case round trips, and rejection of malformed containers.
+"""
+import heapq
+import itertools
+import math
+import os
+from functools import lru_cache
+
+import numpy as np
+import pytest
+
+import oracle
+from lossless_entropy_coded_exponent_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- helpers
+
+def textbook_huffman(counts):
+    """Heap Huffman: (total cost, tree depth).  Independent of package-merge."""
+    items = [(c, i, 0) for i, c in enumerate(counts) if c > 0]
+    if len(items) < 2:
+        return (sum(c for c, _, _ in items), 1 if items else 0)
+    heapq.heapify(items)
+    cost, uid = 0, len(counts)
+    while len(items) > 1:
+        a = heapq.heappop(items)
+        b = heapq.heappop(items)
+        cost += a[0] + b[0]
+        heapq.heappush(items, (a[0] + b[0], uid, max(a[2], b[2]) + 1))
+        uid += 1
+    return cost, items[0][2]
+
+
+def brute_force_min_cost(counts, L):
+    used = [c for c in counts if c > 0]
+    best = None
+    for lens in itertools.product(range(1, L + 1), repeat=len(used)):
+        if sum(2.0 ** -l for l in lens) <= 1.0 + 1e-12:
+            cost = sum(c * l for c, l in zip(used, lens))
+            best = cost if best is None else min(best, cost)
+    return best
+
+
+def dp_length_limited_cost(counts, L):
+    """Optimal cost of a prefix code with lengths <= L by a level-by-level DP:
+    heavier symbols take shallower leaves; at depth d with `a` open nodes,
+    choose how many become leaves, the rest split into 2 nodes each."""
+    w = sorted((c for c in counts if c > 0), reverse=True)
+    m = len(w)
+    prefix = [0]
+    for x in w:
+        prefix.append(prefix[-1] + x)
+
+    @lru_cache(maxsize=None)
+    def f(d, i, a):
+        if i == m:
+            return 0
+        if d > L or a == 0:
+            return math.inf
+        best = math.inf
+        for k in range(0, min(a, m - i) + 1):
+            rest = min(2 * (a - k), m - i - k)
+            best = min(best, d * (prefix[i + k] - prefix[i]) + f(d + 1, i + k, rest))
+        return best
+
+    return f(1, 0, 2)
+
+
+def cost_of(counts, lens):
+    return int(sum(int(c) * int(l) for c, l in zip(counts, lens)))
+
+
+def kraft24(lens):
+    return sum(1 << (24 - int(l)) for l in lens if l > 0)
+
+
+def load_golden_containers():
+    cases, cur = [], None
+    with open(os.path.join(GOLDEN, "tiny_containers.txt")) as fh:
+        for raw in fh:
+            line = raw.split("#", 1)[0].strip()
+            if not line:
+                continue
+            if line.startswith("case "):
+                parts = line.split()
+                kv = dict(p.split("=") for p in parts[2:])
+                cur = {"name": parts[1], "K": int(kv["K"]), "G": int(kv["G"]),
+                       "bytes": np.zeros(int(kv["total"]), dtype=np.uint8)}
+                cases.append(cur)
+            elif line.startswith("input"):
+                cur["input"] = np.array([int(t, 16) for t in line.split()[1:]], dtype=np.uint16)
+            else:
+                off, hexes = line.split(":")
+                vals = [int(t, 16) for t in hexes.split()]
+                cur["bytes"][int(off): int(off) + len(vals)] = vals
+    return cases
+
+
+def load_tie_rules():
+    rows = []
+    with open(os.path.join(GOLDEN, "tie_rule.txt")) as fh:
+        for raw in fh:
+            line = raw.split("#", 1)[0].strip()
+            if not line:
+                continue
+            L, cnt, exp = (p.strip() for p in line.split("|"))
+            counts = np.zeros(256, dtype=np.uint64)
+            for t in cnt.split():
+                s, c = t.split(":")
+                counts[int(s)] = int(c)
+            expected = np.zeros(256, dtype=np.uint8)
+            for t in exp.split():
+                s, l = t.split(":")
+                expected[int(s)] = int(l)
+            rows.append((int(L), counts, expected))
+    return rows
+
+
+# ---------------------------------------------------------------- the split
+
+def test_split_matches_ieee_fields_for_every_pattern():
+    w = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    x = (w.astype(np.uint32) << 16).view(np.float32)
+    e_or = np.array([oracle.exponent(int(v)) for v in w], dtype=np.int64)
+    m_or = np.array([oracle.sign_mantissa(int(v)) for v in w], dtype=np.int64)
+    with np.errstate(all="ignore"):
+        finite = np.isfinite(x)
+        a = np.abs(x.astype(np.float64))
+        normal = finite & (a >= 2.0 ** -126)
+        sub = finite & (a > 0) & ~normal
+        frac, ex = np.frexp(a)
+    exp_e = np.where(normal, ex + 126, 0)
+    exp_e = np.where(finite, exp_e, 255)
+    mant = np.zeros_like(exp_e)
+    mant = np.where(normal, np.rint((frac * 2 - 1) * 128), mant)
+    mant = np.where(sub, np.rint(a / 2.0 ** -133), mant).astype(np.int64)
+    sign = np.signbit(x).astype(np.int64)
+    nan = np.isnan(x)
+    assert np.array_equal(e_or, exp_e)
+    ok = ~nan
+    assert np.array_equal(m_or[ok], (sign[ok] << 7) | mant[ok])
+    assert np.all((m_or[nan] & 0x7F) != 0) and np.array_equal(m_or[nan] >> 7, sign[nan])
+    back = np.array([oracle.merge(int(e), int(m)) for e, m in zip(e_or, m_or)], dtype=np.uint16)
+    assert np.array_equal(back, w)
+
+
+# ---------------------------------------------------------------- code lengths
+
+@pytest.mark.parametrize("row", load_tie_rules(), ids=lambda r: str(r[0]))
+def test_tie_rule_golden(row):
+    L, counts, expected = row
+    assert np.array_equal(oracle.code_lengths(counts, L), expected)
+
+
+def test_brute_force_optimality_tiny_alphabets():
+    rng = np.random.default_rng(123)
+    trials = 0
+    for m in range(2, 8):
+        for L in (3, 4, 5):
+            if (1 << L) < m:
+                continue
+            for _ in range(6 if m < 7 else 2):
+                syms = rng.choice(256, size=m, replace=False)
+                counts = np.zeros(256, dtype=np.uint64)
+                counts[syms] = rng.integers(1, 40, size=m)
+                lens = oracle.code_lengths(counts, L)
+                assert lens.max() <= L and kraft24(lens) == 1 << 24
+                assert np.all((lens > 0) == (counts > 0))
+                assert cost_of(counts, lens) == brute_force_min_cost(counts, L)
+                trials += 1
+    assert trials > 50
+
+
+def test_matches_textbook_huffman_when_tree_fits():
+    w = inputs.small_gaussian()
+    counts = oracle.histogram(w)
+    hcost, depth = textbook_huffman([int(c) for c in counts])
+    assert depth <= 24
+    lens = oracle.code_lengths(counts, 24)
+    assert cost_of(counts, lens) == hcost
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        counts = np.zeros(256, dtype=np.uint64)
+        k = int(rng.integers(2, 257))
+        counts[rng.choice(256, size=k, replace=False)] = rng.integers(1, 10_000, size=k)
+        hcost, depth = textbook_huffman([int(c) for c in counts])
+        if depth <= 24:
+            assert cost_of(counts, oracle.code_lengths(counts, 24)) == hcost
+
+
+def test_fibonacci_counts_force_the_clamp():
+    fib = inputs.fibonacci_counts(28)
+    counts = np.zeros(256, dtype=np.uint64)
+    counts[100:128] = fib
+    hcost, depth = textbook_huffman([int(c) for c in counts])
+    assert depth == 27
+    lens = oracle.code_lengths(counts, 24)
+    assert lens.max() == 24 and kraft24(lens) == 1 << 24
+    cost = cost_of(counts, lens)
+    assert cost > hcost
+    assert cost == dp_length_limited_cost([int(c) for c in counts], 24)
+
+
+def test_dp_agrees_on_random_limited_cases():
+    rng = np.random.default_rng(9)
+    for _ in range(10):
+        m = int(rng.integers(9, 20))
+        L = int(rng.integers(5, 9))
+        counts = np.zeros(256, dtype=np.uint64)
+        counts[rng.choice(256, size=m, replace=False)] = np.maximum(1, (2.0 ** rng.uniform(0, 14, size=m)).astype(np.int64))
+        lens = oracle.code_lengths(counts, L)
+        assert lens.max() <= L and kraft24(lens) == 1 << 24
+        assert cost_of(counts, lens) == dp_length_limited_cost([int(c) for c in counts], L)
+
+
+def test_kraft_equality_and_entropy_bound():
+    for w in (inputs.small_gaussian(), inputs.projection_with_outliers()):
+        counts = oracle.histogram(w)
+        lens = oracle.code_lengths(counts, 24)
+        assert kraft24(lens) == 1 << 24
+        p = counts[counts > 0].astype(np.float64) / w.size
+        H = float(-(p * np.log2(p)).sum())
+        mean = cost_of(counts, lens) / w.size
+        assert H <= mean <= H + 1
+
+
+def test_canonical_codes_prefix_free_and_ordered():
+    for w in (inputs.small_gaussian(), inputs.fibonacci_clamp_tensor(27), inputs.uniform_patterns(1 << 16, 3)):
+        lens = oracle.code_lengths(oracle.histogram(w), 24)
+        code = oracle.canonical_codes(lens)
+        used = [s for s in range(256) if lens[s] > 0]
+        order = sorted(used, key=lambda s: (int(lens[s]), s))
+        left = [int(code[s]) << (24 - int(lens[s])) for s in order]
+        assert left == sorted(left) and len(set(left)) == len(left)
+        for a, b in zip(order, order[1:]):
+            la, lb = int(lens[a]), int(lens[b])
+            # b's code must not start with a's code
+            assert (int(code[b]) >> (lb - la)) != int(code[a])
+        assert int(code[order[0]]) == 0
+        last = order[-1]
+        assert int(code[last]) == (1 << int(lens[last])) - 1  # complete code ends in all ones
+
+
+# ---------------------------------------------------------------- containers
+
+@pytest.mark.parametrize("case", load_golden_containers(), ids=lambda c: c["name"])
+def test_golden_containers(case):
+    got = oracle.encode(case["input"], K=case["K"], G=case["G"])
+    assert got.size == case["bytes"].size
+    assert np.array_equal(got, case["bytes"])
+    assert np.array_equal(oracle.decode(case["bytes"]), case["input"])
+
+
+def test_round_trip_every_bit_pattern():
+    w = inputs.all_patterns_shuffled(26)
+    c = oracle.encode(w)
+    assert np.array_equal(oracle.decode(c), w)
+
+
+@pytest.mark.parametrize("name", list(inputs.edge_cases().keys()))
+def test_round_trip_edge_cases(name):
+    w = inputs.edge_cases()[name]
+    for K, G in ((64, 32), (128, 32), (5, 3)):
+        c = oracle.encode(w, K=K, G=G)
+        assert c.size == oracle.container_bytes(w.size, K, G, int(c[16:24].view(np.uint64)[0]))
+        assert np.array_equal(oracle.decode(c), w)
+
+
+def test_deterministic_and_size_rule():
+    w = inputs.small_gaussian()
+    a = oracle.encode(w)
+    b = oracle.encode(w.copy())
+    assert np.array_equal(a, b)
+    total_bits = int(a[16:24].view(np.uint64)[0])
+    counts = oracle.histogram(w)
+    assert total_bits == cost_of(counts, oracle.code_lengths(counts))
+    assert a.size <= oracle.max_container_bytes(w.size, 64, 32)
+
+
+def test_uniform_exponents_cost_about_eight_bits():
+    w = inputs.uniform_patterns(1 << 20, 24)
+    c = oracle.encode(w)
+    total_bits = int(c[16:24].view(np.uint64)[0])
+    assert 7.99 * w.size <= total_bits <= 8.0 * w.size
+
+
+def test_compression_is_plausible_against_the_pages():
+    """Plausibility, not parity: ~1.5:1 (Liguori, abstract) and ~70 % of the
+    BF16 size (DFloat11 blog, title and section 02)."""
+    w = inputs.small_gaussian()
+    c = oracle.encode(w, K=128)
+    bits_per_weight = 8.0 * c.size / w.size
+    assert 10.0 < bits_per_weight < 11.0
+    assert 1.4 < 16.0 / bits_per_weight < 1.6
+
+
+# ---------------------------------------------------------------- malformed input
+
+def _corrupt_variants(c):
+    n = int(c[8:16].view(np.uint64)[0])
+    out = {}
+    v = c.copy(); v[0] ^= 1; out["magic"] = v
+    v = c.copy(); v[4] = 2; out["version"] = v
+    v = c.copy(); v[8] ^= 1; out["n"] = v
+    v = c.copy(); v[24] ^= 0x10; out["total_bytes"] = v
+    out["truncated"] = c[:-1].copy()
+    used = int(np.flatnonzero(c[64:320])[0])
+    v = c.copy(); v[64 + used] = 0; out["kraft"] = v
+    v = c.copy(); v[64 + used] = 30; out["len_over_limit"] = v
+    v = c.copy(); v[64 + used] += 1; out["kraft_below_one"] = v
+    v = c.copy(); v[320 + 8] ^= 1; out["gbase"] = v
+    nc = int(c[40:44].view(np.uint32)[0]); ng = int(c[44:48].view(np.uint32)[0])
+    off_clen = (320 + 8 * (ng + 1) + 15) // 16 * 16
+    v = c.copy(); v[off_clen] ^= 1; out["clen"] = v
+    v = c.copy(); v[off_clen + 2 * nc] = 1; out["padding"] = v
+    v = c.copy(); v[-1] = 1; out["slack"] = v
+    assert n > 0
+    return out
+
+
+def test_malformed_containers_are_rejected():
+    w = inputs.gaussian(10_000, 0.02, seed=7)
+    c = oracle.encode(w)
+    assert np.array_equal(oracle.decode(c), w)
+    for name, bad in _corrupt_variants(c).items():
+        with pytest.raises(oracle.OracleError) as ei:
+            oracle.decode(bad)
+        assert ei.value.code == oracle.ERR_CORRUPT, name
