@@ -1,0 +1,467 @@
+#!/usr/bin/env python3
+"""Benchmark: dfx_decode throughput on the 70B-shaped layer stream.
+
+Workload: 24 BF16 tensors of 8192 x 28672 (5.64 B weights, 11.3 GB raw), values
+N(0, 1/8192) with 0.05 % N(0, 0.5^2) outliers, each encoded with its own code
+book by dfx_encode.  All 24 containers stay resident in HBM; one step decodes
+them one after another into a single reused 470 MB BF16 buffer on one stream.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  `value` is decoded BF16 GB/s over all ranks
+(each rank decodes its own 24 tensors: weak scaling, no collective on the data
+path).  Timing: CUDA events on the decode stream, W untimed steps first, a
+barrier and a device synchronise on both sides, max over ranks.  Every
+container (~0.32 GB) and the output buffer exceed the 126 MB L2, so no flush is
+needed between steps.
+
+`--impl reference` times the CPU oracle (single-threaded C) decoding a 16 M
+weight sample with the same value distribution; it is the slow reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dfx_decode BF16 GB/s & % of HBM roofline; bits/weight; bit-exact vs oracle"
+UNIT = "GB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+WORKLOAD = "70B-shaped layer stream: 24 x BF16[8192, 28672], N(0, 1/8192) + 0.05% N(0, 0.5^2) outliers"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_dram_traffic.txt")
+DECODE_SOURCES = [os.path.join(ROOT, "lossless_entropy_coded_exponent_b200", "csrc", f)
+                  for f in ("decode.cu", "dfx_common.cuh")]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--tensors", type=int, default=24)
+    ap.add_argument("--chunk-symbols", type=int, default=64)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            v = float(json.load(fh)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in DECODE_SOURCES:
+        with open(p, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic_per_launch(n_weights: int):
+    """DRAM bytes per decode launch from the committed ncu summary, scaled to this
+    launch's weights; None when the kernel source changed since the capture."""
+    try:
+        fields = {}
+        with open(TRAFFIC_FILE) as fh:
+            for line in fh:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip()
+        if fields.get("decode_source_sha256") != decode_source_hash():
+            return None
+        return float(fields["dram_bytes_per_weight"]) * n_weights
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that instead of clocks
+            self._nv = None
+            self.error = repr(e)
+
+    def _handle(self, device_index):
+        import torch
+
+        nv = self._nv
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(device_index)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h) if hasattr(
+                    nv, "nvmlDeviceGetCurrentClocksEventReasons") else nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "no nvml")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------ reference arm
+
+def run_reference(args, world, rank):
+    """The CPU oracle decoding a bounded sample of the workload, single-threaded."""
+    if rank != 0:
+        return None
+    import numpy as np
+
+    import oracle
+    from lossless_entropy_coded_exponent_b200 import inputs
+
+    n = 8192 * 2048
+    w = inputs.layer70b_sample(n, seed=500)
+    c = oracle.encode(w, K=args.chunk_symbols)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        out = oracle.decode(c)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    assert np.array_equal(out, w)
+    t = sum(times)
+    value = 2.0 * n * len(times) / t / 1e9
+    sample = f"one 8192x2048 BF16 tensor ({n} weights) of the same distribution, decoded per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": sample, "chunk_symbols": args.chunk_symbols},
+            "bits_per_weight": 8.0 * c.size / n,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+# ------------------------------------------------------------------------ our arm
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import lossless_entropy_coded_exponent_b200 as dfx
+    from lossless_entropy_coded_exponent_b200 import inputs
+
+    dfx.lib()  # fail loudly if libdfx.so is missing
+    dev = torch.device("cuda", local)
+    rows, cols = inputs.LAYER70B_SHAPE
+    n = rows * cols
+    T = args.tensors
+    K = args.chunk_symbols
+    plan = dfx.dfx_plan(n, chunk_symbols=K)
+    stream = torch.cuda.Stream(device=dev)
+
+    # ---- set-up: generate, encode, keep every container and every input resident
+    xs, comps, sizes = [], [], []
+    scratch = torch.empty(plan.max_compressed_bytes, dtype=torch.uint8, device=dev)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
+    enc_start = torch.cuda.Event(enable_timing=True)
+    enc_end = torch.cuda.Event(enable_timing=True)
+    enc_ms = []
+    with torch.cuda.stream(stream):
+        for i in range(T):
+            x = inputs.layer70b_tensor_cuda(i, seed_base=500 + 1000 * rank, device=dev)
+            enc_start.record(stream)
+            size = dfx.dfx_encode(plan, x, scratch, scratch.numel(), ws, ws.numel(), want_size=False, stream=stream)
+            enc_end.record(stream)
+            stream.synchronize()
+            enc_ms.append(enc_start.elapsed_time(enc_end))
+            size = int(scratch[24:32].cpu().numpy().view(np.uint64)[0])
+            comps.append(scratch[:size].clone())
+            sizes.append(size)
+            xs.append(x)
+    stream.synchronize()
+    if dfx.dfx_device_status(plan, stream=stream):
+        raise RuntimeError("encode reported a device error")
+    del scratch, ws
+    out = torch.empty(n, dtype=torch.int16, device=dev)
+
+    # ---- warm-up
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            for i in range(T):
+                dfx.dfx_decode(plan, comps[i], sizes[i], out, stream=stream)
+    stream.synchronize()
+
+    # ---- timed region: K steps x T decodes, one event per launch boundary
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps * T + 1)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            events[0].record(stream)
+            e = 1
+            for _ in range(args.steps):
+                for i in range(T):
+                    dfx.dfx_decode(plan, comps[i], sizes[i], out, stream=stream)
+                    events[e].record(stream)
+                    e += 1
+        stream.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    launch_ms = [events[j].elapsed_time(events[j + 1]) for j in range(len(events) - 1)]
+    total_ms = events[0].elapsed_time(events[-1])
+    total_ms_max = max_over_ranks(total_ms, world)
+    status = dfx.dfx_device_status(plan, stream=stream)
+
+    # ---- verification: every tensor decodes back to its input, bit for bit
+    roundtrip_ok = status == 0
+    with torch.cuda.stream(stream):
+        for i in range(T):
+            dfx.dfx_decode(plan, comps[i], sizes[i], out, stream=stream)
+            stream.synchronize()
+            roundtrip_ok &= bool(torch.equal(out, xs[i]))
+    roundtrip_ok &= dfx.dfx_device_status(plan, stream=stream) == 0
+
+    decoded_bytes = 2.0 * n * T * args.steps
+    value = sum_over_ranks(decoded_bytes, world) / (total_ms_max * 1e-3) / 1e9
+    comp_total = float(sum(sizes))
+    bits_per_weight = 8.0 * comp_total / (n * T)
+    algo_bytes_per_launch = comp_total / T + 2.0 * n
+    mean_launch_ms = statistics.mean(launch_ms)
+    achieved = algo_bytes_per_launch / (mean_launch_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    traffic = ncu_traffic_per_launch(n)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tensors": T, "weights_per_tensor": n, "chunk_symbols": K,
+                       "group_chunks": 32, "max_len": 24,
+                       "l2": "no flush: each container (~0.32 GB) and the 0.47 GB output exceed the 126 MB L2",
+                       "parallelism": f"replicas x{world} (independent tensors per GPU, no collective)"},
+            "bits_per_weight": bits_per_weight,
+            "hbm_roofline_frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS,
+            "bit_exact_roundtrip": bool(roundtrip_ok),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": algo_bytes_per_launch,
+                         "mean_launch_us": 1e3 * mean_launch_ms, "kernel": "k_decode<64>"},
+            "gpu_launches": args.steps * T,
+            "clocks": clocks.summary(),
+            "encode": {"unit": "GB/s", "value": 2.0 * n / (statistics.median(enc_ms) * 1e-3) / 1e9,
+                       "median_ms_per_tensor": statistics.median(enc_ms),
+                       "note": "dfx_encode (histogram, code book, chunk lengths, group scan, pack), BF16 bytes read / time"}}
+
+    # ---- end to end through the C ABI with host buffers
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, plan, comps, sizes, n, dev, world)
+    # ---- oracle on the host: rank 0 at N=1 only
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        line["cpu_baseline"], line["bit_exact_vs_oracle"] = run_cpu_baseline(xs[0], comps[0], K)
+    plan.free()
+    return line
+
+
+def run_e2e(args, plan, comps, sizes, n, dev, world):
+    """Containers in pinned host memory; per tensor: H2D copy, dfx_decode, D2H
+    copy of the BF16 result, on three streams so copies overlap decoding."""
+    import torch
+
+    import lossless_entropy_coded_exponent_b200 as dfx
+
+    T = len(comps)
+    host_c = [c.cpu().pin_memory() for c in comps]
+    host_out = torch.empty(n, dtype=torch.int16).pin_memory()
+    cap = max(sizes)
+    dev_c = [torch.empty(cap, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dev_o = [torch.empty(n, dtype=torch.int16, device=dev) for _ in range(2)]
+    s_in, s_dec, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+
+    def one_step():
+        h2d_done, dec_done, d2h_done = [], [], []
+        for i in range(T):
+            b = i % 2
+            if i >= 2:
+                s_in.wait_event(dec_done[i - 2])
+            with torch.cuda.stream(s_in):
+                dev_c[b][: sizes[i]].copy_(host_c[i], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(s_in)
+            h2d_done.append(ev)
+            s_dec.wait_event(ev)
+            if i >= 2:
+                s_dec.wait_event(d2h_done[i - 2])
+            dfx.dfx_decode(plan, dev_c[b], sizes[i], dev_o[b], stream=s_dec)
+            ev = torch.cuda.Event()
+            ev.record(s_dec)
+            dec_done.append(ev)
+            s_out.wait_event(ev)
+            with torch.cuda.stream(s_out):
+                host_out.copy_(dev_o[b], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(s_out)
+            d2h_done.append(ev)
+        return d2h_done[-1]
+
+    last = one_step()  # warm-up
+    last.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    s_dec.wait_event(start)
+    s_out.wait_event(start)
+    for _ in range(args.e2e_steps):
+        last = one_step()
+    s_out.wait_event(last)
+    end.record(s_out)
+    end.synchronize()
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(start.elapsed_time(end), world)
+    barrier(world)
+    value = sum_over_ranks(2.0 * n * T * args.e2e_steps, world) / (ms * 1e-3) / 1e9
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": int(sum(sizes)), "d2h_bytes_per_step": int(2 * n * T),
+            "ms_per_step": ms / args.e2e_steps, "steps": args.e2e_steps,
+            "note": "pinned host containers -> H2D -> dfx_decode -> D2H of the BF16 result, copies overlapped"}
+
+
+def run_cpu_baseline(x0, comp0, K):
+    """The oracle (single-threaded C) on tensor 0 of the stream: encode it, compare
+    the bytes with the GPU container, then time its decode."""
+    import numpy as np
+
+    import oracle
+
+    w = x0.cpu().numpy().view(np.uint16)
+    ref = oracle.encode(w, K=K)
+    gpu = comp0.cpu().numpy()
+    exact = bool(ref.size == gpu.size and np.array_equal(ref, gpu))
+    t0 = time.perf_counter()
+    dec = oracle.decode(ref)
+    dt = time.perf_counter() - t0
+    exact &= bool(np.array_equal(dec, w))
+    return ({"value": 2.0 * w.size / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+             "sample": f"tensor 0 of the stream ({w.size} weights), one oracle decode, single thread"}, exact)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+    else:
+        line = run_ours(args, world, rank, local)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,155 @@
+/*
+ * dfx.h -- C ABI of libdfx, a lossless BF16 weight codec for NVIDIA B200 (sm_100a).
+ *
+ * The problem the calls solve: store BF16 network weights smaller, losslessly,
+ * and restore them bit for bit on the GPU before use.  The weight distribution
+ * of trained networks has low entropy, so an entropy code that gives frequent
+ * values short codes removes the redundancy of the 16-bit format without
+ * changing a single bit of the decoded weights ("DFloat11: lossless LLM
+ * compression for GPU", aikraft.ru blog, section 02; a ~1.5:1 ratio on
+ * Llama 2 7B weights is reported in "From a Lossless (~1.5:1) Compression
+ * Algorithm for Llama2 7B Weights to Variable Precision, Variable Range,
+ * Compressed Numeric Data Types for CNNs and LLMs", abstract).  The GPU decoder
+ * uses lookup tables in on-chip shared memory and per-thread auxiliary
+ * position variables (the same blog, section 03, items 1 and 2).
+ *
+ * Coding scheme (this library's reading; the pages leave it open):
+ *   - every BF16 word w is split into its exponent e = (w >> 7) & 0xFF and the
+ *     sign+mantissa byte m = ((w >> 8) & 0x80) | (w & 0x7F);
+ *   - the exponents are coded with a per-tensor canonical Huffman code whose
+ *     lengths come from package-merge with a length limit (24 by default),
+ *     leaves ordered by (count, symbol value), a leaf ahead of a package of
+ *     equal weight, codes assigned in (length, symbol) order; a tensor with a
+ *     single exponent value gets a second, never-used phantom symbol (1 if the
+ *     value is 0, else 0) so both codes are 1 bit long;
+ *   - the m bytes are stored raw.
+ *
+ * Container ("DFX1", all integers little-endian, every section starts on a
+ * 16-byte boundary, every padding byte zero):
+ *   off  0  char[4] "DFX1"; u16 version = 1; u16 header_bytes = 64
+ *   off  8  u64 n                 BF16 elements
+ *   off 16  u64 total_bits        code stream length in bits
+ *   off 24  u64 total_bytes       container size
+ *   off 32  u32 K                 symbols per chunk (one decoding thread)
+ *   off 36  u32 G                 chunks per group (one warp)
+ *   off 40  u32 n_chunk = ceil(n / K);  off 44  u32 n_group = ceil(n_chunk / G)
+ *   off 48  u64 off_m             offset of the sign+mantissa plane
+ *   off 56  u32 max_len;          off 60  u32 reserved = 0
+ *   off 64  u8  len[256]          code length per exponent value, 0 = unused
+ *   off 320 u64 gbase[n_group+1]  start bit of each group; last = total_bits
+ *   then    u16 clen[n_chunk]     bit length of each chunk
+ *   then    u8  m[n]              sign+mantissa bytes in element order
+ *   then    u32 stream[]          codes MSB-first: bit k of the stream is bit
+ *                                 31 - (k mod 32) of word k / 32; the section
+ *                                 is 4*ceil(total_bits/32) bytes rounded up
+ *                                 to 16, plus 16 zero bytes
+ * Two conforming encoders produce identical bytes for the same input and
+ * parameters.
+ *
+ * Memory and streams.  The caller owns every device buffer and the stream.
+ * The library allocates device memory only inside dfx_plan (one small status
+ * buffer per plan) and frees it in dfx_free.  Every call is asynchronous and
+ * stream-ordered unless stated otherwise.  Input and output buffers must not
+ * overlap.  A plan may be used by one host thread at a time.
+ *
+ * Errors.  Every call returns DFX_OK or one of the DFX_ERR_* codes below.
+ * Argument errors are detected on the host before anything is launched.  A
+ * corrupt container is detected by the decode kernel, which never traps and
+ * never reads outside [d_comp, d_comp + comp_bytes): it records a flag in the
+ * plan's sticky device status word, read with dfx_device_status.
+ */
+#ifndef DFX_H_
+#define DFX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA runtime's stream handle (identical to the CUDA headers' typedef). */
+typedef struct CUstream_st *cudaStream_t;
+
+#define DFX_OK 0
+#define DFX_ERR_ARG 1          /* bad pointer, size, alignment or parameter */
+#define DFX_ERR_CAPACITY 2     /* output or workspace buffer too small */
+#define DFX_ERR_CORRUPT 3      /* container malformed (host check or device status) */
+#define DFX_ERR_TOO_LARGE 4    /* n >= 2^32 */
+#define DFX_ERR_CUDA 5         /* a CUDA runtime call failed */
+#define DFX_ERR_UNSUPPORTED 6  /* valid parameters this GPU path does not implement */
+
+/* Bits of the device status word (dfx_device_status). */
+#define DFX_STATUS_HEADER 0x1u  /* header disagrees with the plan or the buffer size */
+#define DFX_STATUS_TABLE 0x2u   /* code lengths above 24 or Kraft sum not exactly 1 */
+#define DFX_STATUS_INDEX 0x4u   /* group start bits or chunk lengths inconsistent */
+#define DFX_STATUS_STREAM 0x8u  /* a bit pattern that is no code, or a chunk that
+                                   did not consume exactly its stated length */
+
+typedef struct dfx_plan_s *dfx_plan_t; /* opaque, host-owned */
+
+typedef struct {
+    uint32_t chunk_symbols; /* K: 32, 64 or 128 on the GPU path (0 -> 64) */
+    uint32_t group_chunks;  /* G: 32 on the GPU path (0 -> 32) */
+    uint32_t max_len;       /* code-length limit, 8..24 (0 -> 24) */
+} dfx_params;
+
+/* Byte offsets of the container sections for given n, params and stream length. */
+typedef struct {
+    uint64_t n, n_chunk, n_group;
+    uint64_t off_len, off_gbase, off_clen, off_m, off_stream;
+    uint64_t stream_bytes, total_bytes;
+} dfx_layout;
+
+/* Library version, (major << 16) | minor. */
+uint32_t dfx_version(void);
+
+/* Static description of an error code; never NULL. */
+const char *dfx_strerror(int code);
+
+/* Host-only: container layout for n elements, params (NULL = defaults) and a
+ * stream of total_bits bits.  Pure arithmetic, no CUDA call. */
+int dfx_container_layout(uint64_t n, const dfx_params *params, uint64_t total_bits, dfx_layout *out);
+
+/* Create a plan for tensors of n BF16 elements on the current CUDA device.
+ *   params                NULL or parameters (see dfx_params; zero fields take defaults)
+ *   max_compressed_bytes  out (may be NULL): capacity an encode output buffer needs;
+ *                         an optimal code never costs more than 8 bits per exponent
+ *   workspace_bytes       out (may be NULL): device scratch size dfx_encode needs
+ * Allocates the plan's device status word.  Argument errors are returned before
+ * any CUDA call.  Synchronous. */
+int dfx_plan(dfx_plan_t *plan, uint64_t n, const dfx_params *params,
+             size_t *max_compressed_bytes, size_t *workspace_bytes);
+
+/* Encode n BF16 elements (d_bf16, device, 16-byte aligned) into a DFX1
+ * container at d_out (device, 16-byte aligned, out_capacity >=
+ * max_compressed_bytes).  d_workspace: device scratch of workspace_bytes
+ * (16-byte aligned), contents on entry ignored.  The bytes of d_out past the
+ * container's end, up to max_compressed_bytes, are zeroed.
+ * h_compressed_bytes: NULL keeps the call asynchronous; otherwise the call
+ * synchronises the stream and stores the container size.  The size is also
+ * in the header at byte offset 24 (u64). */
+int dfx_encode(dfx_plan_t plan, const void *d_bf16, void *d_out, size_t out_capacity,
+               void *d_workspace, size_t workspace_bytes, size_t *h_compressed_bytes,
+               cudaStream_t stream);
+
+/* Decode a DFX1 container (d_comp, device, 16-byte aligned, comp_bytes long,
+ * produced with this plan's n and parameters) into n BF16 elements at d_bf16
+ * (device, 16-byte aligned).  One kernel launch.  A malformed container sets
+ * bits of the plan's device status word and leaves d_bf16 partly unwritten;
+ * the call itself only reports host-side errors. */
+int dfx_decode(dfx_plan_t plan, const void *d_comp, size_t comp_bytes, void *d_bf16,
+               cudaStream_t stream);
+
+/* Synchronise `stream`, return the plan's sticky device status word in
+ * *h_status (0 = no corruption seen since the last read) and clear it. */
+int dfx_device_status(dfx_plan_t plan, cudaStream_t stream, uint32_t *h_status);
+
+/* Release the plan and its device status word.  NULL is accepted. */
+int dfx_free(dfx_plan_t plan);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DFX_H_ */

@@ -1,0 +1,208 @@
+// api.cu -- the C ABI declared in include/dfx.h: argument checks, plans, launches.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#include "dfx.h"
+#include "dfx_common.cuh"
+
+struct dfx_plan_s {
+    uint64_t n;
+    uint32_t K, G, max_len;
+    dfx::Layout L;
+    uint64_t max_bytes;
+    uint64_t ws_bytes;
+    uint32_t* d_status;
+    int device;
+    int decode_grid;
+};
+
+namespace {
+
+int resolve_params(const dfx_params* p, uint32_t* K, uint32_t* G, uint32_t* L) {
+    *K = (p && p->chunk_symbols) ? p->chunk_symbols : 64u;
+    *G = (p && p->group_chunks) ? p->group_chunks : 32u;
+    *L = (p && p->max_len) ? p->max_len : 24u;
+    if (*L < 8 || *L > dfx::kMaxLenLimit) return DFX_ERR_ARG;
+    if ((uint64_t)(*K) * (*L) > 65535u) return DFX_ERR_ARG;  // a chunk's bit length must fit u16
+    return DFX_OK;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int check_device(const dfx_plan_s* plan) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DFX_ERR_CUDA;
+    return dev == plan->device ? DFX_OK : DFX_ERR_ARG;
+}
+
+}  // namespace
+
+extern "C" {
+
+uint32_t dfx_version(void) { return (1u << 16) | 0u; }
+
+const char* dfx_strerror(int code) {
+    switch (code) {
+        case DFX_OK: return "ok";
+        case DFX_ERR_ARG: return "invalid argument (pointer, size, alignment or parameter)";
+        case DFX_ERR_CAPACITY: return "output or workspace buffer too small";
+        case DFX_ERR_CORRUPT: return "container is malformed";
+        case DFX_ERR_TOO_LARGE: return "tensor too large (n must be below 2^32)";
+        case DFX_ERR_CUDA: return "CUDA runtime error";
+        case DFX_ERR_UNSUPPORTED: return "parameters not implemented by the GPU path";
+        default: return "unknown error code";
+    }
+}
+
+int dfx_container_layout(uint64_t n, const dfx_params* params, uint64_t total_bits, dfx_layout* out) {
+    if (!out) return DFX_ERR_ARG;
+    if (n >= (1ull << 32)) return DFX_ERR_TOO_LARGE;
+    uint32_t K, G, L;
+    int rc = resolve_params(params, &K, &G, &L);
+    if (rc) return rc;
+    if (G < 1) return DFX_ERR_ARG;
+    const dfx::Layout lay = dfx::make_layout(n, K, G);
+    out->n = n;
+    out->n_chunk = lay.n_chunk;
+    out->n_group = lay.n_group;
+    out->off_len = dfx::kOffLen;
+    out->off_gbase = dfx::kOffGbase;
+    out->off_clen = lay.off_clen;
+    out->off_m = lay.off_m;
+    out->off_stream = lay.off_stream;
+    out->stream_bytes = dfx::stream_bytes(total_bits);
+    out->total_bytes = lay.off_stream + out->stream_bytes;
+    return DFX_OK;
+}
+
+int dfx_plan(dfx_plan_t* plan, uint64_t n, const dfx_params* params, size_t* max_compressed_bytes,
+             size_t* workspace_bytes) {
+    if (!plan) return DFX_ERR_ARG;
+    *plan = nullptr;
+    if (n >= (1ull << 32)) return DFX_ERR_TOO_LARGE;
+    uint32_t K, G, L;
+    int rc = resolve_params(params, &K, &G, &L);
+    if (rc) return rc;
+    if (!dfx::decode_supports(K, G)) return DFX_ERR_UNSUPPORTED;
+
+    dfx_plan_s* p = (dfx_plan_s*)calloc(1, sizeof(dfx_plan_s));
+    if (!p) return DFX_ERR_ARG;
+    p->n = n;
+    p->K = K;
+    p->G = G;
+    p->max_len = L;
+    p->L = dfx::make_layout(n, K, G);
+    p->max_bytes = p->L.off_stream + dfx::stream_bytes(8 * n);  // optimal codes never exceed 8 bits/symbol
+    p->ws_bytes = dfx::workspace_bytes_for(p->L.n_group);
+    int sms = 0;
+    if (cudaGetDevice(&p->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess ||
+        cudaMalloc((void**)&p->d_status, 256) != cudaSuccess || cudaMemset(p->d_status, 0, 256) != cudaSuccess) {
+        cudaGetLastError();
+        if (p->d_status) cudaFree(p->d_status);
+        free(p);
+        return DFX_ERR_CUDA;
+    }
+    const uint64_t warps = dfx::decode_blocks_per_sm(K) * (uint64_t)sms;  // resident CTAs
+    const uint64_t need = (p->L.n_group + 7) / 8;                          // CTAs with work (8 warps each)
+    p->decode_grid = (int)(need == 0 ? 1 : (need < warps ? need : warps));
+    if (max_compressed_bytes) *max_compressed_bytes = (size_t)p->max_bytes;
+    if (workspace_bytes) *workspace_bytes = (size_t)p->ws_bytes;
+    *plan = p;
+    return DFX_OK;
+}
+
+int dfx_encode(dfx_plan_t plan, const void* d_bf16, void* d_out, size_t out_capacity, void* d_workspace,
+               size_t workspace_bytes, size_t* h_compressed_bytes, cudaStream_t stream) {
+    if (!plan) return DFX_ERR_ARG;
+    if (!d_out || !d_workspace || (!d_bf16 && plan->n)) return DFX_ERR_ARG;
+    if (!aligned16(d_bf16) || !aligned16(d_out) || !aligned16(d_workspace)) return DFX_ERR_ARG;
+    if (out_capacity < plan->max_bytes || workspace_bytes < plan->ws_bytes) return DFX_ERR_CAPACITY;
+    int rc = check_device(plan);
+    if (rc) return rc;
+    dfx::EncodeArgs a;
+    a.in = (const uint16_t*)d_bf16;
+    a.out = (uint8_t*)d_out;
+    a.n = plan->n;
+    a.K = plan->K;
+    a.G = plan->G;
+    a.max_len = plan->max_len;
+    a.n_chunk = (uint32_t)plan->L.n_chunk;
+    a.n_group = (uint32_t)plan->L.n_group;
+    a.off_clen = plan->L.off_clen;
+    a.off_m = plan->L.off_m;
+    a.off_stream = plan->L.off_stream;
+    uint8_t* ws = (uint8_t*)d_workspace;
+    a.ws_counts = (unsigned long long*)(ws + dfx::kWsCounts);
+    a.ws_code = (uint32_t*)(ws + dfx::kWsCode);
+    a.ws_len = ws + dfx::kWsLen;
+    a.ws_group_bits = (uint32_t*)(ws + dfx::kWsGroupBits);
+    a.status = plan->d_status;
+    if (dfx::launch_encode(a, plan->max_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return DFX_ERR_CUDA;
+    }
+    if (h_compressed_bytes) {
+        unsigned long long total = 0;
+        if (cudaMemcpyAsync(&total, a.out + 24, 8, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+            cudaStreamSynchronize(stream) != cudaSuccess) {
+            cudaGetLastError();
+            return DFX_ERR_CUDA;
+        }
+        *h_compressed_bytes = (size_t)total;
+    }
+    return DFX_OK;
+}
+
+int dfx_decode(dfx_plan_t plan, const void* d_comp, size_t comp_bytes, void* d_bf16, cudaStream_t stream) {
+    if (!plan) return DFX_ERR_ARG;
+    if (!d_comp || (!d_bf16 && plan->n)) return DFX_ERR_ARG;
+    if (!aligned16(d_comp) || !aligned16(d_bf16)) return DFX_ERR_ARG;
+    if (comp_bytes < plan->L.off_stream + dfx::stream_bytes(0)) return DFX_ERR_CORRUPT;
+    int rc = check_device(plan);
+    if (rc) return rc;
+    dfx::DecodeArgs a;
+    a.comp = (const uint8_t*)d_comp;
+    a.comp_bytes = comp_bytes;
+    a.out = (uint16_t*)d_bf16;
+    a.n = plan->n;
+    a.K = plan->K;
+    a.G = plan->G;
+    a.n_chunk = (uint32_t)plan->L.n_chunk;
+    a.n_group = (uint32_t)plan->L.n_group;
+    a.off_clen = plan->L.off_clen;
+    a.off_m = plan->L.off_m;
+    a.off_stream = plan->L.off_stream;
+    a.status = plan->d_status;
+    if (dfx::launch_decode(a, plan->decode_grid, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return DFX_ERR_CUDA;
+    }
+    return DFX_OK;
+}
+
+int dfx_device_status(dfx_plan_t plan, cudaStream_t stream, uint32_t* h_status) {
+    if (!plan || !h_status) return DFX_ERR_ARG;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, plan->d_status, 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaMemsetAsync(plan->d_status, 0, 4, stream) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return DFX_ERR_CUDA;
+    }
+    *h_status = v;
+    return DFX_OK;
+}
+
+int dfx_free(dfx_plan_t plan) {
+    if (!plan) return DFX_OK;
+    int rc = DFX_OK;
+    if (plan->d_status && cudaFree(plan->d_status) != cudaSuccess) {
+        cudaGetLastError();
+        rc = DFX_ERR_CUDA;
+    }
+    free(plan);
+    return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,84 @@
+// dfx_common.cuh -- definitions shared by the libdfx CUDA sources (encode,
+// decode, C ABI).  The container rules are stated in include/dfx.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dfx.h"
+
+namespace dfx {
+
+constexpr uint32_t kHeaderBytes = 64;
+constexpr uint32_t kOffLen = 64;
+constexpr uint32_t kOffGbase = 320;
+constexpr uint32_t kMaxLenLimit = 24;   // longest code the decoder tables support
+constexpr uint32_t kWarp = 32;
+
+__host__ __device__ inline uint64_t align16(uint64_t x) { return (x + 15u) & ~uint64_t(15); }
+
+struct Layout {
+    uint64_t n, n_chunk, n_group;
+    uint64_t off_clen, off_m, off_stream;
+    uint32_t K, G;
+};
+
+__host__ __device__ inline Layout make_layout(uint64_t n, uint32_t K, uint32_t G) {
+    Layout L;
+    L.n = n;
+    L.K = K;
+    L.G = G;
+    L.n_chunk = (n + K - 1) / K;
+    L.n_group = (L.n_chunk + G - 1) / G;
+    L.off_clen = align16(kOffGbase + 8 * (L.n_group + 1));
+    L.off_m = align16(L.off_clen + 2 * L.n_chunk);
+    L.off_stream = align16(L.off_m + n);
+    return L;
+}
+
+__host__ __device__ inline uint64_t stream_bytes(uint64_t total_bits) {
+    return align16(4 * ((total_bits + 31) / 32)) + 16;
+}
+
+// Every piece of state a decode launch needs, passed by value.
+struct DecodeArgs {
+    const uint8_t* comp;
+    uint64_t comp_bytes;
+    uint16_t* out;
+    uint64_t n;
+    uint32_t K, G;
+    uint32_t n_chunk, n_group;
+    uint64_t off_clen, off_m, off_stream;
+    uint32_t* status;
+};
+
+struct EncodeArgs {
+    const uint16_t* in;
+    uint8_t* out;
+    uint64_t n;
+    uint32_t K, G, max_len;
+    uint32_t n_chunk, n_group;
+    uint64_t off_clen, off_m, off_stream;
+    unsigned long long* ws_counts;  // [256]
+    uint32_t* ws_code;              // [256]
+    uint8_t* ws_len;                // [256]
+    uint32_t* ws_group_bits;        // [n_group]
+    uint32_t* status;
+};
+
+// Workspace layout for encode.
+constexpr uint64_t kWsCounts = 0;
+constexpr uint64_t kWsCode = 2048;
+constexpr uint64_t kWsLen = 3072;
+constexpr uint64_t kWsGroupBits = 4096;
+inline uint64_t workspace_bytes_for(uint64_t n_group) {
+    return (kWsGroupBits + 4 * n_group + 255) & ~uint64_t(255);
+}
+
+// Launchers (encode.cu / decode.cu).
+cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, int grid, cudaStream_t s);
+int decode_blocks_per_sm(uint32_t K);
+bool decode_supports(uint32_t K, uint32_t G);
+
+}  // namespace dfx

@@ -1,0 +1,442 @@
+// encode.cu -- GPU encoder for DFX1 containers (sm_100a).
+//
+// Passes, all stream-ordered on the caller's stream:
+//   0. zero the container's index region and everything after the m plane;
+//   1. k_histogram      exponent histogram, warp-aggregated shared-memory atomics;
+//   2. k_build_codebook one CTA: package-merge code lengths (limit max_len), canonical codes,
+//                       len[256] and the constant header fields;
+//   3. k_chunk_bits     per chunk of K elements its code bits (clen), per group of 32 chunks
+//                       the sum;
+//   4. k_group_scan     one CTA: exclusive scan of the group sums -> gbase, total_bits,
+//                       total_bytes;
+//   5. k_pack           per chunk: start bit from gbase + warp scan of clen, codes packed
+//                       MSB-first into 32-bit words, m bytes written.
+// The method: frequent exponent values get short codes ("DFloat11: lossless LLM
+// compression for GPU", aikraft.ru blog, section 02); the exact code and layout rules
+// are the ones stated in include/dfx.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dfx_common.cuh"
+
+namespace dfx {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, unsigned lane) {
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        uint32_t y = __shfl_up_sync(kFull, v, d);
+        if (lane >= (unsigned)d) v += y;
+    }
+    return v;
+}
+
+__device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long long v, unsigned lane) {
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        unsigned long long y = __shfl_up_sync(kFull, v, d);
+        if (lane >= (unsigned)d) v += y;
+    }
+    return v;
+}
+
+// ---------------------------------------------------------------- 1. histogram
+
+constexpr int kHistThreads = 512;
+
+__global__ void __launch_bounds__(kHistThreads) k_histogram(const uint16_t* __restrict__ in, uint64_t n,
+                                                          unsigned long long* __restrict__ counts) {
+    __shared__ uint32_t h[256];
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0;
+    __syncthreads();
+    const unsigned lane = threadIdx.x & 31;
+    const uint4* in4 = reinterpret_cast<const uint4*>(in);
+    const uint64_t n8 = n / 8;
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    // `base` is warp-uniform, so every lane reaches each __match_any_sync together.
+    for (uint64_t base = (uint64_t)blockIdx.x * blockDim.x; base < n8; base += stride) {
+        const uint64_t i = base + threadIdx.x;
+        const bool valid = i < n8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (valid) v = __ldg(in4 + i);
+        const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            const uint32_t e = valid ? ((words[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu) : 256u;
+            const unsigned peers = __match_any_sync(kFull, e);
+            if (e < 256u && lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&h[e], (uint32_t)__popc(peers));
+        }
+    }
+    if (blockIdx.x == 0 && threadIdx.x < (n & 7)) {
+        const uint64_t i = n8 * 8 + threadIdx.x;
+        atomicAdd(&h[(in[i] >> 7) & 0xFFu], 1u);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256; i += blockDim.x)
+        if (h[i]) atomicAdd(&counts[i], (unsigned long long)h[i]);
+}
+
+// ---------------------------------------------------------------- 2. code book
+//
+// Package-merge, computed level by level with merge ranks instead of explicit
+// package trees.  List 0 is the leaves sorted by (count, symbol).  List j merges
+// the leaves with the packages of list j-1 (pairs of consecutive items, a trailing
+// odd item dropped), a leaf ahead of a package of equal weight.  A leaf's rank in
+// list j is its index plus the number of packages lighter than it; a package's
+// rank is its index plus the number of leaves not heavier than it.  The first
+// 2m-2 items of the last list are selected.  Selected items of every list form a
+// prefix, and the packages inside the prefix of list j are its first p_j packages,
+// which expand to the first 2 p_j items of list j-1.  So walking back from the
+// last list, q_j = number of leaves in the selected prefix of list j, and the
+// length of the leaf of sorted rank i is the number of lists with i < q_j.
+
+__global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
+    __shared__ unsigned long long cnt[256];
+    __shared__ unsigned long long leafw[256];
+    __shared__ uint8_t leafsym[256];
+    __shared__ unsigned long long lw[2][512];
+    __shared__ unsigned long long pkw[256];
+    __shared__ uint16_t leafpos[kMaxLenLimit][256];
+    __shared__ int qsel[kMaxLenLimit];
+    __shared__ uint8_t lens[256];
+    __shared__ uint32_t nlen[kMaxLenLimit + 1];
+    __shared__ uint32_t firstc[kMaxLenLimit + 1];
+
+    const int t = threadIdx.x;
+    const int L = (int)a.max_len;
+    const unsigned long long c = a.ws_counts[t];
+    cnt[t] = c;
+    lens[t] = 0;
+    if (t <= (int)kMaxLenLimit) nlen[t] = 0;
+    const bool used = c > 0;
+    const int m = __syncthreads_count(used);
+
+    if (m == 1) {
+        // one exponent value: it and a phantom partner both get 1-bit codes
+        if (used) {
+            lens[t] = 1;
+            lens[t == 0 ? 1 : 0] = 1;
+        }
+    } else if (m >= 2) {
+        if (used) {
+            int r = 0;
+            for (int s = 0; s < 256; s++) {
+                const unsigned long long cs = cnt[s];
+                r += (cs > 0) && (cs < c || (cs == c && s < t));
+            }
+            leafw[r] = c;
+            leafsym[r] = (uint8_t)t;
+        }
+        __syncthreads();
+        if (t < m) lw[0][t] = leafw[t];
+        int size = m;
+        __syncthreads();
+        for (int j = 1; j < L; j++) {
+            const unsigned long long* prev = lw[(j - 1) & 1];
+            unsigned long long* cur = lw[j & 1];
+            const int np = size / 2;
+            if (t < np) pkw[t] = prev[2 * t] + prev[2 * t + 1];
+            __syncthreads();
+            if (t < m) {
+                const unsigned long long w = leafw[t];
+                int lo = 0, hi = np;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (pkw[mid] < w) lo = mid + 1;
+                    else hi = mid;
+                }
+                cur[t + lo] = w;
+                leafpos[j][t] = (uint16_t)(t + lo);
+            }
+            if (t < np) {
+                const unsigned long long w = pkw[t];
+                int lo = 0, hi = m;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (leafw[mid] <= w) lo = mid + 1;
+                    else hi = mid;
+                }
+                cur[t + lo] = w;
+            }
+            size = m + np;
+            __syncthreads();
+        }
+        if (t == 0) {
+            int s = 2 * m - 2;
+            for (int j = L - 1; j >= 1; j--) {
+                int lo = 0, hi = m;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (leafpos[j][mid] < s) lo = mid + 1;
+                    else hi = mid;
+                }
+                qsel[j] = lo;
+                s = 2 * (s - lo);
+            }
+            qsel[0] = s;
+        }
+        __syncthreads();
+        if (t < m) {
+            int l = 0;
+            for (int j = 0; j < L; j++) l += (t < qsel[j]);
+            lens[leafsym[t]] = (uint8_t)l;
+        }
+    }
+    __syncthreads();
+
+    // canonical codes: first code per length, then rank among equal lengths by symbol
+    const uint32_t l = lens[t];
+    if (l) atomicAdd(&nlen[l], 1u);
+    __syncthreads();
+    if (t == 0) {
+        uint32_t code = 0;
+        for (int k = 1; k <= (int)kMaxLenLimit; k++) {
+            firstc[k] = code;
+            code = (code + nlen[k]) << 1;
+        }
+    }
+    __syncthreads();
+    uint32_t code = 0;
+    if (l) {
+        uint32_t r = 0;
+        for (int s = 0; s < t; s++) r += (lens[s] == l);
+        code = firstc[l] + r;
+    }
+    a.ws_code[t] = code;
+    a.ws_len[t] = (uint8_t)l;
+    a.out[kOffLen + t] = (uint8_t)l;
+
+    if (t == 0) {
+        uint8_t* h = a.out;
+        *reinterpret_cast<uint32_t*>(h + 0) = 0x31584644u;  // "DFX1"
+        *reinterpret_cast<uint16_t*>(h + 4) = 1;
+        *reinterpret_cast<uint16_t*>(h + 6) = (uint16_t)kHeaderBytes;
+        *reinterpret_cast<unsigned long long*>(h + 8) = a.n;
+        *reinterpret_cast<uint32_t*>(h + 32) = a.K;
+        *reinterpret_cast<uint32_t*>(h + 36) = a.G;
+        *reinterpret_cast<uint32_t*>(h + 40) = a.n_chunk;
+        *reinterpret_cast<uint32_t*>(h + 44) = a.n_group;
+        *reinterpret_cast<unsigned long long*>(h + 48) = a.off_m;
+        *reinterpret_cast<uint32_t*>(h + 56) = a.max_len;
+        *reinterpret_cast<uint32_t*>(h + 60) = 0;
+    }
+}
+
+// ---------------------------------------------------------------- 3. chunk bit lengths
+
+constexpr int kChunkThreads = 256;
+
+__device__ __forceinline__ uint32_t bits8(uint4 v, const uint8_t* lt) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t b = 0;
+#pragma unroll
+    for (int k = 0; k < 4; k++) b += lt[(w[k] >> 7) & 0xFFu] + lt[(w[k] >> 23) & 0xFFu];
+    return b;
+}
+
+template <int K>
+__global__ void __launch_bounds__(kChunkThreads) k_chunk_bits(EncodeArgs a) {
+    __shared__ uint8_t lt[256];
+    lt[threadIdx.x] = a.ws_len[threadIdx.x];
+    __syncthreads();
+    const uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const unsigned lane = threadIdx.x & 31;
+    uint32_t bits = 0;
+    if (c < a.n_chunk) {
+        const uint64_t i0 = c * K;
+        if (i0 + K <= a.n) {
+            const uint4* p = reinterpret_cast<const uint4*>(a.in + i0);
+#pragma unroll 4
+            for (int v = 0; v < K / 8; v++) bits += bits8(__ldg(p + v), lt);
+        } else {
+            for (uint64_t i = i0; i < a.n; i++) bits += lt[(a.in[i] >> 7) & 0xFFu];
+        }
+        reinterpret_cast<uint16_t*>(a.out + a.off_clen)[c] = (uint16_t)bits;
+    }
+    const uint32_t incl = warp_incl_scan(bits, lane);
+    const uint64_t g = c / 32;
+    if (lane == 31 && g < a.n_group) a.ws_group_bits[g] = incl;
+}
+
+// ---------------------------------------------------------------- 4. group scan
+
+constexpr int kScanThreads = 1024;
+constexpr int kScanItems = 4;
+
+__global__ void __launch_bounds__(kScanThreads) k_group_scan(EncodeArgs a) {
+    __shared__ unsigned long long wsum[32];
+    const unsigned t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    unsigned long long* gbase = reinterpret_cast<unsigned long long*>(a.out + kOffGbase);
+    unsigned long long carry = 0;
+    for (uint64_t base = 0; base < a.n_group; base += (uint64_t)kScanThreads * kScanItems) {
+        const uint64_t i = base + (uint64_t)t * kScanItems;
+        uint32_t v[kScanItems];
+        unsigned long long local = 0;
+#pragma unroll
+        for (int k = 0; k < kScanItems; k++) {
+            v[k] = (i + k < a.n_group) ? a.ws_group_bits[i + k] : 0u;
+            local += v[k];
+        }
+        const unsigned long long incl = warp_incl_scan64(local, lane);
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) wsum[lane] = warp_incl_scan64(wsum[lane], lane);
+        __syncthreads();
+        unsigned long long run = carry + (warp ? wsum[warp - 1] : 0ull) + incl - local;
+#pragma unroll
+        for (int k = 0; k < kScanItems; k++)
+            if (i + k < a.n_group) {
+                gbase[i + k] = run;
+                run += v[k];
+            }
+        carry += wsum[31];
+        __syncthreads();
+    }
+    if (t == 0) {
+        gbase[a.n_group] = carry;
+        *reinterpret_cast<unsigned long long*>(a.out + 16) = carry;
+        *reinterpret_cast<unsigned long long*>(a.out + 24) = a.off_stream + stream_bytes(carry);
+    }
+}
+
+// ---------------------------------------------------------------- 5. pack
+
+constexpr int kPackThreads = 256;
+
+struct BitWriter {
+    uint32_t* stream;
+    uint64_t wi;     // index of the word being assembled
+    uint32_t fill;   // bits already in `cur`
+    uint32_t cur;
+    bool first;      // the first emitted word may hold bits of the previous chunk
+
+    __device__ __forceinline__ void emit() {
+        if (first) {
+            atomicOr(stream + wi, cur);
+            first = false;
+        } else {
+            stream[wi] = cur;
+        }
+        wi++;
+    }
+    __device__ __forceinline__ void put(uint32_t code, uint32_t l) {
+        const uint32_t total = fill + l;
+        if (total < 32) {
+            cur |= code << (32 - total);
+            fill = total;
+        } else {
+            const uint32_t over = total - 32;
+            cur |= code >> over;
+            emit();
+            cur = over ? (code << (32 - over)) : 0u;
+            fill = over;
+        }
+    }
+    __device__ __forceinline__ void finish() {
+        if (fill) atomicOr(stream + wi, cur);  // shared with the next chunk
+    }
+};
+
+template <int K>
+__global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
+    __shared__ uint32_t code_sh[256];
+    __shared__ uint8_t len_sh[256];
+    code_sh[threadIdx.x] = a.ws_code[threadIdx.x];
+    len_sh[threadIdx.x] = a.ws_len[threadIdx.x];
+    __syncthreads();
+    const uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const unsigned lane = threadIdx.x & 31;
+    const uint16_t* clen = reinterpret_cast<const uint16_t*>(a.out + a.off_clen);
+    const uint32_t cl = (c < a.n_chunk) ? clen[c] : 0u;
+    const uint32_t incl = warp_incl_scan(cl, lane);
+    if (c >= a.n_chunk) return;
+    const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.out + kOffGbase);
+    const uint64_t start = gbase[c / 32] + (incl - cl);
+
+    BitWriter bw;
+    bw.stream = reinterpret_cast<uint32_t*>(a.out + a.off_stream);
+    bw.wi = start >> 5;
+    bw.fill = (uint32_t)(start & 31);
+    bw.cur = 0;
+    bw.first = true;
+    uint8_t* mpl = a.out + a.off_m;
+
+    const uint64_t i0 = c * K;
+    if (i0 + K <= a.n) {
+        const uint4* p = reinterpret_cast<const uint4*>(a.in + i0);
+        for (int v = 0; v < K / 8; v++) {
+            const uint4 x = __ldg(p + v);
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+            uint32_t mb[2] = {0u, 0u};
+#pragma unroll
+            for (int k = 0; k < 8; k++) {
+                const uint32_t h = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+                const uint32_t e = (h >> 7) & 0xFFu;
+                const uint32_t m = ((h >> 8) & 0x80u) | (h & 0x7Fu);
+                bw.put(code_sh[e], len_sh[e]);
+                mb[k >> 2] |= m << (8 * (k & 3));
+            }
+            *reinterpret_cast<uint2*>(mpl + i0 + 8 * v) = make_uint2(mb[0], mb[1]);
+        }
+    } else {
+        for (uint64_t i = i0; i < a.n; i++) {
+            const uint32_t h = a.in[i];
+            const uint32_t e = (h >> 7) & 0xFFu;
+            bw.put(code_sh[e], len_sh[e]);
+            mpl[i] = (uint8_t)(((h >> 8) & 0x80u) | (h & 0x7Fu));
+        }
+    }
+    bw.finish();
+}
+
+template <int K>
+cudaError_t launch_chunk_passes(const EncodeArgs& a, int phase, cudaStream_t s) {
+    const unsigned blocks = (unsigned)((a.n_chunk + kChunkThreads - 1) / kChunkThreads);
+    if (phase == 0) k_chunk_bits<K><<<blocks, kChunkThreads, 0, s>>>(a);
+    else k_pack<K><<<blocks, kPackThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t s) {
+    cudaError_t err;
+    // index region (header .. clen padding) and everything after the m plane start at zero
+    if ((err = cudaMemsetAsync(a.out, 0, a.off_m, s)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(a.out + a.off_m + a.n, 0, max_bytes - (a.off_m + a.n), s)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(a.ws_counts, 0, 256 * sizeof(unsigned long long), s)) != cudaSuccess) return err;
+
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const uint64_t units = (a.n / 8 + kHistThreads - 1) / kHistThreads;
+    const unsigned hist_blocks = (unsigned)(units == 0 ? 1 : (units < (uint64_t)sms * 4 ? units : (uint64_t)sms * 4));
+    k_histogram<<<hist_blocks, kHistThreads, 0, s>>>(a.in, a.n, a.ws_counts);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    k_build_codebook<<<1, 256, 0, s>>>(a);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (a.n_chunk) {
+        switch (a.K) {
+            case 32: err = launch_chunk_passes<32>(a, 0, s); break;
+            case 64: err = launch_chunk_passes<64>(a, 0, s); break;
+            case 128: err = launch_chunk_passes<128>(a, 0, s); break;
+            default: return cudaErrorInvalidValue;
+        }
+        if (err != cudaSuccess) return err;
+    }
+    k_group_scan<<<1, kScanThreads, 0, s>>>(a);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (a.n_chunk) {
+        switch (a.K) {
+            case 32: err = launch_chunk_passes<32>(a, 1, s); break;
+            case 64: err = launch_chunk_passes<64>(a, 1, s); break;
+            case 128: err = launch_chunk_passes<128>(a, 1, s); break;
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    return err;
+}
+
+}  // namespace dfx

@@ -1,0 +1,86 @@
+"""Host-side checks of libdfx that need no GPU: the shared library loads, exports
+every symbol include/dfx.h declares, its layout arithmetic agrees with the
+oracle's, and argument errors come back before any CUDA call."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import lossless_entropy_coded_exponent_b200 as dfx
+from lossless_entropy_coded_exponent_b200 import build as dfx_build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "dfx.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dfx_build.build()
+    return dfx.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(dfx_\w+)\s*\(", src, flags=re.M)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(dfx.EXPORTS)
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_version_and_strerror(lib):
+    assert dfx.dfx_version() >> 16 == 1
+    for code in range(0, 8):
+        assert isinstance(dfx.dfx_strerror(code), str) and dfx.dfx_strerror(code)
+    assert dfx.dfx_strerror(dfx.DFX_OK) == "ok"
+
+
+@pytest.mark.parametrize("n", [0, 1, 7, 4097, 1_000_003, 1 << 20, 234_881_024])
+@pytest.mark.parametrize("K", [32, 64, 128])
+def test_layout_agrees_with_oracle(lib, n, K):
+    for total_bits in (0, 1, 31, 32, 33, 8 * n):
+        lay = dfx.dfx_container_layout(n, total_bits, chunk_symbols=K)
+        assert lay["total_bytes"] == oracle.container_bytes(n, K, 32, total_bits)
+        assert lay["n_chunk"] == -(-n // K) and lay["n_group"] == -(-lay["n_chunk"] // 32)
+        for key in ("off_clen", "off_m", "off_stream"):
+            assert lay[key] % 16 == 0
+    assert dfx.dfx_container_layout(n, 8 * n, chunk_symbols=K)["total_bytes"] == oracle.max_container_bytes(n, K, 32)
+
+
+def test_layout_matches_an_oracle_container(lib):
+    w = np.arange(5000, dtype=np.uint16)
+    c = oracle.encode(w, K=64)
+    total_bits = int(c[16:24].view(np.uint64)[0])
+    lay = dfx.dfx_container_layout(w.size, total_bits, chunk_symbols=64)
+    assert lay["total_bytes"] == c.size
+    assert lay["off_m"] == int(c[48:56].view(np.uint64)[0])
+
+
+def test_host_argument_errors_precede_cuda(lib):
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_plan(1 << 32)
+    assert e.value.code == dfx.DFX_ERR_TOO_LARGE
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_plan(1000, max_len=7)
+    assert e.value.code == dfx.DFX_ERR_ARG
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_plan(1000, chunk_symbols=96)
+    assert e.value.code == dfx.DFX_ERR_UNSUPPORTED
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_plan(1000, group_chunks=16)
+    assert e.value.code == dfx.DFX_ERR_UNSUPPORTED
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_container_layout(10, 0, chunk_symbols=4000)
+    assert e.value.code == dfx.DFX_ERR_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(dfx, "_lib_handle", None)
+    monkeypatch.setattr(dfx, "LIB_PATH", str(tmp_path / "libdfx.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        dfx.dfx_version()
