@@ -148,6 +148,24 @@ int dfx_device_status(dfx_plan_t plan, cudaStream_t stream, uint32_t *h_status);
 /* Release the plan and its device status word.  NULL is accepted. */
 int dfx_free(dfx_plan_t plan);
 
+/* dfx_encode for callers that cannot allocate device memory.  No page has a
+ * counterpart: it exists for processes whose device memory belongs to another
+ * allocator (a serving pool that reserves nearly all HBM up front) or that must
+ * never risk the implicit synchronisation of cudaFree.  It needs no plan and no
+ * workspace; its scratch is a fixed array in the library's device memory
+ * (1 MiB + 4.25 KiB per GPU that loads the library, held until exit).
+ *   d_bf16, n, params, d_out, out_capacity, h_compressed_bytes, stream: as in
+ *   dfx_plan + dfx_encode (out_capacity >= the plan's max_compressed_bytes).
+ * Limit: at most 262144 groups of 32 chunks (n <= 2^28 with K = 32, 2^29 with
+ * K = 64, 2^30 with K = 128); larger n returns DFX_ERR_CAPACITY before any work.
+ * All calls on a device share the scratch array and it keeps the last call's
+ * contents; calls whose GPU work overlaps race and corrupt each other, so order
+ * them on one stream.  The first call on a device looks up the array's address
+ * with that device current; make it before any stream capture.  Produces the
+ * same bytes as dfx_encode. */
+int dfx_encode_static(const void *d_bf16, uint64_t n, const dfx_params *params, void *d_out,
+                      size_t out_capacity, size_t *h_compressed_bytes, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

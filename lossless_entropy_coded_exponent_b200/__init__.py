@@ -38,6 +38,7 @@ EXPORTS = (
     "dfx_decode",
     "dfx_device_status",
     "dfx_free",
+    "dfx_encode_static",
 )
 
 
@@ -82,7 +83,10 @@ def lib() -> ctypes.CDLL:
         L.dfx_decode.argtypes = [vp, vp, ctypes.c_size_t, vp, vp]
         L.dfx_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.dfx_free.argtypes = [vp]
-        for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_device_status", "dfx_free"):
+        L.dfx_encode_static.argtypes = [vp, ctypes.c_uint64, ctypes.POINTER(dfx_params), vp, ctypes.c_size_t,
+                                        ctypes.POINTER(ctypes.c_size_t), vp]
+        for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_device_status", "dfx_free",
+                  "dfx_encode_static"):
             getattr(L, f).restype = ctypes.c_int
         _lib_handle = L
     return _lib_handle
@@ -187,6 +191,18 @@ def dfx_device_status(plan: Plan, stream=None) -> int:
 
 def dfx_free(plan: Plan) -> None:
     plan.free()
+
+
+def dfx_encode_static(d_bf16, n: int, d_out, out_capacity: int, want_size: bool = False, stream=None,
+                      chunk_symbols: int = 0, group_chunks: int = 0, max_len: int = 0) -> int | None:
+    """Encode without any device allocation by the library (no plan, no workspace);
+    for callers whose device memory is owned by another allocator."""
+    size = ctypes.c_size_t()
+    p = _params(chunk_symbols, group_chunks, max_len)
+    rc = lib().dfx_encode_static(_ptr(d_bf16), n, ctypes.byref(p), _ptr(d_out), out_capacity,
+                                 ctypes.byref(size) if want_size else None, _stream(stream))
+    _check(rc, "dfx_encode_static")
+    return size.value if want_size else None
 
 
 # ---------------------------------------------------------------- tensor helpers

@@ -1,0 +1,114 @@
+// encode_static.cu -- dfx_encode_static: the encoder for callers that cannot allocate
+// device memory.
+//
+// Some callers of a weight codec may not call cudaMalloc or cudaFree at all: a serving
+// process whose device memory belongs to its own pool allocator (it reserves nearly all
+// of HBM at start-up, so a raw cudaMalloc either fails or carves memory out from under
+// the pool), or a component that must never trigger the implicit device-wide
+// synchronisation cudaFree can cause.  dfx_plan allocates a status word and dfx_encode
+// needs a workspace from the caller; this entry point needs neither.  Its scratch (the
+// exponent histogram, the code tables and the per-group bit counts) lives in a
+// fixed-size array in the library's own device memory, created with the module.
+//
+// Limits and sharing:
+//   * at most kStaticMaxGroups = 262144 groups of 32 chunks, i.e. n <= 2^28 with K = 32,
+//     2^29 with K = 64 and 2^30 with K = 128; larger tensors get DFX_ERR_CAPACITY;
+//   * the array costs 1 MiB + 4.25 KiB on every GPU that loads the library, until the
+//     process exits;
+//   * every call on a device uses the same array, and the array keeps the previous call's
+//     contents (the histogram is cleared by each call; everything else is overwritten
+//     before it is read).  Two calls whose GPU work overlaps (different streams, or host
+//     threads without ordering between them) race on it and corrupt each other's output:
+//     order them on one stream or with events;
+//   * the first call on each device looks up the array's device address with that device
+//     current (cudaGetSymbolAddress); make that first call before any stream capture.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "dfx.h"
+#include "dfx_common.cuh"
+
+namespace {
+
+constexpr uint64_t kStaticMaxGroups = 262144;
+constexpr uint64_t kStaticWorkspace = dfx::kWsGroupBits + 4 * kStaticMaxGroups;
+constexpr uint64_t kStaticStatus = kStaticWorkspace;          // one u32, unused by encode kernels
+constexpr uint64_t kStaticBytes = kStaticWorkspace + 256;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticBytes];
+
+std::mutex g_lock;
+uint8_t* g_scratch_addr[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" int dfx_encode_static(const void* d_bf16, uint64_t n, const dfx_params* params, void* d_out,
+                                 size_t out_capacity, size_t* h_compressed_bytes, cudaStream_t stream) {
+    if (n >= (1ull << 32)) return DFX_ERR_TOO_LARGE;
+    const uint32_t K = (params && params->chunk_symbols) ? params->chunk_symbols : 64u;
+    const uint32_t G = (params && params->group_chunks) ? params->group_chunks : 32u;
+    const uint32_t L = (params && params->max_len) ? params->max_len : 24u;
+    if (L < 8 || L > dfx::kMaxLenLimit) return DFX_ERR_ARG;
+    if (!dfx::decode_supports(K, G)) return DFX_ERR_UNSUPPORTED;
+    if (!d_out || (!d_bf16 && n)) return DFX_ERR_ARG;
+    if (((uintptr_t)d_bf16 & 15u) || ((uintptr_t)d_out & 15u)) return DFX_ERR_ARG;
+    const dfx::Layout lay = dfx::make_layout(n, K, G);
+    if (lay.n_group > kStaticMaxGroups) return DFX_ERR_CAPACITY;
+    const uint64_t max_bytes = lay.off_stream + dfx::stream_bytes(8 * n);
+    if (out_capacity < max_bytes) return DFX_ERR_CAPACITY;
+
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return DFX_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return DFX_ERR_ARG;
+    uint8_t* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> guard(g_lock);
+        if (!g_scratch_addr[dev]) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+                cudaGetLastError();
+                return DFX_ERR_CUDA;
+            }
+            g_scratch_addr[dev] = (uint8_t*)p;
+        }
+        scratch = g_scratch_addr[dev];
+    }
+
+    dfx::EncodeArgs a;
+    a.in = (const uint16_t*)d_bf16;
+    a.out = (uint8_t*)d_out;
+    a.n = n;
+    a.K = K;
+    a.G = G;
+    a.max_len = L;
+    a.n_chunk = (uint32_t)lay.n_chunk;
+    a.n_group = (uint32_t)lay.n_group;
+    a.off_clen = lay.off_clen;
+    a.off_m = lay.off_m;
+    a.off_stream = lay.off_stream;
+    a.ws_counts = (unsigned long long*)(scratch + dfx::kWsCounts);
+    a.ws_code = (uint32_t*)(scratch + dfx::kWsCode);
+    a.ws_len = scratch + dfx::kWsLen;
+    a.ws_group_bits = (uint32_t*)(scratch + dfx::kWsGroupBits);
+    a.status = (uint32_t*)(scratch + kStaticStatus);
+    if (dfx::launch_encode(a, max_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return DFX_ERR_CUDA;
+    }
+    if (h_compressed_bytes) {
+        unsigned long long total = 0;
+        if (cudaMemcpyAsync(&total, a.out + 24, 8, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+            cudaStreamSynchronize(stream) != cudaSuccess) {
+            cudaGetLastError();
+            return DFX_ERR_CUDA;
+        }
+        *h_compressed_bytes = (size_t)total;
+    }
+    return DFX_OK;
+}
