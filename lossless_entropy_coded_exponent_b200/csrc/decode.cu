@@ -3,19 +3,23 @@
 // Design (B200-first; the pages' GPU decoder is prior art, "DFloat11: lossless LLM
 // compression for GPU", aikraft.ru blog, section 03):
 //   * persistent grid, 8 warps per CTA; each CTA first builds its decoding tables in
-//     shared memory from len[256]: a direct lookup table on the next 11 bits for every
-//     code of length <= 11 and, for longer codes, the canonical per-length limits (the
+//     shared memory from len[256]: a direct lookup table on the next 12 bits for every
+//     code of length <= 12 and, for longer codes, the canonical per-length limits (the
 //     two levels of the hierarchical table of section 03, item 1);
 //   * one warp decodes one group of 32 chunks; lane i owns chunk i of the group and
 //     decodes exactly K codes.  Its read position is the group's start bit plus the
 //     warp's exclusive scan of the chunk bit lengths (the "lightweight auxiliary
 //     variables" that coordinate read positions, section 03, item 2).  Output positions
 //     need no scan: chunk i writes elements [i*K, i*K + K) of the group;
+//   * each lane keeps a 64-bit window of its stream in registers and refills it with
+//     one word when at most 32 bits are left, once per two codes, so the common path
+//     has no per-code branch besides the rare long-code test;
+//   * the next group's index and first stream words are loaded while the current group
+//     decodes; its sign+mantissa bytes arrive in shared memory by cp.async;
 //   * decoded exponents go to a per-warp shared-memory stash laid out so that both the
 //     lane-per-chunk writes and the coalesced reads of the merge step are free of bank
-//     conflicts; the merge joins them with the sign+mantissa bytes (8-byte loads, issued
-//     before decoding starts so they are in flight while the warp decodes) and writes
-//     BF16 with 16-byte stores, 512 contiguous bytes per warp instruction.
+//     conflicts; the merge joins them with the sign+mantissa bytes and writes BF16 with
+//     16-byte stores, 512 contiguous bytes per warp instruction.
 // Every read of the container is bounded by the header-checked section sizes; a bad
 // container sets bits of the status word and the kernel finishes normally.
 #include <cuda_runtime.h>
@@ -26,7 +30,7 @@
 namespace dfx {
 namespace {
 
-constexpr int kLutBits = 11;
+constexpr int kLutBits = 12;
 constexpr int kDecodeWarps = 8;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 constexpr unsigned kFull = 0xffffffffu;
@@ -40,8 +44,16 @@ struct StashShape {
     static constexpr int kWords = (K / 4) * kStride;
 };
 
+// Pair table entry (u32), indexed by the next kLutBits stream bits:
+//   bits 0-7   first symbol        bits 8-15  second symbol
+//   bits 16-20 length of the first code (0: the first code is longer than kLutBits)
+//   bits 26-30 bits the fast path consumes: both codes' lengths when both fit in the
+//              index bits, else the first code's length (0 for a long first code)
+//   bit  31    set when the entry does not hold two complete codes
+constexpr uint32_t kNotPair = 0x80000000u;
+
 struct Tables {
-    uint16_t lut[1 << kLutBits];              // (len << 8) | symbol, or 0 for codes longer than kLutBits
+    uint32_t lut[1 << kLutBits];
     uint32_t limit[kMaxLenLimit + 1];         // left-justified 24-bit end of the codes of length l
     uint32_t first[kMaxLenLimit + 1];         // first canonical code of length l
     uint32_t index[kMaxLenLimit + 1];         // rank in `sorted` of the first symbol of length l
@@ -121,11 +133,24 @@ __device__ bool build_tables(const DecodeArgs& a, Tables& T) {
     }
     __syncthreads();
     for (int e = t; e < (1 << kLutBits); e += blockDim.x) {
+        // first code: smallest length whose left-justified limit exceeds the bits
         const uint32_t v = (uint32_t)e << (kMaxLenLimit - kLutBits);
-        int l = 1;
-        while (l <= kLutBits && v >= T.limit[l]) l++;
-        uint16_t ent = 0;
-        if (l <= kLutBits) ent = (uint16_t)((l << 8) | T.sorted[T.index[l] + (v >> (kMaxLenLimit - l)) - T.first[l]]);
+        int l0 = 1;
+        while (l0 <= kLutBits && v >= T.limit[l0]) l0++;
+        uint32_t ent = kNotPair;  // long first code
+        if (l0 <= kLutBits) {
+            const uint32_t s0 = T.sorted[T.index[l0] + (v >> (kMaxLenLimit - l0)) - T.first[l0]];
+            // second code: decoded from the remaining kLutBits - l0 known bits only
+            const uint32_t v2 = (((uint32_t)e << l0) & ((1u << kLutBits) - 1)) << (kMaxLenLimit - kLutBits);
+            int l1 = 1;
+            while (l1 <= kLutBits && v2 >= T.limit[l1]) l1++;
+            if (l0 + l1 <= kLutBits) {
+                const uint32_t s1 = T.sorted[T.index[l1] + (v2 >> (kMaxLenLimit - l1)) - T.first[l1]];
+                ent = s0 | (s1 << 8) | ((uint32_t)l0 << 16) | ((uint32_t)(l0 + l1) << 26);
+            } else {
+                ent = kNotPair | s0 | ((uint32_t)l0 << 16) | ((uint32_t)l0 << 26);
+            }
+        }
         T.lut[e] = ent;
     }
     __syncthreads();
@@ -161,20 +186,37 @@ __device__ __forceinline__ uint4 merge8(uint2 m, uint32_t e0, uint32_t e1) {
     return o;
 }
 
+
+// ---------------------------------------------------------------- group index
+
+struct GroupIndex {
+    unsigned long long gb0;  // start bit of the group
+    uint32_t span;           // group bits, or 0xFFFFFFFF if the group's entries are inconsistent
+    uint32_t clen;           // this lane's chunk bits
+};
+
+__device__ __forceinline__ GroupIndex load_index(const DecodeArgs& a, const Tables& T, uint64_t g, unsigned lane,
+                                                 bool has_chunk) {
+    const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.comp + kOffGbase);
+    const uint16_t* clen = reinterpret_cast<const uint16_t*>(a.comp + a.off_clen);
+    GroupIndex r;
+    r.gb0 = __ldg(gbase + g);
+    const unsigned long long gb1 = __ldg(gbase + g + 1);
+    const bool bad = gb1 < r.gb0 || gb1 > T.total_bits || gb1 - r.gb0 >= 0xFFFFFFFFull;
+    r.span = bad ? 0xFFFFFFFFu : (uint32_t)(gb1 - r.gb0);
+    r.clen = has_chunk ? (uint32_t)__ldg(clen + g * 32 + lane) : 0u;
+    return r;
+}
+
 struct GroupStart {
-    uint64_t start;  // first bit of this lane's chunk
+    unsigned long long start;  // first bit of this lane's chunk
     uint32_t clen;
     bool ok;
 };
 
-__device__ __forceinline__ GroupStart group_start(const DecodeArgs& a, const Tables& T, uint64_t g, unsigned lane,
-                                                  bool has_chunk) {
-    const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.comp + kOffGbase);
-    const uint16_t* clen = reinterpret_cast<const uint16_t*>(a.comp + a.off_clen);
-    const uint64_t c = g * 32 + lane;
-    const unsigned long long gb0 = __ldg(gbase + g), gb1 = __ldg(gbase + g + 1);
-    const uint32_t cl = has_chunk ? (uint32_t)__ldg(clen + c) : 0u;
-    uint32_t incl = cl;
+// Warp exclusive scan of the chunk lengths: the lane's read position.
+__device__ __forceinline__ GroupStart scan_index(const GroupIndex& x, unsigned lane) {
+    uint32_t incl = x.clen;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
         const uint32_t y = __shfl_up_sync(kFull, incl, d);
@@ -182,117 +224,243 @@ __device__ __forceinline__ GroupStart group_start(const DecodeArgs& a, const Tab
     }
     const uint32_t sum = __shfl_sync(kFull, incl, 31);
     GroupStart r;
-    r.ok = gb0 <= gb1 && gb1 - gb0 == sum && gb1 <= T.total_bits;
-    r.start = gb0 + (incl - cl);
-    r.clen = cl;
+    r.ok = x.span == sum;
+    r.start = x.gb0 + (incl - x.clen);
+    r.clen = x.clen;
     return r;
 }
 
+// ---------------------------------------------------------------- bit reader
+//
+// hi:lo is a 64-bit window whose top 32 - g bits are the next bits of the stream and
+// whose other bits are zero (g = 32 - valid bits, kept in [-32, 32]); `nxt` is the next
+// stream word, already loaded.  A refill (g >= 0, i.e. at most 32 valid bits) shifts
+// `nxt` in under the valid bits.  Codes are decoded two per table lookup; every pair
+// that the table resolves consumes at most kLutBits = 12 bits, so one refill check per
+// two pairs keeps enough bits in the window.  Pairs the table cannot resolve (the
+// second code does not fit the index bits, or the first code is longer than 12 bits)
+// take a rare branch that decodes code by code and refills as it needs.
+template <bool kClamp>
 struct BitReader {
     const uint32_t* sw;
-    uint32_t maxw, wi, wi0, off0, off;
-    uint32_t w0, w1, w2;
+    uint32_t maxw;
+    uint32_t hi, lo, nxt, wp, wp0, o0;
+    int32_t g;
 
-    __device__ __forceinline__ void init(const uint32_t* s, uint32_t mw, uint64_t start) {
+    __device__ __forceinline__ uint32_t load(uint32_t i) const {
+        return kClamp ? __ldg(sw + min(i, maxw)) : __ldg(sw + i);
+    }
+    // w0, w1, w2: the stream words holding bit `start` and the two after it.
+    __device__ __forceinline__ void init(const uint32_t* s, uint32_t mw, unsigned long long start, uint32_t w0,
+                                         uint32_t w1, uint32_t w2) {
         sw = s;
         maxw = mw;
-        wi = (uint32_t)(start >> 5);
-        wi0 = wi;
-        off0 = off = (uint32_t)start & 31u;
-        w0 = ld_word(sw, wi, maxw);
-        w1 = ld_word(sw, wi + 1, maxw);
-        w2 = ld_word(sw, wi + 2, maxw);
-        wi += 3;
+        o0 = (uint32_t)start & 31u;
+        hi = __funnelshift_l(w1, w0, o0);  // the window ends where w1 ends
+        lo = w1 << o0;
+        g = (int32_t)o0 - 32;              // 64 - o0 valid bits
+        nxt = w2;
+        wp0 = wp = (uint32_t)(start >> 5) + 3;
     }
-    // Decode one code: returns (len << 8) | symbol and advances.
-    __device__ __forceinline__ uint32_t next(const Tables& T, uint32_t& err) {
-        const uint32_t peek = __funnelshift_l(w1, w0, off);
-        uint32_t ent = T.lut[peek >> (32 - kLutBits)];
-        if (ent == 0) {
-            ent = decode_long(peek, T);
+    __device__ __forceinline__ void refill() {  // requires g >= 0
+        hi |= __funnelshift_lc(nxt, 0u, (uint32_t)g);
+        lo |= __funnelshift_lc(0u, nxt, (uint32_t)g);
+        g -= 32;
+        nxt = load(wp);
+        wp++;
+    }
+    __device__ __forceinline__ void consume(uint32_t len) {  // len in 0..31
+        hi = __funnelshift_l(lo, hi, len);
+        lo = __funnelshift_l(0u, lo, len);
+        g += (int32_t)len;
+    }
+    // One code, the general way: returns its symbol.
+    __device__ __forceinline__ uint32_t one(const Tables& T, uint32_t& err) {
+        if (g > 32 - (int)kMaxLenLimit) refill();  // at least 24 valid bits
+        const uint32_t e = T.lut[hi >> (32 - kLutBits)];
+        uint32_t len, sym;
+        if ((e & 0x001F0000u) == 0) {
+            uint32_t ent = decode_long(hi, T);
             if (ent >> 16) {
                 err |= DFX_STATUS_STREAM;
                 ent &= 0xFFFFu;
             }
+            len = ent >> 8;
+            sym = ent & 0xFFu;
+        } else {
+            len = (e >> 16) & 31u;
+            sym = e & 0xFFu;
         }
-        off += ent >> 8;
-        if (off >= 32) {
-            off -= 32;
-            w0 = w1;
-            w1 = w2;
-            w2 = ld_word(sw, wi, maxw);
-            wi++;
-        }
-        return ent;
+        consume(len);
+        if (g > 32 - kLutBits) refill();  // at least 12 valid bits for the next pair
+        return sym;
     }
-    __device__ __forceinline__ uint32_t consumed() const { return (wi - 3 - wi0) * 32 + off - off0; }
+    // Two codes: returns acc with their symbols in bytes 2j and 2j+1.
+    template <int j>
+    __device__ __forceinline__ uint32_t pair(uint32_t acc, const Tables& T, uint32_t& err) {
+        constexpr uint32_t sel = j == 0 ? 0x3254u : 0x5410u;
+        const uint32_t e = T.lut[hi >> (32 - kLutBits)];
+        const uint32_t len = e >> 26;  // wraps to the first code's length (or 0) when bit 31 is set
+        consume(len);
+        acc = __byte_perm(acc, e, sel);
+        if ((int32_t)e < 0) {
+            g -= 32;  // undo bit 31 of `len`
+            uint32_t s0 = e & 0xFFu;
+            if ((e & 0x001F0000u) == 0) s0 = one(T, err);
+            const uint32_t s1 = one(T, err);
+            acc = __byte_perm(acc, s0 | (s1 << 8), sel);
+        }
+        return acc;
+    }
+    // Bits consumed since init.
+    __device__ __forceinline__ uint32_t consumed() const {
+        return 32u + 32u * (wp - wp0) - o0 + (uint32_t)g;
+    }
 };
 
-// A group whose 32 chunks all hold K codes.
-template <int K>
-__device__ __forceinline__ void decode_full_group(const DecodeArgs& a, const Tables& T, uint32_t* stash, uint64_t g,
-                                                  unsigned lane, uint32_t& err) {
+// Decode the K codes of this lane's chunk into the stash.
+template <int K, bool kClamp>
+__device__ __forceinline__ void decode_chunk(BitReader<kClamp>& br, const Tables& T, uint32_t* stash,
+                                             unsigned lane, uint32_t& err) {
     constexpr int S = StashShape<K>::kStride;
-    constexpr int R = K / 8;              // 8-element output slots per lane
-    constexpr bool kPrefetchM = K <= 64;  // keeps the register budget for K = 128
-
-    const GroupStart gs = group_start(a, T, g, lane, true);
-    if (!gs.ok) {
-        err |= DFX_STATUS_INDEX;
-        return;
-    }
-    const uint2* mp = reinterpret_cast<const uint2*>(a.comp + a.off_m) + g * (32 * K / 8) + lane;
-    uint2 mreg[kPrefetchM ? R : 1];
-    if (kPrefetchM) {
-#pragma unroll
-        for (int r = 0; r < R; r++) mreg[r] = __ldg(mp + 32 * r);
-    }
-
-    BitReader br;
-    br.init(reinterpret_cast<const uint32_t*>(a.comp + a.off_stream), T.n_words - 1, gs.start);
 #pragma unroll 2
     for (int q = 0; q < K / 4; q++) {
         uint32_t acc = 0;
-#pragma unroll
-        for (int j = 0; j < 4; j++) acc |= (br.next(T, err) & 0xFFu) << (8 * j);
+        acc = br.template pair<0>(acc, T, err);
+        acc = br.template pair<1>(acc, T, err);
+        if (br.g >= 0) br.refill();
         stash[q * S + lane] = acc;
     }
-    if (br.consumed() != gs.clen) err |= DFX_STATUS_STREAM;
-    __syncwarp();
+}
 
-    uint4* out4 = reinterpret_cast<uint4*>(a.out) + g * (32 * K / 8) + lane;
+// ---------------------------------------------------------------- per-warp buffers
+
+template <int K>
+struct WarpBuffers {
+    uint32_t stash[StashShape<K>::kWords];      // decoded exponents
+    __align__(16) uint8_t m[32 * K];            // the group's sign+mantissa bytes
+};
+
+template <int K>
+__host__ __device__ constexpr size_t warp_buffer_bytes() {
+    return (sizeof(WarpBuffers<K>) + 15) & ~size_t(15);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// Full groups (all 32 chunks hold K codes), one warp at a time, with the next
+// group's index and first stream words in flight while this group decodes.
+template <int K>
+__device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, WarpBuffers<K>& wb, uint64_t g,
+                                   uint64_t step, uint64_t n_full, unsigned lane, uint32_t& err) {
+    constexpr int S = StashShape<K>::kStride;
+    constexpr int kMChunks = (32 * K) / 16 / 32;  // 16-byte copies per lane
+    if (g >= n_full) return;
+    const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
+    const uint32_t maxw = T.n_words - 1;
+    const uint8_t* mplane = a.comp + a.off_m;
+
+    GroupStart st = scan_index(load_index(a, T, g, lane, true), lane);
+    uint32_t w0 = ld_word(sw, (uint32_t)(st.start >> 5), maxw);
+    uint32_t w1 = ld_word(sw, (uint32_t)(st.start >> 5) + 1, maxw);
+    uint32_t w2 = ld_word(sw, (uint32_t)(st.start >> 5) + 2, maxw);
+    uint64_t gn = g + step;
+    GroupIndex idx_n;
+    if (gn < n_full) idx_n = load_index(a, T, gn, lane, true);
+
+    while (true) {
+        // the sign+mantissa bytes of this group go to shared memory asynchronously
+        const uint8_t* msrc = mplane + g * (32ull * K);
 #pragma unroll
-    for (int r = 0; r < R; r++) {
-        const int j0 = 8 * (int)lane + 256 * r;
-        const int t = j0 / K, q0 = (j0 % K) / 4;
-        const uint32_t e0 = stash[q0 * S + t], e1 = stash[(q0 + 1) * S + t];
-        const uint2 m = kPrefetchM ? mreg[kPrefetchM ? r : 0] : __ldg(mp + 32 * r);
-        out4[32 * r] = merge8(m, e0, e1);
+        for (int i = 0; i < kMChunks; i++) cp_async16(wb.m + 16 * (lane + 32 * i), msrc + 16 * (lane + 32 * i));
+        cp_async_commit();
+
+        // the next group's read positions and first words
+        const bool has_next = gn < n_full;
+        const uint64_t gnn = gn + step;
+        GroupStart st_n;
+        uint32_t nw0 = 0, nw1 = 0, nw2 = 0;
+        GroupIndex idx_nn;
+        if (has_next) {
+            st_n = scan_index(idx_n, lane);
+            const uint32_t wi = (uint32_t)(st_n.start >> 5);
+            nw0 = ld_word(sw, wi, maxw);
+            nw1 = ld_word(sw, wi + 1, maxw);
+            nw2 = ld_word(sw, wi + 2, maxw);
+            if (gnn < n_full) idx_nn = load_index(a, T, gnn, lane, true);
+        }
+
+        if (st.ok) {
+            // A chunk refills at most 3K/4 times (24-bit codes); lane 31 starts last.  When
+            // the warp's last possible read is inside the stream, the loads need no clamp.
+            const uint32_t last_wp0 = __shfl_sync(kFull, (uint32_t)(st.start >> 5) + 3u, 31);
+            if (last_wp0 + (3u * K) / 4u + 3u <= maxw) {
+                BitReader<false> br;
+                br.init(sw, maxw, st.start, w0, w1, w2);
+                decode_chunk<K, false>(br, T, wb.stash, lane, err);
+                if (br.consumed() != st.clen) err |= DFX_STATUS_STREAM;
+            } else {
+                BitReader<true> br;
+                br.init(sw, maxw, st.start, w0, w1, w2);
+                decode_chunk<K, true>(br, T, wb.stash, lane, err);
+                if (br.consumed() != st.clen) err |= DFX_STATUS_STREAM;
+            }
+        } else {
+            err |= DFX_STATUS_INDEX;
+        }
+        cp_async_wait_all();
+        __syncwarp();
+        if (st.ok) {
+            uint4* out4 = reinterpret_cast<uint4*>(a.out) + g * (32 * K / 8) + lane;
+#pragma unroll
+            for (int r = 0; r < K / 8; r++) {
+                const int j0 = 8 * (int)lane + 256 * r;
+                const int t = j0 / K, q0 = (j0 % K) / 4;
+                const uint2 m = *reinterpret_cast<const uint2*>(wb.m + j0);
+                out4[32 * r] = merge8(m, wb.stash[q0 * S + t], wb.stash[(q0 + 1) * S + t]);
+            }
+        }
+        __syncwarp();
+        if (!has_next) break;
+        g = gn;
+        gn = gnn;
+        st = st_n;
+        w0 = nw0;
+        w1 = nw1;
+        w2 = nw2;
+        idx_n = idx_nn;
     }
-    __syncwarp();
 }
 
 // The last group when it is ragged: chunks may be short or absent, outputs stop at n.
 template <int K>
-__device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, uint32_t* stash, uint64_t g, unsigned lane,
-                                  uint32_t& err) {
+__device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, WarpBuffers<K>& wb, uint64_t g,
+                                  unsigned lane, uint32_t& err) {
     constexpr int S = StashShape<K>::kStride;
     const uint64_t c = g * 32 + lane;
     const bool has = c < a.n_chunk;
     const uint32_t cnt = has ? (uint32_t)min((uint64_t)K, a.n - c * K) : 0u;
-    const GroupStart gs = group_start(a, T, g, lane, has);
+    const GroupStart gs = scan_index(load_index(a, T, g, lane, has), lane);
     if (!gs.ok) {
         err |= DFX_STATUS_INDEX;
         return;
     }
     if (has) {
-        BitReader br;
-        br.init(reinterpret_cast<const uint32_t*>(a.comp + a.off_stream), T.n_words - 1, gs.start);
+        const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
+        const uint32_t maxw = T.n_words - 1;
+        const uint32_t wi = (uint32_t)(gs.start >> 5);
+        BitReader<true> br;
+        br.init(sw, maxw, gs.start, ld_word(sw, wi, maxw), ld_word(sw, wi + 1, maxw), ld_word(sw, wi + 2, maxw));
         for (int q = 0; q < K / 4; q++) {
             uint32_t acc = 0;
-            for (int j = 0; j < 4; j++)
-                if ((uint32_t)(4 * q + j) < cnt) acc |= (br.next(T, err) & 0xFFu) << (8 * j);
-            stash[q * S + lane] = acc;
+            for (int k = 0; k < 4; k++)
+                if ((uint32_t)(4 * q + k) < cnt) acc |= br.one(T, err) << (8 * k);
+            wb.stash[q * S + lane] = acc;
         }
         if (br.consumed() != gs.clen) err |= DFX_STATUS_STREAM;
     }
@@ -305,12 +473,12 @@ __device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, uint32_t
         const int t = j0 / K, q0 = (j0 % K) / 4;
         if (elem + 8 <= a.n) {
             const uint2 m = __ldg(reinterpret_cast<const uint2*>(mplane + elem));
-            reinterpret_cast<uint4*>(a.out)[elem / 8] = merge8(m, stash[q0 * S + t], stash[(q0 + 1) * S + t]);
+            reinterpret_cast<uint4*>(a.out)[elem / 8] = merge8(m, wb.stash[q0 * S + t], wb.stash[(q0 + 1) * S + t]);
         } else {
             for (int i = 0; i < 8; i++) {
                 if (elem + i >= a.n) break;
                 const int k = (j0 + i) % K;
-                const uint32_t e = (stash[(k / 4) * S + t] >> (8 * (k % 4))) & 0xFFu;
+                const uint32_t e = (wb.stash[(k / 4) * S + t] >> (8 * (k % 4))) & 0xFFu;
                 const uint32_t m = mplane[elem + i];
                 a.out[elem + i] = (uint16_t)(((m & 0x80u) << 8) | (e << 7) | (m & 0x7Fu));
             }
@@ -320,27 +488,52 @@ __device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, uint32_t
 }
 
 template <int K>
-__global__ void __launch_bounds__(kDecodeThreads) k_decode(DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, 5) k_decode(DecodeArgs a) {
     __shared__ Tables T;
-    __shared__ uint32_t stash_all[kDecodeWarps][StashShape<K>::kWords];
+    extern __shared__ __align__(16) uint8_t dyn_smem[];
     if (!build_tables(a, T)) return;
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint32_t* stash = stash_all[warp];
+    WarpBuffers<K>& wb = *reinterpret_cast<WarpBuffers<K>*>(dyn_smem + warp * warp_buffer_bytes<K>());
     uint32_t err = 0;
     const uint64_t n_full = (a.n % (32ull * K) == 0) ? a.n_group : a.n_group - 1;
     const uint64_t step = (uint64_t)gridDim.x * kDecodeWarps;
-    for (uint64_t g = (uint64_t)blockIdx.x * kDecodeWarps + warp; g < a.n_group; g += step) {
-        if (g < n_full) decode_full_group<K>(a, T, stash, g, lane, err);
-        else decode_tail_group<K>(a, T, stash, g, lane, err);
-    }
+    const uint64_t gw = (uint64_t)blockIdx.x * kDecodeWarps + warp;
+    decode_full_groups<K>(a, T, wb, gw, step, n_full, lane, err);
+    if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, wb, n_full, lane, err);
     if (err) atomicOr(a.status, err);
+}
+
+template <int K>
+constexpr size_t dyn_smem_bytes() {
+    return kDecodeWarps * warp_buffer_bytes<K>();
 }
 
 template <int K>
 int blocks_per_sm() {
     int b = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k_decode<K>, kDecodeThreads, 0) != cudaSuccess) return 1;
+    if (cudaFuncSetAttribute(k_decode<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem_bytes<K>()) !=
+        cudaSuccess)
+        return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k_decode<K>, kDecodeThreads, dyn_smem_bytes<K>()) !=
+        cudaSuccess)
+        return 1;
     return b > 0 ? b : 1;
+}
+
+template <int K>
+cudaError_t launch_k(const DecodeArgs& a, int grid, cudaStream_t s) {
+    // the dynamic shared-memory limit is raised once per device (needed above 48 KiB)
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k_decode<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)dyn_smem_bytes<K>());
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    k_decode<K><<<grid, kDecodeThreads, dyn_smem_bytes<K>(), s>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -360,12 +553,12 @@ int decode_warps_per_block() { return kDecodeWarps; }
 
 cudaError_t launch_decode(const DecodeArgs& a, int grid, cudaStream_t s) {
     switch (a.K) {
-        case 32: k_decode<32><<<grid, kDecodeThreads, 0, s>>>(a); break;
-        case 64: k_decode<64><<<grid, kDecodeThreads, 0, s>>>(a); break;
-        case 128: k_decode<128><<<grid, kDecodeThreads, 0, s>>>(a); break;
+        case 32: return launch_k<32>(a, grid, s);
+        case 64: return launch_k<64>(a, grid, s);
+        case 128: return launch_k<128>(a, grid, s);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
+
 
 }  // namespace dfx
