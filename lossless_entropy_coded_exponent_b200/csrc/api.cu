@@ -104,9 +104,10 @@ int dfx_plan(dfx_plan_t* plan, uint64_t n, const dfx_params* params, size_t* max
         free(p);
         return DFX_ERR_CUDA;
     }
-    const uint64_t warps = dfx::decode_blocks_per_sm(K) * (uint64_t)sms;  // resident CTAs
-    const uint64_t need = (p->L.n_group + 7) / 8;                          // CTAs with work (8 warps each)
-    p->decode_grid = (int)(need == 0 ? 1 : (need < warps ? need : warps));
+    const uint64_t resident = dfx::decode_blocks_per_sm(K) * (uint64_t)sms;  // CTAs that fit at once
+    const uint64_t wpb = (uint64_t)dfx::decode_warps_per_block(K);
+    const uint64_t need = (p->L.n_group + wpb - 1) / wpb;                    // CTAs with work (a warp per group)
+    p->decode_grid = (int)(need == 0 ? 1 : (need < resident ? need : resident));
     if (max_compressed_bytes) *max_compressed_bytes = (size_t)p->max_bytes;
     if (workspace_bytes) *workspace_bytes = (size_t)p->ws_bytes;
     *plan = p;

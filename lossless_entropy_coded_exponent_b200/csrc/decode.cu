@@ -30,9 +30,14 @@
 namespace dfx {
 namespace {
 
-constexpr int kLutBits = 12;
-constexpr int kDecodeWarps = 8;
-constexpr int kDecodeThreads = kDecodeWarps * 32;
+constexpr int kLutBits = 14;
+// Warps per CTA: one CTA per SM holds the 64 KiB pair table once; K = 128 needs twice
+// the per-warp buffers, so it runs 16 warps to stay inside 227 KiB of shared memory.
+template <int K>
+struct DecodeShape {
+    static constexpr int kWarps = K == 128 ? 16 : 32;
+    static constexpr int kThreads = kWarps * 32;
+};
 constexpr unsigned kFull = 0xffffffffu;
 
 // Stash row stride (words): row q holds symbols 4q..4q+3 of every lane.  32 + 128/K
@@ -53,7 +58,6 @@ struct StashShape {
 constexpr uint32_t kNotPair = 0x80000000u;
 
 struct Tables {
-    uint32_t lut[1 << kLutBits];
     uint32_t limit[kMaxLenLimit + 1];         // left-justified 24-bit end of the codes of length l
     uint32_t first[kMaxLenLimit + 1];         // first canonical code of length l
     uint32_t index[kMaxLenLimit + 1];         // rank in `sorted` of the first symbol of length l
@@ -65,7 +69,10 @@ struct Tables {
     uint32_t bad;
 };
 
-__device__ bool build_tables(const DecodeArgs& a, Tables& T) {
+// Builds the decoding tables in shared memory: the per-length canonical tables in T and
+// the pair table `lut` (1 << kLutBits entries).  `scratch` (2 << kLutBits bytes) holds the
+// one-code table the pair table is built from.
+__device__ bool build_tables(const DecodeArgs& a, Tables& T, uint32_t* lut, uint16_t* scratch) {
     const int t = threadIdx.x;
     if (t == 0) {
         const uint8_t* h = a.comp;
@@ -132,26 +139,36 @@ __device__ bool build_tables(const DecodeArgs& a, Tables& T) {
         }
     }
     __syncthreads();
+    // one-code table: (len << 8) | symbol for the code the next kLutBits bits start with,
+    // 0 when that code is longer; the length is the smallest l whose limit exceeds the bits
     for (int e = t; e < (1 << kLutBits); e += blockDim.x) {
-        // first code: smallest length whose left-justified limit exceeds the bits
         const uint32_t v = (uint32_t)e << (kMaxLenLimit - kLutBits);
-        int l0 = 1;
-        while (l0 <= kLutBits && v >= T.limit[l0]) l0++;
-        uint32_t ent = kNotPair;  // long first code
-        if (l0 <= kLutBits) {
-            const uint32_t s0 = T.sorted[T.index[l0] + (v >> (kMaxLenLimit - l0)) - T.first[l0]];
-            // second code: decoded from the remaining kLutBits - l0 known bits only
-            const uint32_t v2 = (((uint32_t)e << l0) & ((1u << kLutBits) - 1)) << (kMaxLenLimit - kLutBits);
-            int l1 = 1;
-            while (l1 <= kLutBits && v2 >= T.limit[l1]) l1++;
-            if (l0 + l1 <= kLutBits) {
-                const uint32_t s1 = T.sorted[T.index[l1] + (v2 >> (kMaxLenLimit - l1)) - T.first[l1]];
-                ent = s0 | (s1 << 8) | ((uint32_t)l0 << 16) | ((uint32_t)(l0 + l1) << 26);
-            } else {
-                ent = kNotPair | s0 | ((uint32_t)l0 << 16) | ((uint32_t)l0 << 26);
-            }
+        int lo = 1, hi = kLutBits + 1;  // limit[] is non-decreasing in l
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (v < T.limit[mid]) hi = mid;
+            else lo = mid + 1;
         }
-        T.lut[e] = ent;
+        scratch[e] = lo <= kLutBits
+                         ? (uint16_t)((lo << 8) | T.sorted[T.index[lo] + (v >> (kMaxLenLimit - lo)) - T.first[lo]])
+                         : (uint16_t)0;
+    }
+    __syncthreads();
+    // pair table: the second code is read from the kLutBits - l0 bits left after the
+    // first; a code of length l1 <= kLutBits - l0 depends only on those known bits
+    for (int e = t; e < (1 << kLutBits); e += blockDim.x) {
+        const uint32_t s0 = scratch[e];
+        uint32_t ent = kNotPair;  // long first code
+        if (s0) {
+            const uint32_t l0 = s0 >> 8;
+            const uint32_t s1 = scratch[((uint32_t)e << l0) & ((1u << kLutBits) - 1)];
+            const uint32_t l1 = s1 >> 8;
+            if (s1 && l0 + l1 <= kLutBits)
+                ent = (s0 & 0xFFu) | ((s1 & 0xFFu) << 8) | (l0 << 16) | ((l0 + l1) << 26);
+            else
+                ent = kNotPair | (s0 & 0xFFu) | (l0 << 16) | (l0 << 26);
+        }
+        lut[e] = ent;
     }
     __syncthreads();
     return true;
@@ -242,6 +259,7 @@ __device__ __forceinline__ GroupStart scan_index(const GroupIndex& x, unsigned l
 // take a rare branch that decodes code by code and refills as it needs.
 template <bool kClamp>
 struct BitReader {
+    const uint32_t* lut;  // pair table in shared memory
     const uint32_t* sw;
     uint32_t maxw;
     uint32_t hi, lo, nxt, wp, wp0, o0;
@@ -251,8 +269,9 @@ struct BitReader {
         return kClamp ? __ldg(sw + min(i, maxw)) : __ldg(sw + i);
     }
     // w0, w1, w2: the stream words holding bit `start` and the two after it.
-    __device__ __forceinline__ void init(const uint32_t* s, uint32_t mw, unsigned long long start, uint32_t w0,
-                                         uint32_t w1, uint32_t w2) {
+    __device__ __forceinline__ void init(const uint32_t* table, const uint32_t* s, uint32_t mw,
+                                         unsigned long long start, uint32_t w0, uint32_t w1, uint32_t w2) {
+        lut = table;
         sw = s;
         maxw = mw;
         o0 = (uint32_t)start & 31u;
@@ -277,7 +296,7 @@ struct BitReader {
     // One code, the general way: returns its symbol.
     __device__ __forceinline__ uint32_t one(const Tables& T, uint32_t& err) {
         if (g > 32 - (int)kMaxLenLimit) refill();  // at least 24 valid bits
-        const uint32_t e = T.lut[hi >> (32 - kLutBits)];
+        const uint32_t e = lut[hi >> (32 - kLutBits)];
         uint32_t len, sym;
         if ((e & 0x001F0000u) == 0) {
             uint32_t ent = decode_long(hi, T);
@@ -299,7 +318,7 @@ struct BitReader {
     template <int j>
     __device__ __forceinline__ uint32_t pair(uint32_t acc, const Tables& T, uint32_t& err) {
         constexpr uint32_t sel = j == 0 ? 0x3254u : 0x5410u;
-        const uint32_t e = T.lut[hi >> (32 - kLutBits)];
+        const uint32_t e = lut[hi >> (32 - kLutBits)];
         const uint32_t len = e >> 26;  // wraps to the first code's length (or 0) when bit 31 is set
         consume(len);
         acc = __byte_perm(acc, e, sel);
@@ -323,7 +342,7 @@ template <int K, bool kClamp>
 __device__ __forceinline__ void decode_chunk(BitReader<kClamp>& br, const Tables& T, uint32_t* stash,
                                              unsigned lane, uint32_t& err) {
     constexpr int S = StashShape<K>::kStride;
-#pragma unroll 2
+#pragma unroll 4
     for (int q = 0; q < K / 4; q++) {
         uint32_t acc = 0;
         acc = br.template pair<0>(acc, T, err);
@@ -356,7 +375,8 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // Full groups (all 32 chunks hold K codes), one warp at a time, with the next
 // group's index and first stream words in flight while this group decodes.
 template <int K>
-__device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, WarpBuffers<K>& wb, uint64_t g,
+__device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const uint32_t* lut, WarpBuffers<K>& wb,
+                                   uint64_t g,
                                    uint64_t step, uint64_t n_full, unsigned lane, uint32_t& err) {
     constexpr int S = StashShape<K>::kStride;
     constexpr int kMChunks = (32 * K) / 16 / 32;  // 16-byte copies per lane
@@ -401,12 +421,12 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, WarpBuf
             const uint32_t last_wp0 = __shfl_sync(kFull, (uint32_t)(st.start >> 5) + 3u, 31);
             if (last_wp0 + (3u * K) / 4u + 3u <= maxw) {
                 BitReader<false> br;
-                br.init(sw, maxw, st.start, w0, w1, w2);
+                br.init(lut, sw, maxw, st.start, w0, w1, w2);
                 decode_chunk<K, false>(br, T, wb.stash, lane, err);
                 if (br.consumed() != st.clen) err |= DFX_STATUS_STREAM;
             } else {
                 BitReader<true> br;
-                br.init(sw, maxw, st.start, w0, w1, w2);
+                br.init(lut, sw, maxw, st.start, w0, w1, w2);
                 decode_chunk<K, true>(br, T, wb.stash, lane, err);
                 if (br.consumed() != st.clen) err |= DFX_STATUS_STREAM;
             }
@@ -439,7 +459,8 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, WarpBuf
 
 // The last group when it is ragged: chunks may be short or absent, outputs stop at n.
 template <int K>
-__device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, WarpBuffers<K>& wb, uint64_t g,
+__device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, const uint32_t* lut, WarpBuffers<K>& wb,
+                                  uint64_t g,
                                   unsigned lane, uint32_t& err) {
     constexpr int S = StashShape<K>::kStride;
     const uint64_t c = g * 32 + lane;
@@ -455,7 +476,7 @@ __device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, WarpBuff
         const uint32_t maxw = T.n_words - 1;
         const uint32_t wi = (uint32_t)(gs.start >> 5);
         BitReader<true> br;
-        br.init(sw, maxw, gs.start, ld_word(sw, wi, maxw), ld_word(sw, wi + 1, maxw), ld_word(sw, wi + 2, maxw));
+        br.init(lut, sw, maxw, gs.start, ld_word(sw, wi, maxw), ld_word(sw, wi + 1, maxw), ld_word(sw, wi + 2, maxw));
         for (int q = 0; q < K / 4; q++) {
             uint32_t acc = 0;
             for (int k = 0; k < 4; k++)
@@ -487,26 +508,37 @@ __device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, WarpBuff
     __syncwarp();
 }
 
+constexpr size_t kLutBytes = sizeof(uint32_t) << kLutBits;
+
 template <int K>
-__global__ void __launch_bounds__(kDecodeThreads, 5) k_decode(DecodeArgs a) {
+__global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeArgs a) {
+    constexpr int kDecodeWarps = DecodeShape<K>::kWarps;
     __shared__ Tables T;
+    // dynamic shared memory: the pair table, then one buffer per warp (the buffers
+    // double as scratch for the one-code table while the tables are built)
     extern __shared__ __align__(16) uint8_t dyn_smem[];
-    if (!build_tables(a, T)) return;
+    uint32_t* lut = reinterpret_cast<uint32_t*>(dyn_smem);
+    uint8_t* warp_area = dyn_smem + kLutBytes;
+    if (!build_tables(a, T, lut, reinterpret_cast<uint16_t*>(warp_area))) return;
+    __syncthreads();  // the scratch is reused as warp buffers
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    WarpBuffers<K>& wb = *reinterpret_cast<WarpBuffers<K>*>(dyn_smem + warp * warp_buffer_bytes<K>());
+    WarpBuffers<K>& wb = *reinterpret_cast<WarpBuffers<K>*>(warp_area + warp * warp_buffer_bytes<K>());
     uint32_t err = 0;
     const uint64_t n_full = (a.n % (32ull * K) == 0) ? a.n_group : a.n_group - 1;
     const uint64_t step = (uint64_t)gridDim.x * kDecodeWarps;
     const uint64_t gw = (uint64_t)blockIdx.x * kDecodeWarps + warp;
-    decode_full_groups<K>(a, T, wb, gw, step, n_full, lane, err);
-    if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, wb, n_full, lane, err);
+    decode_full_groups<K>(a, T, lut, wb, gw, step, n_full, lane, err);
+    if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, lut, wb, n_full, lane, err);
     if (err) atomicOr(a.status, err);
 }
 
 template <int K>
 constexpr size_t dyn_smem_bytes() {
-    return kDecodeWarps * warp_buffer_bytes<K>();
+    return kLutBytes + DecodeShape<K>::kWarps * warp_buffer_bytes<K>();
 }
+static_assert(DecodeShape<32>::kWarps * warp_buffer_bytes<32>() >= (2u << kLutBits), "scratch for the one-code table");
+static_assert(DecodeShape<128>::kWarps * warp_buffer_bytes<128>() >= (2u << kLutBits), "scratch for the one-code table");
+static_assert(dyn_smem_bytes<64>() + 1024 <= 227 * 1024 && dyn_smem_bytes<128>() + 1024 <= 227 * 1024, "shared memory");
 
 template <int K>
 int blocks_per_sm() {
@@ -514,7 +546,7 @@ int blocks_per_sm() {
     if (cudaFuncSetAttribute(k_decode<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem_bytes<K>()) !=
         cudaSuccess)
         return 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k_decode<K>, kDecodeThreads, dyn_smem_bytes<K>()) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k_decode<K>, DecodeShape<K>::kThreads, dyn_smem_bytes<K>()) !=
         cudaSuccess)
         return 1;
     return b > 0 ? b : 1;
@@ -532,7 +564,7 @@ cudaError_t launch_k(const DecodeArgs& a, int grid, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    k_decode<K><<<grid, kDecodeThreads, dyn_smem_bytes<K>(), s>>>(a);
+    k_decode<K><<<grid, DecodeShape<K>::kThreads, dyn_smem_bytes<K>(), s>>>(a);
     return cudaGetLastError();
 }
 
@@ -549,7 +581,9 @@ int decode_blocks_per_sm(uint32_t K) {
     }
 }
 
-int decode_warps_per_block() { return kDecodeWarps; }
+int decode_warps_per_block(uint32_t K) {
+    return K == 32 ? DecodeShape<32>::kWarps : K == 64 ? DecodeShape<64>::kWarps : DecodeShape<128>::kWarps;
+}
 
 cudaError_t launch_decode(const DecodeArgs& a, int grid, cudaStream_t s) {
     switch (a.K) {

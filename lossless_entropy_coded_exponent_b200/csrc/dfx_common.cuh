@@ -79,6 +79,7 @@ inline uint64_t workspace_bytes_for(uint64_t n_group) {
 cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int grid, cudaStream_t s);
 int decode_blocks_per_sm(uint32_t K);
+int decode_warps_per_block(uint32_t K);
 bool decode_supports(uint32_t K, uint32_t G);
 
 }  // namespace dfx
