@@ -185,9 +185,6 @@ __device__ __noinline__ uint32_t decode_long(uint32_t peek, const Tables& T) {
     return ((uint32_t)l << 8) | T.sorted[T.index[l] + (v >> (kMaxLenLimit - l)) - T.first[l]];
 }
 
-__device__ __forceinline__ uint32_t ld_word(const uint32_t* sw, uint32_t i, uint32_t maxw) {
-    return __ldg(sw + min(i, maxw));
-}
 
 // Two BF16 from x = [m0, e0, m1, e1] (bytes, low to high).
 __device__ __forceinline__ uint32_t bf16_pair(uint32_t x) {
@@ -227,6 +224,8 @@ __device__ __forceinline__ GroupIndex load_index(const DecodeArgs& a, const Tabl
 
 struct GroupStart {
     unsigned long long start;  // first bit of this lane's chunk
+    unsigned long long gb0;    // first bit of the group
+    uint32_t span;             // bits of the group
     uint32_t clen;
     bool ok;
 };
@@ -243,6 +242,8 @@ __device__ __forceinline__ GroupStart scan_index(const GroupIndex& x, unsigned l
     GroupStart r;
     r.ok = x.span == sum;
     r.start = x.gb0 + (incl - x.clen);
+    r.gb0 = x.gb0;
+    r.span = x.span;
     r.clen = x.clen;
     return r;
 }
@@ -257,29 +258,44 @@ __device__ __forceinline__ GroupStart scan_index(const GroupIndex& x, unsigned l
 // two pairs keeps enough bits in the window.  Pairs the table cannot resolve (the
 // second code does not fit the index bits, or the first code is longer than 12 bits)
 // take a rare branch that decodes code by code and refills as it needs.
-template <bool kClamp>
+// Where a bit reader takes its stream words from: the global stream (with or without a
+// bound clamp) or a warp's shared-memory copy of its group's slice of the stream.
+struct GlobalWords {
+    const uint32_t* p;
+    __device__ __forceinline__ uint32_t operator()(uint32_t i) const { return __ldg(p + i); }
+};
+struct ClampedGlobalWords {
+    const uint32_t* p;
+    uint32_t maxw;
+    __device__ __forceinline__ uint32_t operator()(uint32_t i) const { return __ldg(p + min(i, maxw)); }
+};
+constexpr uint32_t kSliceWords = 256;  // 1 KiB per staged group slice
+struct SharedWords {
+    const uint32_t* s;  // the slice buffer
+    uint32_t base;      // stream word index of s[0]
+    // Well-formed groups read inside the slice; the clamp keeps a corrupt one in the buffer.
+    __device__ __forceinline__ uint32_t operator()(uint32_t i) const { return s[min(i - base, kSliceWords - 1)]; }
+};
+
+template <class Words>
 struct BitReader {
     const uint32_t* lut;  // pair table in shared memory
-    const uint32_t* sw;
-    uint32_t maxw;
+    Words words;
     uint32_t hi, lo, nxt, wp, wp0, o0;
     int32_t g;
 
-    __device__ __forceinline__ uint32_t load(uint32_t i) const {
-        return kClamp ? __ldg(sw + min(i, maxw)) : __ldg(sw + i);
-    }
-    // w0, w1, w2: the stream words holding bit `start` and the two after it.
-    __device__ __forceinline__ void init(const uint32_t* table, const uint32_t* s, uint32_t mw,
-                                         unsigned long long start, uint32_t w0, uint32_t w1, uint32_t w2) {
+    __device__ __forceinline__ uint32_t load(uint32_t i) const { return words(i); }
+    __device__ __forceinline__ void init(const uint32_t* table, const Words& w, unsigned long long start) {
         lut = table;
-        sw = s;
-        maxw = mw;
+        words = w;
+        const uint32_t wi = (uint32_t)(start >> 5);
+        const uint32_t w0 = load(wi), w1 = load(wi + 1);
         o0 = (uint32_t)start & 31u;
         hi = __funnelshift_l(w1, w0, o0);  // the window ends where w1 ends
         lo = w1 << o0;
         g = (int32_t)o0 - 32;              // 64 - o0 valid bits
-        nxt = w2;
-        wp0 = wp = (uint32_t)(start >> 5) + 3;
+        nxt = load(wi + 2);
+        wp0 = wp = wi + 3;
     }
     __device__ __forceinline__ void refill() {  // requires g >= 0
         hi |= __funnelshift_lc(nxt, 0u, (uint32_t)g);
@@ -338,8 +354,8 @@ struct BitReader {
 };
 
 // Decode the K codes of this lane's chunk into the stash.
-template <int K, bool kClamp>
-__device__ __forceinline__ void decode_chunk(BitReader<kClamp>& br, const Tables& T, uint32_t* stash,
+template <int K, class Words>
+__device__ __forceinline__ void decode_chunk(BitReader<Words>& br, const Tables& T, uint32_t* stash,
                                              unsigned lane, uint32_t& err) {
     constexpr int S = StashShape<K>::kStride;
 #pragma unroll 4
@@ -356,8 +372,8 @@ __device__ __forceinline__ void decode_chunk(BitReader<kClamp>& br, const Tables
 
 template <int K>
 struct WarpBuffers {
-    uint32_t stash[StashShape<K>::kWords];      // decoded exponents
-    __align__(16) uint8_t m[32 * K];            // the group's sign+mantissa bytes
+    uint32_t stash[StashShape<K>::kWords];     // decoded exponents
+    __align__(16) uint32_t slice[2][kSliceWords];  // stream slices of this group and the next
 };
 
 template <int K>
@@ -371,78 +387,106 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prior() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
+}
 
-// Full groups (all 32 chunks hold K codes), one warp at a time, with the next
-// group's index and first stream words in flight while this group decodes.
+// Stage the stream words of one group, [gb0 >> 5, ((gb0 + span) >> 5) + 4), in a slice
+// buffer (16-byte cp.async chunks, bypassing L1).  Returns false, and copies nothing,
+// when the group is inconsistent or its words do not fit; the group is then decoded
+// straight from global memory.
+struct Slice {
+    uint32_t base;  // stream word index of the first staged word
+    bool staged;
+};
+
+__device__ __forceinline__ Slice stage_slice(const DecodeArgs& a, const Tables& T, uint32_t* buf,
+                                             unsigned long long gb0, uint32_t span, bool ok, unsigned lane) {
+    Slice r;
+    const uint32_t beg = ((uint32_t)(gb0 >> 5) * 4u) & ~15u;  // bytes into the stream section
+    const uint32_t end = min((((uint32_t)((gb0 + span) >> 5) + 4u) * 4u + 15u) & ~15u, T.n_words * 4u);
+    r.base = beg / 4u;
+    r.staged = ok && end > beg && end - beg <= kSliceWords * 4u;
+    if (r.staged) {
+        const uint8_t* src = a.comp + a.off_stream + beg;
+        for (uint32_t c = lane; c < (end - beg) / 16u; c += 32) cp_async16(buf + 4 * c, src + 16 * c);
+    }
+    return r;
+}
+
+// Full groups (all 32 chunks hold K codes), one warp at a time.  While group g decodes,
+// the stream slice of the warp's next group is copied into the other slice buffer and
+// the index of the group after that is loaded; the sign+mantissa bytes of g are
+// prefetched into L2 when g starts and read by the merge.
 template <int K>
 __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const uint32_t* lut, WarpBuffers<K>& wb,
-                                   uint64_t g,
-                                   uint64_t step, uint64_t n_full, unsigned lane, uint32_t& err) {
+                                   uint32_t g, uint32_t step, uint32_t n_full, unsigned lane, uint32_t& err) {
     constexpr int S = StashShape<K>::kStride;
-    constexpr int kMChunks = (32 * K) / 16 / 32;  // 16-byte copies per lane
     if (g >= n_full) return;
     const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
     const uint32_t maxw = T.n_words - 1;
     const uint8_t* mplane = a.comp + a.off_m;
 
     GroupStart st = scan_index(load_index(a, T, g, lane, true), lane);
-    uint32_t w0 = ld_word(sw, (uint32_t)(st.start >> 5), maxw);
-    uint32_t w1 = ld_word(sw, (uint32_t)(st.start >> 5) + 1, maxw);
-    uint32_t w2 = ld_word(sw, (uint32_t)(st.start >> 5) + 2, maxw);
-    uint64_t gn = g + step;
+    Slice sl = stage_slice(a, T, wb.slice[0], st.gb0, st.span, st.ok, lane);
+    cp_async_commit();
+    uint32_t gn = g + step;
     GroupIndex idx_n;
     if (gn < n_full) idx_n = load_index(a, T, gn, lane, true);
+    uint32_t b = 0;
 
     while (true) {
-        // the sign+mantissa bytes of this group go to shared memory asynchronously
-        const uint8_t* msrc = mplane + g * (32ull * K);
-#pragma unroll
-        for (int i = 0; i < kMChunks; i++) cp_async16(wb.m + 16 * (lane + 32 * i), msrc + 16 * (lane + 32 * i));
-        cp_async_commit();
-
-        // the next group's read positions and first words
+        if (lane == 0) prefetch_l2(mplane + (uint64_t)g * (32u * K), 32u * K);
         const bool has_next = gn < n_full;
-        const uint64_t gnn = gn + step;
+        const uint32_t gnn = gn + step;
         GroupStart st_n;
-        uint32_t nw0 = 0, nw1 = 0, nw2 = 0;
+        Slice sl_n;
         GroupIndex idx_nn;
         if (has_next) {
             st_n = scan_index(idx_n, lane);
-            const uint32_t wi = (uint32_t)(st_n.start >> 5);
-            nw0 = ld_word(sw, wi, maxw);
-            nw1 = ld_word(sw, wi + 1, maxw);
-            nw2 = ld_word(sw, wi + 2, maxw);
+            sl_n = stage_slice(a, T, wb.slice[b ^ 1], st_n.gb0, st_n.span, st_n.ok, lane);
             if (gnn < n_full) idx_nn = load_index(a, T, gnn, lane, true);
         }
+        cp_async_commit();
+        cp_async_wait_prior();  // this group's slice has landed
+        __syncwarp();
 
         if (st.ok) {
-            // A chunk refills at most 3K/4 times (24-bit codes); lane 31 starts last.  When
-            // the warp's last possible read is inside the stream, the loads need no clamp.
-            const uint32_t last_wp0 = __shfl_sync(kFull, (uint32_t)(st.start >> 5) + 3u, 31);
-            if (last_wp0 + (3u * K) / 4u + 3u <= maxw) {
-                BitReader<false> br;
-                br.init(lut, sw, maxw, st.start, w0, w1, w2);
-                decode_chunk<K, false>(br, T, wb.stash, lane, err);
-                if (br.consumed() != st.clen) err |= DFX_STATUS_STREAM;
+            uint32_t used;
+            if (sl.staged) {
+                BitReader<SharedWords> br;
+                br.init(lut, SharedWords{wb.slice[b], sl.base}, st.start);
+                decode_chunk<K>(br, T, wb.stash, lane, err);
+                used = br.consumed();
             } else {
-                BitReader<true> br;
-                br.init(lut, sw, maxw, st.start, w0, w1, w2);
-                decode_chunk<K, true>(br, T, wb.stash, lane, err);
-                if (br.consumed() != st.clen) err |= DFX_STATUS_STREAM;
+                // A chunk refills at most 3K/4 times (24-bit codes); lane 31 starts last.
+                const uint32_t last = __shfl_sync(kFull, (uint32_t)(st.start >> 5), 31);
+                if (last + (3u * K) / 4u + 8u <= maxw) {
+                    BitReader<GlobalWords> br;
+                    br.init(lut, GlobalWords{sw}, st.start);
+                    decode_chunk<K>(br, T, wb.stash, lane, err);
+                    used = br.consumed();
+                } else {
+                    BitReader<ClampedGlobalWords> br;
+                    br.init(lut, ClampedGlobalWords{sw, maxw}, st.start);
+                    decode_chunk<K>(br, T, wb.stash, lane, err);
+                    used = br.consumed();
+                }
             }
+            if (used != st.clen) err |= DFX_STATUS_STREAM;
         } else {
             err |= DFX_STATUS_INDEX;
         }
-        cp_async_wait_all();
         __syncwarp();
         if (st.ok) {
-            uint4* out4 = reinterpret_cast<uint4*>(a.out) + g * (32 * K / 8) + lane;
+            const uint2* mp = reinterpret_cast<const uint2*>(mplane) + (uint64_t)g * (32u * K / 8u) + lane;
+            uint4* out4 = reinterpret_cast<uint4*>(a.out) + (uint64_t)g * (32u * K / 8u) + lane;
 #pragma unroll
             for (int r = 0; r < K / 8; r++) {
                 const int j0 = 8 * (int)lane + 256 * r;
                 const int t = j0 / K, q0 = (j0 % K) / 4;
-                const uint2 m = *reinterpret_cast<const uint2*>(wb.m + j0);
-                out4[32 * r] = merge8(m, wb.stash[q0 * S + t], wb.stash[(q0 + 1) * S + t]);
+                out4[32 * r] = merge8(__ldg(mp + 32 * r), wb.stash[q0 * S + t], wb.stash[(q0 + 1) * S + t]);
             }
         }
         __syncwarp();
@@ -450,11 +494,11 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
         g = gn;
         gn = gnn;
         st = st_n;
-        w0 = nw0;
-        w1 = nw1;
-        w2 = nw2;
+        sl = sl_n;
         idx_n = idx_nn;
+        b ^= 1;
     }
+    cp_async_wait_all();
 }
 
 // The last group when it is ragged: chunks may be short or absent, outputs stop at n.
@@ -474,9 +518,8 @@ __device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, const ui
     if (has) {
         const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
         const uint32_t maxw = T.n_words - 1;
-        const uint32_t wi = (uint32_t)(gs.start >> 5);
-        BitReader<true> br;
-        br.init(lut, sw, maxw, gs.start, ld_word(sw, wi, maxw), ld_word(sw, wi + 1, maxw), ld_word(sw, wi + 2, maxw));
+        BitReader<ClampedGlobalWords> br;
+        br.init(lut, ClampedGlobalWords{sw, maxw}, gs.start);
         for (int q = 0; q < K / 4; q++) {
             uint32_t acc = 0;
             for (int k = 0; k < 4; k++)
@@ -524,9 +567,9 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     WarpBuffers<K>& wb = *reinterpret_cast<WarpBuffers<K>*>(warp_area + warp * warp_buffer_bytes<K>());
     uint32_t err = 0;
-    const uint64_t n_full = (a.n % (32ull * K) == 0) ? a.n_group : a.n_group - 1;
-    const uint64_t step = (uint64_t)gridDim.x * kDecodeWarps;
-    const uint64_t gw = (uint64_t)blockIdx.x * kDecodeWarps + warp;
+    const uint32_t n_full = (a.n % (32ull * K) == 0) ? a.n_group : a.n_group - 1;
+    const uint32_t step = gridDim.x * kDecodeWarps;
+    const uint32_t gw = blockIdx.x * kDecodeWarps + warp;
     decode_full_groups<K>(a, T, lut, wb, gw, step, n_full, lane, err);
     if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, lut, wb, n_full, lane, err);
     if (err) atomicOr(a.status, err);
