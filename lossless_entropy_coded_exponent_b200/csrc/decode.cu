@@ -3,19 +3,22 @@
 // Design (B200-first; the pages' GPU decoder is prior art, "DFloat11: lossless LLM
 // compression for GPU", aikraft.ru blog, section 03):
 //   * persistent grid, 8 warps per CTA; each CTA first builds its decoding tables in
-//     shared memory from len[256]: a direct lookup table on the next 12 bits for every
-//     code of length <= 12 and, for longer codes, the canonical per-length limits (the
-//     two levels of the hierarchical table of section 03, item 1);
+//     shared memory from len[256]: a pair table on the next 14 bits that resolves two
+//     codes at once when both fit, a one-code view of it, and, for codes longer than 14
+//     bits, the canonical per-length limits (the levels of the hierarchical table of
+//     section 03, item 1);
 //   * one warp decodes one group of 32 chunks; lane i owns chunk i of the group and
 //     decodes exactly K codes.  Its read position is the group's start bit plus the
 //     warp's exclusive scan of the chunk bit lengths (the "lightweight auxiliary
 //     variables" that coordinate read positions, section 03, item 2).  Output positions
 //     need no scan: chunk i writes elements [i*K, i*K + K) of the group;
-//   * each lane keeps a 64-bit window of its stream in registers and refills it with
-//     one word when at most 32 bits are left, once per two codes, so the common path
-//     has no per-code branch besides the rare long-code test;
-//   * the next group's index and first stream words are loaded while the current group
-//     decodes; its sign+mantissa bytes arrive in shared memory by cp.async;
+//   * each lane keeps its bit position and a 32-bit peek of the stream; the peek is
+//     reloaded from the warp's shared-memory copy of the group's stream slice once per
+//     two pair lookups, so the common path has no per-code branch besides the rare
+//     unresolved-pair test;
+//   * the next group's stream slice is copied into shared memory (cp.async) and its
+//     index loaded while the current group decodes; the group's sign+mantissa bytes are
+//     prefetched into L2 when it starts;
 //   * decoded exponents go to a per-warp shared-memory stash laid out so that both the
 //     lane-per-chunk writes and the coalesced reads of the merge step are free of bank
 //     conflicts; the merge joins them with the sign+mantissa bytes and writes BF16 with
@@ -250,72 +253,59 @@ __device__ __forceinline__ GroupStart scan_index(const GroupIndex& x, unsigned l
 
 // ---------------------------------------------------------------- bit reader
 //
-// hi:lo is a 64-bit window whose top 32 - g bits are the next bits of the stream and
-// whose other bits are zero (g = 32 - valid bits, kept in [-32, 32]); `nxt` is the next
-// stream word, already loaded.  A refill (g >= 0, i.e. at most 32 valid bits) shifts
-// `nxt` in under the valid bits.  Codes are decoded two per table lookup; every pair
-// that the table resolves consumes at most kLutBits = 12 bits, so one refill check per
-// two pairs keeps enough bits in the window.  Pairs the table cannot resolve (the
-// second code does not fit the index bits, or the first code is longer than 12 bits)
-// take a rare branch that decodes code by code and refills as it needs.
-// Where a bit reader takes its stream words from: the global stream (with or without a
-// bound clamp) or a warp's shared-memory copy of its group's slice of the stream.
+// A lane's state is its bit position p, relative to the first word of its word source,
+// and `peek`, the 32 stream bits starting at p.  Once per round of two pairs, peek is
+// reloaded from the two words holding bit p (two loads and one funnel shift).  Every
+// pair the table resolves consumes at most kLutBits = 14 bits, so after the first pair
+// of a round at least 18 valid bits remain for the second.  Pairs the table cannot
+// resolve (the second code does not fit the index bits, or the first code is longer)
+// take a rare branch that reloads and decodes code by code.
+//
+// Word sources: the global stream (with or without a bound clamp) or a warp's
+// shared-memory copy of its group's slice of the stream.
 struct GlobalWords {
-    const uint32_t* p;
-    __device__ __forceinline__ uint32_t operator()(uint32_t i) const { return __ldg(p + i); }
+    const uint32_t* p;  // first word of the source
+    __device__ __forceinline__ uint32_t load(uint32_t i) const { return __ldg(p + i); }
 };
 struct ClampedGlobalWords {
     const uint32_t* p;
-    uint32_t maxw;
-    __device__ __forceinline__ uint32_t operator()(uint32_t i) const { return __ldg(p + min(i, maxw)); }
+    uint32_t maxw;  // last readable index
+    __device__ __forceinline__ uint32_t load(uint32_t i) const { return __ldg(p + min(i, maxw)); }
 };
 constexpr uint32_t kSliceWords = 256;  // 1 KiB per staged group slice
 struct SharedWords {
-    const uint32_t* s;  // the slice buffer
-    uint32_t base;      // stream word index of s[0]
-    // Well-formed groups read inside the slice; the clamp keeps a corrupt one in the buffer.
-    __device__ __forceinline__ uint32_t operator()(uint32_t i) const { return s[min(i - base, kSliceWords - 1)]; }
+    uint32_t s;  // shared-memory address of the slice buffer
+    // Well-formed groups read inside the slice.  A corrupt one reads at most 3K/4 + 2
+    // words past its start, into the next buffers or the guard pad after the last warp's
+    // buffers: never outside the CTA's shared memory.
+    __device__ __forceinline__ uint32_t load(uint32_t i) const {
+        uint32_t v;
+        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(s + 4u * i));
+        return v;
+    }
 };
 
 template <class Words>
 struct BitReader {
     const uint32_t* lut;  // pair table in shared memory
     Words words;
-    uint32_t hi, lo, nxt, wp, wp0, o0;
-    int32_t g;
+    uint32_t p, p0, peek;
 
-    __device__ __forceinline__ uint32_t load(uint32_t i) const { return words(i); }
-    __device__ __forceinline__ void init(const uint32_t* table, const Words& w, unsigned long long start) {
+    __device__ __forceinline__ void init(const uint32_t* table, const Words& w, uint32_t start) {
         lut = table;
         words = w;
-        const uint32_t wi = (uint32_t)(start >> 5);
-        const uint32_t w0 = load(wi), w1 = load(wi + 1);
-        o0 = (uint32_t)start & 31u;
-        hi = __funnelshift_l(w1, w0, o0);  // the window ends where w1 ends
-        lo = w1 << o0;
-        g = (int32_t)o0 - 32;              // 64 - o0 valid bits
-        nxt = load(wi + 2);
-        wp0 = wp = wi + 3;
+        p = p0 = start;
     }
-    __device__ __forceinline__ void refill() {  // requires g >= 0
-        hi |= __funnelshift_lc(nxt, 0u, (uint32_t)g);
-        lo |= __funnelshift_lc(0u, nxt, (uint32_t)g);
-        g -= 32;
-        nxt = load(wp);
-        wp++;
+    __device__ __forceinline__ void reload() {
+        const uint32_t wi = p >> 5;
+        peek = __funnelshift_l(words.load(wi + 1), words.load(wi), p);  // shift uses p & 31
     }
-    __device__ __forceinline__ void consume(uint32_t len) {  // len in 0..31
-        hi = __funnelshift_l(lo, hi, len);
-        lo = __funnelshift_l(0u, lo, len);
-        g += (int32_t)len;
-    }
-    // One code, the general way: returns its symbol.
+    // One code, the general way (peek must be current): returns its symbol.
     __device__ __forceinline__ uint32_t one(const Tables& T, uint32_t& err) {
-        if (g > 32 - (int)kMaxLenLimit) refill();  // at least 24 valid bits
-        const uint32_t e = lut[hi >> (32 - kLutBits)];
+        const uint32_t e = lut[peek >> (32 - kLutBits)];
         uint32_t len, sym;
         if ((e & 0x001F0000u) == 0) {
-            uint32_t ent = decode_long(hi, T);
+            uint32_t ent = decode_long(peek, T);
             if (ent >> 16) {
                 err |= DFX_STATUS_STREAM;
                 ent &= 0xFFFFu;
@@ -326,20 +316,22 @@ struct BitReader {
             len = (e >> 16) & 31u;
             sym = e & 0xFFu;
         }
-        consume(len);
-        if (g > 32 - kLutBits) refill();  // at least 12 valid bits for the next pair
+        p += len;
+        reload();
         return sym;
     }
     // Two codes: returns acc with their symbols in bytes 2j and 2j+1.
     template <int j>
     __device__ __forceinline__ uint32_t pair(uint32_t acc, const Tables& T, uint32_t& err) {
         constexpr uint32_t sel = j == 0 ? 0x3254u : 0x5410u;
-        const uint32_t e = lut[hi >> (32 - kLutBits)];
-        const uint32_t len = e >> 26;  // wraps to the first code's length (or 0) when bit 31 is set
-        consume(len);
+        const uint32_t e = lut[peek >> (32 - kLutBits)];
+        const uint32_t len = e >> 26;           // bit 5 is set when the entry is not a pair
+        peek = __funnelshift_l(0u, peek, len);  // shifts by len & 31
+        p += len;
         acc = __byte_perm(acc, e, sel);
         if ((int32_t)e < 0) {
-            g -= 32;  // undo bit 31 of `len`
+            p -= 32;  // undo bit 5 of `len`
+            reload();
             uint32_t s0 = e & 0xFFu;
             if ((e & 0x001F0000u) == 0) s0 = one(T, err);
             const uint32_t s1 = one(T, err);
@@ -347,10 +339,7 @@ struct BitReader {
         }
         return acc;
     }
-    // Bits consumed since init.
-    __device__ __forceinline__ uint32_t consumed() const {
-        return 32u + 32u * (wp - wp0) - o0 + (uint32_t)g;
-    }
+    __device__ __forceinline__ uint32_t consumed() const { return p - p0; }
 };
 
 // Decode the K codes of this lane's chunk into the stash.
@@ -360,10 +349,10 @@ __device__ __forceinline__ void decode_chunk(BitReader<Words>& br, const Tables&
     constexpr int S = StashShape<K>::kStride;
 #pragma unroll 4
     for (int q = 0; q < K / 4; q++) {
+        br.reload();
         uint32_t acc = 0;
         acc = br.template pair<0>(acc, T, err);
         acc = br.template pair<1>(acc, T, err);
-        if (br.g >= 0) br.refill();
         stash[q * S + lane] = acc;
     }
 }
@@ -456,20 +445,24 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
             uint32_t used;
             if (sl.staged) {
                 BitReader<SharedWords> br;
-                br.init(lut, SharedWords{wb.slice[b], sl.base}, st.start);
+                br.init(lut, SharedWords{(uint32_t)__cvta_generic_to_shared(wb.slice[b])},
+                        (uint32_t)(st.start - 32ull * sl.base));
                 decode_chunk<K>(br, T, wb.stash, lane, err);
                 used = br.consumed();
             } else {
-                // A chunk refills at most 3K/4 times (24-bit codes); lane 31 starts last.
+                // A chunk reads at most 3K/4 + 2 words past its start (24-bit codes); lane 31
+                // starts last.  When that stays inside the stream the loads need no clamp.
+                const uint32_t first = (uint32_t)(st.gb0 >> 5);
                 const uint32_t last = __shfl_sync(kFull, (uint32_t)(st.start >> 5), 31);
+                const uint32_t rel = (uint32_t)(st.start - 32ull * first);
                 if (last + (3u * K) / 4u + 8u <= maxw) {
                     BitReader<GlobalWords> br;
-                    br.init(lut, GlobalWords{sw}, st.start);
+                    br.init(lut, GlobalWords{sw + first}, rel);
                     decode_chunk<K>(br, T, wb.stash, lane, err);
                     used = br.consumed();
                 } else {
                     BitReader<ClampedGlobalWords> br;
-                    br.init(lut, ClampedGlobalWords{sw, maxw}, st.start);
+                    br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, rel);
                     decode_chunk<K>(br, T, wb.stash, lane, err);
                     used = br.consumed();
                 }
@@ -518,9 +511,11 @@ __device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, const ui
     if (has) {
         const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
         const uint32_t maxw = T.n_words - 1;
+        const uint32_t first = (uint32_t)(gs.gb0 >> 5);
         BitReader<ClampedGlobalWords> br;
-        br.init(lut, ClampedGlobalWords{sw, maxw}, gs.start);
+        br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, (uint32_t)(gs.start - 32ull * first));
         for (int q = 0; q < K / 4; q++) {
+            br.reload();
             uint32_t acc = 0;
             for (int k = 0; k < 4; k++)
                 if ((uint32_t)(4 * q + k) < cnt) acc |= br.one(T, err) << (8 * k);
@@ -575,10 +570,13 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
     if (err) atomicOr(a.status, err);
 }
 
+constexpr size_t kGuardBytes = 512;  // see SharedWords
+
 template <int K>
 constexpr size_t dyn_smem_bytes() {
-    return kLutBytes + DecodeShape<K>::kWarps * warp_buffer_bytes<K>();
+    return kLutBytes + DecodeShape<K>::kWarps * warp_buffer_bytes<K>() + kGuardBytes;
 }
+static_assert(kGuardBytes >= 4 * (3 * 128 / 4 + 8), "guard covers the longest run past a slice");
 static_assert(DecodeShape<32>::kWarps * warp_buffer_bytes<32>() >= (2u << kLutBits), "scratch for the one-code table");
 static_assert(DecodeShape<128>::kWarps * warp_buffer_bytes<128>() >= (2u << kLutBits), "scratch for the one-code table");
 static_assert(dyn_smem_bytes<64>() + 1024 <= 227 * 1024 && dyn_smem_bytes<128>() + 1024 <= 227 * 1024, "shared memory");
