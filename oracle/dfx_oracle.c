@@ -18,7 +18,7 @@
  * The pages leave the concrete code open.  This codec's reading, written out
  * step by step below, is:
  *   1. split every BF16 word into its 8-bit exponent and an 8-bit
- *      sign+mantissa byte;
+ *      mantissa+sign byte (the low byte of the word rotated left by one);
  *   2. histogram the exponents;
  *   3. length-limited (max_len, default 24) Huffman code lengths by
  *      package-merge, ties broken by symbol value;
@@ -26,7 +26,10 @@
  *   5. concatenate the codes MSB-first into 32-bit words;
  *   6. index: per chunk of K symbols its bit length, per group of G chunks its
  *      start bit (the "lightweight auxiliary variables" that let GPU threads
- *      find their read positions, DFloat11 blog section 03, item 2);
+ *      find their read positions, DFloat11 blog section 03, item 2).  The
+ *      elements of a group (G*K of them) are cut into blocks of 8; block b
+ *      belongs to chunk b mod G, so a chunk holds K/8 blocks spaced G blocks
+ *      apart, and the codes are concatenated chunk after chunk;
  *   7. serialise the DFX1 container;
  *   8. decode bit by bit (canonical first-code/count walk), check the index
  *      against the walk, merge the two bytes back.
@@ -39,17 +42,18 @@
  *   8   u64 n              number of BF16 elements
  *   16  u64 total_bits     length of the code stream in bits
  *   24  u64 total_bytes    size of the whole container
- *   32  u32 K              symbols per chunk
+ *   32  u32 K              symbols per chunk (a multiple of 8)
  *   36  u32 G              chunks per group
- *   40  u32 n_chunk = ceil(n / K)
- *   44  u32 n_group = ceil(n_chunk / G)
+ *   40  u32 n_chunk = G * n_group
+ *   44  u32 n_group = ceil(n / (G * K))
  *   48  u64 off_m          byte offset of the sign+mantissa plane
  *   56  u32 max_len        code-length limit used by the encoder
  *   60  u32 reserved = 0
  *   64  u8  len[256]       code length of every exponent value (0 = unused)
  *   320 u64 gbase[n_group + 1]  start bit of each group, gbase[n_group] = total_bits
- *   .   u16 clen[n_chunk]       bit length of each chunk
- *   .   u8  m[n]                sign+mantissa bytes, element order
+ *   .   u16 clen[n_chunk]       bit length of each chunk (0 for a chunk of the
+ *                               last group that has no element)
+ *   .   u8  m[n]                mantissa+sign bytes, element order
  *   .   u32 stream[...]         codes, bit k of the stream = bit (31 - k % 32)
  *                               of word k / 32; 4*ceil(total_bits/32) bytes
  *                               rounded up to 16, then 16 zero bytes of slack
@@ -87,12 +91,13 @@ static uint64_t get_u64(const uint8_t *p) {
 static uint64_t align16(uint64_t x) { return (x + 15u) & ~(uint64_t)15u; }
 
 /* ------------------------------------------------------------------ */
-/* Step 1: the split.  BF16 = sign(1) | exponent(8) | mantissa(7).      */
+/* Step 1: the split.  BF16 = sign(1) | exponent(8) | mantissa(7).  The other
+ * byte holds the mantissa above the sign: mantissa * 2 + sign.            */
 
 uint8_t dfxo_exponent(uint16_t w) { return (uint8_t)((w >> 7) & 0xFF); }
-uint8_t dfxo_sign_mantissa(uint16_t w) { return (uint8_t)(((w >> 8) & 0x80) | (w & 0x7F)); }
+uint8_t dfxo_sign_mantissa(uint16_t w) { return (uint8_t)(((w & 0x7F) << 1) | (w >> 15)); }
 uint16_t dfxo_merge(uint8_t e, uint8_t m) {
-    return (uint16_t)(((uint16_t)(m & 0x80) << 8) | ((uint16_t)e << 7) | (m & 0x7F));
+    return (uint16_t)(((uint16_t)(m & 1) << 15) | ((uint16_t)e << 7) | (m >> 1));
 }
 
 /* ------------------------------------------------------------------ */
@@ -237,20 +242,25 @@ int dfxo_canonical_codes(const uint8_t len[256], uint32_t code[256]) {
 static int params_ok(uint64_t n, uint32_t K, uint32_t G, uint32_t max_len) {
     if (n >= ((uint64_t)1 << 32)) return 0;
     if (max_len < 1 || max_len > 24) return 0;
-    if (K < 1 || G < 1) return 0;
+    if (K < 8 || K % 8 != 0 || G < 1) return 0;
     if ((uint64_t)K * max_len > 65535u) return 0; /* a chunk length must fit in u16 */
     return 1;
 }
 
-static uint64_t n_chunks(uint64_t n, uint32_t K) { return (n + K - 1) / K; }
-static uint64_t n_groups(uint64_t nc, uint32_t G) { return (nc + G - 1) / G; }
+static uint64_t n_groups(uint64_t n, uint32_t K, uint32_t G) { return (n + (uint64_t)G * K - 1) / ((uint64_t)G * K); }
+
+/* Element of position `pos` (0..K-1) in chunk `lane` of group g: the group's
+ * elements form blocks of 8, block b belongs to chunk b mod G. */
+static uint64_t chunk_element(uint64_t g, uint32_t lane, uint32_t pos, uint32_t K, uint32_t G) {
+    return g * G * K + ((uint64_t)(pos / 8) * G + lane) * 8 + pos % 8;
+}
 static uint64_t off_clen_of(uint64_t ng) { return align16(DFXO_GBASE_OFFSET + 8 * (ng + 1)); }
 static uint64_t off_m_of(uint64_t nc, uint64_t ng) { return align16(off_clen_of(ng) + 2 * nc); }
 static uint64_t off_stream_of(uint64_t n, uint64_t nc, uint64_t ng) { return align16(off_m_of(nc, ng) + n); }
 static uint64_t stream_bytes_of(uint64_t total_bits) { return align16(4 * ((total_bits + 31) / 32)) + 16; }
 
 uint64_t dfxo_container_bytes(uint64_t n, uint32_t K, uint32_t G, uint64_t total_bits) {
-    uint64_t nc = n_chunks(n, K), ng = n_groups(nc, G);
+    uint64_t ng = n_groups(n, K, G), nc = ng * G;
     return off_stream_of(n, nc, ng) + stream_bytes_of(total_bits);
 }
 
@@ -288,7 +298,7 @@ int dfxo_encode(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t 
 
     uint64_t total_bits = 0;
     for (uint64_t i = 0; i < n; i++) total_bits += len[dfxo_exponent(w[i])];
-    uint64_t nc = n_chunks(n, K), ng = n_groups(nc, G);
+    uint64_t ng = n_groups(n, K, G), nc = ng * G;
     uint64_t total = dfxo_container_bytes(n, K, G, total_bits);
     if (out_bytes) *out_bytes = total;
     if (cap < total) return DFXO_ERR_CAPACITY;
@@ -309,28 +319,28 @@ int dfxo_encode(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t 
     put_u32(out + 60, 0);
     memcpy(out + DFXO_LEN_OFFSET, len, 256);
 
-    /* index: chunk bit lengths and group start bits, from the prefix of code lengths */
+    /* stream in chunk order, index: chunk bit lengths and group start bits */
     uint8_t *gbase = out + DFXO_GBASE_OFFSET;
     uint8_t *clen = out + off_clen_of(ng);
-    uint64_t pos = 0;
-    for (uint64_t c = 0; c < nc; c++) {
-        if (c % G == 0) put_u64(gbase + 8 * (c / G), pos);
-        uint64_t start = pos;
-        uint64_t end_i = (c + 1) * K < n ? (c + 1) * K : n;
-        for (uint64_t i = c * K; i < end_i; i++) pos += len[dfxo_exponent(w[i])];
-        put_u16(clen + 2 * c, (uint16_t)(pos - start));
-    }
-    put_u64(gbase + 8 * ng, pos);
-
     uint8_t *mplane = out + off_m_of(nc, ng);
     uint8_t *stream = out + off_stream_of(n, nc, ng);
-    pos = 0;
-    for (uint64_t i = 0; i < n; i++) {
-        uint8_t e = dfxo_exponent(w[i]);
-        mplane[i] = dfxo_sign_mantissa(w[i]);
-        put_bits(stream, pos, code[e], len[e]);
-        pos += len[e];
+    uint64_t pos = 0;
+    for (uint64_t g = 0; g < ng; g++) {
+        put_u64(gbase + 8 * g, pos);
+        for (uint32_t lane = 0; lane < G; lane++) {
+            uint64_t start = pos;
+            for (uint32_t k = 0; k < K; k++) {
+                uint64_t x = chunk_element(g, lane, k, K, G);
+                if (x >= n) break;
+                uint8_t e = dfxo_exponent(w[x]);
+                put_bits(stream, pos, code[e], len[e]);
+                pos += len[e];
+            }
+            put_u16(clen + 2 * (g * G + lane), (uint16_t)(pos - start));
+        }
     }
+    put_u64(gbase + 8 * ng, pos);
+    for (uint64_t i = 0; i < n; i++) mplane[i] = dfxo_sign_mantissa(w[i]);
     return DFXO_OK;
 }
 
@@ -357,7 +367,7 @@ int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, u
     uint32_t max_len = get_u32(c + 56);
     if (!params_ok(n, K, G, max_len)) return DFXO_ERR_CORRUPT;
     if (get_u32(c + 60) != 0) return DFXO_ERR_CORRUPT;
-    uint64_t nc = n_chunks(n, K), ng = n_groups(nc, G);
+    uint64_t ng = n_groups(n, K, G), nc = ng * G;
     if (get_u32(c + 40) != nc || get_u32(c + 44) != ng) return DFXO_ERR_CORRUPT;
     if (get_u64(c + 48) != off_m_of(nc, ng)) return DFXO_ERR_CORRUPT;
     if (total_bits > (uint64_t)max_len * n) return DFXO_ERR_CORRUPT;
@@ -411,29 +421,29 @@ int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, u
     if (get_u64(gbase) != 0 || get_u64(gbase + 8 * ng) != total_bits) return DFXO_ERR_CORRUPT;
 
     uint64_t pos = 0;
-    uint64_t chunk_start = 0;
-    for (uint64_t i = 0; i < n; i++) {
-        if (i % K == 0) {
-            uint64_t ci = i / K;
-            chunk_start = pos;
-            if (ci % G == 0 && get_u64(gbase + 8 * (ci / G)) != pos) return DFXO_ERR_CORRUPT;
-        }
-        uint32_t code = 0;
-        int l = 0, found = -1;
-        while (l < 24) {
-            if (pos >= total_bits) return DFXO_ERR_CORRUPT;
-            code = (code << 1) | get_bit(stream, pos);
-            pos++;
-            l++;
-            if (count[l] && code >= first[l] && code - first[l] < count[l]) {
-                found = sorted[index_of_first[l] + (code - first[l])];
-                break;
+    for (uint64_t g = 0; g < ng; g++) {
+        if (get_u64(gbase + 8 * g) != pos) return DFXO_ERR_CORRUPT;
+        for (uint32_t lane = 0; lane < G; lane++) {
+            uint64_t chunk_start = pos;
+            for (uint32_t k = 0; k < K; k++) {
+                uint64_t x = chunk_element(g, lane, k, K, G);
+                if (x >= n) break;
+                uint32_t code = 0;
+                int l = 0, found = -1;
+                while (l < 24) {
+                    if (pos >= total_bits) return DFXO_ERR_CORRUPT;
+                    code = (code << 1) | get_bit(stream, pos);
+                    pos++;
+                    l++;
+                    if (count[l] && code >= first[l] && code - first[l] < count[l]) {
+                        found = sorted[index_of_first[l] + (code - first[l])];
+                        break;
+                    }
+                }
+                if (found < 0) return DFXO_ERR_CORRUPT;
+                w[x] = dfxo_merge((uint8_t)found, mplane[x]);
             }
-        }
-        if (found < 0) return DFXO_ERR_CORRUPT;
-        w[i] = dfxo_merge((uint8_t)found, mplane[i]);
-        if ((i + 1) % K == 0 || i + 1 == n) {
-            if (get_u16(clen + 2 * (i / K)) != pos - chunk_start) return DFXO_ERR_CORRUPT;
+            if (get_u16(clen + 2 * (g * G + lane)) != pos - chunk_start) return DFXO_ERR_CORRUPT;
         }
     }
     if (pos != total_bits) return DFXO_ERR_CORRUPT;

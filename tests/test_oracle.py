@@ -98,7 +98,11 @@ def load_golden_containers():
                        "bytes": np.zeros(int(kv["total"]), dtype=np.uint8)}
                 cases.append(cur)
             elif line.startswith("input"):
-                cur["input"] = np.array([int(t, 16) for t in line.split()[1:]], dtype=np.uint16)
+                words = []
+                for t in line.split()[1:]:
+                    wv, _, rep = t.partition("*")
+                    words += [int(wv, 16)] * (int(rep) if rep else 1)
+                cur["input"] = np.array(words, dtype=np.uint16)
             else:
                 off, hexes = line.split(":")
                 vals = [int(t, 16) for t in hexes.split()]
@@ -148,8 +152,8 @@ def test_split_matches_ieee_fields_for_every_pattern():
     nan = np.isnan(x)
     assert np.array_equal(e_or, exp_e)
     ok = ~nan
-    assert np.array_equal(m_or[ok], (sign[ok] << 7) | mant[ok])
-    assert np.all((m_or[nan] & 0x7F) != 0) and np.array_equal(m_or[nan] >> 7, sign[nan])
+    assert np.array_equal(m_or[ok], (mant[ok] << 1) | sign[ok])
+    assert np.all((m_or[nan] >> 1) != 0) and np.array_equal(m_or[nan] & 1, sign[nan])
     back = np.array([oracle.merge(int(e), int(m)) for e, m in zip(e_or, m_or)], dtype=np.uint16)
     assert np.array_equal(back, w)
 
@@ -270,7 +274,7 @@ def test_round_trip_every_bit_pattern():
 @pytest.mark.parametrize("name", list(inputs.edge_cases().keys()))
 def test_round_trip_edge_cases(name):
     w = inputs.edge_cases()[name]
-    for K, G in ((64, 32), (128, 32), (5, 3)):
+    for K, G in ((64, 32), (128, 32), (8, 3), (16, 5)):
         c = oracle.encode(w, K=K, G=G)
         assert c.size == oracle.container_bytes(w.size, K, G, int(c[16:24].view(np.uint64)[0]))
         assert np.array_equal(oracle.decode(c), w)
@@ -322,14 +326,19 @@ def _corrupt_variants(c):
     nc = int(c[40:44].view(np.uint32)[0]); ng = int(c[44:48].view(np.uint32)[0])
     off_clen = (320 + 8 * (ng + 1) + 15) // 16 * 16
     v = c.copy(); v[off_clen] ^= 1; out["clen"] = v
-    v = c.copy(); v[off_clen + 2 * nc] = 1; out["padding"] = v
+    off_m = int(c[48:56].view(np.uint64)[0])
+    off_stream = (off_m + n + 15) // 16 * 16
+    pads = [b for b in range(320 + 8 * (ng + 1), off_clen)] + [b for b in range(off_clen + 2 * nc, off_m)] + \
+           [b for b in range(off_m + n, off_stream)]
+    assert pads, "test input must leave a padding byte"
+    v = c.copy(); v[pads[0]] = 1; out["padding"] = v
     v = c.copy(); v[-1] = 1; out["slack"] = v
     assert n > 0
     return out
 
 
 def test_malformed_containers_are_rejected():
-    w = inputs.gaussian(10_000, 0.02, seed=7)
+    w = inputs.gaussian(10_003, 0.02, seed=7)
     c = oracle.encode(w)
     assert np.array_equal(oracle.decode(c), w)
     for name, bad in _corrupt_variants(c).items():
