@@ -15,14 +15,20 @@
  *
  * Coding scheme (this library's reading; the pages leave it open):
  *   - every BF16 word w is split into its exponent e = (w >> 7) & 0xFF and the
- *     sign+mantissa byte m = ((w >> 8) & 0x80) | (w & 0x7F);
+ *     mantissa+sign byte m = ((w & 0x7F) << 1) | (w >> 15), the low byte of w
+ *     rotated left by one bit (so w is (e << 8 | m) rotated right by one);
  *   - the exponents are coded with a per-tensor canonical Huffman code whose
  *     lengths come from package-merge with a length limit (24 by default),
  *     leaves ordered by (count, symbol value), a leaf ahead of a package of
  *     equal weight, codes assigned in (length, symbol) order; a tensor with a
  *     single exponent value gets a second, never-used phantom symbol (1 if the
  *     value is 0, else 0) so both codes are 1 bit long;
- *   - the m bytes are stored raw.
+ *   - the m bytes are stored raw, in element order;
+ *   - the exponent codes are cut into chunks of K codes, 32 chunks to a group:
+ *     a group covers 32*K consecutive elements in 8-element blocks, block b of
+ *     the group belongs to chunk b mod 32, and a chunk's codes follow its
+ *     blocks in order; the chunks of the last group hold only elements below n
+ *     (possibly none).
  *
  * Container ("DFX1", all integers little-endian, every section starts on a
  * 16-byte boundary, every padding byte zero):
@@ -30,15 +36,15 @@
  *   off  8  u64 n                 BF16 elements
  *   off 16  u64 total_bits        code stream length in bits
  *   off 24  u64 total_bytes       container size
- *   off 32  u32 K                 symbols per chunk (one decoding thread)
+ *   off 32  u32 K                 symbols per chunk (one decoding thread), a multiple of 8
  *   off 36  u32 G                 chunks per group (one warp)
- *   off 40  u32 n_chunk = ceil(n / K);  off 44  u32 n_group = ceil(n_chunk / G)
+ *   off 40  u32 n_chunk = G * n_group;  off 44  u32 n_group = ceil(n / (G * K))
  *   off 48  u64 off_m             offset of the sign+mantissa plane
  *   off 56  u32 max_len;          off 60  u32 reserved = 0
  *   off 64  u8  len[256]          code length per exponent value, 0 = unused
  *   off 320 u64 gbase[n_group+1]  start bit of each group; last = total_bits
- *   then    u16 clen[n_chunk]     bit length of each chunk
- *   then    u8  m[n]              sign+mantissa bytes in element order
+ *   then    u16 clen[n_chunk]     bit length of each chunk (0 for an empty chunk)
+ *   then    u8  m[n]              mantissa+sign bytes in element order
  *   then    u32 stream[]          codes MSB-first: bit k of the stream is bit
  *                                 31 - (k mod 32) of word k / 32; the section
  *                                 is 4*ceil(total_bits/32) bytes rounded up
@@ -89,7 +95,7 @@ typedef struct CUstream_st *cudaStream_t;
 typedef struct dfx_plan_s *dfx_plan_t; /* opaque, host-owned */
 
 typedef struct {
-    uint32_t chunk_symbols; /* K: 32, 64 or 128 on the GPU path (0 -> 64) */
+    uint32_t chunk_symbols; /* K: a multiple of 8; 32, 64 or 128 on the GPU path (0 -> 64) */
     uint32_t group_chunks;  /* G: 32 on the GPU path (0 -> 32) */
     uint32_t max_len;       /* code-length limit, 8..24 (0 -> 24) */
 } dfx_params;

@@ -24,6 +24,7 @@ int resolve_params(const dfx_params* p, uint32_t* K, uint32_t* G, uint32_t* L) {
     *G = (p && p->group_chunks) ? p->group_chunks : 32u;
     *L = (p && p->max_len) ? p->max_len : 24u;
     if (*L < 8 || *L > dfx::kMaxLenLimit) return DFX_ERR_ARG;
+    if (*K < 8 || *K % 8 != 0) return DFX_ERR_ARG;  // chunks are made of 8-element blocks
     if ((uint64_t)(*K) * (*L) > 65535u) return DFX_ERR_ARG;  // a chunk's bit length must fit u16
     return DFX_OK;
 }

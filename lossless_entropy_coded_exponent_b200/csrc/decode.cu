@@ -2,27 +2,25 @@
 //
 // Design (B200-first; the pages' GPU decoder is prior art, "DFloat11: lossless LLM
 // compression for GPU", aikraft.ru blog, section 03):
-//   * persistent grid, 8 warps per CTA; each CTA first builds its decoding tables in
-//     shared memory from len[256]: a pair table on the next 14 bits that resolves two
+//   * persistent grid, one CTA of 32 warps per SM that first builds its tables in shared
+//     memory from len[256]: a pair table on the next 14 bits that resolves two
 //     codes at once when both fit, a one-code view of it, and, for codes longer than 14
 //     bits, the canonical per-length limits (the levels of the hierarchical table of
 //     section 03, item 1);
-//   * one warp decodes one group of 32 chunks; lane i owns chunk i of the group and
-//     decodes exactly K codes.  Its read position is the group's start bit plus the
-//     warp's exclusive scan of the chunk bit lengths (the "lightweight auxiliary
-//     variables" that coordinate read positions, section 03, item 2).  Output positions
-//     need no scan: chunk i writes elements [i*K, i*K + K) of the group;
+//   * one warp decodes one group of 32 chunks; lane i owns chunk i of the group: the
+//     group's 8-element blocks i, i+32, ...  Its read position is the group's start bit
+//     plus the warp's exclusive scan of the chunk bit lengths (the "lightweight
+//     auxiliary variables" that coordinate read positions, section 03, item 2).  Write
+//     positions need no scan: after every 8 codes the lane holds 8 consecutive outputs
+//     and the warp's 16-byte stores cover 512 contiguous bytes;
 //   * each lane keeps its bit position and a 32-bit peek of the stream; the peek is
 //     reloaded from the warp's shared-memory copy of the group's stream slice once per
 //     two pair lookups, so the common path has no per-code branch besides the rare
 //     unresolved-pair test;
 //   * the next group's stream slice is copied into shared memory (cp.async) and its
 //     index loaded while the current group decodes; the group's sign+mantissa bytes are
-//     prefetched into L2 when it starts;
-//   * decoded exponents go to a per-warp shared-memory stash laid out so that both the
-//     lane-per-chunk writes and the coalesced reads of the merge step are free of bank
-//     conflicts; the merge joins them with the sign+mantissa bytes and writes BF16 with
-//     16-byte stores, 512 contiguous bytes per warp instruction.
+//     prefetched into L2 when it starts and each block's are loaded a block ahead; the
+//     merge is a byte interleave and a 16-bit rotate.
 // Every read of the container is bounded by the header-checked section sizes; a bad
 // container sets bits of the status word and the kernel finishes normally.
 #include <cuda_runtime.h>
@@ -34,23 +32,13 @@ namespace dfx {
 namespace {
 
 constexpr int kLutBits = 14;
-// Warps per CTA: one CTA per SM holds the 64 KiB pair table once; K = 128 needs twice
-// the per-warp buffers, so it runs 16 warps to stay inside 227 KiB of shared memory.
+// Warps per CTA: one CTA per SM holds the 64 KiB pair table once.
 template <int K>
 struct DecodeShape {
-    static constexpr int kWarps = K == 128 ? 16 : 32;
+    static constexpr int kWarps = 32;
     static constexpr int kThreads = kWarps * 32;
 };
 constexpr unsigned kFull = 0xffffffffu;
-
-// Stash row stride (words): row q holds symbols 4q..4q+3 of every lane.  32 + 128/K
-// makes the merge step's reads (lane l reads rows 2a, 2a+1 of lane l/(K/8) ...) hit
-// 32 distinct banks for K = 32, 64, 128.
-template <int K>
-struct StashShape {
-    static constexpr int kStride = 32 + 128 / K;
-    static constexpr int kWords = (K / 4) * kStride;
-};
 
 // Pair table entry (u32), indexed by the next kLutBits stream bits:
 //   bits 0-7   first symbol        bits 8-15  second symbol
@@ -189,9 +177,10 @@ __device__ __noinline__ uint32_t decode_long(uint32_t peek, const Tables& T) {
 }
 
 
-// Two BF16 from x = [m0, e0, m1, e1] (bytes, low to high).
+// Two BF16 from x = [m0, e0, m1, e1] (bytes, low to high), m = mantissa * 2 + sign:
+// each 16-bit half (e << 8 | m) rotated right by one bit.
 __device__ __forceinline__ uint32_t bf16_pair(uint32_t x) {
-    return ((x >> 1) & 0x7F807F80u) | ((x << 8) & 0x80008000u) | (x & 0x007F007Fu);
+    return ((x >> 1) & 0x7FFF7FFFu) | ((x << 15) & 0x80008000u);
 }
 
 __device__ __forceinline__ uint4 merge8(uint2 m, uint32_t e0, uint32_t e1) {
@@ -272,11 +261,10 @@ struct ClampedGlobalWords {
     uint32_t maxw;  // last readable index
     __device__ __forceinline__ uint32_t load(uint32_t i) const { return __ldg(p + min(i, maxw)); }
 };
-constexpr uint32_t kSliceWords = 256;  // 1 KiB per staged group slice
 struct SharedWords {
     uint32_t s;  // shared-memory address of the slice buffer
     // Well-formed groups read inside the slice.  A corrupt one reads at most 3K/4 + 2
-    // words past its start, into the next buffers or the guard pad after the last warp's
+    // words past its start, into the next buffer or the guard pad after the last warp's
     // buffers: never outside the CTA's shared memory.
     __device__ __forceinline__ uint32_t load(uint32_t i) const {
         uint32_t v;
@@ -342,27 +330,28 @@ struct BitReader {
     __device__ __forceinline__ uint32_t consumed() const { return p - p0; }
 };
 
-// Decode the K codes of this lane's chunk into the stash.
-template <int K, class Words>
-__device__ __forceinline__ void decode_chunk(BitReader<Words>& br, const Tables& T, uint32_t* stash,
-                                             unsigned lane, uint32_t& err) {
-    constexpr int S = StashShape<K>::kStride;
-#pragma unroll 4
-    for (int q = 0; q < K / 4; q++) {
-        br.reload();
-        uint32_t acc = 0;
-        acc = br.template pair<0>(acc, T, err);
-        acc = br.template pair<1>(acc, T, err);
-        stash[q * S + lane] = acc;
-    }
+// Decode the 8 codes of one block: symbols 0-3 in e0, 4-7 in e1.
+template <class Words>
+__device__ __forceinline__ void decode_block(BitReader<Words>& br, const Tables& T, uint32_t& e0, uint32_t& e1,
+                                             uint32_t& err) {
+    br.reload();
+    e0 = br.template pair<1>(br.template pair<0>(0u, T, err), T, err);
+    br.reload();
+    e1 = br.template pair<1>(br.template pair<0>(0u, T, err), T, err);
 }
 
 // ---------------------------------------------------------------- per-warp buffers
 
+// Stream words staged per group: the slice of a K = 64 group averages ~0.7 KiB on
+// Gaussian weights; groups that do not fit decode from global memory.
+template <int K>
+struct SliceShape {
+    static constexpr uint32_t kWords = 4u * K;  // 1 KiB at K = 64
+};
+
 template <int K>
 struct WarpBuffers {
-    uint32_t stash[StashShape<K>::kWords];     // decoded exponents
-    __align__(16) uint32_t slice[2][kSliceWords];  // stream slices of this group and the next
+    __align__(16) uint32_t slice[2][SliceShape<K>::kWords];  // this group's stream words and the next's
 };
 
 template <int K>
@@ -390,13 +379,14 @@ struct Slice {
     bool staged;
 };
 
+template <uint32_t kWords>
 __device__ __forceinline__ Slice stage_slice(const DecodeArgs& a, const Tables& T, uint32_t* buf,
                                              unsigned long long gb0, uint32_t span, bool ok, unsigned lane) {
     Slice r;
     const uint32_t beg = ((uint32_t)(gb0 >> 5) * 4u) & ~15u;  // bytes into the stream section
     const uint32_t end = min((((uint32_t)((gb0 + span) >> 5) + 4u) * 4u + 15u) & ~15u, T.n_words * 4u);
     r.base = beg / 4u;
-    r.staged = ok && end > beg && end - beg <= kSliceWords * 4u;
+    r.staged = ok && end > beg && end - beg <= kWords * 4u;
     if (r.staged) {
         const uint8_t* src = a.comp + a.off_stream + beg;
         for (uint32_t c = lane; c < (end - beg) / 16u; c += 32) cp_async16(buf + 4 * c, src + 16 * c);
@@ -404,21 +394,40 @@ __device__ __forceinline__ Slice stage_slice(const DecodeArgs& a, const Tables& 
     return r;
 }
 
-// Full groups (all 32 chunks hold K codes), one warp at a time.  While group g decodes,
-// the stream slice of the warp's next group is copied into the other slice buffer and
-// the index of the group after that is loaded; the sign+mantissa bytes of g are
-// prefetched into L2 when g starts and read by the merge.
+// Decode one full group's 32 chunks (lane i: blocks i, i+32, ... of the group) and
+// write its BF16 output.  Each lane decodes 8 codes, then stores 8 outputs (16 bytes;
+// 512 contiguous bytes per warp store); the sign+mantissa bytes of the next block are
+// loaded while the current one decodes.
+template <int K, class Words>
+__device__ __forceinline__ void decode_group_blocks(const DecodeArgs& a, const Tables& T, BitReader<Words>& br,
+                                                    uint32_t g, unsigned lane, uint32_t& err) {
+    const uint2* mp = reinterpret_cast<const uint2*>(a.comp + a.off_m) + (uint64_t)g * (32u * K / 8u) + lane;
+    uint4* op = reinterpret_cast<uint4*>(a.out) + (uint64_t)g * (32u * K / 8u) + lane;
+    uint2 m_next = __ldg(mp);
+#pragma unroll 2
+    for (int k = 0; k < K / 8; k++) {
+        const uint2 m = m_next;
+        if (k + 1 < K / 8) m_next = __ldg(mp + 32 * (k + 1));
+        uint32_t e0, e1;
+        decode_block(br, T, e0, e1, err);
+        op[32 * k] = merge8(m, e0, e1);
+    }
+}
+
+// Full groups, one warp at a time.  While group g decodes, the stream slice of the
+// warp's next group is copied into the other slice buffer and the index of the group
+// after that is loaded; the sign+mantissa bytes of g are prefetched into L2 when g starts.
 template <int K>
 __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const uint32_t* lut, WarpBuffers<K>& wb,
                                    uint32_t g, uint32_t step, uint32_t n_full, unsigned lane, uint32_t& err) {
-    constexpr int S = StashShape<K>::kStride;
+    constexpr uint32_t kWords = SliceShape<K>::kWords;
     if (g >= n_full) return;
     const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
     const uint32_t maxw = T.n_words - 1;
     const uint8_t* mplane = a.comp + a.off_m;
 
     GroupStart st = scan_index(load_index(a, T, g, lane, true), lane);
-    Slice sl = stage_slice(a, T, wb.slice[0], st.gb0, st.span, st.ok, lane);
+    Slice sl = stage_slice<kWords>(a, T, wb.slice[0], st.gb0, st.span, st.ok, lane);
     cp_async_commit();
     uint32_t gn = g + step;
     GroupIndex idx_n;
@@ -434,7 +443,7 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
         GroupIndex idx_nn;
         if (has_next) {
             st_n = scan_index(idx_n, lane);
-            sl_n = stage_slice(a, T, wb.slice[b ^ 1], st_n.gb0, st_n.span, st_n.ok, lane);
+            sl_n = stage_slice<kWords>(a, T, wb.slice[b ^ 1], st_n.gb0, st_n.span, st_n.ok, lane);
             if (gnn < n_full) idx_nn = load_index(a, T, gnn, lane, true);
         }
         cp_async_commit();
@@ -447,7 +456,7 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
                 BitReader<SharedWords> br;
                 br.init(lut, SharedWords{(uint32_t)__cvta_generic_to_shared(wb.slice[b])},
                         (uint32_t)(st.start - 32ull * sl.base));
-                decode_chunk<K>(br, T, wb.stash, lane, err);
+                decode_group_blocks<K>(a, T, br, g, lane, err);
                 used = br.consumed();
             } else {
                 // A chunk reads at most 3K/4 + 2 words past its start (24-bit codes); lane 31
@@ -458,12 +467,12 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
                 if (last + (3u * K) / 4u + 8u <= maxw) {
                     BitReader<GlobalWords> br;
                     br.init(lut, GlobalWords{sw + first}, rel);
-                    decode_chunk<K>(br, T, wb.stash, lane, err);
+                    decode_group_blocks<K>(a, T, br, g, lane, err);
                     used = br.consumed();
                 } else {
                     BitReader<ClampedGlobalWords> br;
                     br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, rel);
-                    decode_chunk<K>(br, T, wb.stash, lane, err);
+                    decode_group_blocks<K>(a, T, br, g, lane, err);
                     used = br.consumed();
                 }
             }
@@ -471,18 +480,7 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
         } else {
             err |= DFX_STATUS_INDEX;
         }
-        __syncwarp();
-        if (st.ok) {
-            const uint2* mp = reinterpret_cast<const uint2*>(mplane) + (uint64_t)g * (32u * K / 8u) + lane;
-            uint4* out4 = reinterpret_cast<uint4*>(a.out) + (uint64_t)g * (32u * K / 8u) + lane;
-#pragma unroll
-            for (int r = 0; r < K / 8; r++) {
-                const int j0 = 8 * (int)lane + 256 * r;
-                const int t = j0 / K, q0 = (j0 % K) / 4;
-                out4[32 * r] = merge8(__ldg(mp + 32 * r), wb.stash[q0 * S + t], wb.stash[(q0 + 1) * S + t]);
-            }
-        }
-        __syncwarp();
+        __syncwarp();  // the slice buffer is reused by the copy issued next iteration
         if (!has_next) break;
         g = gn;
         gn = gnn;
@@ -494,56 +492,41 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
     cp_async_wait_all();
 }
 
-// The last group when it is ragged: chunks may be short or absent, outputs stop at n.
+// The last group when it is ragged: a lane's chunk holds the elements of its blocks
+// that are below n (a prefix of the chunk, possibly empty); outputs stop at n.
 template <int K>
-__device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, const uint32_t* lut, WarpBuffers<K>& wb,
-                                  uint64_t g,
+__device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, const uint32_t* lut, uint32_t g,
                                   unsigned lane, uint32_t& err) {
-    constexpr int S = StashShape<K>::kStride;
-    const uint64_t c = g * 32 + lane;
-    const bool has = c < a.n_chunk;
-    const uint32_t cnt = has ? (uint32_t)min((uint64_t)K, a.n - c * K) : 0u;
-    const GroupStart gs = scan_index(load_index(a, T, g, lane, has), lane);
+    const GroupStart gs = scan_index(load_index(a, T, g, lane, true), lane);
     if (!gs.ok) {
         err |= DFX_STATUS_INDEX;
         return;
     }
-    if (has) {
-        const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
-        const uint32_t maxw = T.n_words - 1;
-        const uint32_t first = (uint32_t)(gs.gb0 >> 5);
-        BitReader<ClampedGlobalWords> br;
-        br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, (uint32_t)(gs.start - 32ull * first));
-        for (int q = 0; q < K / 4; q++) {
-            br.reload();
-            uint32_t acc = 0;
-            for (int k = 0; k < 4; k++)
-                if ((uint32_t)(4 * q + k) < cnt) acc |= br.one(T, err) << (8 * k);
-            wb.stash[q * S + lane] = acc;
-        }
-        if (br.consumed() != gs.clen) err |= DFX_STATUS_STREAM;
-    }
-    __syncwarp();
-    const uint64_t gbase_elem = g * 32 * K;
+    const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
+    const uint32_t maxw = T.n_words - 1;
+    const uint32_t first = (uint32_t)(gs.gb0 >> 5);
     const uint8_t* mplane = a.comp + a.off_m;
-    for (int r = 0; r < K / 8; r++) {
-        const int j0 = 8 * (int)lane + 256 * r;
-        const uint64_t elem = gbase_elem + j0;
-        const int t = j0 / K, q0 = (j0 % K) / 4;
-        if (elem + 8 <= a.n) {
-            const uint2 m = __ldg(reinterpret_cast<const uint2*>(mplane + elem));
-            reinterpret_cast<uint4*>(a.out)[elem / 8] = merge8(m, wb.stash[q0 * S + t], wb.stash[(q0 + 1) * S + t]);
+    BitReader<ClampedGlobalWords> br;
+    br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, (uint32_t)(gs.start - 32ull * first));
+    br.reload();
+    for (uint32_t k = 0; k < K / 8; k++) {
+        const uint64_t x0 = block_element(g, K, k, lane);
+        if (x0 >= a.n) break;
+        const uint32_t cnt = (uint32_t)min((uint64_t)8, a.n - x0);
+        uint32_t e[2] = {0u, 0u};
+        for (uint32_t j = 0; j < cnt; j++) e[j >> 2] |= br.one(T, err) << (8 * (j & 3));
+        if (cnt == 8) {
+            reinterpret_cast<uint4*>(a.out)[x0 / 8] =
+                merge8(__ldg(reinterpret_cast<const uint2*>(mplane + x0)), e[0], e[1]);
         } else {
-            for (int i = 0; i < 8; i++) {
-                if (elem + i >= a.n) break;
-                const int k = (j0 + i) % K;
-                const uint32_t e = (wb.stash[(k / 4) * S + t] >> (8 * (k % 4))) & 0xFFu;
-                const uint32_t m = mplane[elem + i];
-                a.out[elem + i] = (uint16_t)(((m & 0x80u) << 8) | (e << 7) | (m & 0x7Fu));
+            for (uint32_t j = 0; j < cnt; j++) {
+                const uint32_t m = mplane[x0 + j];
+                const uint32_t ex = (e[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+                a.out[x0 + j] = (uint16_t)(((m & 1u) << 15) | (ex << 7) | (m >> 1));
             }
         }
     }
-    __syncwarp();
+    if (br.consumed() != gs.clen) err |= DFX_STATUS_STREAM;
 }
 
 constexpr size_t kLutBytes = sizeof(uint32_t) << kLutBits;
@@ -566,7 +549,7 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
     const uint32_t step = gridDim.x * kDecodeWarps;
     const uint32_t gw = blockIdx.x * kDecodeWarps + warp;
     decode_full_groups<K>(a, T, lut, wb, gw, step, n_full, lane, err);
-    if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, lut, wb, n_full, lane, err);
+    if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, lut, n_full, lane, err);
     if (err) atomicOr(a.status, err);
 }
 

@@ -28,12 +28,18 @@ __host__ __device__ inline Layout make_layout(uint64_t n, uint32_t K, uint32_t G
     L.n = n;
     L.K = K;
     L.G = G;
-    L.n_chunk = (n + K - 1) / K;
-    L.n_group = (L.n_chunk + G - 1) / G;
+    // a group holds G * K elements in 8-element blocks; block b belongs to chunk b mod G
+    L.n_group = (n + (uint64_t)G * K - 1) / ((uint64_t)G * K);
+    L.n_chunk = L.n_group * G;
     L.off_clen = align16(kOffGbase + 8 * (L.n_group + 1));
     L.off_m = align16(L.off_clen + 2 * L.n_chunk);
     L.off_stream = align16(L.off_m + n);
     return L;
+}
+
+// Element of the first entry of block k of chunk `lane` in group g (G = 32 chunks).
+__host__ __device__ inline uint64_t block_element(uint64_t g, uint32_t K, uint32_t k, uint32_t lane) {
+    return g * 32ull * K + (32ull * k + lane) * 8;
 }
 
 __host__ __device__ inline uint64_t stream_bytes(uint64_t total_bits) {

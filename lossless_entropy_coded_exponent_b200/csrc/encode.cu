@@ -5,12 +5,15 @@
 //   1. k_histogram      exponent histogram, warp-aggregated shared-memory atomics;
 //   2. k_build_codebook one CTA: package-merge code lengths (limit max_len), canonical codes,
 //                       len[256] and the constant header fields;
-//   3. k_chunk_bits     per chunk of K elements its code bits (clen), per group of 32 chunks
-//                       the sum;
+//   3. k_chunk_bits     per chunk its code bits (clen), per group of 32 chunks the sum;
+//                       a group's elements come in 8-element blocks, block b belongs to
+//                       chunk b mod 32, so lane i of a warp reads blocks i, i+32, ...
+//                       (16-byte loads, 512 contiguous bytes per warp instruction);
 //   4. k_group_scan     one CTA: exclusive scan of the group sums -> gbase, total_bits,
 //                       total_bytes;
 //   5. k_pack           per chunk: start bit from gbase + warp scan of clen, codes packed
-//                       MSB-first into 32-bit words, m bytes written.
+//                       MSB-first into 32-bit words in the same block order; the
+//                       mantissa+sign bytes (mantissa * 2 + sign) written in element order.
 // The method: frequent exponent values get short codes ("DFloat11: lossless LLM
 // compression for GPU", aikraft.ru blog, section 02); the exact code and layout rules
 // are the ones stated in include/dfx.h.
@@ -245,13 +248,15 @@ __global__ void __launch_bounds__(kChunkThreads) k_chunk_bits(EncodeArgs a) {
     const unsigned lane = threadIdx.x & 31;
     uint32_t bits = 0;
     if (c < a.n_chunk) {
-        const uint64_t i0 = c * K;
-        if (i0 + K <= a.n) {
-            const uint4* p = reinterpret_cast<const uint4*>(a.in + i0);
-#pragma unroll 4
-            for (int v = 0; v < K / 8; v++) bits += bits8(__ldg(p + v), lt);
-        } else {
-            for (uint64_t i = i0; i < a.n; i++) bits += lt[(a.in[i] >> 7) & 0xFFu];
+        const uint64_t g = c / 32;
+        for (uint32_t k = 0; k < K / 8; k++) {
+            const uint64_t x0 = block_element(g, K, k, lane);
+            if (x0 + 8 <= a.n) {
+                bits += bits8(__ldg(reinterpret_cast<const uint4*>(a.in + x0)), lt);
+            } else {
+                for (uint64_t x = x0; x < a.n; x++) bits += lt[(a.in[x] >> 7) & 0xFFu];
+                break;
+            }
         }
         reinterpret_cast<uint16_t*>(a.out + a.off_clen)[c] = (uint16_t)bits;
     }
@@ -363,29 +368,28 @@ __global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
     bw.first = true;
     uint8_t* mpl = a.out + a.off_m;
 
-    const uint64_t i0 = c * K;
-    if (i0 + K <= a.n) {
-        const uint4* p = reinterpret_cast<const uint4*>(a.in + i0);
-        for (int v = 0; v < K / 8; v++) {
-            const uint4 x = __ldg(p + v);
-            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    for (uint32_t k = 0; k < K / 8; k++) {
+        const uint64_t x0 = block_element(c / 32, K, k, lane);
+        if (x0 + 8 <= a.n) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.in + x0));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             uint32_t mb[2] = {0u, 0u};
 #pragma unroll
-            for (int k = 0; k < 8; k++) {
-                const uint32_t h = (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+            for (int j = 0; j < 8; j++) {
+                const uint32_t h = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
                 const uint32_t e = (h >> 7) & 0xFFu;
-                const uint32_t m = ((h >> 8) & 0x80u) | (h & 0x7Fu);
                 bw.put(code_sh[e], len_sh[e]);
-                mb[k >> 2] |= m << (8 * (k & 3));
+                mb[j >> 2] |= (((h & 0x7Fu) << 1) | (h >> 15)) << (8 * (j & 3));
             }
-            *reinterpret_cast<uint2*>(mpl + i0 + 8 * v) = make_uint2(mb[0], mb[1]);
-        }
-    } else {
-        for (uint64_t i = i0; i < a.n; i++) {
-            const uint32_t h = a.in[i];
-            const uint32_t e = (h >> 7) & 0xFFu;
-            bw.put(code_sh[e], len_sh[e]);
-            mpl[i] = (uint8_t)(((h >> 8) & 0x80u) | (h & 0x7Fu));
+            *reinterpret_cast<uint2*>(mpl + x0) = make_uint2(mb[0], mb[1]);
+        } else {
+            for (uint64_t x = x0; x < a.n; x++) {
+                const uint32_t h = a.in[x];
+                const uint32_t e = (h >> 7) & 0xFFu;
+                bw.put(code_sh[e], len_sh[e]);
+                mpl[x] = (uint8_t)(((h & 0x7Fu) << 1) | (h >> 15));
+            }
+            break;
         }
     }
     bw.finish();

@@ -51,7 +51,7 @@ extern "C" int dfx_encode_static(const void* d_bf16, uint64_t n, const dfx_param
     const uint32_t K = (params && params->chunk_symbols) ? params->chunk_symbols : 64u;
     const uint32_t G = (params && params->group_chunks) ? params->group_chunks : 32u;
     const uint32_t L = (params && params->max_len) ? params->max_len : 24u;
-    if (L < 8 || L > dfx::kMaxLenLimit) return DFX_ERR_ARG;
+    if (L < 8 || L > dfx::kMaxLenLimit || K < 8 || K % 8 != 0) return DFX_ERR_ARG;
     if (!dfx::decode_supports(K, G)) return DFX_ERR_UNSUPPORTED;
     if (!d_out || (!d_bf16 && n)) return DFX_ERR_ARG;
     if (((uintptr_t)d_bf16 & 15u) || ((uintptr_t)d_out & 15u)) return DFX_ERR_ARG;

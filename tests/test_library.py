@@ -46,7 +46,7 @@ def test_layout_agrees_with_oracle(lib, n, K):
     for total_bits in (0, 1, 31, 32, 33, 8 * n):
         lay = dfx.dfx_container_layout(n, total_bits, chunk_symbols=K)
         assert lay["total_bytes"] == oracle.container_bytes(n, K, 32, total_bits)
-        assert lay["n_chunk"] == -(-n // K) and lay["n_group"] == -(-lay["n_chunk"] // 32)
+        assert lay["n_group"] == -(-n // (32 * K)) and lay["n_chunk"] == 32 * lay["n_group"]
         for key in ("off_clen", "off_m", "off_stream"):
             assert lay[key] % 16 == 0
     assert dfx.dfx_container_layout(n, 8 * n, chunk_symbols=K)["total_bytes"] == oracle.max_container_bytes(n, K, 32)
@@ -76,6 +76,9 @@ def test_host_argument_errors_precede_cuda(lib):
     assert e.value.code == dfx.DFX_ERR_UNSUPPORTED
     with pytest.raises(dfx.DfxError) as e:
         dfx.dfx_container_layout(10, 0, chunk_symbols=4000)
+    assert e.value.code == dfx.DFX_ERR_ARG
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_container_layout(10, 0, chunk_symbols=60)  # not a multiple of 8
     assert e.value.code == dfx.DFX_ERR_ARG
 
 
