@@ -14,9 +14,11 @@
  * position variables (the same blog, section 03, items 1 and 2).
  *
  * Coding scheme (this library's reading; the pages leave it open):
- *   - every BF16 word w is split into its exponent e = (w >> 7) & 0xFF and the
- *     mantissa+sign byte m = ((w & 0x7F) << 1) | (w >> 15), the low byte of w
- *     rotated left by one bit (so w is (e << 8 | m) rotated right by one);
+ *   - every BF16 word w[x] is split into its exponent e = (w[x] >> 7) & 0xFF and
+ *     the mantissa+sign byte m[x] = ((w[x] & 0x7F) << 1) | (w[p] >> 15): its
+ *     mantissa above the sign of its partner p = x ^ 1 (p = x when x ^ 1 >= n).
+ *     For a pair (2i, 2i+1) the 32-bit word m[2i] | e[2i] << 8 | m[2i+1] << 16 |
+ *     e[2i+1] << 24 rotated right by one bit is the two BF16 words;
  *   - the exponents are coded with a per-tensor canonical Huffman code whose
  *     lengths come from package-merge with a length limit (24 by default),
  *     leaves ordered by (count, symbol value), a leaf ahead of a package of
@@ -44,7 +46,7 @@
  *   off 64  u8  len[256]          code length per exponent value, 0 = unused
  *   off 320 u64 gbase[n_group+1]  start bit of each group; last = total_bits
  *   then    u16 clen[n_chunk]     bit length of each chunk (0 for an empty chunk)
- *   then    u8  m[n]              mantissa+sign bytes in element order
+ *   then    u8  m[n]              mantissa+sign bytes in element order (above)
  *   then    u32 stream[]          codes MSB-first: bit k of the stream is bit
  *                                 31 - (k mod 32) of word k / 32; the section
  *                                 is 4*ceil(total_bits/32) bytes rounded up

@@ -19,8 +19,9 @@
 //     unresolved-pair test;
 //   * the next group's stream slice is copied into shared memory (cp.async) and its
 //     index loaded while the current group decodes; the group's sign+mantissa bytes are
-//     prefetched into L2 when it starts and each block's are loaded a block ahead; the
-//     merge is a byte interleave and a 16-bit rotate.
+//     prefetched into L2 when it starts and each block's are loaded a block ahead; each pair
+//     lookup is merged at once: one byte permute of the table entry with the m word and
+//     one 32-bit rotate give two BF16 (the m bytes of a pair carry each other's sign).
 // Every read of the container is bounded by the header-checked section sizes; a bad
 // container sets bits of the status word and the kernel finishes normally.
 #include <cuda_runtime.h>
@@ -55,6 +56,7 @@ struct Tables {
     uint32_t nlen[kMaxLenLimit + 1];
     uint8_t sorted[256];                      // used symbols in (length, symbol) order
     uint8_t lens[256];
+    uint8_t wcount[8][kMaxLenLimit + 1];      // symbols of each length among 32-symbol slices
     unsigned long long total_bits;
     uint32_t n_words;                         // 32-bit words of the stream section
     uint32_t bad;
@@ -96,9 +98,10 @@ __device__ bool build_tables(const DecodeArgs& a, Tables& T, uint32_t* lut, uint
         if (t == 0) atomicOr(a.status, T.bad);
         return false;
     }
-    for (int s = t; s < 256; s += blockDim.x) {
-        const uint32_t l = a.comp[kOffLen + s];
-        T.lens[s] = (uint8_t)l;
+    if (t < 8 * (int)(kMaxLenLimit + 1)) (&T.wcount[0][0])[t] = 0;
+    if (t < 256) {
+        const uint32_t l = a.comp[kOffLen + t];
+        T.lens[t] = (uint8_t)l;
         if (l > kMaxLenLimit) atomicOr(&T.bad, DFX_STATUS_TABLE);
         else if (l) atomicAdd(&T.nlen[l], 1u);
     }
@@ -121,28 +124,43 @@ __device__ bool build_tables(const DecodeArgs& a, Tables& T, uint32_t* lut, uint
         if (t == 0) atomicOr(a.status, T.bad);
         return false;
     }
-    for (int s = t; s < 256; s += blockDim.x) {
-        const uint32_t l = T.lens[s];
-        if (l) {
-            uint32_t r = 0;
-            for (int s2 = 0; s2 < s; s2++) r += (T.lens[s2] == l);
-            T.sorted[T.index[l] + r] = (uint8_t)s;
-        }
+    // rank of each used symbol among the symbols of its length (warps 0-7 hold symbols
+    // 0-255, one per lane): lower lanes of the same warp, then the counts of lower warps
+    const unsigned warp = t >> 5, lane = t & 31;
+    uint32_t l_t = 0, within = 0;
+    if (t < 256) {
+        l_t = T.lens[t];
+        const unsigned peers = __match_any_sync(kFull, l_t);
+        const unsigned below = peers & ((1u << lane) - 1u);
+        within = __popc(below);
+        if (l_t && below == 0) T.wcount[warp][l_t] = (uint8_t)__popc(peers);
+    }
+    // meanwhile zero the one-code table (32-bit words: the scratch is 16-byte aligned)
+    for (int i = t; i < (1 << kLutBits) / 2; i += blockDim.x) reinterpret_cast<uint32_t*>(scratch)[i] = 0u;
+    __syncthreads();
+    if (t < 256 && l_t) {
+        uint32_t r = within;
+        for (unsigned w = 0; w < warp; w++) r += T.wcount[w][l_t];
+        T.sorted[T.index[l_t] + r] = (uint8_t)t;
     }
     __syncthreads();
     // one-code table: (len << 8) | symbol for the code the next kLutBits bits start with,
-    // 0 when that code is longer; the length is the smallest l whose limit exceeds the bits
-    for (int e = t; e < (1 << kLutBits); e += blockDim.x) {
-        const uint32_t v = (uint32_t)e << (kMaxLenLimit - kLutBits);
-        int lo = 1, hi = kLutBits + 1;  // limit[] is non-decreasing in l
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (v < T.limit[mid]) hi = mid;
-            else lo = mid + 1;
+    // 0 (left from the zeroing) where they start a longer code.  Symbol i in (length,
+    // symbol) order has the canonical code c = first[l] + i - index[l], which owns the
+    // entries [c, c + 1) << (kLutBits - l); one warp fills one symbol's entries.
+    for (uint32_t i = warp; i < T.index[kLutBits + 1]; i += blockDim.x >> 5) {
+        uint32_t l = 1;
+        while (T.index[l + 1] <= i) l++;
+        const uint32_t shift = kLutBits - l;
+        const uint32_t lo = (T.first[l] + (i - T.index[l])) << shift;
+        const uint32_t v = (l << 8) | T.sorted[i];
+        if (shift >= 3) {  // 8-entry runs, 16-byte aligned
+            const uint32_t w2 = v | (v << 16);
+            uint4* d = reinterpret_cast<uint4*>(scratch + lo);
+            for (uint32_t j = lane; j < (1u << (shift - 3)); j += 32) d[j] = make_uint4(w2, w2, w2, w2);
+        } else if (lane < (1u << shift)) {
+            scratch[lo + lane] = (uint16_t)v;
         }
-        scratch[e] = lo <= kLutBits
-                         ? (uint16_t)((lo << 8) | T.sorted[T.index[lo] + (v >> (kMaxLenLimit - lo)) - T.first[lo]])
-                         : (uint16_t)0;
     }
     __syncthreads();
     // pair table: the second code is read from the kLutBits - l0 bits left after the
@@ -177,11 +195,11 @@ __device__ __noinline__ uint32_t decode_long(uint32_t peek, const Tables& T) {
 }
 
 
-// Two BF16 from x = [m0, e0, m1, e1] (bytes, low to high), m = mantissa * 2 + sign:
-// each 16-bit half (e << 8 | m) rotated right by one bit.
-__device__ __forceinline__ uint32_t bf16_pair(uint32_t x) {
-    return ((x >> 1) & 0x7FFF7FFFu) | ((x << 15) & 0x80008000u);
-}
+// Two BF16 from x = [m0, e0, m1, e1] (bytes, low to high), where the m byte of each
+// element is its mantissa above its partner's sign: rotating x right by one bit puts
+// both mantissas and exponents in place and moves each partner's sign bit to the top
+// of the other half.
+__device__ __forceinline__ uint32_t bf16_pair(uint32_t x) { return __funnelshift_r(x, x, 1); }
 
 __device__ __forceinline__ uint4 merge8(uint2 m, uint32_t e0, uint32_t e1) {
     uint4 o;
@@ -243,12 +261,18 @@ __device__ __forceinline__ GroupStart scan_index(const GroupIndex& x, unsigned l
 // ---------------------------------------------------------------- bit reader
 //
 // A lane's state is its bit position p, relative to the first word of its word source,
-// and `peek`, the 32 stream bits starting at p.  Once per round of two pairs, peek is
-// reloaded from the two words holding bit p (two loads and one funnel shift).  Every
+// `peek`, the 32 stream bits starting at p, and the two words cur, nxt that hold them
+// (word cw and cw + 1).  Once per round of two pairs, peek is rebuilt from cur and nxt
+// with one funnel shift; only when p has moved into the next word does the lane shift
+// its words along and load one new word.  No reload follows more than 32 consumed bits
+// (two table pairs take at most 28, a single code at most 24), so p moves at most one
+// word between reloads, and about one lane in three loads a word per round.  Every
 // pair the table resolves consumes at most kLutBits = 14 bits, so after the first pair
 // of a round at least 18 valid bits remain for the second.  Pairs the table cannot
 // resolve (the second code does not fit the index bits, or the first code is longer)
-// take a rare branch that reloads and decodes code by code.
+// take a rare branch: it reloads after the first code and, when both codes are at most
+// kLutBits long, reads the second from the table entry at the new position; otherwise
+// it decodes code by code with the canonical limits.
 //
 // Word sources: the global stream (with or without a bound clamp) or a warp's
 // shared-memory copy of its group's slice of the stream.
@@ -278,15 +302,24 @@ struct BitReader {
     const uint32_t* lut;  // pair table in shared memory
     Words words;
     uint32_t p, p0, peek;
+    uint32_t cw, cur, nxt;  // cur = word cw, nxt = word cw + 1
 
     __device__ __forceinline__ void init(const uint32_t* table, const Words& w, uint32_t start) {
         lut = table;
         words = w;
         p = p0 = start;
+        cw = start >> 5;
+        cur = words.load(cw);
+        nxt = words.load(cw + 1);
     }
     __device__ __forceinline__ void reload() {
         const uint32_t wi = p >> 5;
-        peek = __funnelshift_l(words.load(wi + 1), words.load(wi), p);  // shift uses p & 31
+        if (wi != cw) {  // wi == cw + 1
+            cw = wi;
+            cur = nxt;
+            nxt = words.load(wi + 1);
+        }
+        peek = __funnelshift_l(nxt, cur, p);  // shift uses p & 31
     }
     // One code, the general way (peek must be current): returns its symbol.
     __device__ __forceinline__ uint32_t one(const Tables& T, uint32_t& err) {
@@ -308,36 +341,48 @@ struct BitReader {
         reload();
         return sym;
     }
-    // Two codes: returns acc with their symbols in bytes 2j and 2j+1.
+    // Two codes, merged with their m bytes (bytes 2j and 2j+1 of mw): two BF16.
     template <int j>
-    __device__ __forceinline__ uint32_t pair(uint32_t acc, const Tables& T, uint32_t& err) {
-        constexpr uint32_t sel = j == 0 ? 0x3254u : 0x5410u;
+    __device__ __forceinline__ uint32_t pair(uint32_t mw, const Tables& T, uint32_t& err) {
+        constexpr uint32_t sel = j == 0 ? 0x5140u : 0x5342u;  // [mw.2j, sym0, mw.2j+1, sym1]
         const uint32_t e = lut[peek >> (32 - kLutBits)];
         const uint32_t len = e >> 26;           // bit 5 is set when the entry is not a pair
         peek = __funnelshift_l(0u, peek, len);  // shifts by len & 31
         p += len;
-        acc = __byte_perm(acc, e, sel);
+        uint32_t syms = e;
         if ((int32_t)e < 0) {
             p -= 32;  // undo bit 5 of `len`
             reload();
-            uint32_t s0 = e & 0xFFu;
-            if ((e & 0x001F0000u) == 0) s0 = one(T, err);
-            const uint32_t s1 = one(T, err);
-            acc = __byte_perm(acc, s0 | (s1 << 8), sel);
+            // usually both codes fit the table on their own: the second one is the first
+            // code of the entry at the new position, and peek keeps at least 18 valid bits
+            const uint32_t e2 = lut[peek >> (32 - kLutBits)];
+            if ((e & 0x001F0000u) && (e2 & 0x001F0000u)) {
+                const uint32_t l1 = (e2 >> 16) & 31u;
+                p += l1;
+                peek = __funnelshift_l(0u, peek, l1);
+                syms = (e & 0xFFu) | ((e2 & 0xFFu) << 8);
+            } else {
+                uint32_t s0 = e & 0xFFu;
+                if ((e & 0x001F0000u) == 0) s0 = one(T, err);
+                syms = s0 | (one(T, err) << 8);
+            }
         }
-        return acc;
+        return bf16_pair(__byte_perm(mw, syms, sel));
     }
     __device__ __forceinline__ uint32_t consumed() const { return p - p0; }
 };
 
-// Decode the 8 codes of one block: symbols 0-3 in e0, 4-7 in e1.
+// Decode the 8 codes of one block and merge them with the block's m bytes: 8 BF16.
 template <class Words>
-__device__ __forceinline__ void decode_block(BitReader<Words>& br, const Tables& T, uint32_t& e0, uint32_t& e1,
-                                             uint32_t& err) {
+__device__ __forceinline__ uint4 decode_block(BitReader<Words>& br, const Tables& T, uint2 m, uint32_t& err) {
+    uint4 o;
     br.reload();
-    e0 = br.template pair<1>(br.template pair<0>(0u, T, err), T, err);
+    o.x = br.template pair<0>(m.x, T, err);
+    o.y = br.template pair<1>(m.x, T, err);
     br.reload();
-    e1 = br.template pair<1>(br.template pair<0>(0u, T, err), T, err);
+    o.z = br.template pair<0>(m.y, T, err);
+    o.w = br.template pair<1>(m.y, T, err);
+    return o;
 }
 
 // ---------------------------------------------------------------- per-warp buffers
@@ -397,7 +442,8 @@ __device__ __forceinline__ Slice stage_slice(const DecodeArgs& a, const Tables& 
 // Decode one full group's 32 chunks (lane i: blocks i, i+32, ... of the group) and
 // write its BF16 output.  Each lane decodes 8 codes, then stores 8 outputs (16 bytes;
 // 512 contiguous bytes per warp store); the sign+mantissa bytes of the next block are
-// loaded while the current one decodes.
+// loaded while the current one decodes (the group's m plane is prefetched into L2 when
+// the group starts).
 template <int K, class Words>
 __device__ __forceinline__ void decode_group_blocks(const DecodeArgs& a, const Tables& T, BitReader<Words>& br,
                                                     uint32_t g, unsigned lane, uint32_t& err) {
@@ -408,15 +454,13 @@ __device__ __forceinline__ void decode_group_blocks(const DecodeArgs& a, const T
     for (int k = 0; k < K / 8; k++) {
         const uint2 m = m_next;
         if (k + 1 < K / 8) m_next = __ldg(mp + 32 * (k + 1));
-        uint32_t e0, e1;
-        decode_block(br, T, e0, e1, err);
-        op[32 * k] = merge8(m, e0, e1);
+        op[32 * k] = decode_block(br, T, m, err);
     }
 }
 
 // Full groups, one warp at a time.  While group g decodes, the stream slice of the
 // warp's next group is copied into the other slice buffer and the index of the group
-// after that is loaded; the sign+mantissa bytes of g are prefetched into L2 when g starts.
+// after that is loaded; the group's m plane is prefetched into L2 when the group starts.
 template <int K>
 __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const uint32_t* lut, WarpBuffers<K>& wb,
                                    uint32_t g, uint32_t step, uint32_t n_full, unsigned lane, uint32_t& err) {
@@ -520,9 +564,9 @@ __device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, const ui
                 merge8(__ldg(reinterpret_cast<const uint2*>(mplane + x0)), e[0], e[1]);
         } else {
             for (uint32_t j = 0; j < cnt; j++) {
-                const uint32_t m = mplane[x0 + j];
+                const uint64_t x = x0 + j, partner = (x ^ 1u) < a.n ? (x ^ 1u) : x;
                 const uint32_t ex = (e[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-                a.out[x0 + j] = (uint16_t)(((m & 1u) << 15) | (ex << 7) | (m >> 1));
+                a.out[x] = (uint16_t)(((mplane[partner] & 1u) << 15) | (ex << 7) | (mplane[x] >> 1u));
             }
         }
     }
@@ -560,6 +604,8 @@ constexpr size_t dyn_smem_bytes() {
     return kLutBytes + DecodeShape<K>::kWarps * warp_buffer_bytes<K>() + kGuardBytes;
 }
 static_assert(kGuardBytes >= 4 * (3 * 128 / 4 + 8), "guard covers the longest run past a slice");
+static_assert(DecodeShape<32>::kThreads >= 256 && DecodeShape<64>::kThreads >= 256 && DecodeShape<128>::kThreads >= 256,
+              "the table build gives each of the 256 symbols its own thread");
 static_assert(DecodeShape<32>::kWarps * warp_buffer_bytes<32>() >= (2u << kLutBits), "scratch for the one-code table");
 static_assert(DecodeShape<128>::kWarps * warp_buffer_bytes<128>() >= (2u << kLutBits), "scratch for the one-code table");
 static_assert(dyn_smem_bytes<64>() + 1024 <= 227 * 1024 && dyn_smem_bytes<128>() + 1024 <= 227 * 1024, "shared memory");

@@ -13,7 +13,8 @@
 //                       total_bytes;
 //   5. k_pack           per chunk: start bit from gbase + warp scan of clen, codes packed
 //                       MSB-first into 32-bit words in the same block order; the
-//                       mantissa+sign bytes (mantissa * 2 + sign) written in element order.
+//                       mantissa+sign bytes (mantissa * 2 + the sign of the pair partner,
+//                       element x ^ 1) written in element order.
 // The method: frequent exponent values get short codes ("DFloat11: lossless LLM
 // compression for GPU", aikraft.ru blog, section 02); the exact code and layout rules
 // are the ones stated in include/dfx.h.
@@ -377,17 +378,19 @@ __global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
 #pragma unroll
             for (int j = 0; j < 8; j++) {
                 const uint32_t h = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+                const uint32_t partner = (w[j >> 1] >> (16 * ((j & 1) ^ 1))) & 0xFFFFu;  // element j ^ 1
                 const uint32_t e = (h >> 7) & 0xFFu;
                 bw.put(code_sh[e], len_sh[e]);
-                mb[j >> 2] |= (((h & 0x7Fu) << 1) | (h >> 15)) << (8 * (j & 3));
+                mb[j >> 2] |= (((h & 0x7Fu) << 1) | (partner >> 15)) << (8 * (j & 3));
             }
             *reinterpret_cast<uint2*>(mpl + x0) = make_uint2(mb[0], mb[1]);
         } else {
             for (uint64_t x = x0; x < a.n; x++) {
                 const uint32_t h = a.in[x];
+                const uint32_t partner = a.in[(x ^ 1u) < a.n ? (x ^ 1u) : x];
                 const uint32_t e = (h >> 7) & 0xFFu;
                 bw.put(code_sh[e], len_sh[e]);
-                mpl[x] = (uint8_t)(((h & 0x7Fu) << 1) | (h >> 15));
+                mpl[x] = (uint8_t)(((h & 0x7Fu) << 1) | (partner >> 15));
             }
             break;
         }

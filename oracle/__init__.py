@@ -52,9 +52,11 @@ def lib() -> ctypes.CDLL:
         u64p = ctypes.POINTER(ctypes.c_uint64)
         L.dfxo_exponent.argtypes = [ctypes.c_uint16]
         L.dfxo_exponent.restype = ctypes.c_uint8
-        L.dfxo_sign_mantissa.argtypes = [ctypes.c_uint16]
+        L.dfxo_partner.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+        L.dfxo_partner.restype = ctypes.c_uint64
+        L.dfxo_sign_mantissa.argtypes = [ctypes.c_uint16, ctypes.c_uint16]
         L.dfxo_sign_mantissa.restype = ctypes.c_uint8
-        L.dfxo_merge.argtypes = [ctypes.c_uint8, ctypes.c_uint8]
+        L.dfxo_merge.argtypes = [ctypes.c_uint8, ctypes.c_uint8, ctypes.c_uint8]
         L.dfxo_merge.restype = ctypes.c_uint16
         L.dfxo_histogram.argtypes = [u16p, ctypes.c_uint64, u64p]
         L.dfxo_code_lengths.argtypes = [u64p, ctypes.c_uint32, u8p]
@@ -80,12 +82,16 @@ def exponent(w: int) -> int:
     return int(lib().dfxo_exponent(w))
 
 
-def sign_mantissa(w: int) -> int:
-    return int(lib().dfxo_sign_mantissa(w))
+def partner(x: int, n: int) -> int:
+    return int(lib().dfxo_partner(x, n))
 
 
-def merge(e: int, m: int) -> int:
-    return int(lib().dfxo_merge(e, m))
+def sign_mantissa(w: int, partner_w: int) -> int:
+    return int(lib().dfxo_sign_mantissa(w, partner_w))
+
+
+def merge(e: int, m: int, m_partner: int) -> int:
+    return int(lib().dfxo_merge(e, m, m_partner))
 
 
 def histogram(w: np.ndarray) -> np.ndarray:

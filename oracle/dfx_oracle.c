@@ -18,7 +18,10 @@
  * The pages leave the concrete code open.  This codec's reading, written out
  * step by step below, is:
  *   1. split every BF16 word into its 8-bit exponent and an 8-bit
- *      mantissa+sign byte (the low byte of the word rotated left by one);
+ *      mantissa+sign byte: the 7 mantissa bits above one sign bit.  Elements
+ *      2i and 2i+1 are partners and each byte carries its partner's sign (the
+ *      last element of an odd-length tensor has none and keeps its own), so
+ *      that a decoder rebuilds two weights with one 32-bit rotate;
  *   2. histogram the exponents;
  *   3. length-limited (max_len, default 24) Huffman code lengths by
  *      package-merge, ties broken by symbol value;
@@ -53,7 +56,9 @@
  *   320 u64 gbase[n_group + 1]  start bit of each group, gbase[n_group] = total_bits
  *   .   u16 clen[n_chunk]       bit length of each chunk (0 for a chunk of the
  *                               last group that has no element)
- *   .   u8  m[n]                mantissa+sign bytes, element order
+ *   .   u8  m[n]                mantissa+sign bytes, element order:
+ *                               m[x] = mantissa(x) * 2 + sign(partner(x)),
+ *                               partner(x) = x ^ 1 if that is < n, else x
  *   .   u32 stream[...]         codes, bit k of the stream = bit (31 - k % 32)
  *                               of word k / 32; 4*ceil(total_bits/32) bytes
  *                               rounded up to 16, then 16 zero bytes of slack
@@ -92,12 +97,17 @@ static uint64_t align16(uint64_t x) { return (x + 15u) & ~(uint64_t)15u; }
 
 /* ------------------------------------------------------------------ */
 /* Step 1: the split.  BF16 = sign(1) | exponent(8) | mantissa(7).  The other
- * byte holds the mantissa above the sign: mantissa * 2 + sign.            */
+ * byte of element x holds x's mantissa above its partner's sign:
+ * mantissa(x) * 2 + sign(partner(x)).                                     */
 
 uint8_t dfxo_exponent(uint16_t w) { return (uint8_t)((w >> 7) & 0xFF); }
-uint8_t dfxo_sign_mantissa(uint16_t w) { return (uint8_t)(((w & 0x7F) << 1) | (w >> 15)); }
-uint16_t dfxo_merge(uint8_t e, uint8_t m) {
-    return (uint16_t)(((uint16_t)(m & 1) << 15) | ((uint16_t)e << 7) | (m >> 1));
+uint64_t dfxo_partner(uint64_t x, uint64_t n) { return (x ^ 1u) < n ? (x ^ 1u) : x; }
+uint8_t dfxo_sign_mantissa(uint16_t w, uint16_t partner) {
+    return (uint8_t)(((w & 0x7F) << 1) | (partner >> 15));
+}
+/* e: x's exponent; m: x's byte; m_partner: the byte of x's partner */
+uint16_t dfxo_merge(uint8_t e, uint8_t m, uint8_t m_partner) {
+    return (uint16_t)(((uint16_t)(m_partner & 1) << 15) | ((uint16_t)e << 7) | (m >> 1));
 }
 
 /* ------------------------------------------------------------------ */
@@ -340,7 +350,7 @@ int dfxo_encode(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t 
         }
     }
     put_u64(gbase + 8 * ng, pos);
-    for (uint64_t i = 0; i < n; i++) mplane[i] = dfxo_sign_mantissa(w[i]);
+    for (uint64_t i = 0; i < n; i++) mplane[i] = dfxo_sign_mantissa(w[i], w[dfxo_partner(i, n)]);
     return DFXO_OK;
 }
 
@@ -441,7 +451,7 @@ int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, u
                     }
                 }
                 if (found < 0) return DFXO_ERR_CORRUPT;
-                w[x] = dfxo_merge((uint8_t)found, mplane[x]);
+                w[x] = dfxo_merge((uint8_t)found, mplane[x], mplane[dfxo_partner(x, n)]);
             }
             if (get_u16(clen + 2 * (g * G + lane)) != pos - chunk_start) return DFXO_ERR_CORRUPT;
         }

@@ -133,10 +133,15 @@ def load_tie_rules():
 # ---------------------------------------------------------------- the split
 
 def test_split_matches_ieee_fields_for_every_pattern():
+    # every pattern, each with a partner drawn from the patterns (a seeded
+    # permutation): the byte is the pattern's mantissa above the partner's sign
     w = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    q = w[np.random.default_rng(5).permutation(w.size)]
     x = (w.astype(np.uint32) << 16).view(np.float32)
+    xq = (q.astype(np.uint32) << 16).view(np.float32)
     e_or = np.array([oracle.exponent(int(v)) for v in w], dtype=np.int64)
-    m_or = np.array([oracle.sign_mantissa(int(v)) for v in w], dtype=np.int64)
+    m_or = np.array([oracle.sign_mantissa(int(v), int(u)) for v, u in zip(w, q)], dtype=np.int64)
+    mq_or = np.array([oracle.sign_mantissa(int(u), int(v)) for v, u in zip(w, q)], dtype=np.int64)
     with np.errstate(all="ignore"):
         finite = np.isfinite(x)
         a = np.abs(x.astype(np.float64))
@@ -148,14 +153,21 @@ def test_split_matches_ieee_fields_for_every_pattern():
     mant = np.zeros_like(exp_e)
     mant = np.where(normal, np.rint((frac * 2 - 1) * 128), mant)
     mant = np.where(sub, np.rint(a / 2.0 ** -133), mant).astype(np.int64)
-    sign = np.signbit(x).astype(np.int64)
+    sign_q = np.signbit(xq).astype(np.int64)
     nan = np.isnan(x)
     assert np.array_equal(e_or, exp_e)
     ok = ~nan
-    assert np.array_equal(m_or[ok], (mant[ok] << 1) | sign[ok])
-    assert np.all((m_or[nan] >> 1) != 0) and np.array_equal(m_or[nan] & 1, sign[nan])
-    back = np.array([oracle.merge(int(e), int(m)) for e, m in zip(e_or, m_or)], dtype=np.uint16)
+    assert np.array_equal(m_or[ok], (mant[ok] << 1) | sign_q[ok])
+    assert np.all((m_or[nan] >> 1) != 0) and np.array_equal(m_or & 1, sign_q)
+    assert np.mean(np.signbit(x) != np.signbit(xq)) > 0.4  # the partner's sign is really another bit
+    back = np.array([oracle.merge(int(e), int(m), int(mq)) for e, m, mq in zip(e_or, m_or, mq_or)], dtype=np.uint16)
     assert np.array_equal(back, w)
+
+
+def test_partners_are_even_odd_pairs():
+    assert [oracle.partner(x, 6) for x in range(6)] == [1, 0, 3, 2, 5, 4]
+    assert [oracle.partner(x, 5) for x in range(5)] == [1, 0, 3, 2, 4]  # the odd last element keeps its own sign
+    assert oracle.partner(0, 1) == 0
 
 
 # ---------------------------------------------------------------- code lengths
