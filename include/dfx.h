@@ -93,6 +93,8 @@ typedef struct CUstream_st *cudaStream_t;
 #define DFX_STATUS_INDEX 0x4u   /* group start bits or chunk lengths inconsistent */
 #define DFX_STATUS_STREAM 0x8u  /* a bit pattern that is no code, or a chunk that
                                    did not consume exactly its stated length */
+#define DFX_STATUS_TIMEOUT 0x10u /* a copy into shared memory did not complete within the
+                                   kernel's bounded wait; the output is not valid */
 
 typedef struct dfx_plan_s *dfx_plan_t; /* opaque, host-owned */
 

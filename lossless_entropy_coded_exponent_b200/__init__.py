@@ -27,6 +27,7 @@ DFX_STATUS_HEADER = 0x1
 DFX_STATUS_TABLE = 0x2
 DFX_STATUS_INDEX = 0x4
 DFX_STATUS_STREAM = 0x8
+DFX_STATUS_TIMEOUT = 0x10
 
 # The exported C symbols, in include/dfx.h order.
 EXPORTS = (

@@ -53,7 +53,6 @@ struct Tables {
     uint32_t limit[kMaxLenLimit + 1];         // left-justified 24-bit end of the codes of length l
     uint32_t first[kMaxLenLimit + 1];         // first canonical code of length l
     uint32_t index[kMaxLenLimit + 1];         // rank in `sorted` of the first symbol of length l
-    uint32_t nlen[kMaxLenLimit + 1];
     uint8_t sorted[256];                      // used symbols in (length, symbol) order
     uint8_t lens[256];
     uint8_t wcount[8][kMaxLenLimit + 1];      // symbols of each length among 32-symbol slices
@@ -64,11 +63,21 @@ struct Tables {
 
 // Builds the decoding tables in shared memory: the per-length canonical tables in T and
 // the pair table `lut` (1 << kLutBits entries).  `scratch` (2 << kLutBits bytes) holds the
-// one-code table the pair table is built from.
+// one-code table the pair table is built from.  The header, the group index ends and
+// len[256] are read in one round of loads (the host has checked that the buffer holds
+// at least the index and the m plane).
 __device__ bool build_tables(const DecodeArgs& a, Tables& T, uint32_t* lut, uint16_t* scratch) {
     const int t = threadIdx.x;
+    const unsigned warp = t >> 5, lane = t & 31;
+    if (t < 8 * (int)(kMaxLenLimit + 1)) (&T.wcount[0][0])[t] = 0;
+    if (t == 0) T.bad = 0;
+    __syncthreads();
+    uint32_t l_t = 0, within = 0;
+    if (t < 256) l_t = a.comp[kOffLen + t];
     if (t == 0) {
         const uint8_t* h = a.comp;
+        const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(h + kOffGbase);
+        const unsigned long long gb_first = gbase[0], gb_last = gbase[a.n_group];
         uint32_t bad = 0;
         const unsigned long long n = *reinterpret_cast<const unsigned long long*>(h + 8);
         const unsigned long long total_bits = *reinterpret_cast<const unsigned long long*>(h + 16);
@@ -83,61 +92,61 @@ __device__ bool build_tables(const DecodeArgs& a, Tables& T, uint32_t* lut, uint
             bad = DFX_STATUS_HEADER;
         if (max_len < 1 || max_len > kMaxLenLimit || total_bits > (unsigned long long)max_len * a.n) bad = DFX_STATUS_HEADER;
         if (total_bytes != a.off_stream + stream_bytes(total_bits) || total_bytes > a.comp_bytes) bad = DFX_STATUS_HEADER;
-        if (!bad) {
-            // the group index must start at bit 0 and end at total_bits
-            const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(h + kOffGbase);
-            if (gbase[0] != 0 || gbase[a.n_group] != total_bits) bad = DFX_STATUS_INDEX;
-        }
+        // the group index must start at bit 0 and end at total_bits
+        if (!bad && (gb_first != 0 || gb_last != total_bits)) bad = DFX_STATUS_INDEX;
         T.total_bits = total_bits;
         T.n_words = bad ? 0u : (uint32_t)((total_bytes - a.off_stream) / 4);
-        T.bad = bad;
-    }
-    if (t <= (int)kMaxLenLimit) T.nlen[t] = 0;
-    __syncthreads();
-    if (T.bad) {
-        if (t == 0) atomicOr(a.status, T.bad);
-        return false;
-    }
-    if (t < 8 * (int)(kMaxLenLimit + 1)) (&T.wcount[0][0])[t] = 0;
-    if (t < 256) {
-        const uint32_t l = a.comp[kOffLen + t];
-        T.lens[t] = (uint8_t)l;
-        if (l > kMaxLenLimit) atomicOr(&T.bad, DFX_STATUS_TABLE);
-        else if (l) atomicAdd(&T.nlen[l], 1u);
-    }
-    __syncthreads();
-    if (t == 0 && !T.bad) {
-        unsigned long long kraft = 0;
-        for (int l = 1; l <= (int)kMaxLenLimit; l++) kraft += (unsigned long long)T.nlen[l] << (kMaxLenLimit - l);
-        if (a.n > 0 ? kraft != (1ull << kMaxLenLimit) : kraft != 0) T.bad = DFX_STATUS_TABLE;
-        uint32_t code = 0, idx = 0;
-        for (int l = 1; l <= (int)kMaxLenLimit; l++) {
-            T.first[l] = code;
-            T.index[l] = idx;
-            T.limit[l] = (code + T.nlen[l]) << (kMaxLenLimit - l);
-            idx += T.nlen[l];
-            code = (code + T.nlen[l]) << 1;
-        }
-    }
-    __syncthreads();
-    if (T.bad) {
-        if (t == 0) atomicOr(a.status, T.bad);
-        return false;
+        if (bad) atomicOr(&T.bad, bad);
     }
     // rank of each used symbol among the symbols of its length (warps 0-7 hold symbols
-    // 0-255, one per lane): lower lanes of the same warp, then the counts of lower warps
-    const unsigned warp = t >> 5, lane = t & 31;
-    uint32_t l_t = 0, within = 0;
+    // 0-255, one per lane): lower lanes of the same warp now, the counts of lower warps
+    // once every warp has written them
     if (t < 256) {
-        l_t = T.lens[t];
+        T.lens[t] = (uint8_t)l_t;
+        if (l_t > kMaxLenLimit) atomicOr(&T.bad, DFX_STATUS_TABLE);
         const unsigned peers = __match_any_sync(kFull, l_t);
         const unsigned below = peers & ((1u << lane) - 1u);
         within = __popc(below);
-        if (l_t && below == 0) T.wcount[warp][l_t] = (uint8_t)__popc(peers);
+        if (l_t && l_t <= kMaxLenLimit && below == 0) T.wcount[warp][l_t] = (uint8_t)__popc(peers);
     }
-    // meanwhile zero the one-code table (32-bit words: the scratch is 16-byte aligned)
-    for (int i = t; i < (1 << kLutBits) / 2; i += blockDim.x) reinterpret_cast<uint32_t*>(scratch)[i] = 0u;
     __syncthreads();
+    if (T.bad) {
+        if (t == 0) atomicOr(a.status, T.bad);
+        return false;
+    }
+    if (warp == 0) {
+        // canonical tables by a warp scan over the lengths (lane l holds length l):
+        // F = sum over shorter lengths j of nlen[j] << (24 - j) is the left-justified
+        // first code of length l; the Kraft sum is F past the longest length
+        uint32_t nl = 0;
+        if (lane >= 1 && lane <= kMaxLenLimit)
+            for (int w = 0; w < 8; w++) nl += T.wcount[w][lane];
+        const uint32_t weight = (lane >= 1 && lane <= kMaxLenLimit) ? nl << (kMaxLenLimit - lane) : 0u;
+        uint32_t f = weight, c = nl;  // inclusive scans
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t fy = __shfl_up_sync(kFull, f, d), cy = __shfl_up_sync(kFull, c, d);
+            if (lane >= (unsigned)d) {
+                f += fy;
+                c += cy;
+            }
+        }
+        const uint32_t kraft = __shfl_sync(kFull, f, 31);
+        if (lane >= 1 && lane <= kMaxLenLimit) {
+            T.first[lane] = (f - weight) >> (kMaxLenLimit - lane);
+            T.index[lane] = c - nl;
+            T.limit[lane] = f;
+        }
+        if (lane == 0 && (a.n > 0 ? kraft != (1u << kMaxLenLimit) : kraft != 0)) T.bad = DFX_STATUS_TABLE;
+    } else {
+        // meanwhile zero the one-code table (32-bit words: the scratch is 16-byte aligned)
+        for (int i = t - 32; i < (1 << kLutBits) / 2; i += blockDim.x - 32) reinterpret_cast<uint32_t*>(scratch)[i] = 0u;
+    }
+    __syncthreads();
+    if (T.bad) {
+        if (t == 0) atomicOr(a.status, T.bad);
+        return false;
+    }
     if (t < 256 && l_t) {
         uint32_t r = within;
         for (unsigned w = 0; w < warp; w++) r += T.wcount[w][l_t];
@@ -288,8 +297,8 @@ struct ClampedGlobalWords {
 struct SharedWords {
     uint32_t s;  // shared-memory address of the slice buffer
     // Well-formed groups read inside the slice.  A corrupt one reads at most 3K/4 + 2
-    // words past its start, into the next buffer or the guard pad after the last warp's
-    // buffers: never outside the CTA's shared memory.
+    // words past a chunk start, into the other slice buffer or the warp's m units that
+    // follow them: never outside the warp's own buffers.
     __device__ __forceinline__ uint32_t load(uint32_t i) const {
         uint32_t v;
         asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(s + 4u * i));
@@ -386,17 +395,30 @@ __device__ __forceinline__ uint4 decode_block(BitReader<Words>& br, const Tables
 }
 
 // ---------------------------------------------------------------- per-warp buffers
+//
+// Everything a warp reads in bulk is copied into its shared-memory buffers ahead of use by
+// one lane with cp.async.bulk (the 1-D bulk copy engine), each buffer completing on its own
+// mbarrier: the stream slice of the next group (double-buffered) and the sign+mantissa
+// bytes in units of 4 blocks (1 KiB), kMUnits units ahead.  Without that a warp keeps only
+// a few hundred bytes of loads in flight and, at one CTA of 32 warps per SM, the memory
+// system stalls on latency well below its bandwidth.
 
 // Stream words staged per group: the slice of a K = 64 group averages ~0.7 KiB on
 // Gaussian weights; groups that do not fit decode from global memory.
 template <int K>
 struct SliceShape {
-    static constexpr uint32_t kWords = 4u * K;  // 1 KiB at K = 64
+    static constexpr uint32_t kWords = K <= 64 ? 4u * K : 3u * K;  // 1 KiB at K = 64, 1.5 KiB at K = 128
 };
+
+constexpr uint32_t kMUnitBlocks = 4;                      // blocks of one m unit
+constexpr uint32_t kMUnitBytes = kMUnitBlocks * 32 * 8;   // 1 KiB
+constexpr uint32_t kMUnits = 2;                           // m units in flight per warp
 
 template <int K>
 struct WarpBuffers {
     __align__(16) uint32_t slice[2][SliceShape<K>::kWords];  // this group's stream words and the next's
+    uint2 munit[kMUnits][kMUnitBlocks * 32];                  // m bytes, [block][lane]
+    unsigned long long mbar[2 + kMUnits];                     // slice 0, slice 1, m units
 };
 
 template <int K>
@@ -404,82 +426,151 @@ __host__ __device__ constexpr size_t warp_buffer_bytes() {
     return (sizeof(WarpBuffers<K>) + 15) & ~size_t(15);
 }
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(unsigned long long* bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(bar)) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_prior() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory"); }
+// orders this thread's (and, after a warp barrier, the warp's) earlier generic accesses to
+// shared memory before the bulk copies it issues next
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+// arm `bar` for `bytes` and copy them from global `src` to shared `dst` (both 16-byte
+// aligned, bytes a multiple of 16)
+__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+// Wait for the phase with the given parity of `bar` to complete; gives up after a bounded
+// number of polls (the copy engine never took that long here) and reports it.
+constexpr uint32_t kWaitPolls = 1u << 20;
+__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity) {
+    const uint32_t addr = smem_addr(bar);
+    for (uint32_t i = 0; i < kWaitPolls; i++) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done)
+            : "r"(addr), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
 }
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p) : "memory");
+}
+__device__ __forceinline__ uint2 ld_shared_u2(const void* p) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr(p)));
+    return v;
+}
 
-// Stage the stream words of one group, [gb0 >> 5, ((gb0 + span) >> 5) + 4), in a slice
-// buffer (16-byte cp.async chunks, bypassing L1).  Returns false, and copies nothing,
-// when the group is inconsistent or its words do not fit; the group is then decoded
-// straight from global memory.
+// The stream words of one group, [gb0 >> 5, ((gb0 + span) >> 5) + 4), in 16-byte units:
+// staged when the group is consistent and they fit the slice buffer, else the group is
+// decoded straight from global memory.
 struct Slice {
-    uint32_t base;  // stream word index of the first staged word
+    uint32_t base;   // stream word index of the first staged word
+    uint32_t bytes;  // bytes to copy
     bool staged;
 };
 
 template <uint32_t kWords>
-__device__ __forceinline__ Slice stage_slice(const DecodeArgs& a, const Tables& T, uint32_t* buf,
-                                             unsigned long long gb0, uint32_t span, bool ok, unsigned lane) {
+__device__ __forceinline__ Slice plan_slice(const Tables& T, unsigned long long gb0, uint32_t span, bool ok) {
     Slice r;
     const uint32_t beg = ((uint32_t)(gb0 >> 5) * 4u) & ~15u;  // bytes into the stream section
     const uint32_t end = min((((uint32_t)((gb0 + span) >> 5) + 4u) * 4u + 15u) & ~15u, T.n_words * 4u);
     r.base = beg / 4u;
     r.staged = ok && end > beg && end - beg <= kWords * 4u;
-    if (r.staged) {
-        const uint8_t* src = a.comp + a.off_stream + beg;
-        for (uint32_t c = lane; c < (end - beg) / 16u; c += 32) cp_async16(buf + 4 * c, src + 16 * c);
-    }
+    r.bytes = r.staged ? end - beg : 0u;
     return r;
 }
 
-// Decode one full group's 32 chunks (lane i: blocks i, i+32, ... of the group) and
-// write its BF16 output.  Each lane decodes 8 codes, then stores 8 outputs (16 bytes;
-// 512 contiguous bytes per warp store); the sign+mantissa bytes of the next block are
-// loaded while the current one decodes (the group's m plane is prefetched into L2 when
-// the group starts).
+// The m pipeline of one warp: unit j of the warp's sequence (group j / U of the warp,
+// blocks 4 (j % U) .. 4 (j % U) + 3, U = K / 32 units per group) is copied into slot
+// j % kMUnits when unit j - kMUnits has been decoded.
+template <int K>
+struct MPipe {
+    static constexpr uint32_t U = K / 32;
+    uint32_t j;       // next unit to decode
+    uint32_t g0;      // the warp's first group
+    uint32_t step;    // groups between the warp's consecutive groups
+    uint32_t groups;  // full groups of this warp
+
+    // lane 0 only; the slot's previous contents have been read by the whole warp
+    __device__ __forceinline__ void issue(const DecodeArgs& a, WarpBuffers<K>& wb, uint32_t unit) const {
+        if (unit / U < groups) {
+            const uint32_t g = g0 + (unit / U) * step;
+            const uint32_t slot = unit % kMUnits;
+            bulk_copy(wb.munit[slot], a.comp + a.off_m + (uint64_t)g * (32u * K) + (unit % U) * kMUnitBytes,
+                      kMUnitBytes, &wb.mbar[2 + slot]);
+        }
+    }
+};
+
+// Decode one full group's 32 chunks (lane i: blocks i, i+32, ... of the group) and write
+// its BF16 output.  Each lane decodes 8 codes, then stores 8 outputs (16 bytes; 512
+// contiguous bytes per warp store).  The m bytes come from the staged units; once a unit
+// has been decoded, lane 0 refills its slot with the unit kMUnits further on.
 template <int K, class Words>
-__device__ __forceinline__ void decode_group_blocks(const DecodeArgs& a, const Tables& T, BitReader<Words>& br,
-                                                    uint32_t g, unsigned lane, uint32_t& err) {
-    const uint2* mp = reinterpret_cast<const uint2*>(a.comp + a.off_m) + (uint64_t)g * (32u * K / 8u) + lane;
+__device__ __forceinline__ void decode_group_blocks(const DecodeArgs& a, const Tables& T, BitReader<Words>* br,
+                                                    WarpBuffers<K>& wb, MPipe<K>& mp, uint32_t g, unsigned lane,
+                                                    uint32_t& err) {
     uint4* op = reinterpret_cast<uint4*>(a.out) + (uint64_t)g * (32u * K / 8u) + lane;
-    uint2 m_next = __ldg(mp);
+    for (uint32_t u = 0; u < MPipe<K>::U; u++) {
+        const uint32_t slot = mp.j % kMUnits;
+        if (!mbar_wait(&wb.mbar[2 + slot], (mp.j / kMUnits) & 1u)) err |= DFX_STATUS_TIMEOUT;
+        if (br) {
+            const uint2* mu = wb.munit[slot] + lane;
 #pragma unroll 2
-    for (int k = 0; k < K / 8; k++) {
-        const uint2 m = m_next;
-        if (k + 1 < K / 8) m_next = __ldg(mp + 32 * (k + 1));
-        op[32 * k] = decode_block(br, T, m, err);
+            for (uint32_t kk = 0; kk < kMUnitBlocks; kk++)
+                op[32u * (kMUnitBlocks * u + kk)] = decode_block(*br, T, ld_shared_u2(mu + 32u * kk), err);
+        }
+        __syncwarp();
+        if (lane == 0) {
+            fence_proxy_async();
+            mp.issue(a, wb, mp.j + kMUnits);
+        }
+        mp.j++;
     }
 }
 
-// Full groups, one warp at a time.  While group g decodes, the stream slice of the
-// warp's next group is copied into the other slice buffer and the index of the group
-// after that is loaded; the group's m plane is prefetched into L2 when the group starts.
+// Full groups, one warp at a time.  While group g decodes, the stream slice of the warp's
+// next group is copied into the other slice buffer, the index of the group after that is
+// loaded, and the m units run kMUnits units (4 blocks each) ahead of the decode.
 template <int K>
 __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const uint32_t* lut, WarpBuffers<K>& wb,
                                    uint32_t g, uint32_t step, uint32_t n_full, unsigned lane, uint32_t& err) {
     constexpr uint32_t kWords = SliceShape<K>::kWords;
     if (g >= n_full) return;
     const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
+    const uint8_t* sbytes = a.comp + a.off_stream;
     const uint32_t maxw = T.n_words - 1;
-    const uint8_t* mplane = a.comp + a.off_m;
 
+    if (lane == 0) {
+        for (int i = 0; i < 2 + (int)kMUnits; i++) mbar_init(&wb.mbar[i]);
+        fence_mbar_init();
+        fence_proxy_async();  // the buffers were scratch for the table build
+    }
+    __syncwarp();
+    MPipe<K> mp{0u, g, step, (n_full - g + step - 1) / step};
     GroupStart st = scan_index(load_index(a, T, g, lane, true), lane);
-    Slice sl = stage_slice<kWords>(a, T, wb.slice[0], st.gb0, st.span, st.ok, lane);
-    cp_async_commit();
+    Slice sl = plan_slice<kWords>(T, st.gb0, st.span, st.ok);
+    if (lane == 0) {
+        if (sl.staged) bulk_copy(wb.slice[0], sbytes + 4u * sl.base, sl.bytes, &wb.mbar[0]);
+        for (uint32_t u = 0; u < kMUnits; u++) mp.issue(a, wb, u);
+    }
     uint32_t gn = g + step;
     GroupIndex idx_n;
     if (gn < n_full) idx_n = load_index(a, T, gn, lane, true);
-    uint32_t b = 0;
+    uint32_t b = 0, sphase = 0;  // slice buffer in use; parity of each slice buffer's next phase
 
     while (true) {
-        if (lane == 0) prefetch_l2(mplane + (uint64_t)g * (32u * K), 32u * K);
         const bool has_next = gn < n_full;
         const uint32_t gnn = gn + step;
         GroupStart st_n;
@@ -487,20 +578,22 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
         GroupIndex idx_nn;
         if (has_next) {
             st_n = scan_index(idx_n, lane);
-            sl_n = stage_slice<kWords>(a, T, wb.slice[b ^ 1], st_n.gb0, st_n.span, st_n.ok, lane);
+            sl_n = plan_slice<kWords>(T, st_n.gb0, st_n.span, st_n.ok);
+            if (lane == 0 && sl_n.staged)  // buffer b ^ 1 was released at the end of the previous group
+                bulk_copy(wb.slice[b ^ 1], sbytes + 4u * sl_n.base, sl_n.bytes, &wb.mbar[b ^ 1]);
             if (gnn < n_full) idx_nn = load_index(a, T, gnn, lane, true);
         }
-        cp_async_commit();
-        cp_async_wait_prior();  // this group's slice has landed
-        __syncwarp();
+        if (sl.staged) {
+            if (!mbar_wait(&wb.mbar[b], (sphase >> b) & 1u)) err |= DFX_STATUS_TIMEOUT;
+            sphase ^= 1u << b;
+        }
 
         if (st.ok) {
             uint32_t used;
             if (sl.staged) {
                 BitReader<SharedWords> br;
-                br.init(lut, SharedWords{(uint32_t)__cvta_generic_to_shared(wb.slice[b])},
-                        (uint32_t)(st.start - 32ull * sl.base));
-                decode_group_blocks<K>(a, T, br, g, lane, err);
+                br.init(lut, SharedWords{smem_addr(wb.slice[b])}, (uint32_t)(st.start - 32ull * sl.base));
+                decode_group_blocks<K>(a, T, &br, wb, mp, g, lane, err);
                 used = br.consumed();
             } else {
                 // A chunk reads at most 3K/4 + 2 words past its start (24-bit codes); lane 31
@@ -511,20 +604,22 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
                 if (last + (3u * K) / 4u + 8u <= maxw) {
                     BitReader<GlobalWords> br;
                     br.init(lut, GlobalWords{sw + first}, rel);
-                    decode_group_blocks<K>(a, T, br, g, lane, err);
+                    decode_group_blocks<K>(a, T, &br, wb, mp, g, lane, err);
                     used = br.consumed();
                 } else {
                     BitReader<ClampedGlobalWords> br;
                     br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, rel);
-                    decode_group_blocks<K>(a, T, br, g, lane, err);
+                    decode_group_blocks<K>(a, T, &br, wb, mp, g, lane, err);
                     used = br.consumed();
                 }
             }
             if (used != st.clen) err |= DFX_STATUS_STREAM;
         } else {
             err |= DFX_STATUS_INDEX;
+            decode_group_blocks<K, SharedWords>(a, T, nullptr, wb, mp, g, lane, err);  // keeps the m pipeline in step
         }
-        __syncwarp();  // the slice buffer is reused by the copy issued next iteration
+        __syncwarp();  // the slice buffer is refilled by the copy issued next iteration
+        if (lane == 0) fence_proxy_async();
         if (!has_next) break;
         g = gn;
         gn = gnn;
@@ -533,7 +628,6 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
         idx_n = idx_nn;
         b ^= 1;
     }
-    cp_async_wait_all();
 }
 
 // The last group when it is ragged: a lane's chunk holds the elements of its blocks
@@ -584,12 +678,23 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
     extern __shared__ __align__(16) uint8_t dyn_smem[];
     uint32_t* lut = reinterpret_cast<uint32_t*>(dyn_smem);
     uint8_t* warp_area = dyn_smem + kLutBytes;
+    const uint32_t n_full = (a.n % (32ull * K) == 0) ? a.n_group : a.n_group - 1;
+    {
+        // start fetching each warp's first group (index entries, m plane) into L2 while
+        // the tables are built
+        const uint32_t g0 = blockIdx.x * kDecodeWarps + (threadIdx.x >> 5);
+        if ((threadIdx.x & 31) == 0 && g0 < n_full) {
+            prefetch_line_l2(a.comp + kOffGbase + 8ull * g0);
+            prefetch_line_l2(a.comp + a.off_clen + 64ull * g0);
+            prefetch_line_l2(a.comp + a.off_clen + 64ull * g0 + 63);
+            prefetch_l2(a.comp + a.off_m + (uint64_t)g0 * (32u * K), 32u * K);
+        }
+    }
     if (!build_tables(a, T, lut, reinterpret_cast<uint16_t*>(warp_area))) return;
     __syncthreads();  // the scratch is reused as warp buffers
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     WarpBuffers<K>& wb = *reinterpret_cast<WarpBuffers<K>*>(warp_area + warp * warp_buffer_bytes<K>());
     uint32_t err = 0;
-    const uint32_t n_full = (a.n % (32ull * K) == 0) ? a.n_group : a.n_group - 1;
     const uint32_t step = gridDim.x * kDecodeWarps;
     const uint32_t gw = blockIdx.x * kDecodeWarps + warp;
     decode_full_groups<K>(a, T, lut, wb, gw, step, n_full, lane, err);
@@ -597,13 +702,14 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
     if (err) atomicOr(a.status, err);
 }
 
-constexpr size_t kGuardBytes = 512;  // see SharedWords
+constexpr size_t kGuardBytes = 0;  // reads past a warp's slices stay in its m units, see SharedWords
 
 template <int K>
 constexpr size_t dyn_smem_bytes() {
     return kLutBytes + DecodeShape<K>::kWarps * warp_buffer_bytes<K>() + kGuardBytes;
 }
-static_assert(kGuardBytes >= 4 * (3 * 128 / 4 + 8), "guard covers the longest run past a slice");
+static_assert(sizeof(WarpBuffers<128>::munit) >= 4 * (3 * 128 / 4 + 8) && sizeof(WarpBuffers<32>::munit) >= 4 * (3 * 32 / 4 + 8),
+              "the m units after the slices cover the longest run past a slice");
 static_assert(DecodeShape<32>::kThreads >= 256 && DecodeShape<64>::kThreads >= 256 && DecodeShape<128>::kThreads >= 256,
               "the table build gives each of the 256 symbols its own thread");
 static_assert(DecodeShape<32>::kWarps * warp_buffer_bytes<32>() >= (2u << kLutBits), "scratch for the one-code table");
