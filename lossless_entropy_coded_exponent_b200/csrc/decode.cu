@@ -54,6 +54,7 @@ struct Tables {
     uint32_t first[kMaxLenLimit + 1];         // first canonical code of length l
     uint32_t index[kMaxLenLimit + 1];         // rank in `sorted` of the first symbol of length l
     uint8_t sorted[256];                      // used symbols in (length, symbol) order
+    uint8_t slen[256];                        // their code lengths
     uint8_t lens[256];
     uint8_t wcount[8][kMaxLenLimit + 1];      // symbols of each length among 32-symbol slices
     unsigned long long total_bits;
@@ -61,12 +62,11 @@ struct Tables {
     uint32_t bad;
 };
 
-// Builds the decoding tables in shared memory: the per-length canonical tables in T and
-// the pair table `lut` (1 << kLutBits entries).  `scratch` (2 << kLutBits bytes) holds the
-// one-code table the pair table is built from.  The header, the group index ends and
-// len[256] are read in one round of loads (the host has checked that the buffer holds
-// at least the index and the m plane).
-__device__ bool build_tables(const DecodeArgs& a, Tables& T, uint32_t* lut, uint16_t* scratch) {
+// Checks the header and builds the per-length canonical tables in T.  The header, the
+// group index ends and len[256] are read in one round of loads (the host has checked that
+// the buffer holds at least the index and the m plane).  Every thread of the block calls
+// it; false means the container was rejected and its status bits are set.
+__device__ bool build_canonical(const DecodeArgs& a, Tables& T) {
     const int t = threadIdx.x;
     const unsigned warp = t >> 5, lane = t & 31;
     if (t < 8 * (int)(kMaxLenLimit + 1)) (&T.wcount[0][0])[t] = 0;
@@ -138,9 +138,6 @@ __device__ bool build_tables(const DecodeArgs& a, Tables& T, uint32_t* lut, uint
             T.limit[lane] = f;
         }
         if (lane == 0 && (a.n > 0 ? kraft != (1u << kMaxLenLimit) : kraft != 0)) T.bad = DFX_STATUS_TABLE;
-    } else {
-        // meanwhile zero the one-code table (32-bit words: the scratch is 16-byte aligned)
-        for (int i = t - 32; i < (1 << kLutBits) / 2; i += blockDim.x - 32) reinterpret_cast<uint32_t*>(scratch)[i] = 0u;
     }
     __syncthreads();
     if (T.bad) {
@@ -151,46 +148,53 @@ __device__ bool build_tables(const DecodeArgs& a, Tables& T, uint32_t* lut, uint
         uint32_t r = within;
         for (unsigned w = 0; w < warp; w++) r += T.wcount[w][l_t];
         T.sorted[T.index[l_t] + r] = (uint8_t)t;
-    }
-    __syncthreads();
-    // one-code table: (len << 8) | symbol for the code the next kLutBits bits start with,
-    // 0 (left from the zeroing) where they start a longer code.  Symbol i in (length,
-    // symbol) order has the canonical code c = first[l] + i - index[l], which owns the
-    // entries [c, c + 1) << (kLutBits - l); one warp fills one symbol's entries.
-    for (uint32_t i = warp; i < T.index[kLutBits + 1]; i += blockDim.x >> 5) {
-        uint32_t l = 1;
-        while (T.index[l + 1] <= i) l++;
-        const uint32_t shift = kLutBits - l;
-        const uint32_t lo = (T.first[l] + (i - T.index[l])) << shift;
-        const uint32_t v = (l << 8) | T.sorted[i];
-        if (shift >= 3) {  // 8-entry runs, 16-byte aligned
-            const uint32_t w2 = v | (v << 16);
-            uint4* d = reinterpret_cast<uint4*>(scratch + lo);
-            for (uint32_t j = lane; j < (1u << (shift - 3)); j += 32) d[j] = make_uint4(w2, w2, w2, w2);
-        } else if (lane < (1u << shift)) {
-            scratch[lo + lane] = (uint16_t)v;
-        }
-    }
-    __syncthreads();
-    // pair table: the second code is read from the kLutBits - l0 bits left after the
-    // first; a code of length l1 <= kLutBits - l0 depends only on those known bits
-    for (int e = t; e < (1 << kLutBits); e += blockDim.x) {
-        const uint32_t s0 = scratch[e];
-        uint32_t ent = kNotPair;  // long first code
-        if (s0) {
-            const uint32_t l0 = s0 >> 8;
-            const uint32_t s1 = scratch[((uint32_t)e << l0) & ((1u << kLutBits) - 1)];
-            const uint32_t l1 = s1 >> 8;
-            if (s1 && l0 + l1 <= kLutBits)
-                ent = (s0 & 0xFFu) | ((s1 & 0xFFu) << 8) | (l0 << 16) | ((l0 + l1) << 26);
-            else
-                ent = kNotPair | (s0 & 0xFFu) | (l0 << 16) | (l0 << 26);
-        }
-        lut[e] = ent;
+        T.slen[T.index[l_t] + r] = (uint8_t)l_t;
     }
     __syncthreads();
     return true;
 }
+
+// Fill `cnt` entries from `p` with v (cnt a power of two and p aligned to it), the warp's
+// lanes sharing the stores.
+__device__ __forceinline__ void fill_run(uint32_t* p, uint32_t cnt, uint32_t v, unsigned lane) {
+    if (cnt >= 4) {
+        uint4* q = reinterpret_cast<uint4*>(p);
+        for (uint32_t j = lane; j < cnt / 4; j += 32) q[j] = make_uint4(v, v, v, v);
+    } else if (lane < cnt) {
+        p[lane] = v;
+    }
+}
+
+// The pair table `lut` (1 << kLutBits entries) from the canonical tables.  The entries
+// whose index bits start with the code c0 of a first symbol s0 of length l0 <= kLutBits
+// are [c0, c0 + 1) << (kLutBits - l0); one warp per first symbol marks that run "first
+// code only" and then overwrites, for every second symbol whose code c1 fits the
+// remaining r = kLutBits - l0 bits, the sub-run that continues with c1.  Entries no short
+// code starts keep the "long first code" mark.  Every thread of the block calls it.
+__device__ void build_pair_table(const Tables& T, uint32_t* lut) {
+    const int t = threadIdx.x;
+    const unsigned warp = t >> 5, lane = t & 31;
+    for (int i = t; i < (1 << kLutBits) / 4; i += blockDim.x)
+        reinterpret_cast<uint4*>(lut)[i] = make_uint4(kNotPair, kNotPair, kNotPair, kNotPair);
+    __syncthreads();
+    const uint32_t n_short = T.index[kLutBits + 1];  // symbols with codes of at most kLutBits bits
+    for (uint32_t i0 = warp; i0 < n_short; i0 += blockDim.x >> 5) {
+        const uint32_t l0 = T.slen[i0], s0 = T.sorted[i0];
+        const uint32_t r = kLutBits - l0;
+        const uint32_t lo = (T.first[l0] + i0 - T.index[l0]) << r;
+        fill_run(lut + lo, 1u << r, kNotPair | s0 | (l0 << 16) | (l0 << 26), lane);
+        __syncwarp();
+        const uint32_t n1 = T.index[r + 1];  // second symbols with codes of at most r bits
+        for (uint32_t i1 = 0; i1 < n1; i1++) {
+            const uint32_t l1 = T.slen[i1];
+            const uint32_t sh = r - l1;
+            fill_run(lut + lo + ((T.first[l1] + i1 - T.index[l1]) << sh), 1u << sh,
+                     s0 | ((uint32_t)T.sorted[i1] << 8) | (l0 << 16) | ((l0 + l1) << 26), lane);
+        }
+    }
+    __syncthreads();
+}
+
 
 // A code longer than kLutBits: find its length from the canonical limits.  Returns
 // (len << 8) | symbol; bit 16 flags a bit pattern that is no code (Kraft-complete
@@ -540,35 +544,60 @@ __device__ __forceinline__ void decode_group_blocks(const DecodeArgs& a, const T
     }
 }
 
-// Full groups, one warp at a time.  While group g decodes, the stream slice of the warp's
-// next group is copied into the other slice buffer, the index of the group after that is
-// loaded, and the m units run kMUnits units (4 blocks each) ahead of the decode.
+// A warp's position in its sequence of full groups g0, g0 + step, ...
 template <int K>
-__device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const uint32_t* lut, WarpBuffers<K>& wb,
-                                   uint32_t g, uint32_t step, uint32_t n_full, unsigned lane, uint32_t& err) {
-    constexpr uint32_t kWords = SliceShape<K>::kWords;
-    if (g >= n_full) return;
-    const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
-    const uint8_t* sbytes = a.comp + a.off_stream;
-    const uint32_t maxw = T.n_words - 1;
+struct GroupState {
+    MPipe<K> mp;
+    GroupStart st;      // the group to decode next
+    Slice sl;           // its stream slice
+    GroupIndex idx_n;   // the index entries of the group after it
+    uint32_t g, gn;     // those two groups
+    uint32_t b;         // slice buffer of group g
+    uint32_t sphase;    // parity of each slice buffer's next phase
+};
 
+// Start the copies of the warp's first group (stream slice, first kMUnits m units) and
+// load the index of its second group; needs only the canonical tables, so it runs while
+// the block builds the pair table.  The warp has at least one full group.
+template <int K>
+__device__ __forceinline__ void group_prologue(const DecodeArgs& a, const Tables& T, WarpBuffers<K>& wb, uint32_t g,
+                                               uint32_t step, uint32_t n_full, unsigned lane, GroupState<K>& s) {
     if (lane == 0) {
         for (int i = 0; i < 2 + (int)kMUnits; i++) mbar_init(&wb.mbar[i]);
         fence_mbar_init();
-        fence_proxy_async();  // the buffers were scratch for the table build
+        fence_proxy_async();
     }
     __syncwarp();
-    MPipe<K> mp{0u, g, step, (n_full - g + step - 1) / step};
-    GroupStart st = scan_index(load_index(a, T, g, lane, true), lane);
-    Slice sl = plan_slice<kWords>(T, st.gb0, st.span, st.ok);
+    s.mp = MPipe<K>{0u, g, step, (n_full - g + step - 1) / step};
+    s.st = scan_index(load_index(a, T, g, lane, true), lane);
+    s.sl = plan_slice<SliceShape<K>::kWords>(T, s.st.gb0, s.st.span, s.st.ok);
     if (lane == 0) {
-        if (sl.staged) bulk_copy(wb.slice[0], sbytes + 4u * sl.base, sl.bytes, &wb.mbar[0]);
-        for (uint32_t u = 0; u < kMUnits; u++) mp.issue(a, wb, u);
+        if (s.sl.staged) bulk_copy(wb.slice[0], a.comp + a.off_stream + 4u * s.sl.base, s.sl.bytes, &wb.mbar[0]);
+        for (uint32_t u = 0; u < kMUnits; u++) s.mp.issue(a, wb, u);
     }
-    uint32_t gn = g + step;
-    GroupIndex idx_n;
-    if (gn < n_full) idx_n = load_index(a, T, gn, lane, true);
-    uint32_t b = 0, sphase = 0;  // slice buffer in use; parity of each slice buffer's next phase
+    s.g = g;
+    s.gn = g + step;
+    if (s.gn < n_full) s.idx_n = load_index(a, T, s.gn, lane, true);
+    s.b = 0;
+    s.sphase = 0;
+}
+
+// Full groups, one warp at a time, from the state the prologue left.  While group g
+// decodes, the stream slice of the warp's next group is copied into the other slice
+// buffer, the index of the group after that is loaded, and the m units run kMUnits units
+// (4 blocks each) ahead of the decode.
+template <int K>
+__device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const uint32_t* lut, WarpBuffers<K>& wb,
+                                   GroupState<K>& s0, uint32_t step, uint32_t n_full, unsigned lane, uint32_t& err) {
+    constexpr uint32_t kWords = SliceShape<K>::kWords;
+    const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
+    const uint8_t* sbytes = a.comp + a.off_stream;
+    const uint32_t maxw = T.n_words - 1;
+    MPipe<K> mp = s0.mp;
+    GroupStart st = s0.st;
+    Slice sl = s0.sl;
+    GroupIndex idx_n = s0.idx_n;
+    uint32_t g = s0.g, gn = s0.gn, b = s0.b, sphase = s0.sphase;
 
     while (true) {
         const bool has_next = gn < n_full;
@@ -673,8 +702,7 @@ template <int K>
 __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeArgs a) {
     constexpr int kDecodeWarps = DecodeShape<K>::kWarps;
     __shared__ Tables T;
-    // dynamic shared memory: the pair table, then one buffer per warp (the buffers
-    // double as scratch for the one-code table while the tables are built)
+    // dynamic shared memory: the pair table, then one buffer per warp
     extern __shared__ __align__(16) uint8_t dyn_smem[];
     uint32_t* lut = reinterpret_cast<uint32_t*>(dyn_smem);
     uint8_t* warp_area = dyn_smem + kLutBytes;
@@ -690,14 +718,16 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
             prefetch_l2(a.comp + a.off_m + (uint64_t)g0 * (32u * K), 32u * K);
         }
     }
-    if (!build_tables(a, T, lut, reinterpret_cast<uint16_t*>(warp_area))) return;
-    __syncthreads();  // the scratch is reused as warp buffers
+    if (!build_canonical(a, T)) return;
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     WarpBuffers<K>& wb = *reinterpret_cast<WarpBuffers<K>*>(warp_area + warp * warp_buffer_bytes<K>());
     uint32_t err = 0;
     const uint32_t step = gridDim.x * kDecodeWarps;
     const uint32_t gw = blockIdx.x * kDecodeWarps + warp;
-    decode_full_groups<K>(a, T, lut, wb, gw, step, n_full, lane, err);
+    GroupState<K> gs;
+    if (gw < n_full) group_prologue<K>(a, T, wb, gw, step, n_full, lane, gs);
+    build_pair_table(T, lut);
+    if (gw < n_full) decode_full_groups<K>(a, T, lut, wb, gs, step, n_full, lane, err);
     if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, lut, n_full, lane, err);
     if (err) atomicOr(a.status, err);
 }
@@ -712,8 +742,6 @@ static_assert(sizeof(WarpBuffers<128>::munit) >= 4 * (3 * 128 / 4 + 8) && sizeof
               "the m units after the slices cover the longest run past a slice");
 static_assert(DecodeShape<32>::kThreads >= 256 && DecodeShape<64>::kThreads >= 256 && DecodeShape<128>::kThreads >= 256,
               "the table build gives each of the 256 symbols its own thread");
-static_assert(DecodeShape<32>::kWarps * warp_buffer_bytes<32>() >= (2u << kLutBits), "scratch for the one-code table");
-static_assert(DecodeShape<128>::kWarps * warp_buffer_bytes<128>() >= (2u << kLutBits), "scratch for the one-code table");
 static_assert(dyn_smem_bytes<64>() + 1024 <= 227 * 1024 && dyn_smem_bytes<128>() + 1024 <= 227 * 1024, "shared memory");
 
 template <int K>
