@@ -25,9 +25,10 @@ import hashlib
 import json
 import math
 import os
+import shutil
 import statistics
+import subprocess
 import sys
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -68,6 +69,20 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def host_cpu() -> str:
+    """Model name and logical CPU count of this host (the oracle runs on one of them)."""
+    model = "unknown CPU"
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return f"{model}, {os.cpu_count()} logical CPUs"
+
+
 def decode_source_hash() -> str:
     h = hashlib.sha256()
     for p in DECODE_SOURCES:
@@ -93,8 +108,26 @@ def ncu_traffic_per_launch(n_weights: int):
         return None
 
 
+CLOCK_CHILD = r"""
+import json, select, sys
+import pynvml
+pynvml.nvmlInit()
+bus, index, period = sys.argv[1], int(sys.argv[2]), float(sys.argv[3])
+h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode()) if bus != "-" else pynvml.nvmlDeviceGetHandleByIndex(index)
+mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+clk, reasons = [], 0
+print("ready", flush=True)
+while not select.select([sys.stdin], [], [], period)[0]:
+    clk.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+    reasons |= pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+print(json.dumps({"clk": clk, "max": mx, "reasons": reasons}), flush=True)
+"""
+
+
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML while running."""
+    """Samples SM clock and clock-event reasons while running, through NVML in a child
+    interpreter (so the launch loop of this one cannot starve it); stops when its stdin
+    closes."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
@@ -103,59 +136,53 @@ class ClockSampler:
     def __init__(self, device_index: int, period_s: float = 0.01):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
-        self._stop = threading.Event()
-        self._thread = None
+        self.device_index = device_index
+        self.error = None
+        self._proc = None
+
+    @staticmethod
+    def _bus_id(device_index):
         try:
-            import pynvml
+            import torch
 
-            pynvml.nvmlInit()
-            self._nv = pynvml
-            self._h = self._handle(device_index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-        except Exception as e:  # no NVML: report that instead of clocks
-            self._nv = None
-            self.error = repr(e)
-
-    def _handle(self, device_index):
-        import torch
-
-        nv = self._nv
-        try:
             props = torch.cuda.get_device_properties(device_index)
-            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
-            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            return "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
         except Exception:
-            return nv.nvmlDeviceGetHandleByIndex(device_index)
-
-    def _run(self):
-        nv = self._nv
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h) if hasattr(
-                    nv, "nvmlDeviceGetCurrentClocksEventReasons") else nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self.period)
+            return "-"
 
     def __enter__(self):
-        if self._nv is not None:
-            self._thread = threading.Thread(target=self._run, daemon=True)
-            self._thread.start()
+        try:
+            self._proc = subprocess.Popen(
+                [sys.executable, "-c", CLOCK_CHILD, self._bus_id(self.device_index), str(self.device_index),
+                 str(self.period)], stdin=subprocess.PIPE, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+            if self._proc.stdout.readline().strip() != "ready":  # sampling has started
+                raise RuntimeError(self._proc.stderr.read()[-300:])
+        except Exception as e:
+            self.error = repr(e)
+            if self._proc is not None:
+                self._proc.kill()
+            self._proc = None
         return self
 
     def __exit__(self, *exc):
-        self._stop.set()
-        if self._thread:
-            self._thread.join()
+        if self._proc is None:
+            return
+        try:
+            out, _ = self._proc.communicate(input="", timeout=30)  # closes stdin: the child reports and exits
+            d = json.loads(out.strip().splitlines()[-1])
+            self.samples, self.max_mhz = d["clk"], d["max"]
+            for bit, name in self.REASONS.items():
+                if d["reasons"] & bit:
+                    self.reasons.add(name)
+        except Exception as e:
+            self.error = repr(e)
+            self._proc.kill()
 
     def summary(self):
-        if self._nv is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "no nvml")}
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0,
+                    "error": self.error or "no samples"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
@@ -240,7 +267,7 @@ def run_reference(args, world, rank):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "sample": sample, "chunk_symbols": args.chunk_symbols},
             "bits_per_weight": 8.0 * c.size / n,
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "host": host_cpu(), "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     return line
 
@@ -444,7 +471,7 @@ def run_cpu_baseline(x0, comp0, K):
     dec = oracle.decode(ref)
     dt = time.perf_counter() - t0
     exact &= bool(np.array_equal(dec, w))
-    return ({"value": 2.0 * w.size / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+    return ({"value": 2.0 * w.size / dt / 1e9, "unit": UNIT, "cores": 1, "host": host_cpu(), "kind": "oracle",
              "sample": f"tensor 0 of the stream ({w.size} weights), one oracle decode, single thread"}, exact)
 
 

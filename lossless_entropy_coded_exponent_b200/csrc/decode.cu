@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
     {
         // start fetching each warp's first group (index entries, m plane) into L2 while
         // the tables are built
-        const uint32_t g0 = blockIdx.x * kDecodeWarps + (threadIdx.x >> 5);
+        const uint32_t g0 = blockIdx.x + gridDim.x * (threadIdx.x >> 5);
         if ((threadIdx.x & 31) == 0 && g0 < n_full) {
             prefetch_line_l2(a.comp + kOffGbase + 8ull * g0);
             prefetch_line_l2(a.comp + a.off_clen + 64ull * g0);
@@ -723,7 +723,9 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
     WarpBuffers<K>& wb = *reinterpret_cast<WarpBuffers<K>*>(warp_area + warp * warp_buffer_bytes<K>());
     uint32_t err = 0;
     const uint32_t step = gridDim.x * kDecodeWarps;
-    const uint32_t gw = blockIdx.x * kDecodeWarps + warp;
+    // groups are dealt to the CTAs (one per SM) in turn and each CTA's to its warps in
+    // turn, so that every SM gets the same number of groups within one
+    const uint32_t gw = blockIdx.x + gridDim.x * warp;
     GroupState<K> gs;
     if (gw < n_full) group_prologue<K>(a, T, wb, gw, step, n_full, lane, gs);
     build_pair_table(T, lut);
