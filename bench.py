@@ -56,6 +56,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-layer-batch", action="store_true", help="skip the multi-tensor (Llama-3-8B layer) decode measurement")
     return ap.parse_args()
 
 
@@ -385,11 +386,77 @@ def run_ours(args, world, rank, local):
     # ---- end to end through the C ABI with host buffers
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, plan, comps, sizes, n, dev, world)
+    # ---- several tensors per launch: a Llama-3-8B-shaped layer
+    if not args.no_layer_batch and rank == 0:
+        line["layer_batch"] = run_layer_batch(args, dev, stream)
     # ---- oracle on the host: rank 0 at N=1 only
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         line["cpu_baseline"], line["bit_exact_vs_oracle"] = run_cpu_baseline(xs[0], comps[0], K)
     plan.free()
     return line
+
+
+def run_layer_batch(args, dev, stream):
+    """The seven projections of a Llama-3-8B-shaped layer (218 M weights, tensors of 4 M
+    to 59 M weights): per layer, seven dfx_decode launches against one dfx_decode_batch."""
+    import torch
+
+    import lossless_entropy_coded_exponent_b200 as dfx
+    from lossless_entropy_coded_exponent_b200 import inputs
+
+    L = len(inputs.LLAMA3_8B_LAYER)
+    with torch.cuda.stream(stream):  # everything below is ordered on this one stream
+        xs = [inputs.llama3_8b_layer_tensor_cuda(i, device=dev) for i in range(L)]
+    plans = [dfx.dfx_plan(x.numel(), chunk_symbols=args.chunk_symbols) for x in xs]
+    try:
+        comps, sizes = [], []
+        with torch.cuda.stream(stream):
+            for x, p in zip(xs, plans):
+                out = torch.empty(p.max_compressed_bytes, dtype=torch.uint8, device=dev)
+                ws = torch.empty(p.workspace_bytes, dtype=torch.uint8, device=dev)
+                size = dfx.dfx_encode(p, x, out, out.numel(), ws, ws.numel(), want_size=True, stream=stream)
+                comps.append(out[:size].clone())
+                sizes.append(size)
+            outs = [torch.empty_like(x) for x in xs]
+
+        def separate():
+            for i in range(L):
+                dfx.dfx_decode(plans[i], comps[i], sizes[i], outs[i], stream=stream)
+
+        def batch():
+            dfx.dfx_decode_batch(plans, comps, sizes, outs, stream=stream)
+
+        def time_it(fn, reps=20, warm=3):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+            with torch.cuda.stream(stream):
+                for _ in range(warm):
+                    fn()
+                ev[0].record(stream)
+                for r in range(reps):
+                    fn()
+                    ev[r + 1].record(stream)
+            stream.synchronize()
+            return statistics.median(ev[r].elapsed_time(ev[r + 1]) for r in range(reps)) * 1e3
+
+        sep_us, bat_us = time_it(separate), time_it(batch)
+        with torch.cuda.stream(stream):
+            for o in outs:
+                o.fill_(-1)
+            batch()
+        stream.synchronize()
+        exact = all(torch.equal(o, x) for o, x in zip(outs, xs)) and all(dfx.dfx_device_status(p) == 0 for p in plans)
+        n = sum(x.numel() for x in xs)
+        algo = float(sum(sizes)) + 2.0 * n
+        peak, peak_kind = measured_hbm_peak()
+        return {"workload": "Llama-3-8B-shaped layer: q, o 4096x4096; k, v 1024x4096; gate, up 14336x4096; "
+                            "down 4096x14336; N(0, 1/fan_in)", "tensors": L, "weights": n,
+                "separate_us": sep_us, "batch_us": bat_us, "batch_algorithmic_gbs": algo / (bat_us * 1e-6) / 1e9,
+                "batch_frac_of_measured": algo / (bat_us * 1e-6) / 1e9 / peak, "peak_kind": peak_kind,
+                "bit_exact": bool(exact), "note": "median per layer over 20 reps; no L2 flush (0.5 GB of "
+                "containers and outputs per layer exceed the 126 MB L2)"}
+    finally:
+        for p in plans:
+            p.free()
 
 
 def run_e2e(args, plan, comps, sizes, n, dev, world):

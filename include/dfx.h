@@ -151,6 +151,21 @@ int dfx_encode(dfx_plan_t plan, const void *d_bf16, void *d_out, size_t out_capa
 int dfx_decode(dfx_plan_t plan, const void *d_comp, size_t comp_bytes, void *d_bf16,
                cudaStream_t stream);
 
+/* Decode `count` containers (1..32; 0 is a no-op) with one kernel launch: a
+ * whole layer's weights restored before use in one go (the pages decode a
+ * model's compressed weights on the GPU ahead of the computation that reads
+ * them: "DFloat11: lossless LLM compression for GPU", title and section 02).
+ * plans[i], d_comps[i], comp_bytes[i], d_bf16s[i]: as for dfx_decode, one per
+ * tensor (host arrays of count entries; the buffers are device memory).  All
+ * plans must belong to the current device and share chunk_symbols, else
+ * DFX_ERR_UNSUPPORTED; host argument errors of any tensor return before any
+ * launch.  The device's CTAs are split among the tensors in proportion to their
+ * groups, each CTA decoding part of one tensor.  Corruption is reported in each
+ * tensor's own plan status word.  Outputs must not overlap each other or the
+ * containers.  Asynchronous. */
+int dfx_decode_batch(const dfx_plan_t *plans, const void *const *d_comps, const size_t *comp_bytes,
+                     void *const *d_bf16s, uint32_t count, cudaStream_t stream);
+
 /* Synchronise `stream`, return the plan's sticky device status word in
  * *h_status (0 = no corruption seen since the last read) and clear it. */
 int dfx_device_status(dfx_plan_t plan, cudaStream_t stream, uint32_t *h_status);

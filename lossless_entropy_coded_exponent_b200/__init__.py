@@ -37,6 +37,7 @@ EXPORTS = (
     "dfx_plan",
     "dfx_encode",
     "dfx_decode",
+    "dfx_decode_batch",
     "dfx_device_status",
     "dfx_free",
     "dfx_encode_static",
@@ -82,12 +83,14 @@ def lib() -> ctypes.CDLL:
                                ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
         L.dfx_encode.argtypes = [vp, vp, vp, ctypes.c_size_t, vp, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t), vp]
         L.dfx_decode.argtypes = [vp, vp, ctypes.c_size_t, vp, vp]
+        L.dfx_decode_batch.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_size_t),
+                                       ctypes.POINTER(vp), ctypes.c_uint32, vp]
         L.dfx_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.dfx_free.argtypes = [vp]
         L.dfx_encode_static.argtypes = [vp, ctypes.c_uint64, ctypes.POINTER(dfx_params), vp, ctypes.c_size_t,
                                         ctypes.POINTER(ctypes.c_size_t), vp]
-        for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_device_status", "dfx_free",
-                  "dfx_encode_static"):
+        for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_decode_batch",
+                  "dfx_device_status", "dfx_free", "dfx_encode_static"):
             getattr(L, f).restype = ctypes.c_int
         _lib_handle = L
     return _lib_handle
@@ -182,6 +185,19 @@ def dfx_encode(plan: Plan, d_bf16, d_out, out_capacity: int, d_workspace, worksp
 
 def dfx_decode(plan: Plan, d_comp, comp_bytes: int, d_bf16, stream=None) -> None:
     _check(lib().dfx_decode(plan.handle, _ptr(d_comp), comp_bytes, _ptr(d_bf16), _stream(stream)), "dfx_decode")
+
+
+def dfx_decode_batch(plans, d_comps, comp_bytes, d_bf16s, stream=None) -> None:
+    """Decode several containers with one kernel launch (sequences of equal length)."""
+    n = len(plans)
+    if not (len(d_comps) == len(comp_bytes) == len(d_bf16s) == n):
+        raise ValueError("dfx_decode_batch: plans, containers, sizes and outputs differ in length")
+    vp = ctypes.c_void_p
+    hp = (vp * max(n, 1))(*[p.handle if p is not None else None for p in plans])
+    cp = (vp * max(n, 1))(*[_ptr(c) for c in d_comps])
+    sz = (ctypes.c_size_t * max(n, 1))(*[int(b) for b in comp_bytes])
+    op = (vp * max(n, 1))(*[_ptr(o) for o in d_bf16s])
+    _check(lib().dfx_decode_batch(hp, cp, sz, op, n, _stream(stream)), "dfx_decode_batch")
 
 
 def dfx_device_status(plan: Plan, stream=None) -> int:

@@ -15,6 +15,7 @@ struct dfx_plan_s {
     uint32_t* d_status;
     int device;
     int decode_grid;
+    int resident_ctas;  // decode CTAs that fit on the device at once
 };
 
 namespace {
@@ -30,6 +31,9 @@ int resolve_params(const dfx_params* p, uint32_t* K, uint32_t* G, uint32_t* L) {
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Host checks of one decode and its kernel arguments.
+int make_decode_args(const dfx_plan_s* plan, const void* d_comp, size_t comp_bytes, void* d_bf16, dfx::DecodeArgs* a);
 
 int check_device(const dfx_plan_s* plan) {
     int dev = -1;
@@ -106,6 +110,7 @@ int dfx_plan(dfx_plan_t* plan, uint64_t n, const dfx_params* params, size_t* max
         return DFX_ERR_CUDA;
     }
     const uint64_t resident = dfx::decode_blocks_per_sm(K) * (uint64_t)sms;  // CTAs that fit at once
+    p->resident_ctas = (int)resident;
     const uint64_t wpb = (uint64_t)dfx::decode_warps_per_block(K);
     const uint64_t need = (p->L.n_group + wpb - 1) / wpb;                    // CTAs with work (a warp per group)
     p->decode_grid = (int)(need == 0 ? 1 : (need < resident ? need : resident));
@@ -158,26 +163,49 @@ int dfx_encode(dfx_plan_t plan, const void* d_bf16, void* d_out, size_t out_capa
 }
 
 int dfx_decode(dfx_plan_t plan, const void* d_comp, size_t comp_bytes, void* d_bf16, cudaStream_t stream) {
-    if (!plan) return DFX_ERR_ARG;
-    if (!d_comp || (!d_bf16 && plan->n)) return DFX_ERR_ARG;
-    if (!aligned16(d_comp) || !aligned16(d_bf16)) return DFX_ERR_ARG;
-    if (comp_bytes < plan->L.off_stream + dfx::stream_bytes(0)) return DFX_ERR_CORRUPT;
-    int rc = check_device(plan);
-    if (rc) return rc;
     dfx::DecodeArgs a;
-    a.comp = (const uint8_t*)d_comp;
-    a.comp_bytes = comp_bytes;
-    a.out = (uint16_t*)d_bf16;
-    a.n = plan->n;
-    a.K = plan->K;
-    a.G = plan->G;
-    a.n_chunk = (uint32_t)plan->L.n_chunk;
-    a.n_group = (uint32_t)plan->L.n_group;
-    a.off_clen = plan->L.off_clen;
-    a.off_m = plan->L.off_m;
-    a.off_stream = plan->L.off_stream;
-    a.status = plan->d_status;
+    const int rc = make_decode_args(plan, d_comp, comp_bytes, d_bf16, &a);
+    if (rc) return rc;
     if (dfx::launch_decode(a, plan->decode_grid, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return DFX_ERR_CUDA;
+    }
+    return DFX_OK;
+}
+
+int dfx_decode_batch(const dfx_plan_t* plans, const void* const* d_comps, const size_t* comp_bytes,
+                     void* const* d_bf16s, uint32_t count, cudaStream_t stream) {
+    if (count == 0) return DFX_OK;
+    if (!plans || !d_comps || !comp_bytes || !d_bf16s || count > dfx::kMaxBatch) return DFX_ERR_ARG;
+    static_assert(sizeof(dfx::BatchArgs) <= 4000, "the batch descriptor is passed as a kernel parameter");
+    dfx::BatchArgs b;
+    b.count = count;
+    uint64_t groups[dfx::kMaxBatch];
+    for (uint32_t i = 0; i < count; i++) {
+        if (!plans[i]) return DFX_ERR_ARG;
+        if (plans[i]->K != plans[0]->K || plans[i]->device != plans[0]->device) return DFX_ERR_UNSUPPORTED;
+        const int rc = make_decode_args(plans[i], d_comps[i], comp_bytes[i], d_bf16s[i], &b.t[i]);
+        if (rc) return rc;
+        groups[i] = plans[i]->L.n_group;
+    }
+    // CTAs in proportion to the groups: every tensor gets one (an empty one only checks its
+    // header), then each further CTA goes to the tensor with the most groups per CTA.
+    const uint32_t total = (uint32_t)plans[0]->resident_ctas;
+    if (total < count) return DFX_ERR_UNSUPPORTED;
+    uint32_t ctas[dfx::kMaxBatch];
+    for (uint32_t i = 0; i < count; i++) ctas[i] = 1;
+    for (uint32_t left = total - count; left > 0; left--) {
+        int best = -1;
+        for (uint32_t i = 0; i < count; i++) {
+            if (ctas[i] >= (groups[i] + 31) / 32) continue;  // every warp already has a group
+            if (best < 0 || groups[i] * ctas[best] > groups[best] * ctas[i]) best = (int)i;
+        }
+        if (best < 0) break;
+        ctas[best]++;
+    }
+    b.cta_begin[0] = 0;
+    for (uint32_t i = 0; i < count; i++) b.cta_begin[i + 1] = b.cta_begin[i] + ctas[i];
+    if (dfx::launch_decode_batch(b, plans[0]->K, stream) != cudaSuccess) {
         cudaGetLastError();
         return DFX_ERR_CUDA;
     }
@@ -208,3 +236,29 @@ int dfx_free(dfx_plan_t plan) {
 }
 
 }  // extern "C"
+
+namespace {
+
+int make_decode_args(const dfx_plan_s* plan, const void* d_comp, size_t comp_bytes, void* d_bf16, dfx::DecodeArgs* a) {
+    if (!plan) return DFX_ERR_ARG;
+    if (!d_comp || (!d_bf16 && plan->n)) return DFX_ERR_ARG;
+    if (!aligned16(d_comp) || !aligned16(d_bf16)) return DFX_ERR_ARG;
+    if (comp_bytes < plan->L.off_stream + dfx::stream_bytes(0)) return DFX_ERR_CORRUPT;
+    const int rc = check_device(plan);
+    if (rc) return rc;
+    a->comp = (const uint8_t*)d_comp;
+    a->comp_bytes = comp_bytes;
+    a->out = (uint16_t*)d_bf16;
+    a->n = plan->n;
+    a->K = plan->K;
+    a->G = plan->G;
+    a->n_chunk = (uint32_t)plan->L.n_chunk;
+    a->n_group = (uint32_t)plan->L.n_group;
+    a->off_clen = plan->L.off_clen;
+    a->off_m = plan->L.off_m;
+    a->off_stream = plan->L.off_stream;
+    a->status = plan->d_status;
+    return DFX_OK;
+}
+
+}  // namespace

@@ -698,8 +698,10 @@ __device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, const ui
 
 constexpr size_t kLutBytes = sizeof(uint32_t) << kLutBits;
 
+// One tensor's decode by `ctas` CTAs of which this is number `cta`: the body of both
+// kernels below.
 template <int K>
-__global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeArgs a) {
+__device__ __forceinline__ void decode_tensor(const DecodeArgs& a, uint32_t cta, uint32_t ctas) {
     constexpr int kDecodeWarps = DecodeShape<K>::kWarps;
     __shared__ Tables T;
     // dynamic shared memory: the pair table, then one buffer per warp
@@ -710,7 +712,7 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
     {
         // start fetching each warp's first group (index entries, m plane) into L2 while
         // the tables are built
-        const uint32_t g0 = blockIdx.x + gridDim.x * (threadIdx.x >> 5);
+        const uint32_t g0 = cta + ctas * (threadIdx.x >> 5);
         if ((threadIdx.x & 31) == 0 && g0 < n_full) {
             prefetch_line_l2(a.comp + kOffGbase + 8ull * g0);
             prefetch_line_l2(a.comp + a.off_clen + 64ull * g0);
@@ -722,16 +724,30 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     WarpBuffers<K>& wb = *reinterpret_cast<WarpBuffers<K>*>(warp_area + warp * warp_buffer_bytes<K>());
     uint32_t err = 0;
-    const uint32_t step = gridDim.x * kDecodeWarps;
+    const uint32_t step = ctas * kDecodeWarps;
     // groups are dealt to the CTAs (one per SM) in turn and each CTA's to its warps in
     // turn, so that every SM gets the same number of groups within one
-    const uint32_t gw = blockIdx.x + gridDim.x * warp;
+    const uint32_t gw = cta + ctas * warp;
     GroupState<K> gs;
     if (gw < n_full) group_prologue<K>(a, T, wb, gw, step, n_full, lane, gs);
     build_pair_table(T, lut);
     if (gw < n_full) decode_full_groups<K>(a, T, lut, wb, gs, step, n_full, lane, err);
     if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, lut, n_full, lane, err);
     if (err) atomicOr(a.status, err);
+}
+
+template <int K>
+__global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeArgs a) {
+    decode_tensor<K>(a, blockIdx.x, gridDim.x);
+}
+
+// Several tensors in one launch (all with the same K): each CTA decodes its share of one
+// tensor, so it builds that tensor's tables once.
+template <int K>
+__global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode_batch(const __grid_constant__ BatchArgs b) {
+    uint32_t i = 0;
+    while (i + 1 < b.count && blockIdx.x >= b.cta_begin[i + 1]) i++;
+    decode_tensor<K>(b.t[i], blockIdx.x - b.cta_begin[i], b.cta_begin[i + 1] - b.cta_begin[i]);
 }
 
 constexpr size_t kGuardBytes = 0;  // reads past a warp's slices stay in its m units, see SharedWords
@@ -758,19 +774,33 @@ int blocks_per_sm() {
     return b > 0 ? b : 1;
 }
 
-template <int K>
-cudaError_t launch_k(const DecodeArgs& a, int grid, cudaStream_t s) {
-    // the dynamic shared-memory limit is raised once per device (needed above 48 KiB)
-    static bool attr_set[64] = {};
+// The dynamic shared-memory limit of a kernel is raised once per device (needed above
+// 48 KiB).
+template <class F>
+cudaError_t allow_smem(F* kernel, size_t bytes, bool* done) {
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_decode<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)dyn_smem_bytes<K>());
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
+    if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+    return e;
+}
+
+template <int K>
+cudaError_t launch_k(const DecodeArgs& a, int grid, cudaStream_t s) {
+    static bool attr_set[64] = {};
+    const cudaError_t e = allow_smem(k_decode<K>, dyn_smem_bytes<K>(), attr_set);
+    if (e != cudaSuccess) return e;
     k_decode<K><<<grid, DecodeShape<K>::kThreads, dyn_smem_bytes<K>(), s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int K>
+cudaError_t launch_batch_k(const BatchArgs& b, cudaStream_t s) {
+    static bool attr_set[64] = {};
+    const cudaError_t e = allow_smem(k_decode_batch<K>, dyn_smem_bytes<K>(), attr_set);
+    if (e != cudaSuccess) return e;
+    k_decode_batch<K><<<b.cta_begin[b.count], DecodeShape<K>::kThreads, dyn_smem_bytes<K>(), s>>>(b);
     return cudaGetLastError();
 }
 
@@ -789,6 +819,16 @@ int decode_blocks_per_sm(uint32_t K) {
 
 int decode_warps_per_block(uint32_t K) {
     return K == 32 ? DecodeShape<32>::kWarps : K == 64 ? DecodeShape<64>::kWarps : DecodeShape<128>::kWarps;
+}
+
+cudaError_t launch_decode_batch(const BatchArgs& b, uint32_t K, cudaStream_t s) {
+    if (b.count == 0 || b.count > kMaxBatch || b.cta_begin[b.count] == 0) return cudaErrorInvalidValue;
+    switch (K) {
+        case 32: return launch_batch_k<32>(b, s);
+        case 64: return launch_batch_k<64>(b, s);
+        case 128: return launch_batch_k<128>(b, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, int grid, cudaStream_t s) {

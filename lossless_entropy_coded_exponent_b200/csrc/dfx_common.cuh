@@ -72,6 +72,14 @@ struct EncodeArgs {
     uint32_t* status;
 };
 
+// Several tensors decoded by one launch: tensor i gets CTAs [cta_begin[i], cta_begin[i+1]).
+constexpr uint32_t kMaxBatch = 32;
+struct BatchArgs {
+    uint32_t count;
+    uint32_t cta_begin[kMaxBatch + 1];
+    DecodeArgs t[kMaxBatch];
+};
+
 // Workspace layout for encode.
 constexpr uint64_t kWsCounts = 0;
 constexpr uint64_t kWsCode = 2048;
@@ -84,6 +92,7 @@ inline uint64_t workspace_bytes_for(uint64_t n_group) {
 // Launchers (encode.cu / decode.cu).
 cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_decode_batch(const BatchArgs& b, uint32_t K, cudaStream_t s);
 int decode_blocks_per_sm(uint32_t K);
 int decode_warps_per_block(uint32_t K);
 bool decode_supports(uint32_t K, uint32_t G);

@@ -188,6 +188,19 @@ def bf16_from_f32_torch(x):
     return ((u + bias) >> 16).to(torch.int16)
 
 
+def llama3_8b_layer_tensor_cuda(i: int, device="cuda"):
+    """Tensor i of the Llama-3-8B-shaped layer drawn on the device: the same recipe as
+    llama3_8b_layer_tensor (N(0, 1/fan_in), seed 40 + i) with torch's seeded generator."""
+    import torch
+
+    _, rows, cols = LLAMA3_8B_LAYER[i]
+    g = torch.Generator(device=device)
+    g.manual_seed(40 + i)
+    x = torch.randn(rows * cols, device=device, dtype=torch.float32, generator=g)
+    x.mul_(1.0 / math.sqrt(cols))
+    return bf16_from_f32_torch(x)
+
+
 def layer70b_tensor_cuda(i: int, seed_base: int = 500, device="cuda"):
     import torch
 

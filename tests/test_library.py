@@ -1,6 +1,7 @@
 """Host-side checks of libdfx that need no GPU: the shared library loads, exports
 every symbol include/dfx.h declares, its layout arithmetic agrees with the
 oracle's, and argument errors come back before any CUDA call."""
+import ctypes
 import os
 import re
 
@@ -87,3 +88,15 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(dfx, "LIB_PATH", str(tmp_path / "libdfx.so"))
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         dfx.dfx_version()
+
+
+def test_batch_argument_errors_precede_cuda(lib):
+    vp = ctypes.c_void_p
+    assert lib.dfx_decode_batch(None, None, None, None, 0, None) == dfx.DFX_OK  # nothing to do
+    assert lib.dfx_decode_batch(None, None, None, None, 1, None) == dfx.DFX_ERR_ARG
+    arr = (vp * 33)()
+    sizes = (ctypes.c_size_t * 33)()
+    assert lib.dfx_decode_batch(arr, arr, sizes, arr, 33, None) == dfx.DFX_ERR_ARG  # at most 32 tensors
+    assert lib.dfx_decode_batch(arr, arr, sizes, arr, 2, None) == dfx.DFX_ERR_ARG  # null plans
+    with pytest.raises(ValueError):
+        dfx.dfx_decode_batch([None], [], [], [])
