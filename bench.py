@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--tensors", type=int, default=24)
-    ap.add_argument("--chunk-symbols", type=int, default=64)
+    ap.add_argument("--chunk-symbols", type=int, default=128)
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -376,7 +376,7 @@ def run_ours(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": algo_bytes_per_launch,
-                         "mean_launch_us": 1e3 * mean_launch_ms, "kernel": "k_decode<64>"},
+                         "mean_launch_us": 1e3 * mean_launch_ms, "kernel": f"k_decode<{K}>"},
             "gpu_launches": args.steps * T,
             "clocks": clocks.summary(),
             "encode": {"unit": "GB/s", "value": 2.0 * n / (statistics.median(enc_ms) * 1e-3) / 1e9,

@@ -99,7 +99,7 @@ typedef struct CUstream_st *cudaStream_t;
 typedef struct dfx_plan_s *dfx_plan_t; /* opaque, host-owned */
 
 typedef struct {
-    uint32_t chunk_symbols; /* K: a multiple of 8; 32, 64 or 128 on the GPU path (0 -> 64) */
+    uint32_t chunk_symbols; /* K: a multiple of 8; 32, 64 or 128 on the GPU path (0 -> 128) */
     uint32_t group_chunks;  /* G: 32 on the GPU path (0 -> 32) */
     uint32_t max_len;       /* code-length limit, 8..24 (0 -> 24) */
 } dfx_params;

@@ -21,7 +21,7 @@ struct dfx_plan_s {
 namespace {
 
 int resolve_params(const dfx_params* p, uint32_t* K, uint32_t* G, uint32_t* L) {
-    *K = (p && p->chunk_symbols) ? p->chunk_symbols : 64u;
+    *K = (p && p->chunk_symbols) ? p->chunk_symbols : 128u;
     *G = (p && p->group_chunks) ? p->group_chunks : 32u;
     *L = (p && p->max_len) ? p->max_len : 24u;
     if (*L < 8 || *L > dfx::kMaxLenLimit) return DFX_ERR_ARG;

@@ -48,7 +48,7 @@ uint8_t* g_scratch_addr[kMaxDevices] = {};
 extern "C" int dfx_encode_static(const void* d_bf16, uint64_t n, const dfx_params* params, void* d_out,
                                  size_t out_capacity, size_t* h_compressed_bytes, cudaStream_t stream) {
     if (n >= (1ull << 32)) return DFX_ERR_TOO_LARGE;
-    const uint32_t K = (params && params->chunk_symbols) ? params->chunk_symbols : 64u;
+    const uint32_t K = (params && params->chunk_symbols) ? params->chunk_symbols : 128u;
     const uint32_t G = (params && params->group_chunks) ? params->group_chunks : 32u;
     const uint32_t L = (params && params->max_len) ? params->max_len : 24u;
     if (L < 8 || L > dfx::kMaxLenLimit || K < 8 || K % 8 != 0) return DFX_ERR_ARG;

@@ -157,7 +157,7 @@ def test_truncated_buffer_is_a_host_error():
     w = inputs.gaussian(4097, 0.02, seed=8)
     c = oracle.encode(w, K=64)
     comp = torch.from_numpy(c).cuda()
-    with dfx.dfx_plan(w.size) as plan:
+    with dfx.dfx_plan(w.size, chunk_symbols=64) as plan:
         out = torch.empty(w.size, dtype=torch.int16, device="cuda")
         with pytest.raises(dfx.DfxError) as e:
             dfx.dfx_decode(plan, comp, 100, out)
@@ -171,6 +171,6 @@ def test_tensor_helpers_round_trip():
     w = inputs.gaussian(3 * 4096 + 5, 0.02, seed=9)
     x = to_dev(w).view(torch.bfloat16)
     comp = dfx.encode(x)
-    assert np.array_equal(comp.cpu().numpy(), oracle.encode(w))
+    assert np.array_equal(comp.cpu().numpy(), oracle.encode(w, K=128))  # the default chunk size
     y = dfx.decode(comp, w.size)
     assert torch.equal(y.view(torch.int16), x.view(torch.int16))
