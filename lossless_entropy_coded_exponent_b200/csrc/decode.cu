@@ -214,14 +214,6 @@ __device__ __noinline__ uint32_t decode_long(uint32_t peek, const Tables& T) {
 // of the other half.
 __device__ __forceinline__ uint32_t bf16_pair(uint32_t x) { return __funnelshift_r(x, x, 1); }
 
-__device__ __forceinline__ uint4 merge8(uint2 m, uint32_t e0, uint32_t e1) {
-    uint4 o;
-    o.x = bf16_pair(__byte_perm(m.x, e0, 0x5140));
-    o.y = bf16_pair(__byte_perm(m.x, e0, 0x7362));
-    o.z = bf16_pair(__byte_perm(m.y, e1, 0x5140));
-    o.w = bf16_pair(__byte_perm(m.y, e1, 0x7362));
-    return o;
-}
 
 
 // ---------------------------------------------------------------- group index
@@ -659,41 +651,65 @@ __device__ void decode_full_groups(const DecodeArgs& a, const Tables& T, const u
     }
 }
 
-// The last group when it is ragged: a lane's chunk holds the elements of its blocks
-// that are below n (a prefix of the chunk, possibly empty); outputs stop at n.
+// The blocks of the ragged last group: a lane's chunk holds the elements of its blocks
+// that are below n (a prefix of the chunk, possibly empty).  Whole blocks take the pair
+// path; the lane's last, partial block is decoded code by code and stored element-wise.
+template <int K, class Words>
+__device__ __forceinline__ void decode_tail_blocks(const DecodeArgs& a, const Tables& T, BitReader<Words>& br,
+                                                   uint32_t g, unsigned lane, uint32_t& err) {
+    const uint8_t* mplane = a.comp + a.off_m;
+    for (uint32_t k = 0; k < K / 8; k++) {
+        const uint64_t x0 = block_element(g, K, k, lane);
+        if (x0 + 8 <= a.n) {
+            reinterpret_cast<uint4*>(a.out)[x0 / 8] =
+                decode_block(br, T, __ldg(reinterpret_cast<const uint2*>(mplane + x0)), err);
+            continue;
+        }
+        if (x0 < a.n) {
+            const uint32_t cnt = (uint32_t)(a.n - x0);
+            br.reload();
+            for (uint32_t j = 0; j < cnt; j++) {  // decode and store one element at a time
+                const uint32_t ex = br.one(T, err);
+                const uint64_t x = x0 + j, partner = (x ^ 1u) < a.n ? (x ^ 1u) : x;
+                a.out[x] = (uint16_t)(((mplane[partner] & 1u) << 15) | (ex << 7) | (mplane[x] >> 1u));
+            }
+        }
+        break;
+    }
+}
+
+// The last group when it is ragged, by one warp after its full groups: its stream slice
+// is copied into the warp's (now idle) slice buffer when it fits, else read from global
+// memory with clamped loads.
 template <int K>
-__device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, const uint32_t* lut, uint32_t g,
-                                  unsigned lane, uint32_t& err) {
+__device__ void decode_tail_group(const DecodeArgs& a, const Tables& T, const uint32_t* lut, WarpBuffers<K>& wb,
+                                  uint32_t g, unsigned lane, uint32_t& err) {
     const GroupStart gs = scan_index(load_index(a, T, g, lane, true), lane);
     if (!gs.ok) {
         err |= DFX_STATUS_INDEX;
         return;
     }
-    const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
-    const uint32_t maxw = T.n_words - 1;
-    const uint32_t first = (uint32_t)(gs.gb0 >> 5);
-    const uint8_t* mplane = a.comp + a.off_m;
-    BitReader<ClampedGlobalWords> br;
-    br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, (uint32_t)(gs.start - 32ull * first));
-    br.reload();
-    for (uint32_t k = 0; k < K / 8; k++) {
-        const uint64_t x0 = block_element(g, K, k, lane);
-        if (x0 >= a.n) break;
-        const uint32_t cnt = (uint32_t)min((uint64_t)8, a.n - x0);
-        uint32_t e[2] = {0u, 0u};
-        for (uint32_t j = 0; j < cnt; j++) e[j >> 2] |= br.one(T, err) << (8 * (j & 3));
-        if (cnt == 8) {
-            reinterpret_cast<uint4*>(a.out)[x0 / 8] =
-                merge8(__ldg(reinterpret_cast<const uint2*>(mplane + x0)), e[0], e[1]);
-        } else {
-            for (uint32_t j = 0; j < cnt; j++) {
-                const uint64_t x = x0 + j, partner = (x ^ 1u) < a.n ? (x ^ 1u) : x;
-                const uint32_t ex = (e[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-                a.out[x] = (uint16_t)(((mplane[partner] & 1u) << 15) | (ex << 7) | (mplane[x] >> 1u));
-            }
-        }
+    const Slice sl = plan_slice<SliceShape<K>::kWords>(T, gs.gb0, gs.span, gs.ok);
+    uint32_t used;
+    if (sl.staged) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.comp + a.off_stream + 4u * sl.base);
+        uint4* dst = reinterpret_cast<uint4*>(wb.slice[0]);
+        for (uint32_t c = lane; c < sl.bytes / 16u; c += 32) dst[c] = __ldg(src + c);
+        __syncwarp();
+        BitReader<SharedWords> br;
+        br.init(lut, SharedWords{smem_addr(wb.slice[0])}, (uint32_t)(gs.start - 32ull * sl.base));
+        decode_tail_blocks<K>(a, T, br, g, lane, err);
+        used = br.consumed();
+    } else {
+        const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
+        const uint32_t maxw = T.n_words - 1;
+        const uint32_t first = (uint32_t)(gs.gb0 >> 5);
+        BitReader<ClampedGlobalWords> br;
+        br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, (uint32_t)(gs.start - 32ull * first));
+        decode_tail_blocks<K>(a, T, br, g, lane, err);
+        used = br.consumed();
     }
-    if (br.consumed() != gs.clen) err |= DFX_STATUS_STREAM;
+    if (used != gs.clen) err |= DFX_STATUS_STREAM;
 }
 
 constexpr size_t kLutBytes = sizeof(uint32_t) << kLutBits;
@@ -732,7 +748,7 @@ __device__ __forceinline__ void decode_tensor(const DecodeArgs& a, uint32_t cta,
     if (gw < n_full) group_prologue<K>(a, T, wb, gw, step, n_full, lane, gs);
     build_pair_table(T, lut);
     if (gw < n_full) decode_full_groups<K>(a, T, lut, wb, gs, step, n_full, lane, err);
-    if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, lut, n_full, lane, err);
+    if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, lut, wb, n_full, lane, err);
     if (err) atomicOr(a.status, err);
 }
 
