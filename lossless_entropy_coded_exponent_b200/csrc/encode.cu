@@ -47,39 +47,93 @@ __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long lon
 }
 
 // ---------------------------------------------------------------- 1. histogram
+//
+// The exponents of a weight tensor crowd into a few neighbouring values.  Each CTA
+// counts the first 16-byte load of each of its threads into a shared histogram and picks
+// the 8 consecutive exponents [b, b + 8) with the most of that sample.  From then on a
+// thread counts the values in that window in registers, four 8-bit counters per 32-bit
+// word (one shift and one add per value), and folds them into 32-bit counts every 31
+// loads, before a counter can pass 255 (31 x 8 values); values outside the window take
+// a shared-memory atomic.  64 warps per SM keep enough loads in flight.
 
-constexpr int kHistThreads = 512;
+constexpr int kHistThreads = 256;
+constexpr int kHistBlocksPerSm = 8;
 
-__global__ void __launch_bounds__(kHistThreads) k_histogram(const uint16_t* __restrict__ in, uint64_t n,
+__device__ __forceinline__ void fold8(uint32_t& c0, uint32_t& c1, uint32_t (&r)[8]) {
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        r[k] += (c0 >> (8 * k)) & 0xFFu;
+        r[k + 4] += (c1 >> (8 * k)) & 0xFFu;
+    }
+    c0 = c1 = 0u;
+}
+
+__global__ void __launch_bounds__(kHistThreads, kHistBlocksPerSm) k_histogram(const uint16_t* __restrict__ in, uint64_t n,
                                                           unsigned long long* __restrict__ counts) {
     __shared__ uint32_t h[256];
+    __shared__ uint32_t window;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0;
     __syncthreads();
-    const unsigned lane = threadIdx.x & 31;
     const uint4* in4 = reinterpret_cast<const uint4*>(in);
     const uint64_t n8 = n / 8;
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
-    // `base` is warp-uniform, so every lane reaches each __match_any_sync together.
-    for (uint64_t base = (uint64_t)blockIdx.x * blockDim.x; base < n8; base += stride) {
-        const uint64_t i = base + threadIdx.x;
-        const bool valid = i < n8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (valid) v = __ldg(in4 + i);
-        const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+    uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n8) {  // the sample (its counts are kept)
+        const uint4 v = __ldg(in4 + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int k = 0; k < 8; k++) {
-            const uint32_t e = valid ? ((words[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu) : 256u;
-            const unsigned peers = __match_any_sync(kFull, e);
-            if (e < 256u && lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&h[e], (uint32_t)__popc(peers));
-        }
+        for (int k = 0; k < 8; k++) atomicAdd(&h[(w[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu], 1u);
     }
-    if (blockIdx.x == 0 && threadIdx.x < (n & 7)) {
-        const uint64_t i = n8 * 8 + threadIdx.x;
-        atomicAdd(&h[(in[i] >> 7) & 0xFFu], 1u);
+    i += stride;
+    __syncthreads();
+    if (threadIdx.x < 32) {  // the window with the largest sample mass: lane l tries b = l + 32 j
+        uint32_t best = 0, best_b = 0;
+        for (uint32_t b = threadIdx.x; b <= 248; b += 32) {
+            uint32_t m = 0;
+            for (uint32_t k = 0; k < 8; k++) m += h[b + k];
+            if (m > best) {
+                best = m;
+                best_b = b;
+            }
+        }
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1) {
+            const uint32_t ob = __shfl_xor_sync(kFull, best, d), obb = __shfl_xor_sync(kFull, best_b, d);
+            if (ob > best || (ob == best && obb < best_b)) {
+                best = ob;
+                best_b = obb;
+            }
+        }
+        if (threadIdx.x == 0) window = best_b;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < 256; i += blockDim.x)
-        if (h[i]) atomicAdd(&counts[i], (unsigned long long)h[i]);
+    const uint32_t b = window;
+    uint32_t c0 = 0u, c1 = 0u, r[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    uint32_t since = 0;
+    for (; i < n8; i += stride) {
+        const uint4 v = __ldg(in4 + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            const uint32_t e = (w[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu;
+            const uint32_t d = e - b;
+            if (d < 4u) c0 += 1u << (8 * d);
+            else if (d < 8u) c1 += 1u << (8 * (d - 4u));
+            else atomicAdd(&h[e], 1u);
+        }
+        if (++since == 31) {
+            fold8(c0, c1, r);
+            since = 0;
+        }
+    }
+    fold8(c0, c1, r);
+#pragma unroll
+    for (int k = 0; k < 8; k++)
+        if (r[k]) atomicAdd(&h[b + k], r[k]);
+    if (blockIdx.x == 0 && threadIdx.x < (n & 7)) atomicAdd(&h[(in[n8 * 8 + threadIdx.x] >> 7) & 0xFFu], 1u);
+    __syncthreads();
+    for (int k = threadIdx.x; k < 256; k += blockDim.x)
+        if (h[k]) atomicAdd(&counts[k], (unsigned long long)h[k]);
 }
 
 // ---------------------------------------------------------------- 2. code book
@@ -269,7 +323,7 @@ __global__ void __launch_bounds__(kChunkThreads) k_chunk_bits(EncodeArgs a) {
 // ---------------------------------------------------------------- 4. group scan
 
 constexpr int kScanThreads = 1024;
-constexpr int kScanItems = 4;
+constexpr int kScanItems = 16;  // four 16-byte loads per thread per round
 
 __global__ void __launch_bounds__(kScanThreads) k_group_scan(EncodeArgs a) {
     __shared__ unsigned long long wsum[32];
@@ -280,11 +334,22 @@ __global__ void __launch_bounds__(kScanThreads) k_group_scan(EncodeArgs a) {
         const uint64_t i = base + (uint64_t)t * kScanItems;
         uint32_t v[kScanItems];
         unsigned long long local = 0;
+        if (i + kScanItems <= a.n_group) {  // the group sums start 16-byte aligned in the workspace
+            const uint4* q = reinterpret_cast<const uint4*>(a.ws_group_bits + i);
 #pragma unroll
-        for (int k = 0; k < kScanItems; k++) {
-            v[k] = (i + k < a.n_group) ? a.ws_group_bits[i + k] : 0u;
-            local += v[k];
+            for (int k = 0; k < kScanItems / 4; k++) {
+                const uint4 x = q[k];
+                v[4 * k] = x.x;
+                v[4 * k + 1] = x.y;
+                v[4 * k + 2] = x.z;
+                v[4 * k + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < kScanItems; k++) v[k] = (i + k < a.n_group) ? a.ws_group_bits[i + k] : 0u;
         }
+#pragma unroll
+        for (int k = 0; k < kScanItems; k++) local += v[k];
         const unsigned long long incl = warp_incl_scan64(local, lane);
         if (lane == 31) wsum[warp] = incl;
         __syncthreads();
@@ -369,10 +434,20 @@ __global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
     bw.first = true;
     uint8_t* mpl = a.out + a.off_m;
 
-    for (uint32_t k = 0; k < K / 8; k++) {
-        const uint64_t x0 = block_element(c / 32, K, k, lane);
-        if (x0 + 8 <= a.n) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.in + x0));
+    // the chunk's whole blocks (a prefix of its K/8 blocks), their loads one block ahead
+    const uint64_t g = c / 32;
+    uint32_t full = K / 8;
+    if ((g + 1) * 32ull * K > a.n) {
+        full = 0;
+        while (full < K / 8 && block_element(g, K, full, lane) + 8 <= a.n) full++;
+    }
+    uint4 v_next = make_uint4(0u, 0u, 0u, 0u);
+    if (full) v_next = __ldg(reinterpret_cast<const uint4*>(a.in + block_element(g, K, 0, lane)));
+    for (uint32_t k = 0; k <= full && k < K / 8; k++) {
+        const uint64_t x0 = block_element(g, K, k, lane);
+        if (k < full) {
+            const uint4 v = v_next;
+            if (k + 1 < full) v_next = __ldg(reinterpret_cast<const uint4*>(a.in + block_element(g, K, k + 1, lane)));
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             uint32_t mb[2] = {0u, 0u};
 #pragma unroll
@@ -384,7 +459,7 @@ __global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
                 mb[j >> 2] |= (((h & 0x7Fu) << 1) | (partner >> 15)) << (8 * (j & 3));
             }
             *reinterpret_cast<uint2*>(mpl + x0) = make_uint2(mb[0], mb[1]);
-        } else {
+        } else {  // the partial block, if any
             for (uint64_t x = x0; x < a.n; x++) {
                 const uint32_t h = a.in[x];
                 const uint32_t partner = a.in[(x ^ 1u) < a.n ? (x ^ 1u) : x];
@@ -419,7 +494,8 @@ cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t 
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const uint64_t units = (a.n / 8 + kHistThreads - 1) / kHistThreads;
-    const unsigned hist_blocks = (unsigned)(units == 0 ? 1 : (units < (uint64_t)sms * 4 ? units : (uint64_t)sms * 4));
+    const uint64_t resident = (uint64_t)sms * kHistBlocksPerSm;
+    const unsigned hist_blocks = (unsigned)(units == 0 ? 1 : (units < resident ? units : resident));
     k_histogram<<<hist_blocks, kHistThreads, 0, s>>>(a.in, a.n, a.ws_counts);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     k_build_codebook<<<1, 256, 0, s>>>(a);

@@ -174,3 +174,29 @@ def test_tensor_helpers_round_trip():
     assert np.array_equal(comp.cpu().numpy(), oracle.encode(w, K=128))  # the default chunk size
     y = dfx.decode(comp, w.size)
     assert torch.equal(y.view(torch.int16), x.view(torch.int16))
+
+
+HIST_CASES = {
+    "small_gaussian": lambda: inputs.small_gaussian(),
+    "layer70b_sample": lambda: inputs.layer70b_sample(1 << 22, 3),
+    "uniform_patterns": lambda: inputs.uniform_patterns(1 << 20, 21),
+    "special_mix": lambda: inputs.special_mix(1 << 20, 22),
+    "all_patterns": lambda: inputs.all_patterns_shuffled(23),
+    "seven": lambda: inputs.gaussian(7, 0.02, seed=24),
+    "ragged": lambda: inputs.gaussian(1_000_003, 0.02, seed=25),
+}
+
+
+@pytest.mark.parametrize("name", list(HIST_CASES))
+def test_exponent_histogram_counts(name):
+    """The encoder's exponent counts (u64[256] at the start of the workspace, where the
+    encode leaves them) equal a plain count of the exponents."""
+    w = HIST_CASES[name]()
+    x = to_dev(w)
+    with dfx.dfx_plan(w.size) as plan:
+        out = torch.empty(plan.max_compressed_bytes, dtype=torch.uint8, device="cuda")
+        ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+        dfx.dfx_encode(plan, x, out, out.numel(), ws, ws.numel(), want_size=True)
+        counts = ws[:2048].cpu().numpy().view(np.uint64)
+    ref = np.bincount(((w >> 7) & 0xFF).astype(np.int64), minlength=256).astype(np.uint64)
+    assert np.array_equal(counts, ref)
