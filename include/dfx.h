@@ -151,6 +151,22 @@ int dfx_encode(dfx_plan_t plan, const void *d_bf16, void *d_out, size_t out_capa
 int dfx_decode(dfx_plan_t plan, const void *d_comp, size_t comp_bytes, void *d_bf16,
                cudaStream_t stream);
 
+/* Decode part of a container: the elements of groups [first_group, first_group +
+ * group_count) (a group is 32 chunks of chunk_symbols elements, so rows of a
+ * weight matrix whose length is a multiple of 32 * chunk_symbols are whole
+ * groups) into d_bf16, which receives element first_group * 32 *
+ * chunk_symbols at d_bf16[0] and ends at element n at the latest.  This lets a
+ * caller restore a weight matrix slice by slice into a small (L2-sized) buffer
+ * just before the computation that reads it, instead of writing the whole BF16
+ * tensor to HBM (the pages decode weights on the GPU ahead of the computation
+ * that uses them: "DFloat11: lossless LLM compression for GPU", section 02).
+ * d_comp, comp_bytes: the whole container, as for dfx_decode (its header and
+ * index are checked every call).  A range past the last group returns
+ * DFX_ERR_ARG; group_count = 0 is a no-op.  Asynchronous; one kernel launch with
+ * a CTA per 32 groups up to one per SM. */
+int dfx_decode_range(dfx_plan_t plan, const void *d_comp, size_t comp_bytes, uint64_t first_group,
+                     uint64_t group_count, void *d_bf16, cudaStream_t stream);
+
 /* Decode `count` containers (1..32; 0 is a no-op) with one kernel launch: a
  * whole layer's weights restored before use in one go (the pages decode a
  * model's compressed weights on the GPU ahead of the computation that reads

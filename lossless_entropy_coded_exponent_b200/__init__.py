@@ -37,6 +37,7 @@ EXPORTS = (
     "dfx_plan",
     "dfx_encode",
     "dfx_decode",
+    "dfx_decode_range",
     "dfx_decode_batch",
     "dfx_device_status",
     "dfx_free",
@@ -83,13 +84,14 @@ def lib() -> ctypes.CDLL:
                                ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
         L.dfx_encode.argtypes = [vp, vp, vp, ctypes.c_size_t, vp, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t), vp]
         L.dfx_decode.argtypes = [vp, vp, ctypes.c_size_t, vp, vp]
+        L.dfx_decode_range.argtypes = [vp, vp, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_uint64, vp, vp]
         L.dfx_decode_batch.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_size_t),
                                        ctypes.POINTER(vp), ctypes.c_uint32, vp]
         L.dfx_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.dfx_free.argtypes = [vp]
         L.dfx_encode_static.argtypes = [vp, ctypes.c_uint64, ctypes.POINTER(dfx_params), vp, ctypes.c_size_t,
                                         ctypes.POINTER(ctypes.c_size_t), vp]
-        for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_decode_batch",
+        for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_decode_range", "dfx_decode_batch",
                   "dfx_device_status", "dfx_free", "dfx_encode_static"):
             getattr(L, f).restype = ctypes.c_int
         _lib_handle = L
@@ -185,6 +187,22 @@ def dfx_encode(plan: Plan, d_bf16, d_out, out_capacity: int, d_workspace, worksp
 
 def dfx_decode(plan: Plan, d_comp, comp_bytes: int, d_bf16, stream=None) -> None:
     _check(lib().dfx_decode(plan.handle, _ptr(d_comp), comp_bytes, _ptr(d_bf16), _stream(stream)), "dfx_decode")
+
+
+DEFAULT_CHUNK_SYMBOLS = 128  # dfx_params.chunk_symbols = 0 means this (include/dfx.h)
+
+
+def group_elements(plan: Plan) -> int:
+    """Elements per group of the plan's containers (32 chunks of chunk_symbols)."""
+    return 32 * (plan.params[0] or DEFAULT_CHUNK_SYMBOLS)
+
+
+def dfx_decode_range(plan: Plan, d_comp, comp_bytes: int, first_group: int, group_count: int, d_bf16,
+                     stream=None) -> None:
+    """Decode groups [first_group, first_group + group_count) into d_bf16 (which holds
+    element first_group * 32 * chunk_symbols at index 0)."""
+    _check(lib().dfx_decode_range(plan.handle, _ptr(d_comp), comp_bytes, first_group, group_count, _ptr(d_bf16),
+                                  _stream(stream)), "dfx_decode_range")
 
 
 def dfx_decode_batch(plans, d_comps, comp_bytes, d_bf16s, stream=None) -> None:

@@ -173,6 +173,26 @@ int dfx_decode(dfx_plan_t plan, const void* d_comp, size_t comp_bytes, void* d_b
     return DFX_OK;
 }
 
+int dfx_decode_range(dfx_plan_t plan, const void* d_comp, size_t comp_bytes, uint64_t first_group,
+                     uint64_t group_count, void* d_bf16, cudaStream_t stream) {
+    if (!plan) return DFX_ERR_ARG;
+    if (first_group > plan->L.n_group || group_count > plan->L.n_group - first_group) return DFX_ERR_ARG;
+    if (group_count == 0) return DFX_OK;
+    dfx::DecodeArgs a;
+    const int rc = make_decode_args(plan, d_comp, comp_bytes, d_bf16, &a);
+    if (rc) return rc;
+    a.g_begin = (uint32_t)first_group;
+    a.g_end = (uint32_t)(first_group + group_count);
+    a.out_first = first_group * (uint64_t)plan->G * plan->K;
+    const uint64_t need = (group_count + 31) / 32;  // a warp per group
+    const int grid = (int)(need < (uint64_t)plan->resident_ctas ? need : (uint64_t)plan->resident_ctas);
+    if (dfx::launch_decode(a, grid, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return DFX_ERR_CUDA;
+    }
+    return DFX_OK;
+}
+
 int dfx_decode_batch(const dfx_plan_t* plans, const void* const* d_comps, const size_t* comp_bytes,
                      void* const* d_bf16s, uint32_t count, cudaStream_t stream) {
     if (count == 0) return DFX_OK;
@@ -258,6 +278,9 @@ int make_decode_args(const dfx_plan_s* plan, const void* d_comp, size_t comp_byt
     a->off_m = plan->L.off_m;
     a->off_stream = plan->L.off_stream;
     a->status = plan->d_status;
+    a->g_begin = 0;
+    a->g_end = (uint32_t)plan->L.n_group;
+    a->out_first = 0;
     return DFX_OK;
 }
 

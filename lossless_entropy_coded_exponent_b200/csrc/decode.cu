@@ -517,7 +517,7 @@ template <int K, class Words>
 __device__ __forceinline__ void decode_group_blocks(const DecodeArgs& a, const Tables& T, BitReader<Words>* br,
                                                     WarpBuffers<K>& wb, MPipe<K>& mp, uint32_t g, unsigned lane,
                                                     uint32_t& err) {
-    uint4* op = reinterpret_cast<uint4*>(a.out) + (uint64_t)g * (32u * K / 8u) + lane;
+    uint4* op = reinterpret_cast<uint4*>(a.out) + ((uint64_t)g * (32u * K) - a.out_first) / 8u + lane;
     for (uint32_t u = 0; u < MPipe<K>::U; u++) {
         const uint32_t slot = mp.j % kMUnits;
         if (!mbar_wait(&wb.mbar[2 + slot], (mp.j / kMUnits) & 1u)) err |= DFX_STATUS_TIMEOUT;
@@ -661,7 +661,7 @@ __device__ __forceinline__ void decode_tail_blocks(const DecodeArgs& a, const Ta
     for (uint32_t k = 0; k < K / 8; k++) {
         const uint64_t x0 = block_element(g, K, k, lane);
         if (x0 + 8 <= a.n) {
-            reinterpret_cast<uint4*>(a.out)[x0 / 8] =
+            reinterpret_cast<uint4*>(a.out)[(x0 - a.out_first) / 8] =
                 decode_block(br, T, __ldg(reinterpret_cast<const uint2*>(mplane + x0)), err);
             continue;
         }
@@ -671,7 +671,7 @@ __device__ __forceinline__ void decode_tail_blocks(const DecodeArgs& a, const Ta
             for (uint32_t j = 0; j < cnt; j++) {  // decode and store one element at a time
                 const uint32_t ex = br.one(T, err);
                 const uint64_t x = x0 + j, partner = (x ^ 1u) < a.n ? (x ^ 1u) : x;
-                a.out[x] = (uint16_t)(((mplane[partner] & 1u) << 15) | (ex << 7) | (mplane[x] >> 1u));
+                a.out[x - a.out_first] = (uint16_t)(((mplane[partner] & 1u) << 15) | (ex << 7) | (mplane[x] >> 1u));
             }
         }
         break;
@@ -725,11 +725,12 @@ __device__ __forceinline__ void decode_tensor(const DecodeArgs& a, uint32_t cta,
     uint32_t* lut = reinterpret_cast<uint32_t*>(dyn_smem);
     uint8_t* warp_area = dyn_smem + kLutBytes;
     const uint32_t n_full = (a.n % (32ull * K) == 0) ? a.n_group : a.n_group - 1;
+    const uint32_t full_end = min(n_full, a.g_end);  // full groups to decode: [g_begin, full_end)
     {
         // start fetching each warp's first group (index entries, m plane) into L2 while
         // the tables are built
-        const uint32_t g0 = cta + ctas * (threadIdx.x >> 5);
-        if ((threadIdx.x & 31) == 0 && g0 < n_full) {
+        const uint32_t g0 = a.g_begin + cta + ctas * (threadIdx.x >> 5);
+        if ((threadIdx.x & 31) == 0 && g0 < full_end) {
             prefetch_line_l2(a.comp + kOffGbase + 8ull * g0);
             prefetch_line_l2(a.comp + a.off_clen + 64ull * g0);
             prefetch_line_l2(a.comp + a.off_clen + 64ull * g0 + 63);
@@ -743,12 +744,14 @@ __device__ __forceinline__ void decode_tensor(const DecodeArgs& a, uint32_t cta,
     const uint32_t step = ctas * kDecodeWarps;
     // groups are dealt to the CTAs (one per SM) in turn and each CTA's to its warps in
     // turn, so that every SM gets the same number of groups within one
-    const uint32_t gw = cta + ctas * warp;
+    const uint32_t gw = a.g_begin + cta + ctas * warp;
     GroupState<K> gs;
-    if (gw < n_full) group_prologue<K>(a, T, wb, gw, step, n_full, lane, gs);
+    if (gw < full_end) group_prologue<K>(a, T, wb, gw, step, full_end, lane, gs);
     build_pair_table(T, lut);
-    if (gw < n_full) decode_full_groups<K>(a, T, lut, wb, gs, step, n_full, lane, err);
-    if (n_full < a.n_group && gw == n_full % step) decode_tail_group<K>(a, T, lut, wb, n_full, lane, err);
+    if (gw < full_end) decode_full_groups<K>(a, T, lut, wb, gs, step, full_end, lane, err);
+    // the ragged last group, by the warp whose sequence it would continue
+    if (n_full < a.n_group && n_full >= a.g_begin && n_full < a.g_end && gw == a.g_begin + (n_full - a.g_begin) % step)
+        decode_tail_group<K>(a, T, lut, wb, n_full, lane, err);
     if (err) atomicOr(a.status, err);
 }
 

@@ -56,6 +56,8 @@ struct DecodeArgs {
     uint32_t n_chunk, n_group;
     uint64_t off_clen, off_m, off_stream;
     uint32_t* status;
+    uint32_t g_begin, g_end;  // groups to decode (all: 0, n_group)
+    uint64_t out_first;       // element index stored at out[0] (g_begin * G * K)
 };
 
 struct EncodeArgs {

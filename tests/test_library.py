@@ -100,3 +100,7 @@ def test_batch_argument_errors_precede_cuda(lib):
     assert lib.dfx_decode_batch(arr, arr, sizes, arr, 2, None) == dfx.DFX_ERR_ARG  # null plans
     with pytest.raises(ValueError):
         dfx.dfx_decode_batch([None], [], [], [])
+
+
+def test_range_argument_errors_precede_cuda(lib):
+    assert lib.dfx_decode_range(None, None, 0, 0, 1, None, None) == dfx.DFX_ERR_ARG
