@@ -375,9 +375,27 @@ __global__ void __launch_bounds__(kScanThreads) k_group_scan(EncodeArgs a) {
 // ---------------------------------------------------------------- 5. pack
 
 constexpr int kPackThreads = 256;
+constexpr uint32_t kPackSliceWords = 1024;  // a group's stream words staged per warp (4 KiB)
 
-struct BitWriter {
+// Where a chunk's packed words go: the stream in global memory, or the warp's shared
+// copy of its group's words.  The first word of a chunk and its last, partial word may
+// hold bits of the neighbouring chunks and are OR-ed in; the words between belong to the
+// chunk alone.
+struct GlobalSink {
     uint32_t* stream;
+    __device__ __forceinline__ void shared_word(uint64_t wi, uint32_t v) const { atomicOr(stream + wi, v); }
+    __device__ __forceinline__ void own_word(uint64_t wi, uint32_t v) const { stream[wi] = v; }
+};
+struct SharedSink {
+    uint32_t* words;  // the group's first stream word is words[0]
+    uint64_t base;
+    __device__ __forceinline__ void shared_word(uint64_t wi, uint32_t v) const { atomicOr(words + (wi - base), v); }
+    __device__ __forceinline__ void own_word(uint64_t wi, uint32_t v) const { words[wi - base] = v; }
+};
+
+template <class Sink>
+struct BitWriter {
+    Sink sink;
     uint64_t wi;     // index of the word being assembled
     uint32_t fill;   // bits already in `cur`
     uint32_t cur;
@@ -385,10 +403,10 @@ struct BitWriter {
 
     __device__ __forceinline__ void emit() {
         if (first) {
-            atomicOr(stream + wi, cur);
+            sink.shared_word(wi, cur);
             first = false;
         } else {
-            stream[wi] = cur;
+            sink.own_word(wi, cur);
         }
         wi++;
     }
@@ -406,28 +424,17 @@ struct BitWriter {
         }
     }
     __device__ __forceinline__ void finish() {
-        if (fill) atomicOr(stream + wi, cur);  // shared with the next chunk
+        if (fill) sink.shared_word(wi, cur);  // shared with the next chunk
     }
 };
 
-template <int K>
-__global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
-    __shared__ uint32_t code_sh[256];
-    __shared__ uint8_t len_sh[256];
-    code_sh[threadIdx.x] = a.ws_code[threadIdx.x];
-    len_sh[threadIdx.x] = a.ws_len[threadIdx.x];
-    __syncthreads();
-    const uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const unsigned lane = threadIdx.x & 31;
-    const uint16_t* clen = reinterpret_cast<const uint16_t*>(a.out + a.off_clen);
-    const uint32_t cl = (c < a.n_chunk) ? clen[c] : 0u;
-    const uint32_t incl = warp_incl_scan(cl, lane);
-    if (c >= a.n_chunk) return;
-    const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.out + kOffGbase);
-    const uint64_t start = gbase[c / 32] + (incl - cl);
-
-    BitWriter bw;
-    bw.stream = reinterpret_cast<uint32_t*>(a.out + a.off_stream);
+// Pack chunk c (lane `lane` of group c / 32), whose codes start at stream bit `start`,
+// and write its elements' mantissa+sign bytes.
+template <int K, class Sink>
+__device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* code_sh, const uint8_t* len_sh,
+                                           uint64_t c, unsigned lane, uint64_t start, Sink sink) {
+    BitWriter<Sink> bw;
+    bw.sink = sink;
     bw.wi = start >> 5;
     bw.fill = (uint32_t)(start & 31);
     bw.cur = 0;
@@ -471,6 +478,50 @@ __global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
         }
     }
     bw.finish();
+}
+
+// One warp per group: the lanes pack their chunks into the warp's shared copy of the
+// group's stream words, which the warp then writes out with coalesced stores (the group's
+// first and last words, which it may share with the neighbouring groups, are OR-ed in).
+// A group whose words do not fit the copy is packed straight into global memory.
+template <int K>
+__global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
+    __shared__ uint32_t code_sh[256];
+    __shared__ uint8_t len_sh[256];
+    __shared__ uint32_t slice[kPackThreads / 32][kPackSliceWords];
+    code_sh[threadIdx.x] = a.ws_code[threadIdx.x];
+    len_sh[threadIdx.x] = a.ws_len[threadIdx.x];
+    __syncthreads();
+    const uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const unsigned lane = threadIdx.x & 31;
+    if (c >= a.n_chunk) return;  // n_chunk is a multiple of 32: whole warps leave
+    const uint16_t* clen = reinterpret_cast<const uint16_t*>(a.out + a.off_clen);
+    const uint32_t cl = clen[c];
+    const uint32_t incl = warp_incl_scan(cl, lane);
+    const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.out + kOffGbase);
+    const uint64_t gb0 = gbase[c / 32];
+    const uint64_t start = gb0 + (incl - cl);
+    uint32_t* stream = reinterpret_cast<uint32_t*>(a.out + a.off_stream);
+    const uint32_t group_bits = __shfl_sync(kFull, incl, 31);
+    const uint64_t wf = gb0 >> 5, wl = (gb0 + group_bits + 31) >> 5;  // the group's words [wf, wl)
+    const uint32_t count = (uint32_t)(wl - wf);
+    if (count <= kPackSliceWords) {
+        uint32_t* sm = slice[threadIdx.x >> 5];
+        for (uint32_t i = lane; i < count; i += 32) sm[i] = 0u;
+        __syncwarp();
+        pack_chunk<K>(a, code_sh, len_sh, c, lane, start, SharedSink{sm, wf});
+        __syncwarp();
+        for (uint32_t i = lane; i < count; i += 32) {
+            const uint32_t v = sm[i];
+            if (i == 0 || i + 1 == count) {
+                if (v) atomicOr(stream + wf + i, v);
+            } else {
+                stream[wf + i] = v;
+            }
+        }
+    } else {
+        pack_chunk<K>(a, code_sh, len_sh, c, lane, start, GlobalSink{stream});
+    }
 }
 
 template <int K>
