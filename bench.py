@@ -386,6 +386,8 @@ def run_ours(args, world, rank, local):
     # ---- end to end through the C ABI with host buffers
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, plan, comps, sizes, n, dev, world)
+        if rank == 0:
+            line["offload"] = run_offload(plan, comps, sizes, xs, n, dev)
     # ---- several tensors per launch: a Llama-3-8B-shaped layer
     if not args.no_layer_batch and rank == 0:
         line["layer_batch"] = run_layer_batch(args, dev, stream)
@@ -559,6 +561,57 @@ def run_decode_into_gemm(args, dev, tokens=16, slice_rows=3584):
         plan.free()
 
 
+def run_offload(plan, comps, sizes, xs, n, dev, tensors=4, slices=8):
+    """Weights kept in pinned host memory and brought to the GPU: raw BF16 copied over
+    the host link, against the containers streamed with dfx_decode_host (copies of a
+    tensor's slices overlapped with their decoding, two staging buffers)."""
+    import torch
+
+    import lossless_entropy_coded_exponent_b200 as dfx
+
+    T = min(tensors, len(comps))
+    host_c = [comps[i].cpu().pin_memory() for i in range(T)]
+    host_x = [xs[i].cpu().pin_memory() for i in range(T)]
+    cap = max(sizes[:T])
+    staging = [torch.empty(cap, dtype=torch.uint8, device=dev) for _ in range(2)]
+    out = torch.empty(n, dtype=torch.int16, device=dev)
+    s_copy, s_dec = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def raw():
+        with torch.cuda.stream(s_copy):
+            for i in range(T):
+                out.copy_(host_x[i], non_blocking=True)
+        s_copy.synchronize()
+
+    def compressed():
+        for i in range(T):
+            s_copy.wait_stream(s_dec)  # staging[i % 2] was read by the decode two tensors back
+            dfx.dfx_decode_host(plan, host_c[i], sizes[i], staging[i % 2], cap, out, slices=slices,
+                                copy_stream=s_copy, decode_stream=s_dec)
+        s_dec.synchronize()
+
+    def wall(fn, reps=3):
+        fn()
+        best = float("inf")
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            fn()
+            best = min(best, time.perf_counter() - t0)
+        return best
+
+    dfx.dfx_device_status(plan)  # start from a clear status word
+    t_raw, t_comp = wall(raw), wall(compressed)
+    equal = bool(torch.equal(out, xs[T - 1]))
+    status = dfx.dfx_device_status(plan, stream=s_dec)
+    exact = equal and status == 0
+    return {"tensors": T, "bf16_bytes_per_tensor": 2 * n, "container_bytes_per_tensor": float(sum(sizes[:T])) / T,
+            "raw_bf16_h2d_gbs": 2.0 * n * T / t_raw / 1e9, "compressed_stream_gbs": 2.0 * n * T / t_comp / 1e9,
+            "speedup": t_raw / t_comp, "bit_exact": exact, "last_tensor_equal": equal, "device_status": status,
+            "slices_per_tensor": slices,
+            "note": "GB/s of BF16 delivered to the device from pinned host memory (best of 3, host wall clock "
+                    "around a synchronised pass over the tensors)"}
+
+
 def run_e2e(args, plan, comps, sizes, n, dev, world):
     """Containers in pinned host memory; per tensor: H2D copy, dfx_decode, D2H
     copy of the BF16 result, on three streams so copies overlap decoding."""
@@ -574,31 +627,31 @@ def run_e2e(args, plan, comps, sizes, n, dev, world):
     dev_o = [torch.empty(n, dtype=torch.int16, device=dev) for _ in range(2)]
     s_in, s_dec, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
 
+    # per double-buffer slot, the last decode that read dev_c[b] and the last copy that
+    # read dev_o[b], carried across steps: a slot is refilled only after both
+    dec_done, d2h_done = [None, None], [None, None]
+
     def one_step():
-        h2d_done, dec_done, d2h_done = [], [], []
         for i in range(T):
             b = i % 2
-            if i >= 2:
-                s_in.wait_event(dec_done[i - 2])
+            if dec_done[b] is not None:
+                s_in.wait_event(dec_done[b])
             with torch.cuda.stream(s_in):
                 dev_c[b][: sizes[i]].copy_(host_c[i], non_blocking=True)
             ev = torch.cuda.Event()
             ev.record(s_in)
-            h2d_done.append(ev)
             s_dec.wait_event(ev)
-            if i >= 2:
-                s_dec.wait_event(d2h_done[i - 2])
+            if d2h_done[b] is not None:
+                s_dec.wait_event(d2h_done[b])
             dfx.dfx_decode(plan, dev_c[b], sizes[i], dev_o[b], stream=s_dec)
-            ev = torch.cuda.Event()
-            ev.record(s_dec)
-            dec_done.append(ev)
-            s_out.wait_event(ev)
+            dec_done[b] = torch.cuda.Event()
+            dec_done[b].record(s_dec)
+            s_out.wait_event(dec_done[b])
             with torch.cuda.stream(s_out):
                 host_out.copy_(dev_o[b], non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(s_out)
-            d2h_done.append(ev)
-        return d2h_done[-1]
+            d2h_done[b] = torch.cuda.Event()
+            d2h_done[b].record(s_out)
+        return d2h_done[(T - 1) % 2]
 
     last = one_step()  # warm-up
     last.synchronize()
@@ -617,9 +670,10 @@ def run_e2e(args, plan, comps, sizes, n, dev, world):
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(start.elapsed_time(end), world)
     barrier(world)
+    status = dfx.dfx_device_status(plan, stream=s_dec)
     value = sum_over_ranks(2.0 * n * T * args.e2e_steps, world) / (ms * 1e-3) / 1e9
     return {"value": value, "unit": UNIT, "h2d_bytes_per_step": int(sum(sizes)), "d2h_bytes_per_step": int(2 * n * T),
-            "ms_per_step": ms / args.e2e_steps, "steps": args.e2e_steps,
+            "ms_per_step": ms / args.e2e_steps, "steps": args.e2e_steps, "device_status": status,
             "note": "pinned host containers -> H2D -> dfx_decode -> D2H of the BF16 result, copies overlapped"}
 
 

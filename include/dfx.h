@@ -167,6 +167,29 @@ int dfx_decode(dfx_plan_t plan, const void *d_comp, size_t comp_bytes, void *d_b
 int dfx_decode_range(dfx_plan_t plan, const void *d_comp, size_t comp_bytes, uint64_t first_group,
                      uint64_t group_count, void *d_bf16, cudaStream_t stream);
 
+/* Decode a container that sits in host memory, streaming it to the device while
+ * it decodes: the weights of a model kept in host memory and brought to the GPU
+ * compressed, so the host link carries the container instead of the BF16 tensor.
+ * The pages name the slow host-to-GPU link as what limits offloaded weights
+ * ("DFloat11: lossless LLM compression for GPU", section 01) and shorten that
+ * transfer by sending the weights compressed (the Endor abstract, for pruned
+ * weights).  The header and index are copied first, then the groups in
+ * `slices` runs (0 -> 8, at most 64): each run's sign+mantissa bytes and stream
+ * words are copied with cudaMemcpyAsync on copy_stream and decoded with
+ * dfx_decode_range on decode_stream once they have landed, so copies and decoding
+ * overlap.
+ *   h_comp: the container in host memory (pinned, for the copies to run
+ *   asynchronously), comp_bytes long; d_staging: device buffer of staging_bytes
+ *   >= the container's size (16-byte aligned), which receives the container;
+ *   d_bf16: the n BF16 outputs.  The host reads the container's size and group
+ *   index directly from h_comp.  Errors as for dfx_decode; staging too small ->
+ *   DFX_ERR_CAPACITY.  The plan's slice events order copies and decoding, so
+ *   calls on the same plan must not overlap.  Returns after queueing the work;
+ *   h_comp must stay valid until copy_stream has finished it. */
+int dfx_decode_host(dfx_plan_t plan, const void *h_comp, size_t comp_bytes, void *d_staging,
+                    size_t staging_bytes, void *d_bf16, uint32_t slices, cudaStream_t copy_stream,
+                    cudaStream_t decode_stream);
+
 /* Decode `count` containers (1..32; 0 is a no-op) with one kernel launch: a
  * whole layer's weights restored before use in one go (the pages decode a
  * model's compressed weights on the GPU ahead of the computation that reads

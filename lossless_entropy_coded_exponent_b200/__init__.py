@@ -38,6 +38,7 @@ EXPORTS = (
     "dfx_encode",
     "dfx_decode",
     "dfx_decode_range",
+    "dfx_decode_host",
     "dfx_decode_batch",
     "dfx_device_status",
     "dfx_free",
@@ -85,13 +86,14 @@ def lib() -> ctypes.CDLL:
         L.dfx_encode.argtypes = [vp, vp, vp, ctypes.c_size_t, vp, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t), vp]
         L.dfx_decode.argtypes = [vp, vp, ctypes.c_size_t, vp, vp]
         L.dfx_decode_range.argtypes = [vp, vp, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_uint64, vp, vp]
+        L.dfx_decode_host.argtypes = [vp, vp, ctypes.c_size_t, vp, ctypes.c_size_t, vp, ctypes.c_uint32, vp, vp]
         L.dfx_decode_batch.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_size_t),
                                        ctypes.POINTER(vp), ctypes.c_uint32, vp]
         L.dfx_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.dfx_free.argtypes = [vp]
         L.dfx_encode_static.argtypes = [vp, ctypes.c_uint64, ctypes.POINTER(dfx_params), vp, ctypes.c_size_t,
                                         ctypes.POINTER(ctypes.c_size_t), vp]
-        for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_decode_range", "dfx_decode_batch",
+        for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_decode_range", "dfx_decode_host", "dfx_decode_batch",
                   "dfx_device_status", "dfx_free", "dfx_encode_static"):
             getattr(L, f).restype = ctypes.c_int
         _lib_handle = L
@@ -203,6 +205,15 @@ def dfx_decode_range(plan: Plan, d_comp, comp_bytes: int, first_group: int, grou
     element first_group * 32 * chunk_symbols at index 0)."""
     _check(lib().dfx_decode_range(plan.handle, _ptr(d_comp), comp_bytes, first_group, group_count, _ptr(d_bf16),
                                   _stream(stream)), "dfx_decode_range")
+
+
+def dfx_decode_host(plan: Plan, h_comp, comp_bytes: int, d_staging, staging_bytes: int, d_bf16, slices: int = 0,
+                    copy_stream=None, decode_stream=None) -> None:
+    """Stream a container in (pinned) host memory to d_staging slice by slice while
+    decoding the slices into d_bf16 (copies on copy_stream, decoding on decode_stream)."""
+    _check(lib().dfx_decode_host(plan.handle, _ptr(h_comp), comp_bytes, _ptr(d_staging), staging_bytes,
+                                 _ptr(d_bf16), slices, _stream(copy_stream), _stream(decode_stream)),
+           "dfx_decode_host")
 
 
 def dfx_decode_batch(plans, d_comps, comp_bytes, d_bf16s, stream=None) -> None:

@@ -2,6 +2,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include "dfx.h"
 #include "dfx_common.cuh"
@@ -16,6 +17,11 @@ struct dfx_plan_s {
     int device;
     int decode_grid;
     int resident_ctas;  // decode CTAs that fit on the device at once
+    // events ordering dfx_decode_host's copies before the decode of their slices,
+    // created on first use
+    static constexpr uint32_t kHostSlicesMax = 64;
+    cudaEvent_t slice_done[kHostSlicesMax];
+    bool events_made;
 };
 
 namespace {
@@ -193,6 +199,66 @@ int dfx_decode_range(dfx_plan_t plan, const void* d_comp, size_t comp_bytes, uin
     return DFX_OK;
 }
 
+int dfx_decode_host(dfx_plan_t plan, const void* h_comp, size_t comp_bytes, void* d_staging, size_t staging_bytes,
+                    void* d_bf16, uint32_t slices, cudaStream_t copy_stream, cudaStream_t decode_stream) {
+    if (!plan || !h_comp || !d_staging) return DFX_ERR_ARG;
+    if (!aligned16(d_staging)) return DFX_ERR_ARG;
+    const dfx::Layout& L = plan->L;
+    if (comp_bytes < L.off_stream + dfx::stream_bytes(0)) return DFX_ERR_CORRUPT;
+    uint64_t total = 0;  // the container's size from its header
+    memcpy(&total, (const uint8_t*)h_comp + 24, 8);
+    if (total > comp_bytes || total < L.off_stream + dfx::stream_bytes(0)) return DFX_ERR_CORRUPT;
+    if (staging_bytes < total) return DFX_ERR_CAPACITY;
+    dfx::DecodeArgs probe;
+    int rc = make_decode_args(plan, d_staging, total, d_bf16, &probe);
+    if (rc) return rc;
+    if (!plan->events_made) {
+        for (uint32_t i = 0; i < dfx_plan_s::kHostSlicesMax; i++)
+            if (cudaEventCreateWithFlags(&plan->slice_done[i], cudaEventDisableTiming) != cudaSuccess) {
+                cudaGetLastError();
+                for (uint32_t j = 0; j < i; j++) cudaEventDestroy(plan->slice_done[j]);
+                return DFX_ERR_CUDA;
+            }
+        plan->events_made = true;
+    }
+    const uint64_t ng = L.n_group;
+    uint64_t ns = slices ? slices : 8;
+    if (ns > dfx_plan_s::kHostSlicesMax) ns = dfx_plan_s::kHostSlicesMax;
+    if (ns > ng) ns = ng ? ng : 1;
+    const uint8_t* h = (const uint8_t*)h_comp;
+    uint8_t* d = (uint8_t*)d_staging;
+    const uint64_t ge = (uint64_t)L.G * L.K;
+    const uint64_t* gbase = (const uint64_t*)(h + dfx::kOffGbase);
+    auto fail = [] {
+        cudaGetLastError();
+        return DFX_ERR_CUDA;
+    };
+    // header, code lengths and the group index: every slice's decode reads them
+    if (cudaMemcpyAsync(d, h, L.off_m, cudaMemcpyHostToDevice, copy_stream) != cudaSuccess) return fail();
+    for (uint64_t s = 0; s < ns; s++) {
+        const uint64_t g0 = ng * s / ns, g1 = ng * (s + 1) / ns;
+        // the slice's sign+mantissa bytes
+        const uint64_t m0 = L.off_m + g0 * ge, m1 = L.off_m + (g1 * ge < L.n ? g1 * ge : L.n);
+        if (m1 > m0 && cudaMemcpyAsync(d + m0, h + m0, m1 - m0, cudaMemcpyHostToDevice, copy_stream) != cudaSuccess)
+            return fail();
+        // its stream words, from the word of its first bit to a few words past its last
+        // (what the decoder stages), clamped to the container
+        uint64_t b0 = gbase[g0], b1 = gbase[g1];
+        if (b1 < b0 || b1 > total * 8) b0 = 0, b1 = (total - L.off_stream) * 8;  // a bad index: copy everything
+        uint64_t s0 = L.off_stream + ((b0 >> 5) * 4 & ~uint64_t(15));
+        uint64_t s1 = L.off_stream + dfx::align16(((b1 >> 5) + 8) * 4);
+        if (s1 > total) s1 = total;
+        if (s1 > s0 && cudaMemcpyAsync(d + s0, h + s0, s1 - s0, cudaMemcpyHostToDevice, copy_stream) != cudaSuccess)
+            return fail();
+        if (cudaEventRecord(plan->slice_done[s], copy_stream) != cudaSuccess ||
+            cudaStreamWaitEvent(decode_stream, plan->slice_done[s], 0) != cudaSuccess)
+            return fail();
+        rc = dfx_decode_range(plan, d_staging, total, g0, g1 - g0, (uint16_t*)d_bf16 + g0 * ge, decode_stream);
+        if (rc) return rc;
+    }
+    return DFX_OK;
+}
+
 int dfx_decode_batch(const dfx_plan_t* plans, const void* const* d_comps, const size_t* comp_bytes,
                      void* const* d_bf16s, uint32_t count, cudaStream_t stream) {
     if (count == 0) return DFX_OK;
@@ -251,6 +317,8 @@ int dfx_free(dfx_plan_t plan) {
         cudaGetLastError();
         rc = DFX_ERR_CUDA;
     }
+    if (plan->events_made)
+        for (uint32_t i = 0; i < dfx_plan_s::kHostSlicesMax; i++) cudaEventDestroy(plan->slice_done[i]);
     free(plan);
     return rc;
 }

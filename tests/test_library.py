@@ -104,3 +104,7 @@ def test_batch_argument_errors_precede_cuda(lib):
 
 def test_range_argument_errors_precede_cuda(lib):
     assert lib.dfx_decode_range(None, None, 0, 0, 1, None, None) == dfx.DFX_ERR_ARG
+
+
+def test_host_decode_argument_errors_precede_cuda(lib):
+    assert lib.dfx_decode_host(None, None, 0, None, 0, None, 0, None, None) == dfx.DFX_ERR_ARG
