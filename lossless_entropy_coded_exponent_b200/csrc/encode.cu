@@ -387,10 +387,8 @@ struct GlobalSink {
     __device__ __forceinline__ void own_word(uint64_t wi, uint32_t v) const { stream[wi] = v; }
 };
 struct SharedSink {
-    uint32_t* words;  // the group's first stream word is words[0]
+    uint32_t* words;  // the group's first stream word is words[0] (see SharedWriter)
     uint64_t base;
-    __device__ __forceinline__ void shared_word(uint64_t wi, uint32_t v) const { atomicOr(words + (wi - base), v); }
-    __device__ __forceinline__ void own_word(uint64_t wi, uint32_t v) const { words[wi - base] = v; }
 };
 
 template <class Sink>
@@ -428,17 +426,50 @@ struct BitWriter {
     }
 };
 
-// Pack chunk c (lane `lane` of group c / 32), whose codes start at stream bit `start`,
-// and write its elements' mantissa+sign bytes.
-template <int K, class Sink>
-__device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* code_sh, const uint8_t* len_sh,
-                                           uint64_t c, unsigned lane, uint64_t start, Sink sink) {
-    BitWriter<Sink> bw;
+// A chunk's writer into the warp's shared copy of its group's words, without branches:
+// the codes go into a 64-bit accumulator and every completed word is OR-ed in (the copy
+// starts zeroed, and a chunk's first and last words may hold bits of its neighbours).
+struct SharedWriter {
+    uint32_t* words;  // the group's first stream word is words[0]
+    uint64_t base;
+    uint64_t wi;      // stream index of the word being completed
+    uint64_t acc;     // the low `nbits` bits are the pending bits
+    uint32_t nbits;
+
+    __device__ __forceinline__ void put(uint32_t code, uint32_t l) {
+        acc = (acc << l) | code;
+        nbits += l;
+        if (nbits >= 32) {
+            nbits -= 32;
+            atomicOr(words + (wi - base), (uint32_t)(acc >> nbits));
+            wi++;
+        }
+    }
+    __device__ __forceinline__ void finish() {
+        if (nbits) atomicOr(words + (wi - base), (uint32_t)(acc << (32 - nbits)));
+    }
+};
+
+__device__ __forceinline__ BitWriter<GlobalSink> make_writer(GlobalSink sink, uint64_t start) {
+    BitWriter<GlobalSink> bw;
     bw.sink = sink;
     bw.wi = start >> 5;
     bw.fill = (uint32_t)(start & 31);
     bw.cur = 0;
     bw.first = true;
+    return bw;
+}
+__device__ __forceinline__ SharedWriter make_writer(SharedSink sink, uint64_t start) {
+    // the bits of the previous chunk in the first word count as already placed zeros
+    return SharedWriter{sink.words, sink.base, start >> 5, 0ull, (uint32_t)(start & 31)};
+}
+
+// Pack chunk c (lane `lane` of group c / 32), whose codes start at stream bit `start`,
+// and write its elements' mantissa+sign bytes.  cl_sh[e] = code << 8 | length.
+template <int K, class Sink>
+__device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* cl_sh, uint64_t c, unsigned lane,
+                                           uint64_t start, Sink sink) {
+    auto bw = make_writer(sink, start);
     uint8_t* mpl = a.out + a.off_m;
 
     // the chunk's whole blocks (a prefix of its K/8 blocks), their loads one block ahead
@@ -462,7 +493,7 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
                 const uint32_t h = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
                 const uint32_t partner = (w[j >> 1] >> (16 * ((j & 1) ^ 1))) & 0xFFFFu;  // element j ^ 1
                 const uint32_t e = (h >> 7) & 0xFFu;
-                bw.put(code_sh[e], len_sh[e]);
+                bw.put(cl_sh[e] >> 8, cl_sh[e] & 0xFFu);
                 mb[j >> 2] |= (((h & 0x7Fu) << 1) | (partner >> 15)) << (8 * (j & 3));
             }
             *reinterpret_cast<uint2*>(mpl + x0) = make_uint2(mb[0], mb[1]);
@@ -471,7 +502,7 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
                 const uint32_t h = a.in[x];
                 const uint32_t partner = a.in[(x ^ 1u) < a.n ? (x ^ 1u) : x];
                 const uint32_t e = (h >> 7) & 0xFFu;
-                bw.put(code_sh[e], len_sh[e]);
+                bw.put(cl_sh[e] >> 8, cl_sh[e] & 0xFFu);
                 mpl[x] = (uint8_t)(((h & 0x7Fu) << 1) | (partner >> 15));
             }
             break;
@@ -486,11 +517,9 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
 // A group whose words do not fit the copy is packed straight into global memory.
 template <int K>
 __global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
-    __shared__ uint32_t code_sh[256];
-    __shared__ uint8_t len_sh[256];
+    __shared__ uint32_t cl_sh[256];  // code << 8 | length
     __shared__ uint32_t slice[kPackThreads / 32][kPackSliceWords];
-    code_sh[threadIdx.x] = a.ws_code[threadIdx.x];
-    len_sh[threadIdx.x] = a.ws_len[threadIdx.x];
+    cl_sh[threadIdx.x] = (a.ws_code[threadIdx.x] << 8) | a.ws_len[threadIdx.x];
     __syncthreads();
     const uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const unsigned lane = threadIdx.x & 31;
@@ -509,7 +538,7 @@ __global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
         uint32_t* sm = slice[threadIdx.x >> 5];
         for (uint32_t i = lane; i < count; i += 32) sm[i] = 0u;
         __syncwarp();
-        pack_chunk<K>(a, code_sh, len_sh, c, lane, start, SharedSink{sm, wf});
+        pack_chunk<K>(a, cl_sh, c, lane, start, SharedSink{sm, wf});
         __syncwarp();
         for (uint32_t i = lane; i < count; i += 32) {
             const uint32_t v = sm[i];
@@ -520,7 +549,7 @@ __global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
             }
         }
     } else {
-        pack_chunk<K>(a, code_sh, len_sh, c, lane, start, GlobalSink{stream});
+        pack_chunk<K>(a, cl_sh, c, lane, start, GlobalSink{stream});
     }
 }
 
