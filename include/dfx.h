@@ -209,6 +209,16 @@ int dfx_decode_batch(const dfx_plan_t *plans, const void *const *d_comps, const 
  * *h_status (0 = no corruption seen since the last read) and clear it. */
 int dfx_device_status(dfx_plan_t plan, cudaStream_t stream, uint32_t *h_status);
 
+/* Test hook for the decoder's failure detection, with no GPU fault: with
+ * DFX_INJECT_SKIP_SLICE_COPY set, every later decode leaves out the copy of the
+ * stream slice of its first group, so the warp that waits for it runs out its
+ * bounded wait (about a second) and the plan's status word gets
+ * DFX_STATUS_TIMEOUT (that group's output is then not valid).  No copy is left
+ * in flight.  flags = 0 restores normal decoding.  Process-wide, not for
+ * concurrent use; unknown flags return DFX_ERR_ARG. */
+#define DFX_INJECT_SKIP_SLICE_COPY 0x1u
+int dfx_debug_inject(uint32_t flags);
+
 /* Release the plan and its device status word.  NULL is accepted. */
 int dfx_free(dfx_plan_t plan);
 

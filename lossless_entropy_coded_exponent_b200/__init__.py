@@ -28,6 +28,7 @@ DFX_STATUS_TABLE = 0x2
 DFX_STATUS_INDEX = 0x4
 DFX_STATUS_STREAM = 0x8
 DFX_STATUS_TIMEOUT = 0x10
+DFX_INJECT_SKIP_SLICE_COPY = 0x1
 
 # The exported C symbols, in include/dfx.h order.
 EXPORTS = (
@@ -43,6 +44,7 @@ EXPORTS = (
     "dfx_device_status",
     "dfx_free",
     "dfx_encode_static",
+    "dfx_debug_inject",
 )
 
 
@@ -91,10 +93,11 @@ def lib() -> ctypes.CDLL:
                                        ctypes.POINTER(vp), ctypes.c_uint32, vp]
         L.dfx_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.dfx_free.argtypes = [vp]
+        L.dfx_debug_inject.argtypes = [ctypes.c_uint32]
         L.dfx_encode_static.argtypes = [vp, ctypes.c_uint64, ctypes.POINTER(dfx_params), vp, ctypes.c_size_t,
                                         ctypes.POINTER(ctypes.c_size_t), vp]
         for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_decode_range", "dfx_decode_host", "dfx_decode_batch",
-                  "dfx_device_status", "dfx_free", "dfx_encode_static"):
+                  "dfx_device_status", "dfx_free", "dfx_encode_static", "dfx_debug_inject"):
             getattr(L, f).restype = ctypes.c_int
         _lib_handle = L
     return _lib_handle
@@ -227,6 +230,12 @@ def dfx_decode_batch(plans, d_comps, comp_bytes, d_bf16s, stream=None) -> None:
     sz = (ctypes.c_size_t * max(n, 1))(*[int(b) for b in comp_bytes])
     op = (vp * max(n, 1))(*[_ptr(o) for o in d_bf16s])
     _check(lib().dfx_decode_batch(hp, cp, sz, op, n, _stream(stream)), "dfx_decode_batch")
+
+
+def dfx_debug_inject(flags: int) -> None:
+    """Test hook: DFX_INJECT_SKIP_SLICE_COPY makes later decodes leave one stream-slice
+    copy out so that a bounded wait runs out (status DFX_STATUS_TIMEOUT); 0 restores."""
+    _check(lib().dfx_debug_inject(flags), "dfx_debug_inject")
 
 
 def dfx_device_status(plan: Plan, stream=None) -> int:

@@ -38,6 +38,8 @@ int resolve_params(const dfx_params* p, uint32_t* K, uint32_t* G, uint32_t* L) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+uint32_t g_inject = 0;  // dfx_debug_inject
+
 // Host checks of one decode and its kernel arguments.
 int make_decode_args(const dfx_plan_s* plan, const void* d_comp, size_t comp_bytes, void* d_bf16, dfx::DecodeArgs* a);
 
@@ -52,6 +54,12 @@ int check_device(const dfx_plan_s* plan) {
 extern "C" {
 
 uint32_t dfx_version(void) { return (1u << 16) | 0u; }
+
+int dfx_debug_inject(uint32_t flags) {
+    if (flags & ~(uint32_t)DFX_INJECT_SKIP_SLICE_COPY) return DFX_ERR_ARG;
+    g_inject = flags;
+    return DFX_OK;
+}
 
 const char* dfx_strerror(int code) {
     switch (code) {
@@ -349,6 +357,7 @@ int make_decode_args(const dfx_plan_s* plan, const void* d_comp, size_t comp_byt
     a->g_begin = 0;
     a->g_end = (uint32_t)plan->L.n_group;
     a->out_first = 0;
+    a->inject = g_inject;
     return DFX_OK;
 }
 

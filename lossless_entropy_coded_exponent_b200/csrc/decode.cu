@@ -439,19 +439,30 @@ __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t b
                  "l"(src), "r"(bytes), "r"(smem_addr(bar))
                  : "memory");
 }
-// Wait for the phase with the given parity of `bar` to complete; gives up after a bounded
-// number of polls (the copy engine never took that long here) and reports it.
-constexpr uint32_t kWaitPolls = 1u << 20;
+// Wait for the phase with the given parity of `bar` to complete.  One blocking poll first
+// (try_wait, which suspends the warp for at most the 100 us time hint: staged data
+// normally lands within it), then non-blocking polls (test_wait) with a sleep of at most
+// 128 ns between them (__nanosleep(64) lasts at most twice its argument); a wait that
+// never completes gives up after ~0.1 ms + ~0.35 s and the caller reports
+// DFX_STATUS_TIMEOUT.
+constexpr uint32_t kWaitPolls = 1u << 21;
 __device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity) {
     const uint32_t addr = smem_addr(bar);
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 100000;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
     for (uint32_t i = 0; i < kWaitPolls; i++) {
-        uint32_t done;
         asm volatile(
-            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+            "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
             : "=r"(done)
             : "r"(addr), "r"(parity)
             : "memory");
         if (done) return true;
+        __nanosleep(64);
     }
     return false;
 }
@@ -564,7 +575,9 @@ __device__ __forceinline__ void group_prologue(const DecodeArgs& a, const Tables
     s.st = scan_index(load_index(a, T, g, lane, true), lane);
     s.sl = plan_slice<SliceShape<K>::kWords>(T, s.st.gb0, s.st.span, s.st.ok);
     if (lane == 0) {
-        if (s.sl.staged) bulk_copy(wb.slice[0], a.comp + a.off_stream + 4u * s.sl.base, s.sl.bytes, &wb.mbar[0]);
+        // (the test hook leaves one copy out, so that its bounded wait runs out)
+        const bool skip = (a.inject & DFX_INJECT_SKIP_SLICE_COPY) && g == a.g_begin;
+        if (s.sl.staged && !skip) bulk_copy(wb.slice[0], a.comp + a.off_stream + 4u * s.sl.base, s.sl.bytes, &wb.mbar[0]);
         for (uint32_t u = 0; u < kMUnits; u++) s.mp.issue(a, wb, u);
     }
     s.g = g;

@@ -58,6 +58,7 @@ struct DecodeArgs {
     uint32_t* status;
     uint32_t g_begin, g_end;  // groups to decode (all: 0, n_group)
     uint64_t out_first;       // element index stored at out[0] (g_begin * G * K)
+    uint32_t inject;          // test hook flags (dfx_debug_inject), normally 0
 };
 
 struct EncodeArgs {

@@ -200,3 +200,23 @@ def test_exponent_histogram_counts(name):
         counts = ws[:2048].cpu().numpy().view(np.uint64)
     ref = np.bincount(((w >> 7) & 0xFF).astype(np.int64), minlength=256).astype(np.uint64)
     assert np.array_equal(counts, ref)
+
+
+def test_bounded_wait_runs_out_and_reports_timeout():
+    """Failure detection without a GPU fault: the test hook leaves one stream-slice copy
+    out, the warp waiting for it gives up after its bounded wait and the status word says
+    so; afterwards the context is healthy and decoding is exact again."""
+    w = inputs.gaussian(4096 * 10, 0.02, seed=51)  # 10 groups: one per warp of one CTA
+    comp = torch.from_numpy(oracle.encode(w, K=128)).cuda()
+    out = torch.empty(w.size, dtype=torch.int16, device="cuda")
+    with dfx.dfx_plan(w.size) as plan:
+        dfx.dfx_debug_inject(dfx.DFX_INJECT_SKIP_SLICE_COPY)
+        try:
+            dfx.dfx_decode(plan, comp, comp.numel(), out)
+            st = dfx.dfx_device_status(plan)
+        finally:
+            dfx.dfx_debug_inject(0)
+        assert st & dfx.DFX_STATUS_TIMEOUT, hex(st)
+        dfx.dfx_decode(plan, comp, comp.numel(), out)
+        assert dfx.dfx_device_status(plan) == 0
+    assert np.array_equal(to_host_u16(out), w)

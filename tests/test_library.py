@@ -108,3 +108,8 @@ def test_range_argument_errors_precede_cuda(lib):
 
 def test_host_decode_argument_errors_precede_cuda(lib):
     assert lib.dfx_decode_host(None, None, 0, None, 0, None, 0, None, None) == dfx.DFX_ERR_ARG
+
+
+def test_debug_inject_flags(lib):
+    assert lib.dfx_debug_inject(0x2) == dfx.DFX_ERR_ARG
+    assert lib.dfx_debug_inject(0) == dfx.DFX_OK
