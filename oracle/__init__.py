@@ -1,7 +1,8 @@
 """ctypes marshalling for the CPU oracle in ``oracle/dfx_oracle.c``.
 
 TEST INFRASTRUCTURE ONLY.  The oracle is the plain single-threaded CPU
-statement of the DFX1 codec that the CUDA library is checked against.  Only
+statement of the DFX1 codec (both exponent coders: canonical Huffman and
+tANS) that the CUDA library is checked against.  Only
 the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
 may import this module; the product path (``lossless_entropy_coded_exponent_b200``)
 never does, and the two share no code.  Every function here only moves
@@ -68,7 +69,17 @@ def lib() -> ctypes.CDLL:
         L.dfxo_encode.argtypes = [u16p, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint32,
                                   u8p, ctypes.c_uint64, u64p]
         L.dfxo_decode.argtypes = [u8p, ctypes.c_uint64, u16p, ctypes.c_uint64, u64p]
-        for f in ("dfxo_histogram", "dfxo_code_lengths", "dfxo_canonical_codes", "dfxo_encode", "dfxo_decode"):
+        L.dfxo_tans_normalize.argtypes = [u64p, ctypes.c_uint32, u32p]
+        L.dfxo_tans_tables.argtypes = [u32p, ctypes.c_uint32, u8p, u32p]
+        L.dfxo_encode_tans.argtypes = [u16p, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint32,
+                                       u8p, ctypes.c_uint64, u64p]
+        L.dfxo_tans_container_bytes.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint64]
+        L.dfxo_tans_container_bytes.restype = ctypes.c_uint64
+        L.dfxo_tans_max_container_bytes.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
+                                                    ctypes.c_uint32]
+        L.dfxo_tans_max_container_bytes.restype = ctypes.c_uint64
+        for f in ("dfxo_histogram", "dfxo_code_lengths", "dfxo_canonical_codes", "dfxo_encode", "dfxo_decode",
+                  "dfxo_tans_normalize", "dfxo_tans_tables", "dfxo_encode_tans"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -143,6 +154,54 @@ def encode(w: np.ndarray, K: int = 64, G: int = 32, max_len: int = 24) -> np.nda
                            _ptr(out, ctypes.c_uint8), cap, _ptr(used, ctypes.c_uint64))
     if rc:
         raise OracleError(rc, "encode")
+    return out[: int(used[0])].copy()
+
+
+def tans_normalize(counts, table_log: int = 12) -> np.ndarray:
+    """Rule T1: the frequencies (summing to 2**table_log) of a count vector."""
+    c = np.zeros(256, dtype=np.uint64)
+    src = np.asarray(counts, dtype=np.uint64)
+    c[: src.size] = src
+    f = np.zeros(256, dtype=np.uint32)
+    rc = lib().dfxo_tans_normalize(_ptr(c, ctypes.c_uint64), table_log, _ptr(f, ctypes.c_uint32))
+    if rc:
+        raise OracleError(rc, "tans_normalize")
+    return f
+
+
+def tans_tables(freq, table_log: int = 12):
+    """Rules T2 and T3: (symbol, state number k) of every table slot."""
+    f = np.zeros(256, dtype=np.uint32)
+    src = np.asarray(freq, dtype=np.uint32)
+    f[: src.size] = src
+    m = 1 << table_log
+    sym = np.zeros(m, dtype=np.uint8)
+    k = np.zeros(m, dtype=np.uint32)
+    rc = lib().dfxo_tans_tables(_ptr(f, ctypes.c_uint32), table_log, _ptr(sym, ctypes.c_uint8),
+                                _ptr(k, ctypes.c_uint32))
+    if rc:
+        raise OracleError(rc, "tans_tables")
+    return sym, k
+
+
+def tans_container_bytes(n: int, K: int, G: int, total_bits: int) -> int:
+    return int(lib().dfxo_tans_container_bytes(n, K, G, total_bits))
+
+
+def tans_max_container_bytes(n: int, K: int, G: int, table_log: int = 12) -> int:
+    return int(lib().dfxo_tans_max_container_bytes(n, K, G, table_log))
+
+
+def encode_tans(w: np.ndarray, K: int = 128, G: int = 32, table_log: int = 12) -> np.ndarray:
+    """Whole-tensor encode with the tANS exponent coder (coder 1)."""
+    w = np.ascontiguousarray(w, dtype=np.uint16).reshape(-1)
+    cap = tans_max_container_bytes(w.size, K, G, table_log)
+    out = np.empty(cap, dtype=np.uint8)
+    used = np.zeros(1, dtype=np.uint64)
+    rc = lib().dfxo_encode_tans(_ptr(w, ctypes.c_uint16), w.size, K, G, table_log,
+                                _ptr(out, ctypes.c_uint8), cap, _ptr(used, ctypes.c_uint64))
+    if rc:
+        raise OracleError(rc, "encode_tans")
     return out[: int(used[0])].copy()
 
 

@@ -37,6 +37,8 @@
  *   8. decode bit by bit (canonical first-code/count walk), check the index
  *      against the walk, merge the two bytes back.
  * No step is blocked, fused or reordered beyond that list.
+ * A second exponent coder (coder 1, tANS) replaces steps 3-5 and 8 with the
+ * rules T1-T5 stated at the end of this file; everything else is shared.
  *
  * The container layout (all integers little-endian, every section starts at a
  * 16-byte boundary, every padding byte is zero):
@@ -75,6 +77,10 @@
 #define DFXO_HEADER_BYTES 64u
 #define DFXO_LEN_OFFSET 64u
 #define DFXO_GBASE_OFFSET 320u
+#define DFXO_CODER_HUFFMAN 0u
+#define DFXO_CODER_TANS 1u
+#define DFXO_FREQ_OFFSET 64u
+#define DFXO_TANS_GBASE_OFFSET 576u
 
 /* ------------------------------------------------------------------ */
 /* little-endian helpers (the container is little-endian by definition) */
@@ -257,21 +263,32 @@ static int params_ok(uint64_t n, uint32_t K, uint32_t G, uint32_t max_len) {
     return 1;
 }
 
-static uint64_t n_groups(uint64_t n, uint32_t K, uint32_t G) { return (n + (uint64_t)G * K - 1) / ((uint64_t)G * K); }
+/* (0 for parameters no container can have, so that sizing never divides by zero) */
+static uint64_t n_groups(uint64_t n, uint32_t K, uint32_t G) {
+    return (G == 0 || K == 0) ? 0 : (n + (uint64_t)G * K - 1) / ((uint64_t)G * K);
+}
 
 /* Element of position `pos` (0..K-1) in chunk `lane` of group g: the group's
  * elements form blocks of 8, block b belongs to chunk b mod G. */
 static uint64_t chunk_element(uint64_t g, uint32_t lane, uint32_t pos, uint32_t K, uint32_t G) {
     return g * G * K + ((uint64_t)(pos / 8) * G + lane) * 8 + pos % 8;
 }
-static uint64_t off_clen_of(uint64_t ng) { return align16(DFXO_GBASE_OFFSET + 8 * (ng + 1)); }
-static uint64_t off_m_of(uint64_t nc, uint64_t ng) { return align16(off_clen_of(ng) + 2 * nc); }
-static uint64_t off_stream_of(uint64_t n, uint64_t nc, uint64_t ng) { return align16(off_m_of(nc, ng) + n); }
+/* The sections after the code section are the same for both coders; only the
+ * code section's size (len[256] for coder 0, freq[256] for coder 1) moves them. */
+static uint64_t gbase_of(uint32_t coder) { return coder == DFXO_CODER_TANS ? DFXO_TANS_GBASE_OFFSET : DFXO_GBASE_OFFSET; }
+static uint64_t off_clen_of(uint64_t ng, uint32_t coder) { return align16(gbase_of(coder) + 8 * (ng + 1)); }
+static uint64_t off_m_of(uint64_t nc, uint64_t ng, uint32_t coder) { return align16(off_clen_of(ng, coder) + 2 * nc); }
+static uint64_t off_stream_of(uint64_t n, uint64_t nc, uint64_t ng, uint32_t coder) {
+    return align16(off_m_of(nc, ng, coder) + n);
+}
 static uint64_t stream_bytes_of(uint64_t total_bits) { return align16(4 * ((total_bits + 31) / 32)) + 16; }
 
-uint64_t dfxo_container_bytes(uint64_t n, uint32_t K, uint32_t G, uint64_t total_bits) {
+static uint64_t container_bytes_of(uint64_t n, uint32_t K, uint32_t G, uint64_t total_bits, uint32_t coder) {
     uint64_t ng = n_groups(n, K, G), nc = ng * G;
-    return off_stream_of(n, nc, ng) + stream_bytes_of(total_bits);
+    return off_stream_of(n, nc, ng, coder) + stream_bytes_of(total_bits);
+}
+uint64_t dfxo_container_bytes(uint64_t n, uint32_t K, uint32_t G, uint64_t total_bits) {
+    return container_bytes_of(n, K, G, total_bits, DFXO_CODER_HUFFMAN);
 }
 
 /* ------------------------------------------------------------------ */
@@ -324,16 +341,16 @@ int dfxo_encode(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t 
     put_u32(out + 36, G);
     put_u32(out + 40, (uint32_t)nc);
     put_u32(out + 44, (uint32_t)ng);
-    put_u64(out + 48, off_m_of(nc, ng));
+    put_u64(out + 48, off_m_of(nc, ng, 0));
     put_u32(out + 56, max_len);
     put_u32(out + 60, 0);
     memcpy(out + DFXO_LEN_OFFSET, len, 256);
 
     /* stream in chunk order, index: chunk bit lengths and group start bits */
     uint8_t *gbase = out + DFXO_GBASE_OFFSET;
-    uint8_t *clen = out + off_clen_of(ng);
-    uint8_t *mplane = out + off_m_of(nc, ng);
-    uint8_t *stream = out + off_stream_of(n, nc, ng);
+    uint8_t *clen = out + off_clen_of(ng, 0);
+    uint8_t *mplane = out + off_m_of(nc, ng, 0);
+    uint8_t *stream = out + off_stream_of(n, nc, ng, 0);
     uint64_t pos = 0;
     for (uint64_t g = 0; g < ng; g++) {
         put_u64(gbase + 8 * g, pos);
@@ -366,7 +383,11 @@ uint64_t dfxo_max_container_bytes(uint64_t n, uint32_t K, uint32_t G) {
  * time: a code of length l is complete when its value minus the first
  * canonical code of length l is below the number of codes of length l.    */
 
+static int decode_tans(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, uint64_t *n_out);
+
 int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, uint64_t *n_out) {
+    if (bytes >= DFXO_HEADER_BYTES && memcmp(c, "DFX1", 4) == 0 && get_u32(c + 60) == DFXO_CODER_TANS)
+        return decode_tans(c, bytes, w, n_cap, n_out);
     if (bytes < DFXO_GBASE_OFFSET + 8) return DFXO_ERR_CORRUPT;
     if (memcmp(c, "DFX1", 4) != 0) return DFXO_ERR_CORRUPT;
     if (get_u16(c + 4) != 1 || get_u16(c + 6) != DFXO_HEADER_BYTES) return DFXO_ERR_CORRUPT;
@@ -379,7 +400,7 @@ int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, u
     if (get_u32(c + 60) != 0) return DFXO_ERR_CORRUPT;
     uint64_t ng = n_groups(n, K, G), nc = ng * G;
     if (get_u32(c + 40) != nc || get_u32(c + 44) != ng) return DFXO_ERR_CORRUPT;
-    if (get_u64(c + 48) != off_m_of(nc, ng)) return DFXO_ERR_CORRUPT;
+    if (get_u64(c + 48) != off_m_of(nc, ng, 0)) return DFXO_ERR_CORRUPT;
     if (total_bits > (uint64_t)max_len * n) return DFXO_ERR_CORRUPT;
     if (total != dfxo_container_bytes(n, K, G, total_bits) || total > bytes) return DFXO_ERR_CORRUPT;
     if (n_out) *n_out = n;
@@ -420,14 +441,14 @@ int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, u
     }
 
     const uint8_t *gbase = c + DFXO_GBASE_OFFSET;
-    const uint8_t *clen = c + off_clen_of(ng);
-    const uint8_t *mplane = c + off_m_of(nc, ng);
-    const uint8_t *stream = c + off_stream_of(n, nc, ng);
+    const uint8_t *clen = c + off_clen_of(ng, 0);
+    const uint8_t *mplane = c + off_m_of(nc, ng, 0);
+    const uint8_t *stream = c + off_stream_of(n, nc, ng, 0);
 
     /* every padding byte must be zero */
-    for (uint64_t b = DFXO_GBASE_OFFSET + 8 * (ng + 1); b < off_clen_of(ng); b++) if (c[b]) return DFXO_ERR_CORRUPT;
-    for (uint64_t b = off_clen_of(ng) + 2 * nc; b < off_m_of(nc, ng); b++) if (c[b]) return DFXO_ERR_CORRUPT;
-    for (uint64_t b = off_m_of(nc, ng) + n; b < off_stream_of(n, nc, ng); b++) if (c[b]) return DFXO_ERR_CORRUPT;
+    for (uint64_t b = DFXO_GBASE_OFFSET + 8 * (ng + 1); b < off_clen_of(ng, 0); b++) if (c[b]) return DFXO_ERR_CORRUPT;
+    for (uint64_t b = off_clen_of(ng, 0) + 2 * nc; b < off_m_of(nc, ng, 0); b++) if (c[b]) return DFXO_ERR_CORRUPT;
+    for (uint64_t b = off_m_of(nc, ng, 0) + n; b < off_stream_of(n, nc, ng, 0); b++) if (c[b]) return DFXO_ERR_CORRUPT;
     if (get_u64(gbase) != 0 || get_u64(gbase + 8 * ng) != total_bits) return DFXO_ERR_CORRUPT;
 
     uint64_t pos = 0;
@@ -461,4 +482,317 @@ int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, u
     for (uint64_t k = total_bits; k < 32 * ((total_bits + 31) / 32); k++) if (get_bit(stream, k)) return DFXO_ERR_CORRUPT;
     for (uint64_t b = 4 * ((total_bits + 31) / 32); b < stream_bytes_of(total_bits); b++) if (stream[b]) return DFXO_ERR_CORRUPT;
     return DFXO_OK;
+}
+
+/* ================================================================== */
+/* Coder 1: tabled asymmetric numeral systems (tANS) for the exponents.
+ *
+ * One page names ANS as the entropy coder of its compressed number formats'
+ * hardware decoder ("From a Lossless (~1.5:1) Compression Algorithm for Llama2
+ * 7B Weights to Variable Precision, Variable Range, Compressed Numeric Data
+ * Types for CNNs and LLMs", abstract) without giving a construction.  This
+ * coder is the published tabled variant (J. Duda, "Asymmetric numeral
+ * systems", 2013) with these rules, each a reading of this codec:
+ *   T1. frequencies: M = 2^R (R = table_log, 4..12).  Every used exponent s
+ *       gets f[s] = counts[s] * M / n rounded half up, at least 1; then the
+ *       largest f (the smallest symbol among equal ones) takes the whole
+ *       shortfall to M, or gives up an excess one unit at a time, until the
+ *       f sum to M.  More used exponents than M: no table (argument error);
+ *   T2. spread: list every symbol f[s] times in symbol order; occurrence i
+ *       goes to table slot (i * step) mod M, step = M/2 + M/8 + 3 (odd, so
+ *       for M >= 16, so every slot is hit once; the stride of Y. Collet's FSE
+ *       coder);
+ *   T3. states: the slots of symbol s, in ascending slot order, are numbered
+ *       k = f[s], f[s] + 1, ..., 2 f[s] - 1;
+ *   T4. a chunk's symbols are encoded from its last to its first, starting
+ *       from state X = M: for symbol s take the nb >= 0 with
+ *       f[s] <= X >> nb < 2 f[s], emit the low nb bits of X, and move to
+ *       X = M + the slot of s numbered X >> nb.  The chunk's bits are the
+ *       final X - M (R bits), then the emitted fields in symbol order
+ *       (first symbol's first), each MSB-first; an empty chunk has no bits;
+ *   T5. decoding a chunk: x = its first R bits; for each symbol, slot x holds
+ *       symbol s with number k; with nb = R - floor(log2 k), x becomes
+ *       k * 2^nb + (the next nb bits) - M.  After the last symbol x is 0.
+ * The container is the DFX1 layout with u32 coder = 1 at offset 60, the table
+ * log in the max_len word (offset 56), u16 freq[256] at offset 64 and the
+ * group start bits at offset 576; the chunks, groups and blocks are those of
+ * coder 0.                                                               */
+
+static int tans_params_ok(uint64_t n, uint32_t K, uint32_t G, uint32_t R) {
+    if (n >= ((uint64_t)1 << 32)) return 0;
+    if (R < 4 || R > 12) return 0;
+    if (K < 8 || K % 8 != 0 || G < 1) return 0;
+    if ((uint64_t)(K + 1) * R > 65535u) return 0; /* a chunk length must fit in u16 */
+    return 1;
+}
+
+/* T1 */
+int dfxo_tans_normalize(const uint64_t counts[256], uint32_t R, uint32_t f[256]) {
+    if (R < 4 || R > 12) return DFXO_ERR_ARG;
+    const uint64_t M = (uint64_t)1 << R;
+    uint64_t n = 0, used = 0;
+    for (int s = 0; s < 256; s++) {
+        f[s] = 0;
+        if (counts[s] >= ((uint64_t)1 << 40)) return DFXO_ERR_ARG;
+        n += counts[s];
+        used += counts[s] > 0;
+    }
+    if (n == 0) return DFXO_OK;
+    if (used > M) return DFXO_ERR_ARG;
+    uint64_t sum = 0;
+    for (int s = 0; s < 256; s++) {
+        if (!counts[s]) continue;
+        uint64_t q = (2 * counts[s] * M + n) / (2 * n);
+        f[s] = (uint32_t)(q ? q : 1);
+        sum += f[s];
+    }
+    while (sum != M) {
+        int big = 0;
+        for (int s = 1; s < 256; s++)
+            if (f[s] > f[big]) big = s;
+        if (sum < M) {
+            f[big] += (uint32_t)(M - sum);
+            sum = M;
+        } else { /* sum > M >= used, so f[big] >= 2 */
+            f[big] -= 1;
+            sum -= 1;
+        }
+    }
+    return DFXO_OK;
+}
+
+/* T2 and T3: slot_sym[j] and slot_k[j] for the M slots.  f must sum to M. */
+int dfxo_tans_tables(const uint32_t f[256], uint32_t R, uint8_t *slot_sym, uint32_t *slot_k) {
+    if (R < 4 || R > 12) return DFXO_ERR_ARG;
+    const uint32_t M = 1u << R;
+    uint64_t sum = 0;
+    for (int s = 0; s < 256; s++) sum += f[s];
+    if (sum != M) return DFXO_ERR_ARG;
+    const uint32_t step = (M >> 1) + (M >> 3) + 3;
+    uint32_t i = 0;
+    for (int s = 0; s < 256; s++)
+        for (uint32_t r = 0; r < f[s]; r++, i++) slot_sym[(i * step) & (M - 1)] = (uint8_t)s;
+    uint32_t next[256];
+    for (int s = 0; s < 256; s++) next[s] = f[s];
+    for (uint32_t j = 0; j < M; j++) slot_k[j] = next[slot_sym[j]]++;
+    return DFXO_OK;
+}
+
+/* T4 for one chunk of cnt symbols e[]: its bit length; when stream is not
+ * NULL the bits are also written from stream bit `pos` on.  enc[cs[s] + k -
+ * f[s]] is the slot of s numbered k; v and nb hold cnt fields. */
+static uint64_t tans_chunk(const uint32_t f[256], const uint32_t cs[256], const uint32_t *enc, uint32_t R,
+                           const uint8_t *e, uint32_t cnt, uint8_t *stream, uint64_t pos, uint32_t *v, uint8_t *nb) {
+    if (cnt == 0) return 0;
+    const uint32_t M = 1u << R;
+    uint32_t X = M;
+    uint64_t bits = R;
+    for (uint32_t i = cnt; i-- > 0;) {
+        const uint32_t s = e[i];
+        uint32_t b = 0;
+        while ((X >> b) >= 2 * f[s]) b++;
+        v[i] = X & ((1u << b) - 1u);
+        nb[i] = (uint8_t)b;
+        bits += b;
+        X = M + enc[cs[s] + (X >> b) - f[s]];
+    }
+    if (stream) {
+        put_bits(stream, pos, X - M, R);
+        pos += R;
+        for (uint32_t i = 0; i < cnt; i++) {
+            put_bits(stream, pos, v[i], nb[i]);
+            pos += nb[i];
+        }
+    }
+    return bits;
+}
+
+uint64_t dfxo_tans_container_bytes(uint64_t n, uint32_t K, uint32_t G, uint64_t total_bits) {
+    return container_bytes_of(n, K, G, total_bits, DFXO_CODER_TANS);
+}
+
+uint64_t dfxo_tans_max_container_bytes(uint64_t n, uint32_t K, uint32_t G, uint32_t R) {
+    /* a field is at most R bits (k >= 1), plus R bits of state per chunk */
+    uint64_t nc = n_groups(n, K, G) * G;
+    return container_bytes_of(n, K, G, (uint64_t)R * (n + nc), DFXO_CODER_TANS);
+}
+
+/* The symbols of chunk `lane` of group g, in chunk order; returns how many. */
+static uint32_t chunk_symbols(const uint16_t *w, uint64_t n, uint64_t g, uint32_t lane, uint32_t K, uint32_t G,
+                              uint8_t *e) {
+    uint32_t cnt = 0;
+    for (uint32_t k = 0; k < K; k++) {
+        uint64_t x = chunk_element(g, lane, k, K, G);
+        if (x >= n) break;
+        e[cnt++] = dfxo_exponent(w[x]);
+    }
+    return cnt;
+}
+
+int dfxo_encode_tans(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t R, uint8_t *out, uint64_t cap,
+                     uint64_t *out_bytes) {
+    if (!tans_params_ok(n, K, G, R)) return DFXO_ERR_ARG;
+    const uint32_t M = 1u << R;
+    uint64_t counts[256];
+    uint32_t f[256], cs[256];
+    dfxo_histogram(w, n, counts);
+    int rc = dfxo_tans_normalize(counts, R, f);
+    if (rc) return rc;
+    uint8_t *slot_sym = (uint8_t *)malloc(M);
+    uint32_t *slot_k = (uint32_t *)malloc(4 * (size_t)M), *enc = (uint32_t *)malloc(4 * (size_t)M);
+    uint32_t *v = (uint32_t *)malloc(4 * (size_t)K);
+    uint8_t *e = (uint8_t *)malloc(K), *nb = (uint8_t *)malloc(K);
+    if (!slot_sym || !slot_k || !enc || !v || !e || !nb) {
+        rc = DFXO_ERR_ARG;
+        goto done;
+    }
+    {
+        uint32_t run = 0;
+        for (int s = 0; s < 256; s++) {
+            cs[s] = run;
+            run += f[s];
+        }
+    }
+    if (n > 0) {
+        dfxo_tans_tables(f, R, slot_sym, slot_k);
+        for (uint32_t j = 0; j < M; j++) enc[cs[slot_sym[j]] + slot_k[j] - f[slot_sym[j]]] = j;
+    }
+    uint64_t ng = n_groups(n, K, G), nc = ng * G;
+    uint64_t total_bits = 0;
+    for (uint64_t g = 0; g < ng; g++)
+        for (uint32_t lane = 0; lane < G; lane++) {
+            uint32_t cnt = chunk_symbols(w, n, g, lane, K, G, e);
+            total_bits += tans_chunk(f, cs, enc, R, e, cnt, NULL, 0, v, nb);
+        }
+    uint64_t total = container_bytes_of(n, K, G, total_bits, DFXO_CODER_TANS);
+    if (out_bytes) *out_bytes = total;
+    if (cap < total) {
+        rc = DFXO_ERR_CAPACITY;
+        goto done;
+    }
+    memset(out, 0, (size_t)total);
+    memcpy(out, "DFX1", 4);
+    put_u16(out + 4, 1);
+    put_u16(out + 6, DFXO_HEADER_BYTES);
+    put_u64(out + 8, n);
+    put_u64(out + 16, total_bits);
+    put_u64(out + 24, total);
+    put_u32(out + 32, K);
+    put_u32(out + 36, G);
+    put_u32(out + 40, (uint32_t)nc);
+    put_u32(out + 44, (uint32_t)ng);
+    put_u64(out + 48, off_m_of(nc, ng, DFXO_CODER_TANS));
+    put_u32(out + 56, R);
+    put_u32(out + 60, DFXO_CODER_TANS);
+    for (int s = 0; s < 256; s++) put_u16(out + DFXO_FREQ_OFFSET + 2 * s, (uint16_t)f[s]);
+    {
+        uint8_t *gbase = out + DFXO_TANS_GBASE_OFFSET;
+        uint8_t *clen = out + off_clen_of(ng, DFXO_CODER_TANS);
+        uint8_t *mplane = out + off_m_of(nc, ng, DFXO_CODER_TANS);
+        uint8_t *stream = out + off_stream_of(n, nc, ng, DFXO_CODER_TANS);
+        uint64_t pos = 0;
+        for (uint64_t g = 0; g < ng; g++) {
+            put_u64(gbase + 8 * g, pos);
+            for (uint32_t lane = 0; lane < G; lane++) {
+                uint32_t cnt = chunk_symbols(w, n, g, lane, K, G, e);
+                uint64_t bits = tans_chunk(f, cs, enc, R, e, cnt, stream, pos, v, nb);
+                put_u16(clen + 2 * (g * G + lane), (uint16_t)bits);
+                pos += bits;
+            }
+        }
+        put_u64(gbase + 8 * ng, pos);
+        for (uint64_t i = 0; i < n; i++) mplane[i] = dfxo_sign_mantissa(w[i], w[dfxo_partner(i, n)]);
+    }
+    rc = DFXO_OK;
+done:
+    free(slot_sym);
+    free(slot_k);
+    free(enc);
+    free(v);
+    free(e);
+    free(nb);
+    return rc;
+}
+
+/* T5, with every header field, the frequency table, the index and the
+ * padding checked. */
+static int decode_tans(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, uint64_t *n_out) {
+    if (bytes < DFXO_TANS_GBASE_OFFSET + 8) return DFXO_ERR_CORRUPT;
+    if (get_u16(c + 4) != 1 || get_u16(c + 6) != DFXO_HEADER_BYTES) return DFXO_ERR_CORRUPT;
+    uint64_t n = get_u64(c + 8), total_bits = get_u64(c + 16), total = get_u64(c + 24);
+    uint32_t K = get_u32(c + 32), G = get_u32(c + 36), R = get_u32(c + 56);
+    if (!tans_params_ok(n, K, G, R)) return DFXO_ERR_CORRUPT;
+    uint64_t ng = n_groups(n, K, G), nc = ng * G;
+    if (get_u32(c + 40) != nc || get_u32(c + 44) != ng) return DFXO_ERR_CORRUPT;
+    if (get_u64(c + 48) != off_m_of(nc, ng, DFXO_CODER_TANS)) return DFXO_ERR_CORRUPT;
+    if (total_bits > (uint64_t)R * (n + nc)) return DFXO_ERR_CORRUPT;
+    if (total != container_bytes_of(n, K, G, total_bits, DFXO_CODER_TANS) || total > bytes) return DFXO_ERR_CORRUPT;
+    if (n_out) *n_out = n;
+    if (n > n_cap) return DFXO_ERR_CAPACITY;
+
+    const uint32_t M = 1u << R;
+    uint32_t f[256];
+    uint64_t sum = 0;
+    for (int s = 0; s < 256; s++) {
+        f[s] = get_u16(c + DFXO_FREQ_OFFSET + 2 * s);
+        sum += f[s];
+    }
+    if (sum != (n > 0 ? M : 0)) return DFXO_ERR_CORRUPT;
+    uint8_t *slot_sym = (uint8_t *)malloc(M);
+    uint32_t *slot_k = (uint32_t *)malloc(4 * (size_t)M);
+    int rc = DFXO_ERR_CORRUPT;
+    if (!slot_sym || !slot_k) goto done;
+    if (n > 0) dfxo_tans_tables(f, R, slot_sym, slot_k);
+
+    const uint8_t *gbase = c + DFXO_TANS_GBASE_OFFSET;
+    const uint8_t *clen = c + off_clen_of(ng, DFXO_CODER_TANS);
+    const uint8_t *mplane = c + off_m_of(nc, ng, DFXO_CODER_TANS);
+    const uint8_t *stream = c + off_stream_of(n, nc, ng, DFXO_CODER_TANS);
+    for (uint64_t b = DFXO_TANS_GBASE_OFFSET + 8 * (ng + 1); b < off_clen_of(ng, DFXO_CODER_TANS); b++)
+        if (c[b]) goto done;
+    for (uint64_t b = off_clen_of(ng, DFXO_CODER_TANS) + 2 * nc; b < off_m_of(nc, ng, DFXO_CODER_TANS); b++)
+        if (c[b]) goto done;
+    for (uint64_t b = off_m_of(nc, ng, DFXO_CODER_TANS) + n; b < off_stream_of(n, nc, ng, DFXO_CODER_TANS); b++)
+        if (c[b]) goto done;
+    if (get_u64(gbase) != 0 || get_u64(gbase + 8 * ng) != total_bits) goto done;
+
+    uint64_t pos = 0;
+    for (uint64_t g = 0; g < ng; g++) {
+        if (get_u64(gbase + 8 * g) != pos) goto done;
+        for (uint32_t lane = 0; lane < G; lane++) {
+            uint64_t chunk_start = pos;
+            uint32_t x = 0;
+            for (uint32_t k = 0; k < K; k++) {
+                uint64_t xe = chunk_element(g, lane, k, K, G);
+                if (xe >= n) break;
+                if (k == 0) { /* the chunk's first R bits: the decoder's start state */
+                    for (uint32_t b = 0; b < R; b++) {
+                        if (pos >= total_bits) goto done;
+                        x = (x << 1) | get_bit(stream, pos++);
+                    }
+                }
+                uint32_t s = slot_sym[x], kk = slot_k[x], nbits = R, t = kk;
+                while (t >>= 1) nbits--;
+                uint32_t val = 0;
+                for (uint32_t b = 0; b < nbits; b++) {
+                    if (pos >= total_bits) goto done;
+                    val = (val << 1) | get_bit(stream, pos++);
+                }
+                x = (kk << nbits) + val - M;
+                w[xe] = dfxo_merge((uint8_t)s, mplane[xe], mplane[dfxo_partner(xe, n)]);
+            }
+            if (x != 0) goto done; /* every chunk ends in the encoder's start state */
+            if (get_u16(clen + 2 * (g * G + lane)) != pos - chunk_start) goto done;
+        }
+    }
+    if (pos != total_bits) goto done;
+    for (uint64_t k = total_bits; k < 32 * ((total_bits + 31) / 32); k++)
+        if (get_bit(stream, k)) goto done;
+    for (uint64_t b = 4 * ((total_bits + 31) / 32); b < stream_bytes_of(total_bits); b++)
+        if (stream[b]) goto done;
+    rc = DFXO_OK;
+done:
+    free(slot_sym);
+    free(slot_k);
+    return rc;
 }

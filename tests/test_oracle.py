@@ -6,7 +6,11 @@
 * equality with the textbook (heap) Huffman cost when the tree fits the limit;
 * an independent dynamic program for the length-limited optimum (Fibonacci clamp);
 * Kraft equality, the entropy bound, canonical-code prefix-freedom;
-* exhaustive and edge-case round trips, and rejection of malformed containers.
+* exhaustive and edge-case round trips, and rejection of malformed containers;
+* for the tANS exponent coder: hand-worked containers and frequency vectors, the
+  state-numbering and tiling properties of its tables, exact field lengths on dyadic
+  distributions (equal to the package-merge code's), a rate within a hair of the
+  entropy, round trips and rejection of malformed containers.
 """
 import heapq
 import itertools
@@ -84,9 +88,9 @@ def kraft24(lens):
     return sum(1 << (24 - int(l)) for l in lens if l > 0)
 
 
-def load_golden_containers():
+def load_golden_containers(name="tiny_containers.txt"):
     cases, cur = [], None
-    with open(os.path.join(GOLDEN, "tiny_containers.txt")) as fh:
+    with open(os.path.join(GOLDEN, name)) as fh:
         for raw in fh:
             line = raw.split("#", 1)[0].strip()
             if not line:
@@ -94,7 +98,7 @@ def load_golden_containers():
             if line.startswith("case "):
                 parts = line.split()
                 kv = dict(p.split("=") for p in parts[2:])
-                cur = {"name": parts[1], "K": int(kv["K"]), "G": int(kv["G"]),
+                cur = {"name": parts[1], "K": int(kv["K"]), "G": int(kv["G"]), "R": int(kv.get("R", 0)),
                        "bytes": np.zeros(int(kv["total"]), dtype=np.uint8)}
                 cases.append(cur)
             elif line.startswith("input"):
@@ -356,4 +360,227 @@ def test_malformed_containers_are_rejected():
     for name, bad in _corrupt_variants(c).items():
         with pytest.raises(oracle.OracleError) as ei:
             oracle.decode(bad)
+        assert ei.value.code == oracle.ERR_CORRUPT, name
+
+
+# ---------------------------------------------------------------- tANS exponent coder
+
+def load_tans_frequencies():
+    rows = []
+    with open(os.path.join(GOLDEN, "tans_frequencies.txt")) as fh:
+        for raw in fh:
+            line = raw.split("#", 1)[0].strip()
+            if not line:
+                continue
+            R, cnt, exp = (p.strip() for p in line.split("|"))
+            counts = np.zeros(256, dtype=np.uint64)
+            for t in cnt.split():
+                sym, c = t.split(":")
+                counts[int(sym)] = int(c)
+            if exp == "refused":
+                expected = None
+            else:
+                expected = np.zeros(256, dtype=np.uint32)
+                for t in exp.split():
+                    sym, f = t.split(":")
+                    expected[int(sym)] = int(f)
+            rows.append((int(R), counts, expected))
+    return rows
+
+
+@pytest.mark.parametrize("row", load_tans_frequencies(), ids=lambda r: f"R{r[0]}-{int((r[1] > 0).sum())}sym")
+def test_tans_frequency_golden(row):
+    R, counts, expected = row
+    if expected is None:
+        with pytest.raises(oracle.OracleError) as ei:
+            oracle.tans_normalize(counts, R)
+        assert ei.value.code == oracle.ERR_ARG
+    else:
+        assert np.array_equal(oracle.tans_normalize(counts, R), expected)
+
+
+@pytest.mark.parametrize("case", load_golden_containers("tans_containers.txt"), ids=lambda c: c["name"])
+def test_tans_golden_containers(case):
+    got = oracle.encode_tans(case["input"], K=case["K"], G=case["G"], table_log=case["R"])
+    assert got.size == case["bytes"].size
+    assert np.array_equal(got, case["bytes"])
+    assert np.array_equal(oracle.decode(case["bytes"]), case["input"])
+
+
+def test_tans_table_golden():
+    """The M = 16 table worked by hand in tans_containers.txt."""
+    f = np.zeros(256, dtype=np.uint32)
+    f[127], f[128] = 13, 3
+    sym, k = oracle.tans_tables(f, 4)
+    slots_128 = [3, 6, 9]
+    assert [j for j in range(16) if sym[j] == 128] == slots_128
+    assert all(sym[j] == 127 for j in range(16) if j not in slots_128)
+    assert [int(k[j]) for j in slots_128] == [3, 4, 5]
+    assert [int(k[j]) for j in range(16) if j not in slots_128] == list(range(13, 26))
+
+
+def decode_entries(sym, k, R):
+    """(symbol, nb, base) of every slot, from the state numbers alone."""
+    M = 1 << R
+    out = []
+    for j in range(M):
+        kk = int(k[j])
+        nb = R - (kk.bit_length() - 1)
+        out.append((int(sym[j]), nb, (kk << nb) - M))
+    return out
+
+
+def random_frequencies(rng, R, used):
+    M = 1 << R
+    syms = rng.choice(256, size=used, replace=False)
+    cuts = np.sort(rng.choice(np.arange(1, M), size=used - 1, replace=False))
+    f = np.zeros(256, dtype=np.uint32)
+    f[syms] = np.diff(np.concatenate([[0], cuts, [M]]))
+    return f
+
+
+@pytest.mark.parametrize("R", [4, 5, 8, 11, 12])
+def test_tans_tables_number_and_tile(R):
+    """Each symbol holds exactly f[s] slots numbered f[s] .. 2 f[s] - 1 in ascending slot
+    order, and for every symbol the decoder's next-state ranges [base, base + 2^nb) of its
+    slots tile [0, M) exactly: from any state, every symbol has exactly one encoding."""
+    rng = np.random.default_rng(100 + R)
+    M = 1 << R
+    for used in sorted({1, 2, 3, min(16, M), min(200, M), min(256, M)}):
+        f = random_frequencies(rng, R, used)
+        sym, k = oracle.tans_tables(f, R)
+        ent = decode_entries(sym, k, R)
+        for s in np.flatnonzero(f):
+            slots = [j for j in range(M) if sym[j] == s]
+            assert len(slots) == f[s]
+            assert [int(k[j]) for j in slots] == list(range(int(f[s]), 2 * int(f[s])))
+            cover = np.zeros(M, dtype=np.int64)
+            for j in slots:
+                _, nb, base = ent[j]
+                assert 0 <= base and base + (1 << nb) <= M
+                cover[base: base + (1 << nb)] += 1
+            assert np.all(cover == 1)
+
+
+def test_tans_normalize_properties():
+    rng = np.random.default_rng(7)
+    for R in (4, 8, 12):
+        M = 1 << R
+        for trial in range(40):
+            used = int(rng.integers(1, min(M, 256) + 1))
+            counts = np.zeros(256, dtype=np.uint64)
+            syms = rng.choice(256, size=used, replace=False)
+            counts[syms] = rng.integers(1, 10 ** int(rng.integers(1, 7)), size=used)
+            f = oracle.tans_normalize(counts, R)
+            assert int(f.sum()) == M
+            assert np.array_equal(f > 0, counts > 0)
+        # counts proportional to a frequency vector come back unchanged
+        f0 = random_frequencies(rng, R, min(10, M))
+        assert np.array_equal(oracle.tans_normalize(f0.astype(np.uint64) * 37, R), f0)
+    assert not oracle.tans_normalize(np.zeros(256, dtype=np.uint64), 12).any()
+
+
+def dyadic_tensor(n, seed):
+    """Exponents 127, 126, 125, 128 with probabilities exactly 1/2, 1/4, 1/8, 1/8."""
+    rng = np.random.default_rng(seed)
+    e = np.array([127] * (n // 2) + [126] * (n // 4) + [125] * (n // 8) + [128] * (n // 8), dtype=np.uint16)
+    rng.shuffle(e)
+    low = rng.integers(0, 128, size=n, dtype=np.uint16)
+    sign = rng.integers(0, 2, size=n, dtype=np.uint16) << 15
+    return (sign | (e << 7) | low).astype(np.uint16)
+
+
+@pytest.mark.parametrize("K,G,R", [(128, 32, 12), (8, 3, 4), (64, 5, 8)])
+def test_tans_dyadic_fields_equal_the_huffman_lengths(K, G, R):
+    """With f[s] = M 2^-l exactly, a tANS step for s emits exactly l bits (f <= X >> l <
+    2f for every state X in [M, 2M)), so each chunk is R bits longer than its
+    package-merge code: checked chunk by chunk against the Huffman oracle."""
+    n = 8 * 1000 + 8 * (K // 8) * 3
+    w = dyadic_tensor(n, seed=K + R)
+    t = oracle.encode_tans(w, K=K, G=G, table_log=R)
+    h = oracle.encode(w, K=K, G=G)
+    counts = oracle.histogram(w)
+    assert list(oracle.code_lengths(counts)[[127, 126, 125, 128]]) == [1, 2, 3, 3]
+    ng = int(t[44:48].view(np.uint32)[0])
+    nc = ng * G
+    off_t = (576 + 8 * (ng + 1) + 15) // 16 * 16
+    off_h = (320 + 8 * (ng + 1) + 15) // 16 * 16
+    clen_t = t[off_t: off_t + 2 * nc].view(np.uint16).astype(np.int64)
+    clen_h = h[off_h: off_h + 2 * nc].view(np.uint16).astype(np.int64)
+    assert np.array_equal(clen_t, np.where(clen_h > 0, clen_h + R, 0))
+    assert np.array_equal(oracle.decode(t), w)
+
+
+def test_tans_rate_is_near_the_entropy():
+    """On N(0, 0.02^2) exponents the fields cost within 0.003 bits of the empirical
+    entropy H (a coder that numbers the states in spread order instead of ascending
+    order costs ~0.05 bits more, as much as the Huffman code's excess), and below the
+    package-merge code's mean length."""
+    w = inputs.gaussian(1 << 20, 0.02, seed=11)
+    K, R = 4096, 12
+    t = oracle.encode_tans(w, K=K, table_log=R)
+    counts = oracle.histogram(w).astype(np.float64)
+    p = counts[counts > 0] / counts.sum()
+    H = float(-(p * np.log2(p)).sum())
+    chunks = -(-w.size // K)
+    fields = (int(t[16:24].view(np.uint64)[0]) - R * chunks) / w.size
+    huff = cost_of(oracle.histogram(w), oracle.code_lengths(oracle.histogram(w))) / w.size
+    assert H - 0.003 <= fields <= H + 0.003, (H, fields)
+    assert fields < huff - 0.02
+
+
+def test_tans_round_trip_every_bit_pattern():
+    w = inputs.all_patterns_shuffled(26)
+    for R in (8, 12):  # 256 used exponents: at R = 8 every frequency is 1
+        c = oracle.encode_tans(w, K=128, table_log=R)
+        assert np.array_equal(oracle.decode(c), w)
+
+
+@pytest.mark.parametrize("name", list(inputs.edge_cases().keys()))
+def test_tans_round_trip_edge_cases(name):
+    w = inputs.edge_cases()[name]
+    used = int((oracle.histogram(w) > 0).sum())
+    for K, G, R in ((128, 32, 12), (64, 32, 8), (8, 3, 4), (16, 5, 10)):
+        if used > (1 << R):
+            with pytest.raises(oracle.OracleError) as ei:
+                oracle.encode_tans(w, K=K, G=G, table_log=R)
+            assert ei.value.code == oracle.ERR_ARG
+            continue
+        c = oracle.encode_tans(w, K=K, G=G, table_log=R)
+        assert c.size == oracle.tans_container_bytes(w.size, K, G, int(c[16:24].view(np.uint64)[0]))
+        assert c.size <= oracle.tans_max_container_bytes(w.size, K, G, R)
+        assert np.array_equal(oracle.decode(c), w)
+
+
+def test_tans_parameters_are_checked():
+    w = inputs.gaussian(1000, 0.02, seed=3)
+    for K, G, R in ((128, 32, 3), (128, 32, 13), (12, 32, 12), (5464, 32, 12), (128, 0, 12)):
+        with pytest.raises(oracle.OracleError) as ei:
+            oracle.encode_tans(w, K=K, G=G, table_log=R)
+        assert ei.value.code == oracle.ERR_ARG, (K, G, R)
+    oracle.encode_tans(w, K=5456, G=1, table_log=12)  # the largest K with (K + 1) R <= 65535
+
+
+def test_tans_malformed_containers_are_rejected():
+    w = inputs.gaussian(10_003, 0.02, seed=8)
+    c = oracle.encode_tans(w, K=64)
+    assert np.array_equal(oracle.decode(c), w)
+    ng = int(c[44:48].view(np.uint32)[0])
+    off_clen = (576 + 8 * (ng + 1) + 15) // 16 * 16
+    off_m = int(c[48:56].view(np.uint64)[0])
+    n = w.size
+    off_stream = (off_m + n + 15) // 16 * 16
+    bad = {}
+    v = c.copy(); v[60] = 0; bad["coder"] = v  # read as a Huffman container: no valid code lengths
+    v = c.copy(); v[56] = 13; bad["table_log"] = v
+    used = int(np.flatnonzero(c[64:576:2])[0])
+    v = c.copy(); v[64 + 2 * used] += 1; bad["freq_sum"] = v
+    v = c.copy(); v[576 + 8] ^= 1; bad["gbase"] = v
+    v = c.copy(); v[off_clen] ^= 1; bad["clen"] = v
+    v = c.copy(); v[off_stream] ^= 0x80; bad["stream_bit"] = v  # the first chunk's state
+    v = c.copy(); v[-1] = 1; bad["slack"] = v
+    bad["truncated"] = c[:-1].copy()
+    for name, b in bad.items():
+        with pytest.raises(oracle.OracleError) as ei:
+            oracle.decode(b)
         assert ei.value.code == oracle.ERR_CORRUPT, name
