@@ -42,7 +42,7 @@ FALLBACK_HBM_GBS = 6650.0
 WORKLOAD = "70B-shaped layer stream: 24 x BF16[8192, 28672], N(0, 1/8192) + 0.05% N(0, 0.5^2) outliers"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_dram_traffic.txt")
 DECODE_SOURCES = [os.path.join(ROOT, "lossless_entropy_coded_exponent_b200", "csrc", f)
-                  for f in ("decode.cu", "dfx_common.cuh")]
+                  for f in ("decode.cu", "decode_pipeline.cuh", "dfx_common.cuh")]
 
 
 def parse_args():
@@ -57,6 +57,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-layer-batch", action="store_true", help="skip the multi-tensor (Llama-3-8B layer) decode measurement")
+    ap.add_argument("--no-tans", action="store_true", help="skip the tANS exponent coder comparison")
     return ap.parse_args()
 
 
@@ -376,7 +377,7 @@ def run_ours(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": algo_bytes_per_launch,
-                         "mean_launch_us": 1e3 * mean_launch_ms, "kernel": f"k_decode<{K}>"},
+                         "mean_launch_us": 1e3 * mean_launch_ms, "kernel": f"k_decode<HuffmanCoder, {K}>"},
             "gpu_launches": args.steps * T,
             "clocks": clocks.summary(),
             "encode": {"unit": "GB/s", "value": 2.0 * n / (statistics.median(enc_ms) * 1e-3) / 1e9,
@@ -394,11 +395,84 @@ def run_ours(args, world, rank, local):
     # ---- decode feeding its consumer: slices through an L2-sized buffer into a GEMM
     if not args.no_layer_batch and rank == 0:
         line["decode_into_gemm"] = run_decode_into_gemm(args, dev)
+    # ---- the other exponent coder (tANS) on the same tensors and launch configuration
+    if not args.no_tans and rank == 0:
+        line["tans"] = run_tans_compare(args, dev, stream, xs, sizes, 1e3 * mean_launch_ms, n)
     # ---- oracle on the host: rank 0 at N=1 only
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         line["cpu_baseline"], line["bit_exact_vs_oracle"] = run_cpu_baseline(xs[0], comps[0], K)
     plan.free()
     return line
+
+
+def run_tans_compare(args, dev, stream, xs, huff_sizes, huff_launch_us, n, tensors=4, reps=10):
+    """The tANS exponent coder (4096 states) on the first `tensors` tensors of the workload,
+    with the same chunk size and launch configuration: bits/weight, encode time and decode
+    time per launch (CUDA events, launches back to back into the reused output buffer),
+    next to the Huffman coder's numbers on the same tensors."""
+    import numpy as np
+    import torch
+
+    import lossless_entropy_coded_exponent_b200 as dfx
+
+    T = min(tensors, len(xs))
+    K = args.chunk_symbols
+    plan = dfx.dfx_plan(n, chunk_symbols=K, coder=dfx.DFX_CODER_TANS)
+    try:
+        scratch = torch.empty(plan.max_compressed_bytes, dtype=torch.uint8, device=dev)
+        ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
+        comps, sizes, enc_ms = [], [], []
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for i in range(T):
+                e0.record(stream)
+                dfx.dfx_encode(plan, xs[i], scratch, scratch.numel(), ws, ws.numel(), stream=stream)
+                e1.record(stream)
+                stream.synchronize()
+                enc_ms.append(e0.elapsed_time(e1))
+                size = int(scratch[24:32].cpu().numpy().view(np.uint64)[0])
+                comps.append(scratch[:size].clone())
+                sizes.append(size)
+        del scratch, ws
+        out = torch.empty(n, dtype=torch.int16, device=dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps * T + 1)]
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                for i in range(T):
+                    dfx.dfx_decode(plan, comps[i], sizes[i], out, stream=stream)
+            ev[0].record(stream)
+            k = 1
+            for _ in range(reps):
+                for i in range(T):
+                    dfx.dfx_decode(plan, comps[i], sizes[i], out, stream=stream)
+                    ev[k].record(stream)
+                    k += 1
+        stream.synchronize()
+        launch_us = [1e3 * ev[j].elapsed_time(ev[j + 1]) for j in range(len(ev) - 1)]
+        exact = dfx.dfx_device_status(plan, stream=stream) == 0
+        with torch.cuda.stream(stream):
+            for i in range(T):
+                out.fill_(-1)
+                dfx.dfx_decode(plan, comps[i], sizes[i], out, stream=stream)
+                stream.synchronize()
+                exact &= bool(torch.equal(out, xs[i]))
+        exact &= dfx.dfx_device_status(plan, stream=stream) == 0
+        mean_us = statistics.mean(launch_us)
+        algo = float(sum(sizes)) / T + 2.0 * n
+        achieved = algo / (mean_us * 1e-6) / 1e9
+        peak, peak_kind = measured_hbm_peak()
+        return {"coder": "tANS, 4096 states", "tensors": T, "chunk_symbols": K,
+                "bits_per_weight": 8.0 * sum(sizes) / (n * T),
+                "huffman_bits_per_weight": 8.0 * sum(huff_sizes[:T]) / (n * T),
+                "decode_mean_launch_us": mean_us, "huffman_mean_launch_us": huff_launch_us,
+                "decode_bf16_gbs": 2.0 * n / (mean_us * 1e-6) / 1e9,
+                "decode_algorithmic_gbs": achieved, "decode_frac_of_measured": achieved / peak, "peak_kind": peak_kind,
+                "encode_median_ms_per_tensor": statistics.median(enc_ms), "bit_exact": bool(exact),
+                "kernel": f"k_decode<TansCoder, {K}>",
+                "note": f"{reps} x {T} launches back to back after 3 x {T} warm-up; the Huffman figures are "
+                        "the main measurement's (same shape, K and grid)"}
+    finally:
+        plan.free()
 
 
 def run_layer_batch(args, dev, stream):

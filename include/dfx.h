@@ -25,6 +25,18 @@
  *     equal weight, codes assigned in (length, symbol) order; a tensor with a
  *     single exponent value gets a second, never-used phantom symbol (1 if the
  *     value is 0, else 0) so both codes are 1 bit long;
+ *   - or (coder 1, DFX_CODER_TANS) the exponents are coded with tabled asymmetric
+ *     numeral systems (tANS; one page names ANS as the coder of its compressed
+ *     number formats: the "From a Lossless (~1.5:1) ..." abstract) over a table of
+ *     M = 2^table_log states: every used exponent gets f[s] = count * M / n rounded
+ *     half up (at least 1), the largest f (smallest symbol among equal ones) taking a
+ *     shortfall or giving up an excess one unit at a time; occurrence i of the
+ *     symbol-ordered list of f[s] copies per symbol takes slot (i * step) mod M,
+ *     step = M/2 + M/8 + 3; each symbol's slots, ascending, are states f[s] ..
+ *     2 f[s] - 1; a chunk is encoded from its last symbol to its first from state M
+ *     (for symbol s, nb bits with f[s] <= X >> nb < 2 f[s] are emitted, low bits of
+ *     X, and X becomes M + the slot of state X >> nb) and stored as the final state
+ *     minus M (table_log bits) followed by the fields in symbol order;
  *   - the m bytes are stored raw, in element order;
  *   - the exponent codes are cut into chunks of K codes, 32 chunks to a group:
  *     a group covers 32*K consecutive elements in 8-element blocks, block b of
@@ -42,7 +54,7 @@
  *   off 36  u32 G                 chunks per group (one warp)
  *   off 40  u32 n_chunk = G * n_group;  off 44  u32 n_group = ceil(n / (G * K))
  *   off 48  u64 off_m             offset of the sign+mantissa plane
- *   off 56  u32 max_len;          off 60  u32 reserved = 0
+ *   off 56  u32 max_len;          off 60  u32 coder = 0
  *   off 64  u8  len[256]          code length per exponent value, 0 = unused
  *   off 320 u64 gbase[n_group+1]  start bit of each group; last = total_bits
  *   then    u16 clen[n_chunk]     bit length of each chunk (0 for an empty chunk)
@@ -51,6 +63,9 @@
  *                                 31 - (k mod 32) of word k / 32; the section
  *                                 is 4*ceil(total_bits/32) bytes rounded up
  *                                 to 16, plus 16 zero bytes
+ * Coder 1 changes three things: off 56 holds table_log (4..12), off 60 holds
+ * coder = 1, and u16 freq[256] (summing to 2^table_log, all 0 when n = 0) sits at
+ * off 64 with gbase following at off 576; the other sections are as above.
  * Two conforming encoders produce identical bytes for the same input and
  * parameters.
  *
@@ -89,7 +104,8 @@ typedef struct CUstream_st *cudaStream_t;
 
 /* Bits of the device status word (dfx_device_status). */
 #define DFX_STATUS_HEADER 0x1u  /* header disagrees with the plan or the buffer size */
-#define DFX_STATUS_TABLE 0x2u   /* code lengths above 24 or Kraft sum not exactly 1 */
+#define DFX_STATUS_TABLE 0x2u   /* code lengths above 24 or Kraft sum not exactly 1
+                                   (coder 1: frequencies not summing to 2^table_log) */
 #define DFX_STATUS_INDEX 0x4u   /* group start bits or chunk lengths inconsistent */
 #define DFX_STATUS_STREAM 0x8u  /* a bit pattern that is no code, or a chunk that
                                    did not consume exactly its stated length */
@@ -98,16 +114,24 @@ typedef struct CUstream_st *cudaStream_t;
 
 typedef struct dfx_plan_s *dfx_plan_t; /* opaque, host-owned */
 
+/* Exponent coders. */
+#define DFX_CODER_HUFFMAN 0u /* canonical length-limited Huffman (the default) */
+#define DFX_CODER_TANS 1u    /* tabled asymmetric numeral systems */
+
 typedef struct {
     uint32_t chunk_symbols; /* K: a multiple of 8; 32, 64 or 128 on the GPU path (0 -> 128) */
     uint32_t group_chunks;  /* G: 32 on the GPU path (0 -> 32) */
-    uint32_t max_len;       /* code-length limit, 8..24 (0 -> 24) */
+    uint32_t max_len;       /* coder 0: code-length limit, 8..24 (0 -> 24) */
+    uint32_t coder;         /* DFX_CODER_HUFFMAN or DFX_CODER_TANS */
+    uint32_t table_log;     /* coder 1: log2 of the state table, 4..12 (0 -> 12); dfx_encode
+                               needs 8..12 (room for all 256 exponent values), every value
+                               decodes */
 } dfx_params;
 
 /* Byte offsets of the container sections for given n, params and stream length. */
 typedef struct {
     uint64_t n, n_chunk, n_group;
-    uint64_t off_len, off_gbase, off_clen, off_m, off_stream;
+    uint64_t off_len, off_gbase, off_clen, off_m, off_stream;  /* off_len: the code section */
     uint64_t stream_bytes, total_bytes;
 } dfx_layout;
 
@@ -232,6 +256,7 @@ int dfx_free(dfx_plan_t plan);
  *   dfx_plan + dfx_encode (out_capacity >= the plan's max_compressed_bytes).
  * Limit: at most 262144 groups of 32 chunks (n <= 2^28 with K = 32, 2^29 with
  * K = 64, 2^30 with K = 128); larger n returns DFX_ERR_CAPACITY before any work.
+ * Coder 0 only (coder 1 returns DFX_ERR_UNSUPPORTED).
  * All calls on a device share the scratch array and it keeps the last call's
  * contents; calls whose GPU work overlaps race and corrupt each other, so order
  * them on one stream.  The first call on a device looks up the array's address

@@ -29,6 +29,8 @@ DFX_STATUS_INDEX = 0x4
 DFX_STATUS_STREAM = 0x8
 DFX_STATUS_TIMEOUT = 0x10
 DFX_INJECT_SKIP_SLICE_COPY = 0x1
+DFX_CODER_HUFFMAN = 0
+DFX_CODER_TANS = 1
 
 # The exported C symbols, in include/dfx.h order.
 EXPORTS = (
@@ -55,7 +57,8 @@ class DfxError(RuntimeError):
 
 
 class dfx_params(ctypes.Structure):
-    _fields_ = [("chunk_symbols", ctypes.c_uint32), ("group_chunks", ctypes.c_uint32), ("max_len", ctypes.c_uint32)]
+    _fields_ = [("chunk_symbols", ctypes.c_uint32), ("group_chunks", ctypes.c_uint32), ("max_len", ctypes.c_uint32),
+                ("coder", ctypes.c_uint32), ("table_log", ctypes.c_uint32)]
 
 
 class dfx_layout(ctypes.Structure):
@@ -125,8 +128,8 @@ def _stream(s) -> int | None:
     return s.cuda_stream
 
 
-def _params(chunk_symbols=0, group_chunks=0, max_len=0):
-    return dfx_params(chunk_symbols, group_chunks, max_len)
+def _params(chunk_symbols=0, group_chunks=0, max_len=0, coder=DFX_CODER_HUFFMAN, table_log=0):
+    return dfx_params(chunk_symbols, group_chunks, max_len, coder, table_log)
 
 
 def dfx_version() -> int:
@@ -137,9 +140,10 @@ def dfx_strerror(code: int) -> str:
     return lib().dfx_strerror(code).decode()
 
 
-def dfx_container_layout(n: int, total_bits: int, chunk_symbols=0, group_chunks=0, max_len=0) -> dict:
+def dfx_container_layout(n: int, total_bits: int, chunk_symbols=0, group_chunks=0, max_len=0,
+                         coder=DFX_CODER_HUFFMAN, table_log=0) -> dict:
     out = dfx_layout()
-    p = _params(chunk_symbols, group_chunks, max_len)
+    p = _params(chunk_symbols, group_chunks, max_len, coder, table_log)
     _check(lib().dfx_container_layout(n, ctypes.byref(p), total_bits, ctypes.byref(out)), "dfx_container_layout")
     return {name: int(getattr(out, name)) for name, _ in dfx_layout._fields_}
 
@@ -172,13 +176,14 @@ class Plan:
             pass
 
 
-def dfx_plan(n: int, chunk_symbols: int = 0, group_chunks: int = 0, max_len: int = 0) -> Plan:
+def dfx_plan(n: int, chunk_symbols: int = 0, group_chunks: int = 0, max_len: int = 0,
+             coder: int = DFX_CODER_HUFFMAN, table_log: int = 0) -> Plan:
     h = ctypes.c_void_p()
     mx = ctypes.c_size_t()
     ws = ctypes.c_size_t()
-    p = _params(chunk_symbols, group_chunks, max_len)
+    p = _params(chunk_symbols, group_chunks, max_len, coder, table_log)
     _check(lib().dfx_plan(ctypes.byref(h), n, ctypes.byref(p), ctypes.byref(mx), ctypes.byref(ws)), "dfx_plan")
-    return Plan(h.value, n, mx.value, ws.value, (chunk_symbols, group_chunks, max_len))
+    return Plan(h.value, n, mx.value, ws.value, (chunk_symbols, group_chunks, max_len, coder, table_log))
 
 
 def dfx_encode(plan: Plan, d_bf16, d_out, out_capacity: int, d_workspace, workspace_bytes: int,
@@ -249,11 +254,12 @@ def dfx_free(plan: Plan) -> None:
 
 
 def dfx_encode_static(d_bf16, n: int, d_out, out_capacity: int, want_size: bool = False, stream=None,
-                      chunk_symbols: int = 0, group_chunks: int = 0, max_len: int = 0) -> int | None:
+                      chunk_symbols: int = 0, group_chunks: int = 0, max_len: int = 0,
+                      coder: int = DFX_CODER_HUFFMAN) -> int | None:
     """Encode without any device allocation by the library (no plan, no workspace);
-    for callers whose device memory is owned by another allocator."""
+    for callers whose device memory is owned by another allocator (coder 0 only)."""
     size = ctypes.c_size_t()
-    p = _params(chunk_symbols, group_chunks, max_len)
+    p = _params(chunk_symbols, group_chunks, max_len, coder)
     rc = lib().dfx_encode_static(_ptr(d_bf16), n, ctypes.byref(p), _ptr(d_out), out_capacity,
                                  ctypes.byref(size) if want_size else None, _stream(stream))
     _check(rc, "dfx_encode_static")

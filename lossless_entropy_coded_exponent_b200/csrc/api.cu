@@ -10,6 +10,7 @@
 struct dfx_plan_s {
     uint64_t n;
     uint32_t K, G, max_len;
+    uint32_t coder, table_log;  // exponent coder; tANS table log (coder 1)
     dfx::Layout L;
     uint64_t max_bytes;
     uint64_t ws_bytes;
@@ -26,14 +27,37 @@ struct dfx_plan_s {
 
 namespace {
 
-int resolve_params(const dfx_params* p, uint32_t* K, uint32_t* G, uint32_t* L) {
-    *K = (p && p->chunk_symbols) ? p->chunk_symbols : 128u;
-    *G = (p && p->group_chunks) ? p->group_chunks : 32u;
-    *L = (p && p->max_len) ? p->max_len : 24u;
-    if (*L < 8 || *L > dfx::kMaxLenLimit) return DFX_ERR_ARG;
-    if (*K < 8 || *K % 8 != 0) return DFX_ERR_ARG;  // chunks are made of 8-element blocks
-    if ((uint64_t)(*K) * (*L) > 65535u) return DFX_ERR_ARG;  // a chunk's bit length must fit u16
+struct Params {
+    uint32_t K, G, L, coder, R;
+};
+
+// Defaults and checks of dfx_params.  Only the fields of the chosen coder are checked:
+// max_len for coder 0, table_log for coder 1.
+int resolve_params(const dfx_params* p, Params* r) {
+    r->K = (p && p->chunk_symbols) ? p->chunk_symbols : 128u;
+    r->G = (p && p->group_chunks) ? p->group_chunks : 32u;
+    r->L = (p && p->max_len) ? p->max_len : 24u;
+    r->coder = p ? p->coder : DFX_CODER_HUFFMAN;
+    r->R = (p && p->table_log) ? p->table_log : dfx::kTansMaxLog;
+    if (r->K < 8 || r->K % 8 != 0) return DFX_ERR_ARG;  // chunks are made of 8-element blocks
+    if (r->coder == DFX_CODER_HUFFMAN) {
+        if (r->L < 8 || r->L > dfx::kMaxLenLimit) return DFX_ERR_ARG;
+        if ((uint64_t)r->K * r->L > 65535u) return DFX_ERR_ARG;  // a chunk's bit length must fit u16
+        r->R = 0;
+    } else if (r->coder == DFX_CODER_TANS) {
+        if (r->R < dfx::kTansMinLog || r->R > dfx::kTansMaxLog) return DFX_ERR_ARG;
+        if ((uint64_t)(r->K + 1) * r->R > 65535u) return DFX_ERR_ARG;  // fields and state fit u16
+        r->L = 0;
+    } else {
+        return DFX_ERR_ARG;
+    }
     return DFX_OK;
+}
+
+// Longest stream a coder may produce: at most 8 bits per exponent for an optimal prefix
+// code, at most table_log bits per exponent and per chunk for tANS.
+uint64_t max_stream_bits(const Params& q, uint64_t n, uint64_t n_chunk) {
+    return q.coder == DFX_CODER_TANS ? (uint64_t)q.R * (n + n_chunk) : 8 * n;
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -77,16 +101,16 @@ const char* dfx_strerror(int code) {
 int dfx_container_layout(uint64_t n, const dfx_params* params, uint64_t total_bits, dfx_layout* out) {
     if (!out) return DFX_ERR_ARG;
     if (n >= (1ull << 32)) return DFX_ERR_TOO_LARGE;
-    uint32_t K, G, L;
-    int rc = resolve_params(params, &K, &G, &L);
+    Params q;
+    int rc = resolve_params(params, &q);
     if (rc) return rc;
-    if (G < 1) return DFX_ERR_ARG;
-    const dfx::Layout lay = dfx::make_layout(n, K, G);
+    if (q.G < 1) return DFX_ERR_ARG;
+    const dfx::Layout lay = dfx::make_layout(n, q.K, q.G, q.coder);
     out->n = n;
     out->n_chunk = lay.n_chunk;
     out->n_group = lay.n_group;
-    out->off_len = dfx::kOffLen;
-    out->off_gbase = dfx::kOffGbase;
+    out->off_len = q.coder == DFX_CODER_TANS ? dfx::kOffFreq : dfx::kOffLen;
+    out->off_gbase = lay.off_gbase;
     out->off_clen = lay.off_clen;
     out->off_m = lay.off_m;
     out->off_stream = lay.off_stream;
@@ -100,9 +124,10 @@ int dfx_plan(dfx_plan_t* plan, uint64_t n, const dfx_params* params, size_t* max
     if (!plan) return DFX_ERR_ARG;
     *plan = nullptr;
     if (n >= (1ull << 32)) return DFX_ERR_TOO_LARGE;
-    uint32_t K, G, L;
-    int rc = resolve_params(params, &K, &G, &L);
+    Params q;
+    int rc = resolve_params(params, &q);
     if (rc) return rc;
+    const uint32_t K = q.K, G = q.G;
     if (!dfx::decode_supports(K, G)) return DFX_ERR_UNSUPPORTED;
 
     dfx_plan_s* p = (dfx_plan_s*)calloc(1, sizeof(dfx_plan_s));
@@ -110,10 +135,12 @@ int dfx_plan(dfx_plan_t* plan, uint64_t n, const dfx_params* params, size_t* max
     p->n = n;
     p->K = K;
     p->G = G;
-    p->max_len = L;
-    p->L = dfx::make_layout(n, K, G);
-    p->max_bytes = p->L.off_stream + dfx::stream_bytes(8 * n);  // optimal codes never exceed 8 bits/symbol
-    p->ws_bytes = dfx::workspace_bytes_for(p->L.n_group);
+    p->max_len = q.L;
+    p->coder = q.coder;
+    p->table_log = q.R;
+    p->L = dfx::make_layout(n, K, G, q.coder);
+    p->max_bytes = p->L.off_stream + dfx::stream_bytes(max_stream_bits(q, n, p->L.n_chunk));
+    p->ws_bytes = dfx::workspace_bytes_for(p->L.n_group, q.coder);
     int sms = 0;
     if (cudaGetDevice(&p->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess ||
@@ -123,7 +150,7 @@ int dfx_plan(dfx_plan_t* plan, uint64_t n, const dfx_params* params, size_t* max
         free(p);
         return DFX_ERR_CUDA;
     }
-    const uint64_t resident = dfx::decode_blocks_per_sm(K) * (uint64_t)sms;  // CTAs that fit at once
+    const uint64_t resident = dfx::decode_blocks_per_sm(K, q.coder) * (uint64_t)sms;  // CTAs that fit at once
     p->resident_ctas = (int)resident;
     const uint64_t wpb = (uint64_t)dfx::decode_warps_per_block(K);
     const uint64_t need = (p->L.n_group + wpb - 1) / wpb;                    // CTAs with work (a warp per group)
@@ -140,6 +167,8 @@ int dfx_encode(dfx_plan_t plan, const void* d_bf16, void* d_out, size_t out_capa
     if (!d_out || !d_workspace || (!d_bf16 && plan->n)) return DFX_ERR_ARG;
     if (!aligned16(d_bf16) || !aligned16(d_out) || !aligned16(d_workspace)) return DFX_ERR_ARG;
     if (out_capacity < plan->max_bytes || workspace_bytes < plan->ws_bytes) return DFX_ERR_CAPACITY;
+    // all 256 exponent values must fit a tANS table
+    if (plan->coder == DFX_CODER_TANS && plan->table_log < 8) return DFX_ERR_UNSUPPORTED;
     int rc = check_device(plan);
     if (rc) return rc;
     dfx::EncodeArgs a;
@@ -149,8 +178,11 @@ int dfx_encode(dfx_plan_t plan, const void* d_bf16, void* d_out, size_t out_capa
     a.K = plan->K;
     a.G = plan->G;
     a.max_len = plan->max_len;
+    a.coder = plan->coder;
+    a.table_log = plan->table_log;
     a.n_chunk = (uint32_t)plan->L.n_chunk;
     a.n_group = (uint32_t)plan->L.n_group;
+    a.off_gbase = plan->L.off_gbase;
     a.off_clen = plan->L.off_clen;
     a.off_m = plan->L.off_m;
     a.off_stream = plan->L.off_stream;
@@ -159,6 +191,7 @@ int dfx_encode(dfx_plan_t plan, const void* d_bf16, void* d_out, size_t out_capa
     a.ws_code = (uint32_t*)(ws + dfx::kWsCode);
     a.ws_len = ws + dfx::kWsLen;
     a.ws_group_bits = (uint32_t*)(ws + dfx::kWsGroupBits);
+    a.ws_tans = (uint32_t*)(ws + dfx::ws_tans_offset(plan->L.n_group));
     a.status = plan->d_status;
     if (dfx::launch_encode(a, plan->max_bytes, stream) != cudaSuccess) {
         cudaGetLastError();
@@ -180,7 +213,7 @@ int dfx_decode(dfx_plan_t plan, const void* d_comp, size_t comp_bytes, void* d_b
     dfx::DecodeArgs a;
     const int rc = make_decode_args(plan, d_comp, comp_bytes, d_bf16, &a);
     if (rc) return rc;
-    if (dfx::launch_decode(a, plan->decode_grid, stream) != cudaSuccess) {
+    if (dfx::launch_decode(a, plan->coder, plan->decode_grid, stream) != cudaSuccess) {
         cudaGetLastError();
         return DFX_ERR_CUDA;
     }
@@ -200,7 +233,7 @@ int dfx_decode_range(dfx_plan_t plan, const void* d_comp, size_t comp_bytes, uin
     a.out_first = first_group * (uint64_t)plan->G * plan->K;
     const uint64_t need = (group_count + 31) / 32;  // a warp per group
     const int grid = (int)(need < (uint64_t)plan->resident_ctas ? need : (uint64_t)plan->resident_ctas);
-    if (dfx::launch_decode(a, grid, stream) != cudaSuccess) {
+    if (dfx::launch_decode(a, plan->coder, grid, stream) != cudaSuccess) {
         cudaGetLastError();
         return DFX_ERR_CUDA;
     }
@@ -236,12 +269,12 @@ int dfx_decode_host(dfx_plan_t plan, const void* h_comp, size_t comp_bytes, void
     const uint8_t* h = (const uint8_t*)h_comp;
     uint8_t* d = (uint8_t*)d_staging;
     const uint64_t ge = (uint64_t)L.G * L.K;
-    const uint64_t* gbase = (const uint64_t*)(h + dfx::kOffGbase);
+    const uint64_t* gbase = (const uint64_t*)(h + L.off_gbase);
     auto fail = [] {
         cudaGetLastError();
         return DFX_ERR_CUDA;
     };
-    // header, code lengths and the group index: every slice's decode reads them
+    // header, code section and the group index: every slice's decode reads them
     if (cudaMemcpyAsync(d, h, L.off_m, cudaMemcpyHostToDevice, copy_stream) != cudaSuccess) return fail();
     for (uint64_t s = 0; s < ns; s++) {
         const uint64_t g0 = ng * s / ns, g1 = ng * (s + 1) / ns;
@@ -277,7 +310,8 @@ int dfx_decode_batch(const dfx_plan_t* plans, const void* const* d_comps, const 
     uint64_t groups[dfx::kMaxBatch];
     for (uint32_t i = 0; i < count; i++) {
         if (!plans[i]) return DFX_ERR_ARG;
-        if (plans[i]->K != plans[0]->K || plans[i]->device != plans[0]->device) return DFX_ERR_UNSUPPORTED;
+        if (plans[i]->K != plans[0]->K || plans[i]->coder != plans[0]->coder || plans[i]->device != plans[0]->device)
+            return DFX_ERR_UNSUPPORTED;
         const int rc = make_decode_args(plans[i], d_comps[i], comp_bytes[i], d_bf16s[i], &b.t[i]);
         if (rc) return rc;
         groups[i] = plans[i]->L.n_group;
@@ -299,7 +333,7 @@ int dfx_decode_batch(const dfx_plan_t* plans, const void* const* d_comps, const 
     }
     b.cta_begin[0] = 0;
     for (uint32_t i = 0; i < count; i++) b.cta_begin[i + 1] = b.cta_begin[i] + ctas[i];
-    if (dfx::launch_decode_batch(b, plans[0]->K, stream) != cudaSuccess) {
+    if (dfx::launch_decode_batch(b, plans[0]->K, plans[0]->coder, stream) != cudaSuccess) {
         cudaGetLastError();
         return DFX_ERR_CUDA;
     }

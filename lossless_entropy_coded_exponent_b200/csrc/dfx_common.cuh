@@ -10,28 +10,35 @@
 namespace dfx {
 
 constexpr uint32_t kHeaderBytes = 64;
-constexpr uint32_t kOffLen = 64;
-constexpr uint32_t kOffGbase = 320;
+constexpr uint32_t kOffLen = 64;        // coder 0: u8 len[256]
+constexpr uint32_t kOffGbase = 320;     // coder 0: group start bits
+constexpr uint32_t kOffFreq = 64;       // coder 1: u16 freq[256]
+constexpr uint32_t kOffGbaseTans = 576; // coder 1: group start bits
 constexpr uint32_t kMaxLenLimit = 24;   // longest code the decoder tables support
+constexpr uint32_t kTansMinLog = 4, kTansMaxLog = 12;  // tANS table sizes 2^4 .. 2^12
 constexpr uint32_t kWarp = 32;
+
+__host__ __device__ inline uint32_t gbase_offset(uint32_t coder) { return coder == DFX_CODER_TANS ? kOffGbaseTans : kOffGbase; }
 
 __host__ __device__ inline uint64_t align16(uint64_t x) { return (x + 15u) & ~uint64_t(15); }
 
 struct Layout {
     uint64_t n, n_chunk, n_group;
-    uint64_t off_clen, off_m, off_stream;
-    uint32_t K, G;
+    uint64_t off_gbase, off_clen, off_m, off_stream;
+    uint32_t K, G, coder;
 };
 
-__host__ __device__ inline Layout make_layout(uint64_t n, uint32_t K, uint32_t G) {
+__host__ __device__ inline Layout make_layout(uint64_t n, uint32_t K, uint32_t G, uint32_t coder = DFX_CODER_HUFFMAN) {
     Layout L;
     L.n = n;
     L.K = K;
     L.G = G;
+    L.coder = coder;
+    L.off_gbase = gbase_offset(coder);
     // a group holds G * K elements in 8-element blocks; block b belongs to chunk b mod G
     L.n_group = (n + (uint64_t)G * K - 1) / ((uint64_t)G * K);
     L.n_chunk = L.n_group * G;
-    L.off_clen = align16(kOffGbase + 8 * (L.n_group + 1));
+    L.off_clen = align16(L.off_gbase + 8 * (L.n_group + 1));
     L.off_m = align16(L.off_clen + 2 * L.n_chunk);
     L.off_stream = align16(L.off_m + n);
     return L;
@@ -66,12 +73,14 @@ struct EncodeArgs {
     uint8_t* out;
     uint64_t n;
     uint32_t K, G, max_len;
+    uint32_t coder, table_log;      // DFX_CODER_*; tANS table log (coder 1)
     uint32_t n_chunk, n_group;
-    uint64_t off_clen, off_m, off_stream;
+    uint64_t off_gbase, off_clen, off_m, off_stream;
     unsigned long long* ws_counts;  // [256]
     uint32_t* ws_code;              // [256]
     uint8_t* ws_len;                // [256]
     uint32_t* ws_group_bits;        // [n_group]
+    uint32_t* ws_tans;              // coder 1: [kWsTansWords] encode tables
     uint32_t* status;
 };
 
@@ -88,16 +97,29 @@ constexpr uint64_t kWsCounts = 0;
 constexpr uint64_t kWsCode = 2048;
 constexpr uint64_t kWsLen = 3072;
 constexpr uint64_t kWsGroupBits = 4096;
-inline uint64_t workspace_bytes_for(uint64_t n_group) {
-    return (kWsGroupBits + 4 * n_group + 255) & ~uint64_t(255);
+// coder 1: per symbol (threshold << 16 | nb_hi, cs << 16 | f) and the slot of every
+// (symbol, state number) pair, after the group sums
+constexpr uint64_t kWsTansWords = 2 * 256 + (1u << kTansMaxLog);
+inline uint64_t ws_tans_offset(uint64_t n_group) { return (kWsGroupBits + 4 * n_group + 255) & ~uint64_t(255); }
+inline uint64_t workspace_bytes_for(uint64_t n_group, uint32_t coder = DFX_CODER_HUFFMAN) {
+    const uint64_t base = ws_tans_offset(n_group);
+    return coder == DFX_CODER_TANS ? base + 4 * kWsTansWords : base;
 }
 
-// Launchers (encode.cu / decode.cu).
+// Launchers (encode.cu, encode_tans.cu / decode.cu, decode_tans.cu); `coder` selects the
+// exponent coder's kernels.
 cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t s);
-cudaError_t launch_decode(const DecodeArgs& a, int grid, cudaStream_t s);
-cudaError_t launch_decode_batch(const BatchArgs& b, uint32_t K, cudaStream_t s);
-int decode_blocks_per_sm(uint32_t K);
+cudaError_t launch_encode_tans(const EncodeArgs& a, int phase, cudaStream_t s);  // 0: before the group scan, 1: after
+cudaError_t launch_decode(const DecodeArgs& a, uint32_t coder, int grid, cudaStream_t s);
+cudaError_t launch_decode_batch(const BatchArgs& b, uint32_t K, uint32_t coder, cudaStream_t s);
+int decode_blocks_per_sm(uint32_t K, uint32_t coder);
 int decode_warps_per_block(uint32_t K);
 bool decode_supports(uint32_t K, uint32_t G);
+cudaError_t launch_decode_huffman(const DecodeArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_decode_batch_huffman(const BatchArgs& b, uint32_t K, cudaStream_t s);
+int decode_blocks_per_sm_huffman(uint32_t K);
+cudaError_t launch_decode_tans(const DecodeArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_decode_batch_tans(const BatchArgs& b, uint32_t K, cudaStream_t s);
+int decode_blocks_per_sm_tans(uint32_t K);
 
 }  // namespace dfx

@@ -10,7 +10,8 @@
 //                       chunk b mod 32, so lane i of a warp reads blocks i, i+32, ...
 //                       (16-byte loads, 512 contiguous bytes per warp instruction);
 //   4. k_group_scan     one CTA: exclusive scan of the group sums -> gbase, total_bits,
-//                       total_bytes;
+//                       total_bytes (shared with the tANS coder, whose passes 2, 3 and 5
+//                       are in encode_tans.cu);
 //   5. k_pack           per chunk: start bit from gbase + warp scan of clen, codes packed
 //                       MSB-first into 32-bit words in the same block order; the
 //                       mantissa+sign bytes (mantissa * 2 + the sign of the pair partner,
@@ -328,7 +329,7 @@ constexpr int kScanItems = 16;  // four 16-byte loads per thread per round
 __global__ void __launch_bounds__(kScanThreads) k_group_scan(EncodeArgs a) {
     __shared__ unsigned long long wsum[32];
     const unsigned t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    unsigned long long* gbase = reinterpret_cast<unsigned long long*>(a.out + kOffGbase);
+    unsigned long long* gbase = reinterpret_cast<unsigned long long*>(a.out + a.off_gbase);
     unsigned long long carry = 0;
     for (uint64_t base = 0; base < a.n_group; base += (uint64_t)kScanThreads * kScanItems) {
         const uint64_t i = base + (uint64_t)t * kScanItems;
@@ -578,6 +579,12 @@ cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t 
     const unsigned hist_blocks = (unsigned)(units == 0 ? 1 : (units < resident ? units : resident));
     k_histogram<<<hist_blocks, kHistThreads, 0, s>>>(a.in, a.n, a.ws_counts);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (a.coder == DFX_CODER_TANS) {  // the tANS passes around the same group scan
+        if ((err = launch_encode_tans(a, 0, s)) != cudaSuccess) return err;
+        k_group_scan<<<1, kScanThreads, 0, s>>>(a);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        return launch_encode_tans(a, 1, s);
+    }
     k_build_codebook<<<1, 256, 0, s>>>(a);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (a.n_chunk) {

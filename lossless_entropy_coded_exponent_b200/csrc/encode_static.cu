@@ -52,6 +52,8 @@ extern "C" int dfx_encode_static(const void* d_bf16, uint64_t n, const dfx_param
     const uint32_t G = (params && params->group_chunks) ? params->group_chunks : 32u;
     const uint32_t L = (params && params->max_len) ? params->max_len : 24u;
     if (L < 8 || L > dfx::kMaxLenLimit || K < 8 || K % 8 != 0) return DFX_ERR_ARG;
+    if (params && params->coder == DFX_CODER_TANS) return DFX_ERR_UNSUPPORTED;
+    if (params && params->coder != DFX_CODER_HUFFMAN) return DFX_ERR_ARG;
     if (!dfx::decode_supports(K, G)) return DFX_ERR_UNSUPPORTED;
     if (!d_out || (!d_bf16 && n)) return DFX_ERR_ARG;
     if (((uintptr_t)d_bf16 & 15u) || ((uintptr_t)d_out & 15u)) return DFX_ERR_ARG;
@@ -87,8 +89,11 @@ extern "C" int dfx_encode_static(const void* d_bf16, uint64_t n, const dfx_param
     a.K = K;
     a.G = G;
     a.max_len = L;
+    a.coder = DFX_CODER_HUFFMAN;
+    a.table_log = 0;
     a.n_chunk = (uint32_t)lay.n_chunk;
     a.n_group = (uint32_t)lay.n_group;
+    a.off_gbase = lay.off_gbase;
     a.off_clen = lay.off_clen;
     a.off_m = lay.off_m;
     a.off_stream = lay.off_stream;
@@ -96,6 +101,7 @@ extern "C" int dfx_encode_static(const void* d_bf16, uint64_t n, const dfx_param
     a.ws_code = (uint32_t*)(scratch + dfx::kWsCode);
     a.ws_len = scratch + dfx::kWsLen;
     a.ws_group_bits = (uint32_t*)(scratch + dfx::kWsGroupBits);
+    a.ws_tans = nullptr;
     a.status = (uint32_t*)(scratch + kStaticStatus);
     if (dfx::launch_encode(a, max_bytes, stream) != cudaSuccess) {
         cudaGetLastError();

@@ -113,3 +113,43 @@ def test_host_decode_argument_errors_precede_cuda(lib):
 def test_debug_inject_flags(lib):
     assert lib.dfx_debug_inject(0x2) == dfx.DFX_ERR_ARG
     assert lib.dfx_debug_inject(0) == dfx.DFX_OK
+
+
+@pytest.mark.parametrize("n", [0, 5, 4097, 1_000_003, 234_881_024])
+@pytest.mark.parametrize("K,R", [(32, 12), (128, 12), (64, 8), (128, 4)])
+def test_tans_layout_agrees_with_oracle(lib, n, K, R):
+    nc = 32 * -(-n // (32 * K))
+    for total_bits in (0, 1, 33, R * (n + nc)):
+        lay = dfx.dfx_container_layout(n, total_bits, chunk_symbols=K, coder=dfx.DFX_CODER_TANS, table_log=R)
+        assert lay["total_bytes"] == oracle.tans_container_bytes(n, K, 32, total_bits)
+        assert lay["off_len"] == 64 and lay["off_gbase"] == 576
+    lay = dfx.dfx_container_layout(n, R * (n + nc), chunk_symbols=K, coder=dfx.DFX_CODER_TANS, table_log=R)
+    assert lay["total_bytes"] == oracle.tans_max_container_bytes(n, K, 32, R)
+
+
+def test_tans_layout_matches_an_oracle_container(lib):
+    w = np.arange(5000, dtype=np.uint16) % 1024
+    c = oracle.encode_tans(w, K=64)
+    total_bits = int(c[16:24].view(np.uint64)[0])
+    lay = dfx.dfx_container_layout(w.size, total_bits, chunk_symbols=64, coder=dfx.DFX_CODER_TANS)
+    assert lay["total_bytes"] == c.size
+    assert lay["off_m"] == int(c[48:56].view(np.uint64)[0])
+
+
+def test_tans_argument_errors_precede_cuda(lib):
+    for kw in ({"table_log": 3}, {"table_log": 13}, {"chunk_symbols": 5464}):
+        with pytest.raises(dfx.DfxError) as e:
+            dfx.dfx_plan(1000, coder=dfx.DFX_CODER_TANS, **kw)
+        assert e.value.code == dfx.DFX_ERR_ARG, kw
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_plan(1000, coder=2)
+    assert e.value.code == dfx.DFX_ERR_ARG
+    # the tANS coder ignores max_len, the Huffman coder table_log
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_container_layout(10, 0, chunk_symbols=5464, coder=dfx.DFX_CODER_TANS)  # 5465 x 12 > 65535
+    assert e.value.code == dfx.DFX_ERR_ARG
+    dfx.dfx_container_layout(10, 0, chunk_symbols=4000, max_len=99, coder=dfx.DFX_CODER_TANS)
+    dfx.dfx_container_layout(10, 0, table_log=99)
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_encode_static(None, 10, None, 0, coder=dfx.DFX_CODER_TANS)
+    assert e.value.code == dfx.DFX_ERR_UNSUPPORTED
