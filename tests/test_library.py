@@ -153,3 +153,28 @@ def test_tans_argument_errors_precede_cuda(lib):
     with pytest.raises(dfx.DfxError) as e:
         dfx.dfx_encode_static(None, 10, None, 0, coder=dfx.DFX_CODER_TANS)
     assert e.value.code == dfx.DFX_ERR_UNSUPPORTED
+
+
+def header_struct_fields(name):
+    """(type, field) pairs of `typedef struct { ... } name;` in include/dfx.h, in order."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    body = re.search(r"typedef struct \{([^{}]*)\}\s*" + name + r"\s*;", src).group(1)
+    out = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        ctype, names = decl.split(None, 1)
+        out += [(ctype, n.strip()) for n in names.split(",")]
+    return out
+
+
+@pytest.mark.parametrize("name", ["dfx_params", "dfx_layout"])
+def test_ctypes_structs_mirror_the_header(name):
+    """The binding's ctypes structures have the header's fields, in order, with the same
+    widths: a field added on one side only would shift every later one."""
+    widths = {"uint32_t": ctypes.c_uint32, "uint64_t": ctypes.c_uint64}
+    declared = header_struct_fields(name)
+    mirror = getattr(dfx, name)._fields_
+    assert [n for _, n in declared] == [n for n, _ in mirror]
+    assert all(widths[t] is c for (t, _), (_, c) in zip(declared, mirror))
