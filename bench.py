@@ -15,6 +15,13 @@ barrier and a device synchronise on both sides, max over ranks.  Every
 container (~0.32 GB) and the output buffer exceed the 126 MB L2, so no flush is
 needed between steps.
 
+The line also reports, on rank 0: `e2e` (pinned host containers through H2D, decode
+and D2H), `offload` (weights streamed from pinned host memory, raw against
+compressed), `layer_batch` (a Llama-3-8B-shaped layer as 7 launches and as one
+batched launch), `decode_into_gemm` (a weight restored ahead of its GEMM), `tans`
+(the tANS exponent coder on 4 of the tensors against the Huffman figures) and
+`cpu_baseline` (the oracle, one host core).
+
 `--impl reference` times the CPU oracle (single-threaded C) decoding a 16 M
 weight sample with the same value distribution; it is the slow reference arm.
 """
