@@ -178,3 +178,15 @@ def test_ctypes_structs_mirror_the_header(name):
     mirror = getattr(dfx, name)._fields_
     assert [n for _, n in declared] == [n for n, _ in mirror]
     assert all(widths[t] is c for (t, _), (_, c) in zip(declared, mirror))
+
+
+def test_binding_constants_match_the_header():
+    """Every DFX_* constant of the binding has the value include/dfx.h defines."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    defined = {name: int(val.rstrip("uU"), 0)
+               for name, val in re.findall(r"^#define\s+(DFX_\w+)\s+(0x[0-9a-fA-F]+u?|\d+u?)\s*$", src, flags=re.M)}
+    mirrored = {k: v for k, v in vars(dfx).items() if k.startswith("DFX_") and isinstance(v, int)}
+    assert mirrored, "the binding defines no DFX_ constants"
+    for name, value in mirrored.items():
+        assert name in defined, f"{name} is not defined in include/dfx.h"
+        assert defined[name] == value, (name, value, defined[name])
