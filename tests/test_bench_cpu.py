@@ -1,0 +1,32 @@
+"""Host-side pieces of bench.py: the DRAM traffic figure is reported only while the decode
+sources still match the ones the committed ncu capture was taken on."""
+import os
+import shutil
+
+import bench
+
+
+def test_traffic_matches_the_committed_capture():
+    n = 234_881_024
+    t = bench.ncu_traffic_per_launch(n)
+    assert t is not None, "the committed traffic file no longer matches the decode sources"
+    assert abs(t / n - 3.0967) < 0.01  # bytes per weight read + written per launch
+    assert abs(bench.ncu_traffic_per_launch(2 * n) - 2 * t) < 1.0
+
+
+def test_traffic_is_null_once_a_decode_source_changes(tmp_path, monkeypatch):
+    srcs = []
+    for p in bench.DECODE_SOURCES:
+        q = tmp_path / os.path.basename(p)
+        shutil.copy(p, q)
+        srcs.append(str(q))
+    monkeypatch.setattr(bench, "DECODE_SOURCES", srcs)
+    assert bench.ncu_traffic_per_launch(1000) is not None
+    with open(srcs[0], "a") as fh:
+        fh.write("\n")
+    assert bench.ncu_traffic_per_launch(1000) is None
+
+
+def test_traffic_is_null_without_the_file(monkeypatch, tmp_path):
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.txt"))
+    assert bench.ncu_traffic_per_launch(1000) is None
