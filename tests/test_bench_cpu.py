@@ -13,7 +13,9 @@ def test_traffic_matches_the_committed_capture():
     t = bench.ncu_traffic_per_launch(n)
     if t is None:  # the kernel changed since the capture: the bench reports null, as it should
         pytest.skip("decode sources changed since the committed ncu capture")
-    assert abs(t / n - 3.0967) < 0.01  # bytes per weight read + written per launch
+    # DRAM bytes per weight read + written per launch: near the algorithmic ~3.34 (container
+    # once, output once, part of it still in L2 at kernel end), not above it (no re-reads)
+    assert 2.5 < t / n < 1.1 * 3.34
     assert abs(bench.ncu_traffic_per_launch(2 * n) - 2 * t) < 1.0
 
 
