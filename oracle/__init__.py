@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.dfxo_tans_tables.argtypes = [u32p, ctypes.c_uint32, u8p, u32p]
         L.dfxo_encode_tans.argtypes = [u16p, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint32,
                                        u8p, ctypes.c_uint64, u64p]
+        L.dfxo_tans_encode_chunk.argtypes = [u32p, ctypes.c_uint32, u8p, ctypes.c_uint32, u8p, u64p]
+        L.dfxo_tans_encode_chunk.restype = ctypes.c_int
         L.dfxo_tans_container_bytes.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint64]
         L.dfxo_tans_container_bytes.restype = ctypes.c_uint64
         L.dfxo_tans_max_container_bytes.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
@@ -182,6 +184,24 @@ def tans_tables(freq, table_log: int = 12):
     if rc:
         raise OracleError(rc, "tans_tables")
     return sym, k
+
+
+def tans_encode_chunk(freq, symbols, table_log: int = 12) -> str:
+    """Rule T4 for one chunk with a given frequency table: its bits as a '0'/'1' string."""
+    f = np.zeros(256, dtype=np.uint32)
+    src = np.asarray(freq, dtype=np.uint32)
+    f[: src.size] = src
+    syms = np.ascontiguousarray(symbols, dtype=np.uint8)
+    out = np.zeros((table_log * (syms.size + 1) + 7) // 8 + 8, dtype=np.uint8)
+    bits = np.zeros(1, dtype=np.uint64)
+    rc = lib().dfxo_tans_encode_chunk(_ptr(f, ctypes.c_uint32), table_log, _ptr(syms, ctypes.c_uint8), syms.size,
+                                      _ptr(out, ctypes.c_uint8), _ptr(bits, ctypes.c_uint64))
+    if rc:
+        raise OracleError(rc, "tans_encode_chunk")
+    nbits = int(bits[0])
+    # the stream layout: bit k is bit 31 - k % 32 of little-endian 32-bit word k / 32
+    words = np.frombuffer(out[: (out.size // 4) * 4].tobytes(), dtype="<u4")
+    return "".join(str((int(words[k // 32]) >> (31 - k % 32)) & 1) for k in range(nbits))
 
 
 def tans_container_bytes(n: int, K: int, G: int, total_bits: int) -> int:

@@ -607,6 +607,38 @@ static uint64_t tans_chunk(const uint32_t f[256], const uint32_t cs[256], const 
     return bits;
 }
 
+/* T4 for one chunk of cnt symbols with a given frequency table f (summing to M):
+ * writes the chunk's bits MSB-first from bit 0 of `out` (zeroed by the caller, at least
+ * R * (cnt + 1) bits long) and returns their number. */
+int dfxo_tans_encode_chunk(const uint32_t f[256], uint32_t R, const uint8_t *syms, uint32_t cnt, uint8_t *out,
+                           uint64_t *bits) {
+    if (R < 4 || R > 12) return DFXO_ERR_ARG;
+    const uint32_t M = 1u << R;
+    uint32_t cs[256], run = 0;
+    for (int s = 0; s < 256; s++) {
+        cs[s] = run;
+        run += f[s];
+    }
+    for (uint32_t i = 0; i < cnt; i++)
+        if (f[syms[i]] == 0) return DFXO_ERR_ARG;
+    uint8_t *slot_sym = (uint8_t *)malloc(M);
+    uint32_t *slot_k = (uint32_t *)malloc(4 * (size_t)M), *enc = (uint32_t *)malloc(4 * (size_t)M);
+    uint32_t *v = (uint32_t *)malloc(4 * (size_t)(cnt + 1));
+    uint8_t *nb = (uint8_t *)malloc(cnt + 1);
+    int rc = DFXO_ERR_ARG;
+    if (slot_sym && slot_k && enc && v && nb && dfxo_tans_tables(f, R, slot_sym, slot_k) == DFXO_OK) {
+        for (uint32_t j = 0; j < M; j++) enc[cs[slot_sym[j]] + slot_k[j] - f[slot_sym[j]]] = j;
+        *bits = tans_chunk(f, cs, enc, R, syms, cnt, out, 0, v, nb);
+        rc = DFXO_OK;
+    }
+    free(slot_sym);
+    free(slot_k);
+    free(enc);
+    free(v);
+    free(nb);
+    return rc;
+}
+
 uint64_t dfxo_tans_container_bytes(uint64_t n, uint32_t K, uint32_t G, uint64_t total_bits) {
     return container_bytes_of(n, K, G, total_bits, DFXO_CODER_TANS);
 }

@@ -584,3 +584,30 @@ def test_tans_malformed_containers_are_rejected():
         with pytest.raises(oracle.OracleError) as ei:
             oracle.decode(b)
         assert ei.value.code == oracle.ERR_CORRUPT, name
+
+
+def test_tans_chunk_codes_brute_force():
+    """For a fixed 16-state table, the chunk codes of every sequence of a given length
+    (3 symbols, lengths 1..5: up to 243 sequences) are distinct and prefix-free, as any
+    decodable code must be; each code's length is R plus, per symbol s, between
+    R - floor(log2(2f-1)) and R - floor(log2 f) bits (the state number k lies in
+    [f, 2f) and a step emits R - floor(log2 k) bits); with the dyadic table f = (8, 4, 4)
+    every symbol costs exactly its -log2(f / M) bits."""
+    R = 4
+    for freqs in ({1: 8, 2: 5, 3: 3}, {1: 8, 2: 4, 3: 4}, {1: 14, 2: 1, 3: 1}):
+        f = np.zeros(256, dtype=np.uint32)
+        for s_, v in freqs.items():
+            f[s_] = v
+        lo = {s_: R - int(math.floor(math.log2(2 * v - 1))) for s_, v in freqs.items()}
+        hi = {s_: R - int(math.floor(math.log2(v))) for s_, v in freqs.items()}
+        for L in range(1, 6):
+            codes = {}
+            for seq in itertools.product(sorted(freqs), repeat=L):
+                c = oracle.tans_encode_chunk(f, np.array(seq, dtype=np.uint8), R)
+                assert R + sum(lo[x] for x in seq) <= len(c) <= R + sum(hi[x] for x in seq), (freqs, seq, c)
+                codes[seq] = c
+            vals = sorted(codes.values())
+            assert len(set(vals)) == len(vals)
+            assert all(not b.startswith(a) for a, b in zip(vals, vals[1:])), (freqs, L)
+            if freqs == {1: 8, 2: 4, 3: 4}:
+                assert all(len(c) == R + sum(1 if x == 1 else 2 for x in seq) for seq, c in codes.items())
