@@ -36,7 +36,8 @@
  *     2 f[s] - 1; a chunk is encoded from its last symbol to its first from state M
  *     (for symbol s, nb bits with f[s] <= X >> nb < 2 f[s] are emitted, low bits of
  *     X, and X becomes M + the slot of state X >> nb) and stored as the final state
- *     minus M (table_log bits) followed by the fields in symbol order;
+ *     minus M (table_log bits) followed by the fields in symbol order (a chunk of the
+ *     last group with no element has no bits);
  *   - the m bytes are stored raw, in element order;
  *   - the exponent codes are cut into chunks of K codes, 32 chunks to a group:
  *     a group covers 32*K consecutive elements in 8-element blocks, block b of
