@@ -208,9 +208,13 @@ int dfx_decode_range(dfx_plan_t plan, const void *d_comp, size_t comp_bytes, uin
  *   >= the container's size (16-byte aligned), which receives the container;
  *   d_bf16: the n BF16 outputs.  The host reads the container's size and group
  *   index directly from h_comp.  Errors as for dfx_decode; staging too small ->
- *   DFX_ERR_CAPACITY.  The plan's slice events order copies and decoding, so
- *   calls on the same plan must not overlap.  Returns after queueing the work;
- *   h_comp must stay valid until copy_stream has finished it. */
+ *   DFX_ERR_CAPACITY.  The copies into d_staging wait for the work already
+ *   queued on decode_stream when the call starts, so a call may reuse the
+ *   staging buffer of an earlier call on that stream (work queued on other
+ *   streams that reads d_staging is the caller's to order).  The plan's slice
+ *   events order copies and decoding, so calls on the same plan must be issued
+ *   from one host thread at a time.  Returns after queueing the work; h_comp
+ *   must stay valid until copy_stream has finished it. */
 int dfx_decode_host(dfx_plan_t plan, const void *h_comp, size_t comp_bytes, void *d_staging,
                     size_t staging_bytes, void *d_bf16, uint32_t slices, cudaStream_t copy_stream,
                     cudaStream_t decode_stream);
@@ -260,9 +264,11 @@ int dfx_free(dfx_plan_t plan);
  * Coder 0 only (coder 1 returns DFX_ERR_UNSUPPORTED).
  * All calls on a device share the scratch array and it keeps the last call's
  * contents; calls whose GPU work overlaps race and corrupt each other, so order
- * them on one stream.  The first call on a device looks up the array's address
- * with that device current; make it before any stream capture.  Produces the
- * same bytes as dfx_encode. */
+ * them on one stream.  Every call looks up the array's address in the current
+ * context, so calls after a cudaDeviceReset or from another context on the same
+ * device find the array that context holds; the first call in a context loads
+ * the library's module there, so make it before any stream capture.  Produces
+ * the same bytes as dfx_encode. */
 int dfx_encode_static(const void *d_bf16, uint64_t n, const dfx_params *params, void *d_out,
                       size_t out_capacity, size_t *h_compressed_bytes, cudaStream_t stream);
 

@@ -22,6 +22,10 @@ struct dfx_plan_s {
     // created on first use
     static constexpr uint32_t kHostSlicesMax = 64;
     cudaEvent_t slice_done[kHostSlicesMax];
+    // recorded on the decode stream when dfx_decode_host starts: its copies into the
+    // staging buffer wait for the decoding already queued there (an earlier call's
+    // slices may still be reading the buffer)
+    cudaEvent_t decode_idle;
     bool events_made;
 };
 
@@ -254,10 +258,15 @@ int dfx_decode_host(dfx_plan_t plan, const void* h_comp, size_t comp_bytes, void
     int rc = make_decode_args(plan, d_staging, total, d_bf16, &probe);
     if (rc) return rc;
     if (!plan->events_made) {
+        if (cudaEventCreateWithFlags(&plan->decode_idle, cudaEventDisableTiming) != cudaSuccess) {
+            cudaGetLastError();
+            return DFX_ERR_CUDA;
+        }
         for (uint32_t i = 0; i < dfx_plan_s::kHostSlicesMax; i++)
             if (cudaEventCreateWithFlags(&plan->slice_done[i], cudaEventDisableTiming) != cudaSuccess) {
                 cudaGetLastError();
                 for (uint32_t j = 0; j < i; j++) cudaEventDestroy(plan->slice_done[j]);
+                cudaEventDestroy(plan->decode_idle);
                 return DFX_ERR_CUDA;
             }
         plan->events_made = true;
@@ -274,6 +283,11 @@ int dfx_decode_host(dfx_plan_t plan, const void* h_comp, size_t comp_bytes, void
         cudaGetLastError();
         return DFX_ERR_CUDA;
     };
+    // the staging buffer is overwritten only once the decoding queued before this call
+    // (which may read it) has finished
+    if (cudaEventRecord(plan->decode_idle, decode_stream) != cudaSuccess ||
+        cudaStreamWaitEvent(copy_stream, plan->decode_idle, 0) != cudaSuccess)
+        return fail();
     // header, code section and the group index: every slice's decode reads them
     if (cudaMemcpyAsync(d, h, L.off_m, cudaMemcpyHostToDevice, copy_stream) != cudaSuccess) return fail();
     for (uint64_t s = 0; s < ns; s++) {
@@ -359,8 +373,10 @@ int dfx_free(dfx_plan_t plan) {
         cudaGetLastError();
         rc = DFX_ERR_CUDA;
     }
-    if (plan->events_made)
+    if (plan->events_made) {
         for (uint32_t i = 0; i < dfx_plan_s::kHostSlicesMax; i++) cudaEventDestroy(plan->slice_done[i]);
+        cudaEventDestroy(plan->decode_idle);
+    }
     free(plan);
     return rc;
 }

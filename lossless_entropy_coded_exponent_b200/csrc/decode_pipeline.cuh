@@ -6,9 +6,10 @@
 //     memory first (while the first group's copies are already in flight);
 //   * one warp decodes one group of 32 chunks; lane i owns chunk i of the group: the
 //     group's 8-element blocks i, i+32, ...  Its read position is the group's start bit
-//     plus the warp's exclusive scan of the chunk bit lengths (the "lightweight
-//     auxiliary variables" that coordinate read positions, "DFloat11: lossless LLM
-//     compression for GPU", aikraft.ru blog, section 03, item 2).  Write positions need
+//     plus the warp's exclusive scan of the chunk bit lengths: the per-group start bits
+//     and per-chunk bit lengths are the small position records with which each thread
+//     finds where to read ("DFloat11: lossless LLM compression for GPU", aikraft.ru
+//     blog, section 03, item 2).  Write positions need
 //     no scan: after every 8 codes the lane holds 8 consecutive outputs and the warp's
 //     16-byte stores cover 512 contiguous bytes;
 //   * the next group's stream slice and the sign+mantissa bytes are copied into the warp's

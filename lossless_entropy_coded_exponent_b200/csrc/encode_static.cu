@@ -20,12 +20,13 @@
 //     before it is read).  Two calls whose GPU work overlaps (different streams, or host
 //     threads without ordering between them) race on it and corrupt each other's output:
 //     order them on one stream or with events;
-//   * the first call on each device looks up the array's device address with that device
-//     current (cudaGetSymbolAddress); make that first call before any stream capture.
+//   * every call looks up the array's device address in the current context
+//     (cudaGetSymbolAddress) instead of keeping it from an earlier call: after a
+//     cudaDeviceReset, or in another context on the same device, the module and its array
+//     are loaded again at another address.  The first call in a context loads the module
+//     there; make that first call before any stream capture.
 #include <cuda_runtime.h>
 #include <stdint.h>
-
-#include <mutex>
 
 #include "dfx.h"
 #include "dfx_common.cuh"
@@ -36,12 +37,8 @@ constexpr uint64_t kStaticMaxGroups = 262144;
 constexpr uint64_t kStaticWorkspace = dfx::kWsGroupBits + 4 * kStaticMaxGroups;
 constexpr uint64_t kStaticStatus = kStaticWorkspace;          // one u32, unused by encode kernels
 constexpr uint64_t kStaticBytes = kStaticWorkspace + 256;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticBytes];
-
-std::mutex g_lock;
-uint8_t* g_scratch_addr[kMaxDevices] = {};
 
 }  // namespace
 
@@ -62,24 +59,16 @@ extern "C" int dfx_encode_static(const void* d_bf16, uint64_t n, const dfx_param
     const uint64_t max_bytes = lay.off_stream + dfx::stream_bytes(8 * n);
     if (out_capacity < max_bytes) return DFX_ERR_CAPACITY;
 
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
-        cudaGetLastError();
-        return DFX_ERR_CUDA;
-    }
-    if (dev < 0 || dev >= kMaxDevices) return DFX_ERR_ARG;
+    // In host code g_static_scratch names a host-side stand-in, not device memory: the
+    // kernels get the array's address in the current context, looked up on every call.
     uint8_t* scratch = nullptr;
     {
-        std::lock_guard<std::mutex> guard(g_lock);
-        if (!g_scratch_addr[dev]) {
-            void* p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
-                cudaGetLastError();
-                return DFX_ERR_CUDA;
-            }
-            g_scratch_addr[dev] = (uint8_t*)p;
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return DFX_ERR_CUDA;
         }
-        scratch = g_scratch_addr[dev];
+        scratch = (uint8_t*)p;
     }
 
     dfx::EncodeArgs a;

@@ -28,8 +28,8 @@
  *   4. canonical codes from the lengths;
  *   5. concatenate the codes MSB-first into 32-bit words;
  *   6. index: per chunk of K symbols its bit length, per group of G chunks its
- *      start bit (the "lightweight auxiliary variables" that let GPU threads
- *      find their read positions, DFloat11 blog section 03, item 2).  The
+ *      start bit: the small per-thread position records with which the GPU
+ *      threads find where to read (DFloat11 blog, section 03, item 2).  The
  *      elements of a group (G*K of them) are cut into blocks of 8; block b
  *      belongs to chunk b mod G, so a chunk holds K/8 blocks spaced G blocks
  *      apart, and the codes are concatenated chunk after chunk;

@@ -26,7 +26,12 @@ def test_traffic_is_null_once_a_decode_source_changes(tmp_path, monkeypatch):
         shutil.copy(p, q)
         srcs.append(str(q))
     monkeypatch.setattr(bench, "DECODE_SOURCES", srcs)
-    assert bench.ncu_traffic_per_launch(1000) is not None
+    # a capture record keyed to these sources
+    rec = tmp_path / "traffic.txt"
+    rec.write_text(f"# test record\ndecode_source_sha256: {bench.decode_source_hash()}\n"
+                   "dram_bytes_per_weight: 3.0\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(rec))
+    assert bench.ncu_traffic_per_launch(1000) == 3000.0
     with open(srcs[0], "a") as fh:
         fh.write("\n")
     assert bench.ncu_traffic_per_launch(1000) is None

@@ -65,9 +65,9 @@ def test_special_values_and_long_codes_in_one_batch():
 
 
 def test_llama3_8b_layer_in_one_launch():
-    """The seven projections of a Llama-3-8B-shaped layer (218 M weights) in one launch;
-    each container written by the GPU encoder, which the parity suite checks byte for
-    byte against the oracle on the same tensors."""
+    """The seven projections of a Llama-3-8B-shaped layer (218 M weights) in one launch.
+    Each container is written by the GPU encoder at the default chunk size K = 128 and
+    is first checked byte for byte against the oracle's container of the same tensor."""
     ws = [inputs.llama3_8b_layer_tensor(i) for i in range(len(inputs.LLAMA3_8B_LAYER))]
     plans = [dfx.dfx_plan(w.size) for w in ws]
     try:
@@ -76,6 +76,7 @@ def test_llama3_8b_layer_in_one_launch():
             out = torch.empty(p.max_compressed_bytes, dtype=torch.uint8, device="cuda")
             ws_ = torch.empty(p.workspace_bytes, dtype=torch.uint8, device="cuda")
             size = dfx.dfx_encode(p, to_dev(w), out, out.numel(), ws_, ws_.numel(), want_size=True)
+            assert np.array_equal(out[:size].cpu().numpy(), oracle.encode(w, K=128))
             comps.append(out[:size].clone())
             sizes.append(size)
         outs = [torch.empty(w.size, dtype=torch.int16, device="cuda") for w in ws]

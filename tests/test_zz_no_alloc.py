@@ -3,14 +3,15 @@
 It serves callers that may not call cudaMalloc/cudaFree (their HBM belongs to
 their own pool allocator, or they must avoid cudaFree's implicit device
 synchronisation).  Its scratch is a fixed array inside the library that every
-call reuses, so this checks it against dfx_encode on two calls in a row: the
-second call starts from the first call's leftovers in that array.  The file is
-named to run last in a full test run.
+call reuses, so this checks it against dfx_encode, and against the CPU oracle's
+container, on two calls in a row: the second call starts from the first call's
+leftovers in that array.  The file is named to run last in a full test run.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import lossless_entropy_coded_exponent_b200 as dfx
 from lossless_entropy_coded_exponent_b200 import build as dfx_build
 from lossless_entropy_coded_exponent_b200 import inputs
@@ -43,6 +44,7 @@ def test_static_encoder_matches_dfx_encode_on_two_calls_in_a_row():
         assert size == ref.size
         assert np.array_equal(got[:size], ref)
         assert np.all(got[size:] == 0)
+        assert np.array_equal(got[:size], oracle.encode(w, K=K))
 
 
 def test_static_encoder_rejects_sizes_beyond_its_scratch():
