@@ -547,10 +547,12 @@ def run_layer_batch(args, dev, stream):
 
 def run_decode_into_gemm(args, dev, tokens=16, slice_rows=3584):
     """Y = X W^T for the gate projection of the Llama-3-8B-shaped layer (W 14336x4096
-    BF16, X 16x4096), three ways, each replayed from a CUDA graph: W resident as BF16;
+    BF16, X 16x4096), four ways, each replayed from a CUDA graph: W resident as BF16;
     W decoded whole into HBM, then the GEMM; W decoded 3584 rows at a time
     (dfx_decode_range) into two 29 MB buffers that stay in L2, each slice's GEMM (a
-    torch/cuBLAS matmul on a second stream) overlapping the next slice's decode."""
+    torch/cuBLAS matmul on a second stream) overlapping the next slice's decode; and
+    dfx_decode_gemm, one kernel that decodes W into shared-memory tiles and multiplies
+    them on the tensor cores (W never written to HBM)."""
     import torch
 
     import lossless_entropy_coded_exponent_b200 as dfx
@@ -575,6 +577,7 @@ def run_decode_into_gemm(args, dev, tokens=16, slice_rows=3584):
         bufs = [torch.empty(slice_rows * cols, dtype=torch.int16, device=dev) for _ in range(2)]
         y = torch.empty(tokens, rows, dtype=torch.bfloat16, device=dev)
         ys = [torch.empty(tokens, slice_rows, dtype=torch.bfloat16, device=dev) for _ in range(n_slices)]
+        yf = torch.empty(tokens, rows, dtype=torch.float32, device=dev)
         torch.cuda.synchronize(dev)
 
         def resident():
@@ -603,6 +606,9 @@ def run_decode_into_gemm(args, dev, tokens=16, slice_rows=3584):
                 freed[b].record(side)
             s.wait_stream(side)
 
+        def fused():
+            dfx.dfx_decode_gemm(plan, comp, size, rows, cols, x, tokens, yf, stream=torch.cuda.current_stream())
+
         def graph_time(fn, reps=20):
             cap = torch.cuda.Stream(device=dev)
             with torch.cuda.stream(cap):
@@ -624,6 +630,14 @@ def run_decode_into_gemm(args, dev, tokens=16, slice_rows=3584):
             return ev[0].elapsed_time(ev[1]) * 1e3 / reps
 
         t_res, t_whole, t_sliced = graph_time(resident), graph_time(whole), graph_time(sliced)
+        t_fused = graph_time(fused)
+        # the fused product against an FP32 product of the same BF16 values
+        y32 = x.float() @ wb.float().t()
+        fused_rel = float((yf - y32).abs().max() / y32.abs().max())
+        w_check = torch.empty(rows * cols, dtype=torch.int16, device=dev)
+        dfx.dfx_decode_gemm(plan, comp, size, rows, cols, x, tokens, yf, w_check)
+        fused_exact = bool(torch.equal(w_check, w.view(-1))) and dfx.dfx_device_status(plan) == 0
+        del w_check
         y_ref = x @ wb.t()
         exact = all(torch.equal(bufs[(n_slices - 2 + k) % 2].view(slice_rows, cols),
                                 w.view(rows, cols)[(n_slices - 2 + k) * slice_rows:(n_slices - 1 + k) * slice_rows])
@@ -631,7 +645,11 @@ def run_decode_into_gemm(args, dev, tokens=16, slice_rows=3584):
         diff = float((torch.cat(ys, dim=1).float() - y_ref.float()).abs().max())
         return {"workload": f"Y = X W^T, W 14336x4096 BF16 (gate projection of the Llama-3-8B-shaped layer), "
                             f"X {tokens}x4096", "resident_bf16_us": t_res, "decode_whole_then_gemm_us": t_whole,
-                "decode_slices_into_gemm_us": t_sliced, "slice_rows": slice_rows,
+                "decode_slices_into_gemm_us": t_sliced, "fused_decode_gemm_us": t_fused,
+                "fused_decoded_w_bit_exact": fused_exact, "fused_y_max_rel_diff_vs_fp32_gemm": fused_rel,
+                "fused_container_gbs": size / t_fused / 1e3,
+                "fused_frac_of_measured": size / t_fused / 1e3 / measured_hbm_peak()[0],
+                "slice_rows": slice_rows,
                 "container_mb": size / 1e6, "bf16_mb": 2 * rows * cols / 1e6,
                 "decoded_slices_bit_exact": bool(exact), "y_max_abs_diff_vs_resident_gemm": diff,
                 "note": "per product, CUDA-graph replays, mean over 20; the sliced path keeps the decoded weights "

@@ -219,6 +219,31 @@ int dfx_decode_host(dfx_plan_t plan, const void *h_comp, size_t comp_bytes, void
                     size_t staging_bytes, void *d_bf16, uint32_t slices, cudaStream_t copy_stream,
                     cudaStream_t decode_stream);
 
+/* Y = X W^T with the weight matrix W restored from its container inside the kernel
+ * that multiplies it: the decoded BF16 weights go from the decoding threads into
+ * shared-memory tiles read by the tensor cores (tcgen05.mma, FP32 accumulation in
+ * tensor memory) and are never written to HBM.  The pages decompress weights on
+ * the GPU just before the computation that uses them, rebuilding them in a form
+ * ready for that computation ("DFloat11: lossless LLM compression for GPU",
+ * aikraft.ru blog, section 02 and section 03, item 2).
+ *   plan, d_comp, comp_bytes: as for dfx_decode; coder 0 (Huffman) only, else
+ *     DFX_ERR_UNSUPPORTED.
+ *   rows, cols: W's shape, row-major in the container's element order (rows * cols
+ *     must equal the plan's n, else DFX_ERR_ARG); cols must be a multiple of
+ *     32 * chunk_symbols (every group inside one row), else DFX_ERR_UNSUPPORTED.
+ *   d_x: X, tokens x cols BF16, row-major, device, 16-byte aligned; 1 <= tokens <= 32,
+ *     else DFX_ERR_ARG.
+ *   d_y: Y, tokens x rows FP32, row-major, device, 16-byte aligned; written whole.
+ *   d_w_out: NULL, or a device buffer (16-byte aligned) of rows * cols BF16 that also
+ *     receives the decoded W (for checking the decode; costs the 2n-byte write the
+ *     fused path otherwise avoids).
+ * Y is the exact product rounded by FP32 accumulation in an order of the hardware's
+ * choosing.  A corrupt container sets the plan's status word as dfx_decode does (Y
+ * is then not valid).  Asynchronous; one kernel launch of one CTA per SM, each
+ * decoding a tile of at most 120 rows once and feeding it to the tensor cores. */
+int dfx_decode_gemm(dfx_plan_t plan, const void *d_comp, size_t comp_bytes, uint64_t rows, uint64_t cols,
+                    const void *d_x, uint32_t tokens, float *d_y, void *d_w_out, cudaStream_t stream);
+
 /* Decode `count` containers (1..32; 0 is a no-op) with one kernel launch: a
  * whole layer's weights restored before use in one go (the pages decode a
  * model's compressed weights on the GPU ahead of the computation that reads

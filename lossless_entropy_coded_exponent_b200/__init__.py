@@ -42,6 +42,7 @@ EXPORTS = (
     "dfx_decode",
     "dfx_decode_range",
     "dfx_decode_host",
+    "dfx_decode_gemm",
     "dfx_decode_batch",
     "dfx_device_status",
     "dfx_free",
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
         L.dfx_decode.argtypes = [vp, vp, ctypes.c_size_t, vp, vp]
         L.dfx_decode_range.argtypes = [vp, vp, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_uint64, vp, vp]
         L.dfx_decode_host.argtypes = [vp, vp, ctypes.c_size_t, vp, ctypes.c_size_t, vp, ctypes.c_uint32, vp, vp]
+        L.dfx_decode_gemm.argtypes = [vp, vp, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_uint64, vp, ctypes.c_uint32, vp,
+                                      vp, vp]
         L.dfx_decode_batch.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_size_t),
                                        ctypes.POINTER(vp), ctypes.c_uint32, vp]
         L.dfx_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -99,7 +102,8 @@ def lib() -> ctypes.CDLL:
         L.dfx_debug_inject.argtypes = [ctypes.c_uint32]
         L.dfx_encode_static.argtypes = [vp, ctypes.c_uint64, ctypes.POINTER(dfx_params), vp, ctypes.c_size_t,
                                         ctypes.POINTER(ctypes.c_size_t), vp]
-        for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_decode_range", "dfx_decode_host", "dfx_decode_batch",
+        for f in ("dfx_container_layout", "dfx_plan", "dfx_encode", "dfx_decode", "dfx_decode_range", "dfx_decode_host",
+                  "dfx_decode_gemm", "dfx_decode_batch",
                   "dfx_device_status", "dfx_free", "dfx_encode_static", "dfx_debug_inject"):
             getattr(L, f).restype = ctypes.c_int
         _lib_handle = L
@@ -222,6 +226,15 @@ def dfx_decode_host(plan: Plan, h_comp, comp_bytes: int, d_staging, staging_byte
     _check(lib().dfx_decode_host(plan.handle, _ptr(h_comp), comp_bytes, _ptr(d_staging), staging_bytes,
                                  _ptr(d_bf16), slices, _stream(copy_stream), _stream(decode_stream)),
            "dfx_decode_host")
+
+
+def dfx_decode_gemm(plan: Plan, d_comp, comp_bytes: int, rows: int, cols: int, d_x, tokens: int, d_y,
+                    d_w_out=None, stream=None) -> None:
+    """Y = X W^T with W (rows x cols BF16) decoded from its container inside the GEMM
+    kernel; X tokens x cols BF16, Y tokens x rows FP32; d_w_out (optional) also
+    receives the decoded W."""
+    _check(lib().dfx_decode_gemm(plan.handle, _ptr(d_comp), comp_bytes, rows, cols, _ptr(d_x), tokens, _ptr(d_y),
+                                 _ptr(d_w_out), _stream(stream)), "dfx_decode_gemm")
 
 
 def dfx_decode_batch(plans, d_comps, comp_bytes, d_bf16s, stream=None) -> None:

@@ -16,6 +16,7 @@ struct dfx_plan_s {
     uint64_t ws_bytes;
     uint32_t* d_status;
     int device;
+    int sms;  // streaming multiprocessors of the device
     int decode_grid;
     int resident_ctas;  // decode CTAs that fit on the device at once
     // events ordering dfx_decode_host's copies before the decode of their slices,
@@ -154,6 +155,7 @@ int dfx_plan(dfx_plan_t* plan, uint64_t n, const dfx_params* params, size_t* max
         free(p);
         return DFX_ERR_CUDA;
     }
+    p->sms = sms;
     const uint64_t resident = dfx::decode_blocks_per_sm(K, q.coder) * (uint64_t)sms;  // CTAs that fit at once
     p->resident_ctas = (int)resident;
     const uint64_t wpb = (uint64_t)dfx::decode_warps_per_block(K);
@@ -310,6 +312,31 @@ int dfx_decode_host(dfx_plan_t plan, const void* h_comp, size_t comp_bytes, void
             return fail();
         rc = dfx_decode_range(plan, d_staging, total, g0, g1 - g0, (uint16_t*)d_bf16 + g0 * ge, decode_stream);
         if (rc) return rc;
+    }
+    return DFX_OK;
+}
+
+int dfx_decode_gemm(dfx_plan_t plan, const void* d_comp, size_t comp_bytes, uint64_t rows, uint64_t cols,
+                    const void* d_x, uint32_t tokens, float* d_y, void* d_w_out, cudaStream_t stream) {
+    if (!plan) return DFX_ERR_ARG;
+    if (plan->coder != DFX_CODER_HUFFMAN) return DFX_ERR_UNSUPPORTED;
+    if (rows == 0 || cols == 0 || rows * cols != plan->n || rows >= (1ull << 31) || cols >= (1ull << 31))
+        return DFX_ERR_ARG;
+    if (tokens == 0 || tokens > dfx::kGemmMaxTokens) return DFX_ERR_ARG;
+    if (cols % (32ull * plan->K) != 0) return DFX_ERR_UNSUPPORTED;  // every group inside one row
+    if (!d_x || !d_y || !aligned16(d_x) || !aligned16(d_y) || !aligned16(d_w_out)) return DFX_ERR_ARG;
+    dfx::DecodeArgs a;
+    const int rc = make_decode_args(plan, d_comp, comp_bytes, d_w_out ? d_w_out : d_y, &a);
+    if (rc) return rc;
+    // one CTA per SM, each a tile of at most kGemmMaxRows rows; more CTAs (several waves)
+    // only when the rows need them
+    uint64_t grid = rows < (uint64_t)plan->sms ? rows : (uint64_t)plan->sms;
+    const uint64_t need = (rows + dfx::kGemmMaxRows - 1) / dfx::kGemmMaxRows;
+    if (need > grid) grid = need;
+    if (dfx::launch_decode_gemm(a, (const uint16_t*)d_x, d_y, (uint16_t*)d_w_out, (uint32_t)rows, (uint32_t)cols, tokens,
+                                (int)grid, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return DFX_ERR_CUDA;
     }
     return DFX_OK;
 }

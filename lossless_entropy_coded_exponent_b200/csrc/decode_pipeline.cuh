@@ -45,8 +45,6 @@
 namespace dfx {
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
-
 // One CTA of 32 warps per SM.
 template <int K>
 struct DecodeShape {

@@ -17,6 +17,7 @@ constexpr uint32_t kOffGbaseTans = 576; // coder 1: group start bits
 constexpr uint32_t kMaxLenLimit = 24;   // longest code the decoder tables support
 constexpr uint32_t kTansMinLog = 4, kTansMaxLog = 12;  // tANS table sizes 2^4 .. 2^12
 constexpr uint32_t kWarp = 32;
+constexpr unsigned kFull = 0xffffffffu;  // all lanes of a warp
 
 __host__ __device__ inline uint32_t gbase_offset(uint32_t coder) { return coder == DFX_CODER_TANS ? kOffGbaseTans : kOffGbase; }
 
@@ -121,5 +122,11 @@ int decode_blocks_per_sm_huffman(uint32_t K);
 cudaError_t launch_decode_tans(const DecodeArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_decode_batch_tans(const BatchArgs& b, uint32_t K, cudaStream_t s);
 int decode_blocks_per_sm_tans(uint32_t K);
+// Y = X W^T from W's container (decode_gemm.cu): at most kGemmMaxTokens tokens, at most
+// kGemmMaxRows rows of W per CTA
+constexpr uint32_t kGemmMaxTokens = 32;
+constexpr uint32_t kGemmMaxRows = 120;
+cudaError_t launch_decode_gemm(const DecodeArgs& d, const uint16_t* x, float* y, uint16_t* w_out, uint32_t rows,
+                               uint32_t cols, uint32_t tokens, int grid, cudaStream_t s);
 
 }  // namespace dfx

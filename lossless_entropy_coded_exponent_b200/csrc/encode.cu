@@ -27,8 +27,6 @@
 namespace dfx {
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
-
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, unsigned lane) {
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
