@@ -49,7 +49,7 @@ FALLBACK_HBM_GBS = 6650.0
 WORKLOAD = "70B-shaped layer stream: 24 x BF16[8192, 28672], N(0, 1/8192) + 0.05% N(0, 0.5^2) outliers"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_dram_traffic.txt")
 DECODE_SOURCES = [os.path.join(ROOT, "lossless_entropy_coded_exponent_b200", "csrc", f)
-                  for f in ("decode.cu", "decode_pipeline.cuh", "dfx_common.cuh")]
+                  for f in ("decode.cu", "decode_pipeline.cuh", "huffman_reader.cuh", "huffman_tables.cuh", "bulk.cuh", "dfx_common.cuh")]
 
 
 def parse_args():
@@ -65,6 +65,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-layer-batch", action="store_true", help="skip the multi-tensor (Llama-3-8B layer) decode measurement")
     ap.add_argument("--no-tans", action="store_true", help="skip the tANS exponent coder comparison")
+    ap.add_argument("--no-config-table", action="store_true",
+                    help="skip the per-configuration decode table and the pinned oracle table")
     return ap.parse_args()
 
 
@@ -331,23 +333,23 @@ def run_ours(args, world, rank, local):
                 dfx.dfx_decode(plan, comps[i], sizes[i], out, stream=stream)
     stream.synchronize()
 
-    # ---- timed region: K steps x T decodes, one event per launch boundary
-    events = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps * T + 1)]
+    # ---- timed region: K steps x T decodes back to back, one event per step boundary (an
+    # event between two launches would keep the next decode from starting while the
+    # previous one finishes; the decode kernels are launched as programmatic dependents)
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     barrier(world)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
         with torch.cuda.stream(stream):
             events[0].record(stream)
-            e = 1
-            for _ in range(args.steps):
+            for e in range(1, args.steps + 1):
                 for i in range(T):
                     dfx.dfx_decode(plan, comps[i], sizes[i], out, stream=stream)
-                    events[e].record(stream)
-                    e += 1
+                events[e].record(stream)
         stream.synchronize()
     torch.cuda.synchronize(dev)
     barrier(world)
-    launch_ms = [events[j].elapsed_time(events[j + 1]) for j in range(len(events) - 1)]
+    launch_ms = [events[j].elapsed_time(events[j + 1]) / T for j in range(len(events) - 1)]  # per launch, by step
     total_ms = events[0].elapsed_time(events[-1])
     total_ms_max = max_over_ranks(total_ms, world)
     status = dfx.dfx_device_status(plan, stream=stream)
@@ -405,11 +407,129 @@ def run_ours(args, world, rank, local):
     # ---- the other exponent coder (tANS) on the same tensors and launch configuration
     if not args.no_tans and rank == 0:
         line["tans"] = run_tans_compare(args, dev, stream, xs, sizes, 1e3 * mean_launch_ms, n)
+    # ---- the smaller configurations, with and without an L2 flush
+    if not args.no_config_table and rank == 0:
+        line["config_table"] = run_config_table(args, dev, stream)
     # ---- oracle on the host: rank 0 at N=1 only
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         line["cpu_baseline"], line["bit_exact_vs_oracle"] = run_cpu_baseline(xs[0], comps[0], K)
+        if not args.no_config_table:
+            line["cpu_baseline_table"] = run_oracle_table()
     plan.free()
     return line
+
+
+CONFIG_TABLE = [
+    # name, generator (inputs module, seeded), note
+    ("cfg1 1024x1024 N(0, 0.02^2)", "small_gaussian", ()),
+    ("cfg2 length 1000003", "gaussian", (1_000_003, 0.02, 23)),
+    ("cfg2 all-zero 65536", "edge:all_zero", ()),
+    ("cfg2 uniform 16-bit patterns 2^20", "edge:uniform_exponents", ()),
+    ("cfg2 +-0/subnormal/+-Inf/NaN mix 2^20", "edge:special_mix", ()),
+    ("cfg2 Fibonacci counts (24-bit limit)", "edge:fibonacci_clamp", ()),
+    ("cfg3 4096x4096 + 0.1% N(0, 1) outliers", "projection_with_outliers", ()),
+    ("cfg4 Llama-3-8B layer gate_proj 14336x4096", "llama3_8b_layer_tensor", (4,)),
+    ("cfg4 Llama-3-8B layer k_proj 1024x4096", "llama3_8b_layer_tensor", (2,)),
+]
+
+
+def config_input(spec):
+    """The seeded BF16 input (as uint16) of one row of CONFIG_TABLE."""
+    from lossless_entropy_coded_exponent_b200 import inputs
+
+    gen, args = spec[1], spec[2]
+    if gen.startswith("edge:"):
+        return inputs.edge_cases()[gen[5:]]
+    return getattr(inputs, gen)(*args)
+
+
+def run_config_table(args, dev, stream, reps=20, flush_mib=512):
+    """Decode of each smaller configuration on the GPU (container from dfx_encode, checked
+    against the input): median launch time back to back (inputs partly L2-resident) and
+    with the L2 flushed before every launch (a 512 MiB buffer written between launches,
+    outside the timed region), as decoded BF16 GB/s and as algorithmic GB/s (container +
+    2n) against the measured HBM peak."""
+    import numpy as np
+    import torch
+
+    import lossless_entropy_coded_exponent_b200 as dfx
+
+    peak, peak_kind = measured_hbm_peak()
+    flush = torch.empty(flush_mib << 20, dtype=torch.uint8, device=dev)
+    rows = []
+    for spec in CONFIG_TABLE:
+        w = config_input(spec)
+        n = int(w.size)
+        x = torch.from_numpy(np.ascontiguousarray(w).view(np.int16)).to(dev)
+        with dfx.dfx_plan(n, chunk_symbols=args.chunk_symbols) as plan:
+            out = torch.empty(plan.max_compressed_bytes, dtype=torch.uint8, device=dev)
+            ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
+            size = dfx.dfx_encode(plan, x, out, out.numel(), ws, ws.numel(), want_size=True, stream=stream)
+            comp = out[:size].clone()
+            del out, ws
+            y = torch.empty_like(x)
+
+            def timed(flushed):
+                ts = []
+                with torch.cuda.stream(stream):
+                    for r in range(reps + 3):
+                        if flushed:
+                            flush.fill_(r & 0xFF)
+                        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        e0.record(stream)
+                        dfx.dfx_decode(plan, comp, size, y, stream=stream)
+                        e1.record(stream)
+                        ts.append((e0, e1))
+                stream.synchronize()
+                return statistics.median(a.elapsed_time(b) for a, b in ts[3:]) * 1e3
+
+            warm_us, flushed_us = timed(False), timed(True)
+            exact = bool(torch.equal(y, x)) and dfx.dfx_device_status(plan, stream=stream) == 0
+        algo = float(size) + 2.0 * n
+        rows.append({"config": spec[0], "weights": n, "bits_per_weight": 8.0 * size / max(n, 1),
+                     "decode_us": warm_us, "decode_us_l2_flushed": flushed_us,
+                     "bf16_gbs": 2.0 * n / (warm_us * 1e-6) / 1e9, "bf16_gbs_l2_flushed": 2.0 * n / (flushed_us * 1e-6) / 1e9,
+                     "frac_of_measured": algo / (warm_us * 1e-6) / 1e9 / peak,
+                     "frac_of_measured_l2_flushed": algo / (flushed_us * 1e-6) / 1e9 / peak, "bit_exact": exact})
+        del x, y, comp
+    del flush
+    return {"peak_gbs": peak, "peak_kind": peak_kind, "reps": reps, "rows": rows,
+            "note": "median launch time; 'l2_flushed' writes a 512 MiB buffer before every launch; these tensors "
+                    "(at most 59 M weights) are small enough that launch and table-build costs weigh"}
+
+
+ORACLE_CHILD = r"""
+import json, os, sys, time
+sys.path.insert(0, sys.argv[1])
+core = int(sys.argv[2])
+os.sched_setaffinity(0, {core})
+import bench, oracle
+oracle.lib()
+out = []
+for spec in bench.CONFIG_TABLE:
+    w = bench.config_input(spec)
+    t0 = time.perf_counter(); c = oracle.encode(w, K=128); t1 = time.perf_counter()
+    d = oracle.decode(c); t2 = time.perf_counter()
+    ok = bool((d == w).all())
+    out.append({"config": spec[0], "weights": int(w.size), "encode_weights_per_s": w.size / max(t1 - t0, 1e-9),
+                "decode_weights_per_s": w.size / max(t2 - t1, 1e-9), "decode_bf16_gbs": 2.0 * w.size / max(t2 - t1, 1e-9) / 1e9,
+                "round_trip": ok})
+print(json.dumps({"core": core, "rows": out}))
+"""
+
+
+def run_oracle_table():
+    """The oracle (single-threaded C) encoding and decoding every row of CONFIG_TABLE in a
+    child process pinned to one host core (sched_setaffinity, the same effect as
+    taskset -c): weights/s per config, as the benchmark's CPU-baseline plan asks."""
+    core = sorted(os.sched_getaffinity(0))[-1]
+    r = subprocess.run([sys.executable, "-c", ORACLE_CHILD, ROOT, str(core)], capture_output=True, text=True,
+                       timeout=600)
+    if r.returncode != 0:
+        return {"error": r.stderr[-500:]}
+    res = json.loads(r.stdout.strip().splitlines()[-1])
+    res.update({"cores": 1, "host": host_cpu(), "kind": "oracle", "pinned": f"sched_setaffinity to core {core}"})
+    return res
 
 
 def run_tans_compare(args, dev, stream, xs, huff_sizes, huff_launch_us, n, tensors=4, reps=10):

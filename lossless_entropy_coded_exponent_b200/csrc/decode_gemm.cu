@@ -11,53 +11,52 @@
 // number of groups (32 chunks of K codes), so every group lies inside one row.  X is
 // tokens x cols BF16 (row-major), tokens <= 32; Y is tokens x rows FP32 (row-major).
 //
-// One CTA (one per SM) takes a tile of at most 128 rows of W:
+// One CTA (one per SM) takes a tile of at most 120 rows of W (the MMA's M = 128):
 //   * every thread first helps build the Huffman tables in shared memory (the canonical
 //     per-length limits and the 14-bit pair table of huffman_tables.cuh);
-//   * 15 decoding warps hold up to 8 rows each (row slot i of warp w is tile row w + 15 i;
-//     a tile has at most 120 rows, the MMA's M = 128 rows past them unused).
-//     A warp decodes its rows side by side, one step at a time: in a step each lane
-//     decodes the next 8 codes of its chunk in every row, which are the row's 256
-//     consecutive weights [256 t, 256 t + 256), lane i holding weights 8 i .. 8 i + 7;
-//   * the 8 weights are merged with their sign+mantissa bytes and written as one 16-byte
-//     store into the A tile of the step: 128 rows x 256 K in the canonical K-major layout
-//     with the 128-byte swizzle (four 64-wide K atoms; in each 8-row group of an atom, row
-//     r's 16-byte chunk c sits at chunk c ^ (r mod 8)).  The same threads copy the step's
-//     slice of X into the B tile in the same layout;
-//   * one MMA warp waits for the step's tiles, issues 16 tcgen05.mma (M = 128, N = tokens
-//     rounded up to 16, K = 16 each) accumulating in tensor memory, and commits them to
-//     the stage's "free" barrier, which the decoding warps wait on before reusing the
-//     stage two steps later (two stages of A and B);
-//   * after the last step, decoding warps 0-3 read the accumulator (tensor memory lanes
+//   * 15 decoding warps hold up to 8 rows each, tile row R in warp R mod 15; four lanes
+//     share a row.  A group's 32 chunks are decoded in 8 rounds of 4: in round j lane q of
+//     a row decodes chunk 4 (j mod 8) + q from its first code to its last, 8 codes (one
+//     block) at a time, with the decode kernel's reader, from a shared-memory copy of the
+//     round's stream slice that the bulk-copy engine brought in during the previous round;
+//   * the sum over K of X W^T does not depend on the order of K, so the kernel takes K in
+//     the order it decodes it: two consecutive blocks of the four chunks of a round, 64
+//     weights per row, make one stage of A, 128 rows x 128 bytes (one K atom of the
+//     canonical K-major layout with the 128-byte swizzle: in each 8-row group, row r's
+//     16-byte chunk c sits at chunk c ^ (r mod 8)); the MMA warp gathers the same 64
+//     columns of X into the stage's B tile;
+//   * the MMA warp waits for a stage's A (every decoding warp arrives on its barrier),
+//     issues 4 tcgen05.mma (M = 128, N = tokens rounded up to 16, K = 16) accumulating in
+//     tensor memory and commits them to the stage's "free" barrier, which the decoding
+//     warps wait on before they write the stage again, kStages stages later;
+//   * after the last stage, decoding warps 0-3 read the accumulator (tensor-memory lanes
 //     32 w .. 32 w + 31 are tile rows) and write Y.
-// Each lane's stream words come from global memory with one word of read-ahead (a step's
-// worth of decoding hides its latency); the sign+mantissa bytes and the slice of X of the
-// next step are loaded into registers while the current step decodes.
 // Every wait is bounded: a wait that runs out sets DFX_STATUS_TIMEOUT and the kernel
 // carries on (with a wrong Y) and releases its tensor memory.  A corrupt container sets
-// the same status bits as dfx_decode and never makes the kernel read outside it.
+// the same status bits as dfx_decode and never makes the kernel read outside it or
+// outside its own shared memory.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "decode_pipeline.cuh"
+#include "huffman_reader.cuh"
 #include "huffman_tables.cuh"
 
 namespace dfx {
 namespace {
 
-// 15 decoding warps and the MMA warp: 16 warps, 4 per SM sub-partition, so that each thread
-// may hold up to 128 registers (a 17th warp would cut that to 96).
-constexpr int kGemmDecodeWarps = 15;
-constexpr int kGemmRowSlots = 8;                                     // rows per decoding warp
+constexpr int kGemmDecodeWarps = 15;  // + the MMA warp: 16 warps, up to 128 registers each
+constexpr int kGemmRowSlots = 8;      // rows per decoding warp, four lanes each
 static_assert(kGemmMaxRows == kGemmDecodeWarps * kGemmRowSlots, "rows per tile at most");
-constexpr int kGemmTileRows = 128;                                   // MMA M (rows past the tile's are unused)
-constexpr int kGemmThreads = (kGemmDecodeWarps + 1) * 32;
-constexpr int kGemmDecodeThreads = kGemmDecodeWarps * 32;
-constexpr uint32_t kStepK = 256;                                   // K per step
-constexpr uint32_t kAtomBytes = 128;                               // one swizzle row: 64 BF16
-constexpr uint32_t kAStageBytes = kGemmTileRows * kStepK * 2;      // 64 KiB
-constexpr uint32_t kTmemCols = 32;                                 // FP32 accumulator columns
+constexpr int kGemmTileRows = 128;    // MMA M (tile rows past the tile's own are never stored)
 static_assert(kGemmMaxRows <= kGemmTileRows, "the rows of a tile fit the MMA's M = 128");
+constexpr int kGemmThreads = (kGemmDecodeWarps + 1) * 32;
+constexpr uint32_t kAtomBytes = 128;                           // one swizzle row: 64 BF16
+constexpr uint32_t kAStageBytes = kGemmTileRows * kAtomBytes;  // 16 KiB: 128 rows x 64 K
+constexpr uint32_t kStages = 4;
+constexpr uint32_t kTmemCols = 32;                             // FP32 accumulator columns
+constexpr uint32_t kSliceBytes = 256;                          // a row's stream slice for one round
+constexpr uint32_t kSliceWords = kSliceBytes / 4;
 
 // ---------------------------------------------------------------- tcgen05 helpers
 
@@ -118,99 +117,18 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t rows, uint32_t r, uint
     return a * rows * kAtomBytes + (r >> 3) * 1024u + (r & 7u) * kAtomBytes + ((c ^ (r & 7u)) << 4);
 }
 
-// ---------------------------------------------------------------- stream reader
-//
-// The bit reader of decode.cu over global memory, with one word of read-ahead: a lane
-// holds its bit position p (relative to word `bw` of the stream), the 32-bit peek at p, the
-// words cur, nxt under it (cw and cw + 1) and `ahead` (cw + 2), loaded when the position
-// moves into a new word and first needed when it moves again, about 12 codes later.  No
-// reload follows more than 32 consumed bits, so p moves at most one word between reloads.
-// Loads are clamped to the stream section.
-struct GemmReader {
-    uint32_t bw, p, cw, peek, cur, nxt, ahead;
+// ---------------------------------------------------------------- the kernel
 
-    __device__ __forceinline__ static uint32_t word(const uint32_t* s, uint32_t i, uint32_t maxw) {
-        return __ldg(s + min(i, maxw));
-    }
-    __device__ __forceinline__ void init(const uint32_t* s, uint32_t maxw, uint32_t base_word, uint32_t start) {
-        bw = base_word;
-        p = start;
-        cw = start >> 5;
-        cur = word(s, bw + cw, maxw);
-        nxt = word(s, bw + cw + 1, maxw);
-        ahead = word(s, bw + cw + 2, maxw);
-    }
-    __device__ __forceinline__ void reload(const uint32_t* s, uint32_t maxw) {
-        const uint32_t wi = p >> 5;
-        if (wi != cw) {  // wi == cw + 1
-            cw = wi;
-            cur = nxt;
-            nxt = ahead;
-            ahead = word(s, bw + cw + 2, maxw);
-        }
-        peek = __funnelshift_l(nxt, cur, p);
-    }
-    __device__ __forceinline__ uint32_t one(const uint32_t* lut, const HuffTables& T, const uint32_t* s, uint32_t maxw,
-                                            uint32_t& err) {
-        const uint32_t e = lut[peek >> (32 - kLutBits)];
-        uint32_t len, sym;
-        if ((e & 0x001F0000u) == 0) {
-            uint32_t ent = decode_long(peek, T);
-            if (ent >> 16) {
-                err |= DFX_STATUS_STREAM;
-                ent &= 0xFFFFu;
-            }
-            len = ent >> 8;
-            sym = ent & 0xFFu;
-        } else {
-            len = (e >> 16) & 31u;
-            sym = e & 0xFFu;
-        }
-        p += len;
-        reload(s, maxw);
-        return sym;
-    }
-    // two codes merged with their m bytes (bytes 2j, 2j+1 of mw): two BF16
-    template <int j>
-    __device__ __forceinline__ uint32_t pair(uint32_t mw, const uint32_t* lut, const HuffTables& T, const uint32_t* s,
-                                             uint32_t maxw, uint32_t& err) {
-        constexpr uint32_t sel = j == 0 ? 0x5140u : 0x5342u;
-        const uint32_t e = lut[peek >> (32 - kLutBits)];
-        const uint32_t len = e >> 26;
-        peek = __funnelshift_l(0u, peek, len);
-        p += len;
-        uint32_t syms = e;
-        if ((int32_t)e < 0) {
-            p -= 32;
-            reload(s, maxw);
-            const uint32_t e2 = lut[peek >> (32 - kLutBits)];
-            if ((e & 0x001F0000u) && (e2 & 0x001F0000u)) {
-                const uint32_t l1 = (e2 >> 16) & 31u;
-                p += l1;
-                peek = __funnelshift_l(0u, peek, l1);
-                syms = (e & 0xFFu) | ((e2 & 0xFFu) << 8);
-            } else {
-                uint32_t s0 = e & 0xFFu;
-                if ((e & 0x001F0000u) == 0) s0 = one(lut, T, s, maxw, err);
-                syms = s0 | (one(lut, T, s, maxw, err) << 8);
-            }
-        }
-        return bf16_pair(__byte_perm(mw, syms, sel));
-    }
-    __device__ __forceinline__ uint4 block(uint2 m, const uint32_t* lut, const HuffTables& T, const uint32_t* s,
-                                           uint32_t maxw, uint32_t& err) {
-        uint4 o;
-        reload(s, maxw);
-        o.x = pair<0>(m.x, lut, T, s, maxw, err);
-        o.y = pair<1>(m.x, lut, T, s, maxw, err);
-        reload(s, maxw);
-        o.z = pair<0>(m.y, lut, T, s, maxw, err);
-        o.w = pair<1>(m.y, lut, T, s, maxw, err);
-        return o;
+// A row's staged stream slice: loads clamped to the slot's buffer, so a corrupt stream
+// never reads outside the warp's own buffers.
+struct SlotWords {
+    uint32_t s;  // shared-memory address of the slice
+    __device__ __forceinline__ uint32_t load(uint32_t i) const {
+        uint32_t v;
+        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(s + 4u * min(i, kSliceWords - 1)));
+        return v;
     }
 };
-
-// ---------------------------------------------------------------- the kernel
 
 struct GemmArgs {
     DecodeArgs d;      // the container (whole tensor: g_begin = 0, g_end = n_group)
@@ -221,23 +139,33 @@ struct GemmArgs {
     uint32_t gpr;      // groups per row
 };
 
+// Per decoding warp: the index of its rows' current group and two buffers of round slices.
+struct GemmWarp {
+    uint32_t incl[kGemmRowSlots][32];  // inclusive chunk-bit prefix of each row's group
+    unsigned long long gb0[kGemmRowSlots];
+    uint32_t base[2][kGemmRowSlots];   // per buffer and row: stream word of the first staged word
+    uint32_t staged[2];                // per buffer: bit r set when row r's slice is staged
+    unsigned long long bar[2];
+    __align__(16) uint32_t slice[2][kGemmRowSlots][kSliceWords];
+};
+
 template <int NT>  // N = 16 NT accumulator columns (tokens rounded up to 16)
 __host__ __device__ constexpr uint32_t gemm_b_stage_bytes() {
-    return 16u * NT * kStepK * 2u;
+    return 16u * NT * kAtomBytes;
 }
 template <int NT>
 constexpr size_t gemm_dyn_smem_bytes() {
-    // 1 KiB of alignment slack, two A stages, two B stages, the pair table
-    return 1024 + 2 * (size_t)kAStageBytes + 2 * (size_t)gemm_b_stage_bytes<NT>() + (sizeof(uint32_t) << kLutBits);
+    // 1 KiB of alignment slack, the A and B stages, the pair table, the warps' buffers
+    return 1024 + kStages * (size_t)(kAStageBytes + gemm_b_stage_bytes<NT>()) + (sizeof(uint32_t) << kLutBits) +
+           kGemmDecodeWarps * sizeof(GemmWarp);
 }
 
 template <int NT>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_constant__ GemmArgs ga) {
     constexpr uint32_t N = 16u * NT;
-    constexpr int NX = (int)((N * 32 + kGemmDecodeThreads - 1) / kGemmDecodeThreads);  // B chunks per thread
     constexpr uint32_t kBStage = gemm_b_stage_bytes<NT>();
     __shared__ HuffTables T;
-    __shared__ __align__(8) unsigned long long bar_full[2], bar_free[2], bar_done;
+    __shared__ __align__(8) unsigned long long bar_full[kStages], bar_free[kStages], bar_done;
     __shared__ uint32_t tmem_slot;
     extern __shared__ __align__(16) uint8_t dyn_smem[];
     const DecodeArgs& a = ga.d;
@@ -245,17 +173,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
     // 1024-byte aligned tiles (the swizzle pattern follows address bits 4-9)
     const uint32_t dyn0 = smem_addr(dyn_smem);
     const uint32_t pad = (1024u - (dyn0 & 1023u)) & 1023u;
-    const uint32_t sA = dyn0 + pad;                 // two A stages
-    const uint32_t sB = sA + 2 * kAStageBytes;      // two B stages
-    const uint32_t* lut = reinterpret_cast<const uint32_t*>(dyn_smem + pad + 2 * kAStageBytes + 2 * kBStage);
+    const uint32_t sA = dyn0 + pad;                   // kStages A stages
+    const uint32_t sB = sA + kStages * kAStageBytes;  // kStages B stages
+    uint8_t* after_b = dyn_smem + pad + kStages * (kAStageBytes + kBStage);
+    uint32_t* lut = reinterpret_cast<uint32_t*>(after_b);
+    GemmWarp* warps = reinterpret_cast<GemmWarp*>(after_b + (sizeof(uint32_t) << kLutBits));
 
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lo = (uint32_t)((uint64_t)blockIdx.x * ga.rows / gridDim.x);
     const uint32_t hi = (uint32_t)((uint64_t)(blockIdx.x + 1) * ga.rows / gridDim.x);
-    const uint32_t rows_t = hi - lo;  // <= 128 (the host sizes the grid)
+    const uint32_t rows_t = hi - lo;  // <= 120 (the host sizes the grid)
 
     if (!build_canonical(a, T)) return;
-    build_pair_table(T, const_cast<uint32_t*>(lut));
+    build_pair_table(T, lut);
 
     if (warp == kGemmDecodeWarps) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_addr(&tmem_slot)),
@@ -263,11 +193,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
         if (lane == 0) {
-            for (int i = 0; i < 2; i++) {
+            for (uint32_t i = 0; i < kStages; i++) {
                 mbar_init_count(&bar_full[i], kGemmDecodeWarps);
                 mbar_init_count(&bar_free[i], 1);
             }
             mbar_init_count(&bar_done, 1);
+            fence_mbar_init();
+        }
+    } else {
+        // slices start zeroed: a lane without a row decodes zeros from its never-staged slot
+        uint4* z = reinterpret_cast<uint4*>(&warps[warp].slice[0][0][0]);
+        for (uint32_t k = lane; k < sizeof(warps[warp].slice) / 16; k += 32) z[k] = make_uint4(0, 0, 0, 0);
+        if (lane == 0) {
+            for (int b = 0; b < 2; b++) mbar_init_count(&warps[warp].bar[b], kGemmRowSlots);
             fence_mbar_init();
         }
     }
@@ -276,127 +214,200 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
 
-    const uint32_t S = ga.cols / kStepK;  // steps per row
-    const uint32_t spg = a.K / 8;         // steps per group
+    const uint32_t bpr = a.K / 8;            // blocks per chunk: per round
+    const uint32_t spr = bpr / 2;            // stages per round
+    const uint32_t rounds = ga.gpr * 8;      // rounds per row
+    const uint32_t n_stages = rounds * spr;  // stages per tile
     uint32_t err = 0;
 
     if (warp == kGemmDecodeWarps) {
-        // ------------------------------------------------------------ MMA warp
+        // ------------------------------------------------------------ MMA warp: B tiles, MMAs
         constexpr uint32_t idesc = idesc_bf16_f32(N);
-        for (uint32_t t = 0; t < S; t++) {
-            const uint32_t st = t & 1u;
-            if (!mbar_wait(&bar_full[st], (t >> 1) & 1u)) err |= DFX_STATUS_TIMEOUT;
+        constexpr uint32_t NX = N * 8 / 32;  // 16-byte B chunks per lane per stage
+        uint4 xv[NX];
+        // B chunk q of stage i: token q / 8, column chunk c = q mod 8, which holds block
+        // 2 bp + c / 4 of chunk 4 jj + c mod 4 of group grp (round j = 8 grp + jj = i / spr,
+        // bp = i mod spr)
+        auto load_x = [&](uint32_t i) {
+            const uint32_t j = i / spr, bp = i % spr, grp = j / 8, jj = j % 8;
+#pragma unroll
+            for (uint32_t u = 0; u < NX; u++) {
+                const uint32_t q = lane + 32u * u, t = q / 8, c = q % 8;
+                const uint32_t pos = grp * 32u * a.K + (32u * (2u * bp + c / 4) + 4u * jj + c % 4) * 8u;
+                xv[u] = t < ga.tokens ? __ldg(reinterpret_cast<const uint4*>(ga.x + (uint64_t)t * ga.cols + pos))
+                                      : make_uint4(0, 0, 0, 0);
+            }
+        };
+        load_x(0);
+        for (uint32_t i = 0; i < n_stages; i++) {
+            const uint32_t st = i % kStages, u = i / kStages;
+            // the stage's previous MMAs have read it
+            if (u >= 1 && !mbar_wait(&bar_free[st], (u - 1) & 1u)) err |= DFX_STATUS_TIMEOUT;
+#pragma unroll
+            for (uint32_t v = 0; v < NX; v++) {
+                const uint32_t q = lane + 32u * v;
+                st_shared_v4(sB + st * kBStage + sw128_offset(N, q / 8, 0, q % 8), xv[v]);
+            }
+            if (i + 1 < n_stages) load_x(i + 1);
+            fence_proxy_async();  // B is read by the tensor cores
+            __syncwarp();
+            if (!mbar_wait(&bar_full[st], u & 1u)) err |= DFX_STATUS_TIMEOUT;
             tc_fence_after();
             if (lane == 0) {
 #pragma unroll
-                for (uint32_t at = 0; at < kStepK / 64; at++)
-#pragma unroll
-                    for (uint32_t kk = 0; kk < 4; kk++) {
-                        const uint32_t aa = sA + st * kAStageBytes + at * kGemmTileRows * kAtomBytes + kk * 32u;
-                        const uint32_t bb = sB + st * kBStage + at * N * kAtomBytes + kk * 32u;
-                        mma_bf16(tmem, smem_desc_sw128(aa), smem_desc_sw128(bb), idesc, (t | at | kk) != 0);
-                    }
+                for (uint32_t kk = 0; kk < 4; kk++)
+                    mma_bf16(tmem, smem_desc_sw128(sA + st * kAStageBytes + kk * 32u),
+                             smem_desc_sw128(sB + st * kBStage + kk * 32u), idesc, (i | kk) != 0);
                 mma_commit(&bar_free[st]);
-                if (t + 1 == S) mma_commit(&bar_done);
+                if (i + 1 == n_stages) mma_commit(&bar_done);
             }
             __syncwarp();
         }
     } else {
         // ------------------------------------------------------------ decoding warps
+        GemmWarp& W = warps[warp];
         const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
         const uint32_t maxw = T.n_words - 1;
         const uint8_t* mplane = a.comp + a.off_m;
         const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.comp + kOffGbase);
         const uint16_t* clen = reinterpret_cast<const uint16_t*>(a.comp + a.off_clen);
-        const uint32_t nr = rows_t > warp ? (rows_t - warp + kGemmDecodeWarps - 1) / kGemmDecodeWarps : 0u;
+        const uint32_t slot = lane >> 2, q = lane & 3;
+        const uint32_t R = warp + kGemmDecodeWarps * slot;  // this lane's tile row
+        const bool live = R < rows_t;
+        const uint64_t row = lo + R;
 
-        GemmReader rd[kGemmRowSlots];
-        uint32_t end[kGemmRowSlots];
-        uint2 mcur[kGemmRowSlots], mnext[kGemmRowSlots];
-        uint4 xnext[NX];
-
-        // the B tile entries of this thread: token q / 32, 16-byte chunk q mod 32 of the step
-        auto load_x = [&](uint32_t t) {
+        // group grp's index for every row of the warp (lane = chunk)
+        auto load_group = [&](uint32_t grp) {
+            unsigned long long g0[kGemmRowSlots], g1[kGemmRowSlots];
+            uint32_t cl[kGemmRowSlots];
 #pragma unroll
-            for (int j = 0; j < NX; j++) {
-                const uint32_t q = threadIdx.x + kGemmDecodeThreads * j;
-                const uint32_t tk = q >> 5, c = q & 31u;
-                xnext[j] = q < N * 32 && tk < ga.tokens
-                               ? __ldg(reinterpret_cast<const uint4*>(ga.x + (uint64_t)tk * ga.cols + kStepK * t) + c)
-                               : make_uint4(0, 0, 0, 0);
-            }
-        };
-        auto load_m = [&](uint32_t t, uint2 (&mm)[kGemmRowSlots]) {
-#pragma unroll
-            for (int i = 0; i < kGemmRowSlots; i++)
-                if ((uint32_t)i < nr) {
-                    const uint64_t row = lo + warp + kGemmDecodeWarps * i;
-                    mm[i] = __ldg(reinterpret_cast<const uint2*>(mplane + row * ga.cols + kStepK * t) + lane);
+            for (int r = 0; r < kGemmRowSlots; r++) {
+                if (warp + kGemmDecodeWarps * r < rows_t) {
+                    const uint64_t g = (uint64_t)(lo + warp + kGemmDecodeWarps * r) * ga.gpr + grp;
+                    g0[r] = __ldg(gbase + g);
+                    g1[r] = __ldg(gbase + g + 1);
+                    cl[r] = __ldg(clen + g * 32 + lane);
                 }
-        };
-        load_x(0);
-        load_m(0, mnext);
-
-        for (uint32_t t = 0; t < S; t++) {
-            const uint32_t st = t & 1u;
-            const uint32_t kstep = t % spg;
-#pragma unroll
-            for (int i = 0; i < kGemmRowSlots; i++) mcur[i] = mnext[i];
-            if (kstep == 0) {
-                // a new group in every row: its start bits and this lane's chunk
-#pragma unroll
-                for (int i = 0; i < kGemmRowSlots; i++)
-                    if ((uint32_t)i < nr) {
-                        const uint64_t g = (uint64_t)(lo + warp + kGemmDecodeWarps * i) * ga.gpr + t / spg;
-                        const unsigned long long gb0 = __ldg(gbase + g), gb1 = __ldg(gbase + g + 1);
-                        const uint32_t cl = __ldg(clen + g * 32 + lane);
-                        uint32_t incl = cl;
-#pragma unroll
-                        for (int d = 1; d < 32; d <<= 1) {
-                            const uint32_t yv = __shfl_up_sync(kFull, incl, d);
-                            if (lane >= (unsigned)d) incl += yv;
-                        }
-                        const uint32_t sum = __shfl_sync(kFull, incl, 31);
-                        const bool ok = gb1 >= gb0 && gb1 <= T.total_bits && gb1 - gb0 == (unsigned long long)sum;
-                        if (!ok) err |= DFX_STATUS_INDEX;
-                        const uint32_t start = ok ? (uint32_t)(gb0 & 31u) + incl - cl : 0u;
-                        rd[i].init(sw, maxw, ok ? (uint32_t)(gb0 >> 5) : 0u, start);
-                        end[i] = start + (ok ? cl : 0u);
-                    }
-            }
-            // next step's operands, loaded while this step decodes
-            if (t + 1 < S) {
-                load_m(t + 1, mnext);
-            }
-            uint4 xv[NX];
-#pragma unroll
-            for (int j = 0; j < NX; j++) xv[j] = xnext[j];
-            if (t + 1 < S) load_x(t + 1);
-
-            // stage st was last read by the MMAs of step t - 2
-            if (t >= 2 && !mbar_wait(&bar_free[st], ((t >> 1) - 1) & 1u)) err |= DFX_STATUS_TIMEOUT;
-#pragma unroll
-            for (int j = 0; j < NX; j++) {
-                const uint32_t q = threadIdx.x + kGemmDecodeThreads * j;
-                if (q < N * 32) st_shared_v4(sB + st * kBStage + sw128_offset(N, q >> 5, (q & 31u) >> 3, q & 7u), xv[j]);
             }
 #pragma unroll
-            for (int i = 0; i < kGemmRowSlots; i++)
-                if ((uint32_t)i < nr) {
-                    const uint32_t r = warp + kGemmDecodeWarps * i;  // tile row
-                    const uint4 o = rd[i].block(mcur[i], lut, T, sw, maxw, err);
-                    st_shared_v4(sA + st * kAStageBytes + sw128_offset(kGemmTileRows, r, lane >> 3, lane & 7u), o);
-                    if (ga.w_out)
-                        reinterpret_cast<uint4*>(ga.w_out + (uint64_t)(lo + r) * ga.cols + kStepK * t)[lane] = o;
+            for (int r = 0; r < kGemmRowSlots; r++) {
+                if (warp + kGemmDecodeWarps * r >= rows_t) continue;  // the same for every lane
+                uint32_t incl = cl[r];
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const uint32_t yv = __shfl_up_sync(kFull, incl, d);
+                    if (lane >= (unsigned)d) incl += yv;
                 }
-            if (kstep + 1 == spg) {
-#pragma unroll
-                for (int i = 0; i < kGemmRowSlots; i++)
-                    if ((uint32_t)i < nr && rd[i].p != end[i]) err |= DFX_STATUS_STREAM;
+                const uint32_t sum = __shfl_sync(kFull, incl, 31);
+                const bool ok = g1[r] >= g0[r] && g1[r] <= T.total_bits && g1[r] - g0[r] == (unsigned long long)sum;
+                if (!ok) err |= DFX_STATUS_INDEX;
+                W.incl[r][lane] = ok ? incl : 0u;
+                if (lane == 0) W.gb0[r] = ok ? g0[r] : 0ull;
             }
-            fence_proxy_async();  // the tiles are read by the tensor cores (async proxy)
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_full[st]);
+        };
+        // lanes 0-7: copy round j's slice of row slot `lane` into buffer b (or arrive
+        // without a copy when the row is empty or its slice does not fit)
+        auto stage_round = [&](uint32_t j, uint32_t b) {
+            if (lane < kGemmRowSlots) {
+                const uint32_t r = lane, jj = j % 8;
+                uint32_t bytes = 0;
+                if (warp + kGemmDecodeWarps * r < rows_t) {
+                    const unsigned long long s0 = W.gb0[r] + (jj ? W.incl[r][4 * jj - 1] : 0u);
+                    const unsigned long long s1 = W.gb0[r] + W.incl[r][4 * jj + 3];
+                    const uint32_t beg = ((uint32_t)(s0 >> 5) * 4u) & ~15u;
+                    const uint32_t end = min((((uint32_t)(s1 >> 5) + 4u) * 4u + 15u) & ~15u, T.n_words * 4u);
+                    W.base[b][r] = beg / 4u;
+                    if (end > beg && end - beg <= kSliceBytes) bytes = end - beg;
+                }
+                const uint32_t mask = __ballot_sync(0xFFu, bytes != 0);
+                if (lane == 0) W.staged[b] = mask;
+                __syncwarp(0xFFu);
+                fence_proxy_async();  // the buffer's previous contents were read (generic proxy)
+                if (bytes) bulk_copy(W.slice[b][r], a.comp + a.off_stream + 4ull * W.base[b][r], bytes, &W.bar[b]);
+                else mbar_arrive(&W.bar[b]);
+            }
+            __syncwarp();
+        };
+        // the m bytes of block k of round j of this lane's chunk
+        auto m_of = [&](uint32_t j, uint32_t k) -> uint2 {
+            const uint32_t grp = j / 8, c = 4u * (j % 8) + q;
+            return __ldg(reinterpret_cast<const uint2*>(mplane + row * ga.cols + grp * 32u * a.K + (32u * k + c) * 8u));
+        };
+
+        load_group(0);
+        stage_round(0, 0);
+        uint32_t sphase = 0;  // parity of each round buffer's next phase
+        uint2 m0 = make_uint2(0, 0), m1 = make_uint2(0, 0);
+        if (live) {
+            m0 = m_of(0, 0);
+            m1 = m_of(0, 1);
+        }
+        uint32_t i = 0;  // stage
+        for (uint32_t j = 0; j < rounds; j++) {
+            const uint32_t b = j & 1u, jj = j % 8, c = 4u * jj + q;
+            // this lane's chunk: start (relative to the group) and bits, read before the
+            // next group's index replaces them
+            uint32_t c_start = 0, c_bits = 0;
+            unsigned long long g_start = 0;
+            if (live) {
+                const uint32_t e = W.incl[slot][c];
+                c_start = c ? W.incl[slot][c - 1] : 0u;
+                c_bits = e - c_start;
+                g_start = W.gb0[slot];
+            }
+            __syncwarp();
+            // the next round's slice (a new group's index first)
+            if (j + 1 < rounds) {
+                if ((j + 1) % 8 == 0) load_group((j + 1) / 8);
+                stage_round(j + 1, b ^ 1u);
+            }
+            if (!mbar_wait(&W.bar[b], (sphase >> b) & 1u)) err |= DFX_STATUS_TIMEOUT;
+            sphase ^= 1u << b;
+            const bool staged = (W.staged[b] >> slot) & 1u;
+            const unsigned long long p0 = g_start + c_start;  // the chunk's first stream bit
+            // decode the round: every lane runs the same steps; a lane without a row stores
+            // nothing and its reader reads the slot's buffer (or word 0 of the stream)
+            auto run = [&](auto& br) {
+                for (uint32_t bp = 0; bp < spr; bp++, i++) {
+                    const uint32_t st = i % kStages, u = i / kStages;
+                    if (u >= 1 && !mbar_wait(&bar_free[st], (u - 1) & 1u)) err |= DFX_STATUS_TIMEOUT;
+#pragma unroll
+                    for (uint32_t h = 0; h < 2; h++) {
+                        const uint32_t k = 2u * bp + h;
+                        const uint2 m = h ? m1 : m0;
+                        // the m bytes two blocks on (the next round's first two at a round's end)
+                        if (live) {
+                            const uint2 mn = k + 2 < bpr ? m_of(j, k + 2) : (j + 1 < rounds ? m_of(j + 1, k + 2 - bpr) : m);
+                            if (h) m1 = mn;
+                            else m0 = mn;
+                        }
+                        const uint4 o = decode_block(br, T, m, err);
+                        if (live) {
+                            st_shared_v4(sA + st * kAStageBytes + sw128_offset(kGemmTileRows, R, 0, 4u * h + q), o);
+                            if (ga.w_out)
+                                *reinterpret_cast<uint4*>(ga.w_out + row * ga.cols + ga.cols / ga.gpr * (j / 8) +
+                                                          (32u * k + c) * 8u) = o;
+                        }
+                    }
+                    fence_proxy_async();  // A is read by the tensor cores
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar_full[st]);
+                }
+                if (live && br.consumed() != c_bits) err |= DFX_STATUS_STREAM;
+            };
+            if (__all_sync(kFull, staged || !live)) {
+                BitReader<SlotWords> br;
+                const uint32_t rel = live ? (uint32_t)(p0 - 32ull * W.base[b][slot]) : 0u;
+                br.init(lut, SlotWords{smem_addr(W.slice[b][slot])}, rel);
+                run(br);
+            } else {
+                // a slice that did not fit: the whole warp reads this round from global memory
+                const uint32_t first = live ? (uint32_t)(p0 >> 5) : 0u;
+                BitReader<ClampedGlobalWords> br;
+                br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, live ? (uint32_t)(p0 & 31u) : 0u);
+                run(br);
+            }
         }
 
         // ------------------------------------------------------------ epilogue
@@ -405,14 +416,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
             tc_fence_after();
             const uint32_t r = 32u * warp + lane;  // tile row = tensor-memory lane
 #pragma unroll
-            for (int j = 0; j < NT; j++) {
+            for (int jn = 0; jn < NT; jn++) {
                 uint32_t v[16];
-                tmem_ld16(tmem + ((32u * warp) << 16) + 16u * j, v);
+                tmem_ld16(tmem + ((32u * warp) << 16) + 16u * jn, v);
                 if (r < rows_t)
 #pragma unroll
-                    for (int c = 0; c < 16; c++) {
-                        const uint32_t tk = 16u * j + c;
-                        if (tk < ga.tokens) ga.y[(uint64_t)tk * ga.rows + lo + r] = __uint_as_float(v[c]);
+                    for (int cc = 0; cc < 16; cc++) {
+                        const uint32_t tk = 16u * jn + cc;
+                        if (tk < ga.tokens) ga.y[(uint64_t)tk * ga.rows + lo + r] = __uint_as_float(v[cc]);
                     }
             }
         }

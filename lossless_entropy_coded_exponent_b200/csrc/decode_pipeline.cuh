@@ -40,6 +40,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "bulk.cuh"
 #include "dfx_common.cuh"
 
 namespace dfx {
@@ -163,56 +164,6 @@ __host__ __device__ constexpr size_t warp_buffer_bytes() {
     return (sizeof(WarpBuffers<K>) + 15) & ~size_t(15);
 }
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-__device__ __forceinline__ void mbar_init(unsigned long long* bar) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(bar)) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory"); }
-// orders this thread's (and, after a warp barrier, the warp's) earlier generic accesses to
-// shared memory before the bulk copies it issues next
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
-// arm `bar` for `bytes` and copy them from global `src` to shared `dst` (both 16-byte
-// aligned, bytes a multiple of 16)
-__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                     smem_addr(dst)),
-                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
-                 : "memory");
-}
-// Wait for the phase with the given parity of `bar` to complete.  One blocking poll first
-// (try_wait, which suspends the warp for at most the 100 us time hint: staged data
-// normally lands within it), then non-blocking polls (test_wait) with a sleep of at most
-// 128 ns between them (__nanosleep(64) lasts at most twice its argument); a wait that
-// never completes gives up after ~0.1 ms + ~0.35 s and the caller reports
-// DFX_STATUS_TIMEOUT.
-constexpr uint32_t kWaitPolls = 1u << 21;
-__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity) {
-    const uint32_t addr = smem_addr(bar);
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 100000;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done) return true;
-    for (uint32_t i = 0; i < kWaitPolls; i++) {
-        asm volatile(
-            "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-            : "=r"(done)
-            : "r"(addr), "r"(parity)
-            : "memory");
-        if (done) return true;
-        __nanosleep(64);
-    }
-    return false;
-}
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void prefetch_line_l2(const void* p) {
-    asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p) : "memory");
-}
 __device__ __forceinline__ uint2 ld_shared_u2(const void* p) {
     uint2 v;
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr(p)));
@@ -501,8 +452,10 @@ __device__ __forceinline__ void decode_tensor(const DecodeArgs& a, uint32_t cta,
     uint32_t err = 0;
     const uint32_t step = ctas * kDecodeWarps;
     // groups are dealt to the CTAs (one per SM) in turn and each CTA's to its warps in
-    // turn, so that every SM gets the same number of groups within one
-    const uint32_t gw = a.g_begin + cta + ctas * warp;
+    // turn, highest warp first, so that every SM gets the same number of groups within
+    // one; the warps that get one group more than the rest are the highest-numbered ones,
+    // which the schedulers favour (they finish their groups first)
+    const uint32_t gw = a.g_begin + cta + ctas * (kDecodeWarps - 1 - warp);
     GroupState<K> gs;
     if (gw < full_end) group_prologue<C, K>(a, T, wb, gw, step, full_end, lane, gs);
     C::build(T, table, scratch);
@@ -513,8 +466,18 @@ __device__ __forceinline__ void decode_tensor(const DecodeArgs& a, uint32_t cta,
     if (err) atomicOr(a.status, err);
 }
 
+// Launched as a programmatic dependent of the work before it in the stream: a CTA may be
+// scheduled while the previous kernel is still finishing (back-to-back decodes then lose
+// no time between launches), and waits for that work to complete, memory included,
+// before it reads or writes anything in global memory.
+__device__ __forceinline__ void wait_prior_grid() {
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 template <class C, int K>
 __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeArgs a) {
+    wait_prior_grid();
     decode_tensor<C, K>(a, blockIdx.x, gridDim.x);
 }
 
@@ -522,6 +485,7 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
 // share of one tensor, so it builds that tensor's tables once.
 template <class C, int K>
 __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode_batch(const __grid_constant__ BatchArgs b) {
+    wait_prior_grid();
     uint32_t i = 0;
     while (i + 1 < b.count && blockIdx.x >= b.cta_begin[i + 1]) i++;
     decode_tensor<C, K>(b.t[i], blockIdx.x - b.cta_begin[i], b.cta_begin[i + 1] - b.cta_begin[i]);
@@ -556,13 +520,28 @@ cudaError_t allow_smem(F* kernel, size_t bytes, bool* done) {
     return e;
 }
 
+// Launch with programmatic stream serialisation (the kernel starts with wait_prior_grid).
+template <class Kern, class Arg>
+cudaError_t launch_programmatic(Kern* kernel, int grid, int threads, size_t smem, cudaStream_t s, const Arg& arg) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, arg);
+}
+
 template <class C, int K>
 cudaError_t launch_k(const DecodeArgs& a, int grid, cudaStream_t s) {
     static bool attr_set[64] = {};
     const cudaError_t e = allow_smem(k_decode<C, K>, dyn_smem_bytes<C, K>(), attr_set);
     if (e != cudaSuccess) return e;
-    k_decode<C, K><<<grid, DecodeShape<K>::kThreads, dyn_smem_bytes<C, K>(), s>>>(a);
-    return cudaGetLastError();
+    return launch_programmatic(k_decode<C, K>, grid, DecodeShape<K>::kThreads, dyn_smem_bytes<C, K>(), s, a);
 }
 
 template <class C, int K>
@@ -570,8 +549,8 @@ cudaError_t launch_batch_k(const BatchArgs& b, cudaStream_t s) {
     static bool attr_set[64] = {};
     const cudaError_t e = allow_smem(k_decode_batch<C, K>, dyn_smem_bytes<C, K>(), attr_set);
     if (e != cudaSuccess) return e;
-    k_decode_batch<C, K><<<b.cta_begin[b.count], DecodeShape<K>::kThreads, dyn_smem_bytes<C, K>(), s>>>(b);
-    return cudaGetLastError();
+    return launch_programmatic(k_decode_batch<C, K>, (int)b.cta_begin[b.count], DecodeShape<K>::kThreads,
+                               dyn_smem_bytes<C, K>(), s, b);
 }
 
 // The launchers of one coder for K = 32, 64, 128.

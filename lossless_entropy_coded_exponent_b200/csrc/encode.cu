@@ -2,26 +2,29 @@
 //
 // Passes, all stream-ordered on the caller's stream:
 //   0. zero the container's index region and everything after the m plane;
-//   1. k_histogram      exponent histogram, warp-aggregated shared-memory atomics;
+//   1. k_histogram      exponent histogram: input streamed by the bulk-copy engine, counts
+//                       of the 8 most frequent neighbouring values in registers;
 //   2. k_build_codebook one CTA: package-merge code lengths (limit max_len), canonical codes,
 //                       len[256] and the constant header fields;
-//   3. k_chunk_bits     per chunk its code bits (clen), per group of 32 chunks the sum;
-//                       a group's elements come in 8-element blocks, block b belongs to
-//                       chunk b mod 32, so lane i of a warp reads blocks i, i+32, ...
-//                       (16-byte loads, 512 contiguous bytes per warp instruction);
-//   4. k_group_scan     one CTA: exclusive scan of the group sums -> gbase, total_bits,
-//                       total_bytes (shared with the tANS coder, whose passes 2, 3 and 5
-//                       are in encode_tans.cu);
-//   5. k_pack           per chunk: start bit from gbase + warp scan of clen, codes packed
-//                       MSB-first into 32-bit words in the same block order; the
-//                       mantissa+sign bytes (mantissa * 2 + the sign of the pair partner,
-//                       element x ^ 1) written in element order.
+//   3. k_pack_fused     one warp per group, groups in ticket order: the group's input
+//                       into registers once (a group's elements come in 8-element
+//                       blocks, block b belongs to chunk b mod 32, so lane i reads
+//                       blocks i, i+32, ...: 16-byte loads, 512 contiguous bytes per warp
+//                       instruction), per chunk its code bits (clen), the group's start
+//                       bit by a decoupled look-back over the groups before it (gbase,
+//                       total_bits, total_bytes), codes packed MSB-first into 32-bit
+//                       words in the same block order, and the mantissa+sign bytes
+//                       (mantissa * 2 + the sign of the pair partner, element x ^ 1) in
+//                       element order.
+// The tANS coder shares pass 1 and k_group_scan (a one-CTA scan of per-group sums); its
+// passes 2, 3 and 5 are in encode_tans.cu.
 // The method: frequent exponent values get short codes ("DFloat11: lossless LLM
 // compression for GPU", aikraft.ru blog, section 02); the exact code and layout rules
 // are the ones stated in include/dfx.h.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "bulk.cuh"
 #include "dfx_common.cuh"
 
 namespace dfx {
@@ -47,16 +50,35 @@ __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long lon
 
 // ---------------------------------------------------------------- 1. histogram
 //
-// The exponents of a weight tensor crowd into a few neighbouring values.  Each CTA
-// counts the first 16-byte load of each of its threads into a shared histogram and picks
-// the 8 consecutive exponents [b, b + 8) with the most of that sample.  From then on a
-// thread counts the values in that window in registers, four 8-bit counters per 32-bit
-// word (one shift and one add per value), and folds them into 32-bit counts every 31
-// loads, before a counter can pass 255 (31 x 8 values); values outside the window take
-// a shared-memory atomic.  64 warps per SM keep enough loads in flight.
+// One CTA of 16 warps per SM.  The input's 16-byte units (8 exponents each) are cut into
+// chunks of 128 units (2 KiB); each warp takes a contiguous run of chunks and streams them
+// into its shared-memory buffers with the bulk-copy engine, kHistBufs chunks in flight,
+// so the bytes in flight do not depend on registers.  The exponents of a weight tensor
+// crowd into a few neighbouring values: each CTA counts its warps' first chunks into a
+// shared histogram and picks the 8 consecutive exponents [b, b + 8) with the most of that
+// sample.  From then on a lane counts the values in that window in registers, four 8-bit
+// counters per 32-bit word (one shift and one add per value and word; a shift by 32 or
+// more gives 0, so a value lands in at most one word), and folds them into 32-bit counts
+// every kHistFold chunks (32 values per lane per chunk: no counter passes 255); values
+// outside the window take a shared-memory atomic.
 
-constexpr int kHistThreads = 256;
-constexpr int kHistBlocksPerSm = 8;
+constexpr int kHistWarps = 16;
+constexpr uint32_t kHistChunkUnits = 128;  // 16-byte units per chunk (2 KiB)
+constexpr uint32_t kHistBufs = 4;          // chunks in flight per warp
+constexpr uint32_t kHistFold = 7;          // chunks between folds (7 x 32 < 256)
+
+struct HistWarpBuffers {
+    uint4 chunk[kHistBufs][kHistChunkUnits];
+    unsigned long long bar[kHistBufs];
+};
+constexpr size_t kHistSmem = kHistWarps * sizeof(HistWarpBuffers);
+
+// 1 << s, 0 for s >= 32 (the PTX shift clamps its amount)
+__device__ __forceinline__ uint32_t shl_clamped(uint32_t s) {
+    uint32_t r;
+    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(1u), "r"(s));
+    return r;
+}
 
 __device__ __forceinline__ void fold8(uint32_t& c0, uint32_t& c1, uint32_t (&r)[8]) {
 #pragma unroll
@@ -67,23 +89,51 @@ __device__ __forceinline__ void fold8(uint32_t& c0, uint32_t& c1, uint32_t (&r)[
     c0 = c1 = 0u;
 }
 
-__global__ void __launch_bounds__(kHistThreads, kHistBlocksPerSm) k_histogram(const uint16_t* __restrict__ in, uint64_t n,
-                                                          unsigned long long* __restrict__ counts) {
+__global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t* __restrict__ in, uint64_t n,
+                                                                  unsigned long long* __restrict__ counts,
+                                                                  uint32_t* status) {
     __shared__ uint32_t h[256];
     __shared__ uint32_t window;
+    extern __shared__ __align__(16) uint8_t hist_smem[];
+    const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    HistWarpBuffers& wb = reinterpret_cast<HistWarpBuffers*>(hist_smem)[warp];
     for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0;
-    __syncthreads();
+    const uint64_t units = n / 8;
+    const uint64_t chunks = (units + kHistChunkUnits - 1) / kHistChunkUnits;
+    const uint64_t nw = (uint64_t)gridDim.x * kHistWarps, wg = (uint64_t)blockIdx.x * kHistWarps + warp;
+    const uint64_t c0 = chunks * wg / nw;
+    const uint32_t nc = (uint32_t)(chunks * (wg + 1) / nw - c0);  // this warp's chunks c0 .. c0 + nc - 1
     const uint4* in4 = reinterpret_cast<const uint4*>(in);
-    const uint64_t n8 = n / 8;
-    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
-    uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n8) {  // the sample (its counts are kept)
-        const uint4 v = __ldg(in4 + i);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int k = 0; k < 8; k++) atomicAdd(&h[(w[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu], 1u);
+    auto chunk_units = [&](uint32_t k) -> uint32_t {
+        const uint64_t left = units - (c0 + k) * kHistChunkUnits;
+        return left < kHistChunkUnits ? (uint32_t)left : kHistChunkUnits;
+    };
+    auto issue = [&](uint32_t k) {  // lane 0: chunk k of the warp into buffer k % kHistBufs
+        bulk_copy(wb.chunk[k % kHistBufs], in4 + (c0 + k) * kHistChunkUnits, 16u * chunk_units(k),
+                  &wb.bar[k % kHistBufs]);
+    };
+    if (lane == 0) {
+        for (uint32_t i = 0; i < kHistBufs; i++) mbar_init(&wb.bar[i]);
+        fence_mbar_init();
+        for (uint32_t k = 0; k < kHistBufs && k < nc; k++) issue(k);
     }
-    i += stride;
+    __syncthreads();  // h zeroed
+    uint32_t err = 0;
+    if (nc > 0) {  // the sample: every warp's first chunk (its counts are kept)
+        if (!mbar_wait(&wb.bar[0], 0)) err |= DFX_STATUS_TIMEOUT;
+        const uint32_t nu = chunk_units(0);
+        for (uint32_t u = lane; u < nu; u += 32) {
+            const uint4 v = wb.chunk[0][u];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 8; k++) atomicAdd(&h[(w[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu], 1u);
+        }
+        __syncwarp();
+        if (lane == 0 && kHistBufs < nc) {
+            fence_proxy_async();
+            issue(kHistBufs);
+        }
+    }
     __syncthreads();
     if (threadIdx.x < 32) {  // the window with the largest sample mass: lane l tries b = l + 32 j
         uint32_t best = 0, best_b = 0;
@@ -107,29 +157,45 @@ __global__ void __launch_bounds__(kHistThreads, kHistBlocksPerSm) k_histogram(co
     }
     __syncthreads();
     const uint32_t b = window;
-    uint32_t c0 = 0u, c1 = 0u, r[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    uint32_t c0w = 0u, c1w = 0u, r[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     uint32_t since = 0;
-    for (; i < n8; i += stride) {
-        const uint4 v = __ldg(in4 + i);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (uint32_t k = 1; k < nc; k++) {
+        const uint32_t slot = k % kHistBufs;
+        if (!mbar_wait(&wb.bar[slot], (k / kHistBufs) & 1u)) err |= DFX_STATUS_TIMEOUT;
+        const uint32_t nu = chunk_units(k);
+        uint4 v[kHistChunkUnits / 32];
 #pragma unroll
-        for (int k = 0; k < 8; k++) {
-            const uint32_t e = (w[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu;
-            const uint32_t d = e - b;
-            if (d < 4u) c0 += 1u << (8 * d);
-            else if (d < 8u) c1 += 1u << (8 * (d - 4u));
-            else atomicAdd(&h[e], 1u);
+        for (uint32_t j = 0; j < kHistChunkUnits / 32; j++)
+            v[j] = (lane + 32 * j < nu) ? wb.chunk[slot][lane + 32 * j] : make_uint4(0, 0, 0, 0);
+        __syncwarp();
+        if (lane == 0 && k + kHistBufs < nc) {
+            fence_proxy_async();
+            issue(k + kHistBufs);
         }
-        if (++since == 31) {
-            fold8(c0, c1, r);
+#pragma unroll
+        for (uint32_t j = 0; j < kHistChunkUnits / 32; j++) {
+            if (lane + 32 * j >= nu) break;
+            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                const uint32_t e = (w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu;
+                const uint32_t d = e - b;
+                c0w += shl_clamped(8u * d);
+                c1w += shl_clamped(8u * d - 32u);
+                if (d >= 8u) atomicAdd(&h[e], 1u);
+            }
+        }
+        if (++since == kHistFold) {
+            fold8(c0w, c1w, r);
             since = 0;
         }
     }
-    fold8(c0, c1, r);
+    fold8(c0w, c1w, r);
 #pragma unroll
     for (int k = 0; k < 8; k++)
         if (r[k]) atomicAdd(&h[b + k], r[k]);
-    if (blockIdx.x == 0 && threadIdx.x < (n & 7)) atomicAdd(&h[(in[n8 * 8 + threadIdx.x] >> 7) & 0xFFu], 1u);
+    if (blockIdx.x == 0 && threadIdx.x < (n & 7)) atomicAdd(&h[(in[units * 8 + threadIdx.x] >> 7) & 0xFFu], 1u);
+    if (err) atomicOr(status, err);
     __syncthreads();
     for (int k = threadIdx.x; k < 256; k += blockDim.x)
         if (h[k]) atomicAdd(&counts[k], (unsigned long long)h[k]);
@@ -281,45 +347,7 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     }
 }
 
-// ---------------------------------------------------------------- 3. chunk bit lengths
-
-constexpr int kChunkThreads = 256;
-
-__device__ __forceinline__ uint32_t bits8(uint4 v, const uint8_t* lt) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t b = 0;
-#pragma unroll
-    for (int k = 0; k < 4; k++) b += lt[(w[k] >> 7) & 0xFFu] + lt[(w[k] >> 23) & 0xFFu];
-    return b;
-}
-
-template <int K>
-__global__ void __launch_bounds__(kChunkThreads) k_chunk_bits(EncodeArgs a) {
-    __shared__ uint8_t lt[256];
-    lt[threadIdx.x] = a.ws_len[threadIdx.x];
-    __syncthreads();
-    const uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const unsigned lane = threadIdx.x & 31;
-    uint32_t bits = 0;
-    if (c < a.n_chunk) {
-        const uint64_t g = c / 32;
-        for (uint32_t k = 0; k < K / 8; k++) {
-            const uint64_t x0 = block_element(g, K, k, lane);
-            if (x0 + 8 <= a.n) {
-                bits += bits8(__ldg(reinterpret_cast<const uint4*>(a.in + x0)), lt);
-            } else {
-                for (uint64_t x = x0; x < a.n; x++) bits += lt[(a.in[x] >> 7) & 0xFFu];
-                break;
-            }
-        }
-        reinterpret_cast<uint16_t*>(a.out + a.off_clen)[c] = (uint16_t)bits;
-    }
-    const uint32_t incl = warp_incl_scan(bits, lane);
-    const uint64_t g = c / 32;
-    if (lane == 31 && g < a.n_group) a.ws_group_bits[g] = incl;
-}
-
-// ---------------------------------------------------------------- 4. group scan
+// ---------------------------------------------------------------- group scan (tANS; empty tensors)
 
 constexpr int kScanThreads = 1024;
 constexpr int kScanItems = 16;  // four 16-byte loads per thread per round
@@ -371,9 +399,8 @@ __global__ void __launch_bounds__(kScanThreads) k_group_scan(EncodeArgs a) {
     }
 }
 
-// ---------------------------------------------------------------- 5. pack
+// ---------------------------------------------------------------- bit writers
 
-constexpr int kPackThreads = 256;
 constexpr uint32_t kPackSliceWords = 1024;  // a group's stream words staged per warp (4 KiB)
 
 // Where a chunk's packed words go: the stream in global memory, or the warp's shared
@@ -510,54 +537,181 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
     bw.finish();
 }
 
-// One warp per group: the lanes pack their chunks into the warp's shared copy of the
-// group's stream words, which the warp then writes out with coalesced stores (the group's
-// first and last words, which it may share with the neighbouring groups, are OR-ed in).
-// A group whose words do not fit the copy is packed straight into global memory.
-template <int K>
-__global__ void __launch_bounds__(kPackThreads) k_pack(EncodeArgs a) {
-    __shared__ uint32_t cl_sh[256];  // code << 8 | length
-    __shared__ uint32_t slice[kPackThreads / 32][kPackSliceWords];
-    cl_sh[threadIdx.x] = (a.ws_code[threadIdx.x] << 8) | a.ws_len[threadIdx.x];
-    __syncthreads();
-    const uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const unsigned lane = threadIdx.x & 31;
-    if (c >= a.n_chunk) return;  // n_chunk is a multiple of 32: whole warps leave
-    const uint16_t* clen = reinterpret_cast<const uint16_t*>(a.out + a.off_clen);
-    const uint32_t cl = clen[c];
-    const uint32_t incl = warp_incl_scan(cl, lane);
+// ---------------------------------------------------------------- 3. lengths, scan and pack
+//
+// Chunk lengths, the scan of the group lengths and the pack in one kernel, reading the
+// input once.  A CTA of 8 warps takes the next 8 groups from a ticket counter (so the
+// CTAs holding earlier groups are always running and the scan below always makes
+// progress); a warp loads its group into registers (lane i: the 16-byte blocks i, i + 32,
+// ... of the group), sums its chunk's code lengths, and finds the group's start bit by a
+// decoupled look-back over the group words of the workspace.  A group publishes its bit
+// count as soon as it is known (flag kGroupCount) and, once it has its own start, writes
+// the next group's gbase entry (its inclusive end) and then sets kGroupEnd; a warp adds
+// up its predecessors' counts, 32 at a time, back to the nearest group whose end is
+// published.  Then it packs its codes from the same registers (into the warp's shared
+// copy of its words, as k_pack does) and writes the sign+mantissa bytes.  The ragged last
+// group reads its elements from global memory.
+
+constexpr int kFusedWarps = 8;
+constexpr uint32_t kGroupCount = 1u << 30;  // the group's bit count (bits 0-29) is published
+constexpr uint32_t kGroupEnd = 1u << 31;    // and its end bit is in gbase[g + 1]
+constexpr uint32_t kLookbackPolls = 1u << 20;
+constexpr uint64_t kWsTicket = 3328;        // the pass's CTA ticket counter in the workspace
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned long long ld_relaxed64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// The exclusive start bit of group g: predecessors' published counts back to the nearest
+// published end.  Every wait is bounded (a flag that never comes sets DFX_STATUS_TIMEOUT
+// and counts as 0).
+__device__ uint64_t lookback(const EncodeArgs& a, uint32_t g, unsigned lane, uint32_t& err) {
+    const uint32_t* gw = a.ws_group_bits;
     const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.out + kOffGbase);
-    const uint64_t gb0 = gbase[c / 32];
-    const uint64_t start = gb0 + (incl - cl);
-    uint32_t* stream = reinterpret_cast<uint32_t*>(a.out + a.off_stream);
+    uint64_t excl = 0;
+    int64_t pos = (int64_t)g - 1;
+    while (pos >= 0) {
+        const int64_t i = pos - (int64_t)lane;
+        uint32_t v = kGroupCount | kGroupEnd;  // before group 0: an end at bit 0
+        for (uint32_t it = 0;; it++) {
+            if (i >= 0) v = ld_acquire(gw + i);
+            if (__all_sync(kFull, (v & kGroupCount) != 0)) break;
+            if (it == kLookbackPolls) {
+                err |= DFX_STATUS_TIMEOUT;
+                v = kGroupCount | kGroupEnd;
+                break;
+            }
+            __nanosleep(32);
+        }
+        const uint32_t ends = __ballot_sync(kFull, (v & kGroupEnd) != 0);
+        uint64_t c = 0;
+        if (ends) {
+            const unsigned first = __ffs(ends) - 1;  // the nearest predecessor with its end published
+            if (lane < first) c = v & (kGroupCount - 1);
+            if (lane == first && i >= 0) c = ld_relaxed64(gbase + i + 1);  // ordered after the flag's acquire
+        } else {
+            c = v & (kGroupCount - 1);
+        }
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1) c += __shfl_xor_sync(kFull, c, d);
+        excl += c;
+        if (ends) break;
+        pos -= 32;
+    }
+    return excl;
+}
+
+template <int K>
+__global__ void __launch_bounds__(kFusedWarps * 32) k_pack_fused(EncodeArgs a) {
+    __shared__ uint32_t cl_sh[256];  // code << 8 | length
+    __shared__ uint32_t slice[kFusedWarps][kPackSliceWords];
+    __shared__ uint32_t cta_ticket;
+    cl_sh[threadIdx.x] = (a.ws_code[threadIdx.x] << 8) | a.ws_len[threadIdx.x];
+    if (threadIdx.x == 0) cta_ticket = atomicAdd(reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTicket), 1u);
+    __syncthreads();
+    const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t g = cta_ticket * kFusedWarps + warp;
+    if (g >= a.n_group) return;
+    const uint64_t c = (uint64_t)g * 32 + lane;
+    const bool ragged = (uint64_t)(g + 1) * 32u * K > a.n;
+    uint32_t err = 0;
+
+    // the lane's chunk: its code bits
+    constexpr uint32_t NB = K / 8;
+    uint4 v[NB];
+    uint32_t bits = 0;
+    if (!ragged) {
+#pragma unroll
+        for (uint32_t k = 0; k < NB; k++) v[k] = __ldg(reinterpret_cast<const uint4*>(a.in + block_element(g, K, k, lane)));
+#pragma unroll
+        for (uint32_t k = 0; k < NB; k++) {
+            const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+            for (int q = 0; q < 4; q++) bits += (cl_sh[(w[q] >> 7) & 0xFFu] & 0xFFu) + (cl_sh[(w[q] >> 23) & 0xFFu] & 0xFFu);
+        }
+    } else {
+        for (uint32_t k = 0; k < NB; k++) {
+            const uint64_t x0 = block_element(g, K, k, lane);
+            for (uint64_t x = x0; x < x0 + 8 && x < a.n; x++) bits += cl_sh[(a.in[x] >> 7) & 0xFFu] & 0xFFu;
+            if (x0 + 8 > a.n) break;
+        }
+    }
+    reinterpret_cast<uint16_t*>(a.out + a.off_clen)[c] = (uint16_t)bits;
+    const uint32_t incl = warp_incl_scan(bits, lane);
     const uint32_t group_bits = __shfl_sync(kFull, incl, 31);
+
+    // the group's start bit
+    if (lane == 0) st_release(a.ws_group_bits + g, kGroupCount | group_bits);
+    const uint64_t gb0 = lookback(a, g, lane, err);
+    if (lane == 0) {
+        unsigned long long* gbase = reinterpret_cast<unsigned long long*>(a.out + kOffGbase);
+        gbase[g + 1] = gb0 + group_bits;
+        st_release(a.ws_group_bits + g, kGroupEnd | kGroupCount | group_bits);
+        if (g + 1 == a.n_group) {
+            *reinterpret_cast<unsigned long long*>(a.out + 16) = gb0 + group_bits;
+            *reinterpret_cast<unsigned long long*>(a.out + 24) = a.off_stream + stream_bytes(gb0 + group_bits);
+        }
+    }
+
+    // pack
+    const uint64_t start = gb0 + (incl - bits);
+    uint32_t* stream = reinterpret_cast<uint32_t*>(a.out + a.off_stream);
     const uint64_t wf = gb0 >> 5, wl = (gb0 + group_bits + 31) >> 5;  // the group's words [wf, wl)
     const uint32_t count = (uint32_t)(wl - wf);
-    if (count <= kPackSliceWords) {
-        uint32_t* sm = slice[threadIdx.x >> 5];
+    if (!ragged && count <= kPackSliceWords) {
+        uint32_t* sm = slice[warp];
+        for (uint32_t i = lane; i < count; i += 32) sm[i] = 0u;
+        __syncwarp();
+        SharedWriter bw = make_writer(SharedSink{sm, wf}, start);
+        uint8_t* mpl = a.out + a.off_m;
+#pragma unroll
+        for (uint32_t k = 0; k < NB; k++) {
+            const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+            uint32_t mb[2] = {0u, 0u};
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const uint32_t h = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+                const uint32_t partner = (w[j >> 1] >> (16 * ((j & 1) ^ 1))) & 0xFFFFu;  // element j ^ 1
+                const uint32_t ce = cl_sh[(h >> 7) & 0xFFu];
+                bw.put(ce >> 8, ce & 0xFFu);
+                mb[j >> 2] |= (((h & 0x7Fu) << 1) | (partner >> 15)) << (8 * (j & 3));
+            }
+            *reinterpret_cast<uint2*>(mpl + block_element(g, K, k, lane)) = make_uint2(mb[0], mb[1]);
+        }
+        bw.finish();
+        __syncwarp();
+        for (uint32_t i = lane; i < count; i += 32) {
+            const uint32_t wv = sm[i];
+            if (i == 0 || i + 1 == count) {
+                if (wv) atomicOr(stream + wf + i, wv);
+            } else {
+                stream[wf + i] = wv;
+            }
+        }
+    } else if (count <= kPackSliceWords) {
+        uint32_t* sm = slice[warp];
         for (uint32_t i = lane; i < count; i += 32) sm[i] = 0u;
         __syncwarp();
         pack_chunk<K>(a, cl_sh, c, lane, start, SharedSink{sm, wf});
         __syncwarp();
         for (uint32_t i = lane; i < count; i += 32) {
-            const uint32_t v = sm[i];
-            if (i == 0 || i + 1 == count) {
-                if (v) atomicOr(stream + wf + i, v);
-            } else {
-                stream[wf + i] = v;
-            }
+            const uint32_t wv = sm[i];
+            if (wv) atomicOr(stream + wf + i, wv);
         }
     } else {
         pack_chunk<K>(a, cl_sh, c, lane, start, GlobalSink{stream});
     }
-}
-
-template <int K>
-cudaError_t launch_chunk_passes(const EncodeArgs& a, int phase, cudaStream_t s) {
-    const unsigned blocks = (unsigned)((a.n_chunk + kChunkThreads - 1) / kChunkThreads);
-    if (phase == 0) k_chunk_bits<K><<<blocks, kChunkThreads, 0, s>>>(a);
-    else k_pack<K><<<blocks, kPackThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    if (err) atomicOr(a.status, err);
 }
 
 }  // namespace
@@ -568,14 +722,29 @@ cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t 
     if ((err = cudaMemsetAsync(a.out, 0, a.off_m, s)) != cudaSuccess) return err;
     if ((err = cudaMemsetAsync(a.out + a.off_m + a.n, 0, max_bytes - (a.off_m + a.n), s)) != cudaSuccess) return err;
     if ((err = cudaMemsetAsync(a.ws_counts, 0, 256 * sizeof(unsigned long long), s)) != cudaSuccess) return err;
+    // the fused pass's CTA ticket and group words start at zero
+    if (a.coder != DFX_CODER_TANS &&
+        (err = cudaMemsetAsync(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTicket, 0,
+                               kWsGroupBits - kWsTicket + 4ull * a.n_group, s)) != cudaSuccess)
+        return err;
 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const uint64_t units = (a.n / 8 + kHistThreads - 1) / kHistThreads;
-    const uint64_t resident = (uint64_t)sms * kHistBlocksPerSm;
-    const unsigned hist_blocks = (unsigned)(units == 0 ? 1 : (units < resident ? units : resident));
-    k_histogram<<<hist_blocks, kHistThreads, 0, s>>>(a.in, a.n, a.ws_counts);
+    {
+        static bool attr_set[64] = {};
+        if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+            if ((err = cudaFuncSetAttribute(k_histogram, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kHistSmem)) !=
+                cudaSuccess)
+                return err;
+            attr_set[dev] = true;
+        }
+        // one CTA per SM, fewer for small inputs (at least one chunk per warp)
+        const uint64_t chunks = (a.n / 8 + kHistChunkUnits - 1) / kHistChunkUnits;
+        const uint64_t ctas = (chunks + kHistWarps - 1) / kHistWarps;
+        const unsigned hist_blocks = (unsigned)(ctas == 0 ? 1 : (ctas < (uint64_t)sms ? ctas : (uint64_t)sms));
+        k_histogram<<<hist_blocks, kHistWarps * 32, kHistSmem, s>>>(a.in, a.n, a.ws_counts, a.status);
+    }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (a.coder == DFX_CODER_TANS) {  // the tANS passes around the same group scan
         if ((err = launch_encode_tans(a, 0, s)) != cudaSuccess) return err;
@@ -585,26 +754,18 @@ cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t 
     }
     k_build_codebook<<<1, 256, 0, s>>>(a);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if (a.n_chunk) {
-        switch (a.K) {
-            case 32: err = launch_chunk_passes<32>(a, 0, s); break;
-            case 64: err = launch_chunk_passes<64>(a, 0, s); break;
-            case 128: err = launch_chunk_passes<128>(a, 0, s); break;
-            default: return cudaErrorInvalidValue;
-        }
-        if (err != cudaSuccess) return err;
+    if (a.n_group == 0) {  // an empty tensor: the group scan writes the header totals
+        k_group_scan<<<1, kScanThreads, 0, s>>>(a);
+        return cudaGetLastError();
     }
-    k_group_scan<<<1, kScanThreads, 0, s>>>(a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if (a.n_chunk) {
-        switch (a.K) {
-            case 32: err = launch_chunk_passes<32>(a, 1, s); break;
-            case 64: err = launch_chunk_passes<64>(a, 1, s); break;
-            case 128: err = launch_chunk_passes<128>(a, 1, s); break;
-            default: return cudaErrorInvalidValue;
-        }
+    const unsigned ctas = (a.n_group + kFusedWarps - 1) / kFusedWarps;
+    switch (a.K) {
+        case 32: k_pack_fused<32><<<ctas, kFusedWarps * 32, 0, s>>>(a); break;
+        case 64: k_pack_fused<64><<<ctas, kFusedWarps * 32, 0, s>>>(a); break;
+        case 128: k_pack_fused<128><<<ctas, kFusedWarps * 32, 0, s>>>(a); break;
+        default: return cudaErrorInvalidValue;
     }
-    return err;
+    return cudaGetLastError();
 }
 
 }  // namespace dfx

@@ -120,3 +120,21 @@ def test_mixed_chunk_sizes_are_refused():
     finally:
         a.free()
         b.free()
+
+
+def test_back_to_back_launches_of_one_plan():
+    """Decodes of one plan, ranges and whole tensors, one after another on a stream, into
+    reused buffers."""
+    w = inputs.gaussian(4096 * 333 + 17, 0.02, seed=95)
+    c = torch.from_numpy(oracle.encode(w, K=128)).cuda()
+    x = to_dev(w)
+    with dfx.dfx_plan(w.size) as plan:
+        out = torch.full_like(x, -1)
+        for rep in range(3):
+            out.fill_(-1)
+            dfx.dfx_decode(plan, c, c.numel(), out)
+            assert torch.equal(out, x), rep
+            part = torch.full((4096 * 100,), -1, dtype=torch.int16, device="cuda")
+            dfx.dfx_decode_range(plan, c, c.numel(), 200, 100, part)
+            assert torch.equal(part, x[4096 * 200: 4096 * 300]), rep
+        assert dfx.dfx_device_status(plan) == 0
