@@ -298,7 +298,9 @@ def run_ours(args, world, rank, local):
     n = rows * cols
     T = args.tensors
     K = args.chunk_symbols
-    plan = dfx.dfx_plan(n, chunk_symbols=K)
+    # the containers are written once, before the decoding starts: a decode may read its
+    # container while the decode before it finishes (DFX_DECODE_EARLY_READ)
+    plan = dfx.dfx_plan(n, chunk_symbols=K, decode_flags=dfx.DFX_DECODE_EARLY_READ)
     stream = torch.cuda.Stream(device=dev)
 
     # ---- set-up: generate, encode, keep every container and every input resident
@@ -613,7 +615,8 @@ def run_layer_batch(args, dev, stream):
     L = len(inputs.LLAMA3_8B_LAYER)
     with torch.cuda.stream(stream):  # everything below is ordered on this one stream
         xs = [inputs.llama3_8b_layer_tensor_cuda(i, device=dev) for i in range(L)]
-    plans = [dfx.dfx_plan(x.numel(), chunk_symbols=args.chunk_symbols) for x in xs]
+    plans = [dfx.dfx_plan(x.numel(), chunk_symbols=args.chunk_symbols, decode_flags=dfx.DFX_DECODE_EARLY_READ)
+             for x in xs]
     try:
         comps, sizes = [], []
         with torch.cuda.stream(stream):
@@ -624,6 +627,7 @@ def run_layer_batch(args, dev, stream):
                 comps.append(out[:size].clone())
                 sizes.append(size)
             outs = [torch.empty_like(x) for x in xs]
+        stream.synchronize()  # the containers are complete before any decode starts
 
         def separate():
             for i in range(L):

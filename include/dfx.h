@@ -127,7 +127,19 @@ typedef struct {
     uint32_t table_log;     /* coder 1: log2 of the state table, 4..12 (0 -> 12); dfx_encode
                                needs 8..12 (room for all 256 exponent values), every value
                                decodes */
+    uint32_t decode_flags;  /* 0 or DFX_DECODE_EARLY_READ */
 } dfx_params;
+
+/* Decode flag: the kernel that precedes a decode of this plan in its stream never writes
+ * that decode's container (for instance the containers of a model's weights, written
+ * once before layer-by-layer decoding starts).  The decode kernels are launched as
+ * programmatic dependents of the work before them, so their CTAs can start while the
+ * preceding kernel finishes; with this flag a CTA also reads the container's header,
+ * builds its tables and starts copying its first group during that time, and waits for
+ * the preceding kernel only before its first output write.  Without it (the default)
+ * the CTA waits before it reads anything, which is always safe.  Applies to dfx_decode,
+ * dfx_decode_range, dfx_decode_batch and dfx_decode_host; dfx_decode_gemm ignores it. */
+#define DFX_DECODE_EARLY_READ 0x1u
 
 /* Byte offsets of the container sections for given n, params and stream length. */
 typedef struct {

@@ -31,6 +31,7 @@ DFX_STATUS_TIMEOUT = 0x10
 DFX_INJECT_SKIP_SLICE_COPY = 0x1
 DFX_CODER_HUFFMAN = 0
 DFX_CODER_TANS = 1
+DFX_DECODE_EARLY_READ = 0x1
 
 # The exported C symbols, in include/dfx.h order.
 EXPORTS = (
@@ -59,7 +60,7 @@ class DfxError(RuntimeError):
 
 class dfx_params(ctypes.Structure):
     _fields_ = [("chunk_symbols", ctypes.c_uint32), ("group_chunks", ctypes.c_uint32), ("max_len", ctypes.c_uint32),
-                ("coder", ctypes.c_uint32), ("table_log", ctypes.c_uint32)]
+                ("coder", ctypes.c_uint32), ("table_log", ctypes.c_uint32), ("decode_flags", ctypes.c_uint32)]
 
 
 class dfx_layout(ctypes.Structure):
@@ -132,8 +133,8 @@ def _stream(s) -> int | None:
     return s.cuda_stream
 
 
-def _params(chunk_symbols=0, group_chunks=0, max_len=0, coder=DFX_CODER_HUFFMAN, table_log=0):
-    return dfx_params(chunk_symbols, group_chunks, max_len, coder, table_log)
+def _params(chunk_symbols=0, group_chunks=0, max_len=0, coder=DFX_CODER_HUFFMAN, table_log=0, decode_flags=0):
+    return dfx_params(chunk_symbols, group_chunks, max_len, coder, table_log, decode_flags)
 
 
 def dfx_version() -> int:
@@ -181,11 +182,11 @@ class Plan:
 
 
 def dfx_plan(n: int, chunk_symbols: int = 0, group_chunks: int = 0, max_len: int = 0,
-             coder: int = DFX_CODER_HUFFMAN, table_log: int = 0) -> Plan:
+             coder: int = DFX_CODER_HUFFMAN, table_log: int = 0, decode_flags: int = 0) -> Plan:
     h = ctypes.c_void_p()
     mx = ctypes.c_size_t()
     ws = ctypes.c_size_t()
-    p = _params(chunk_symbols, group_chunks, max_len, coder, table_log)
+    p = _params(chunk_symbols, group_chunks, max_len, coder, table_log, decode_flags)
     _check(lib().dfx_plan(ctypes.byref(h), n, ctypes.byref(p), ctypes.byref(mx), ctypes.byref(ws)), "dfx_plan")
     return Plan(h.value, n, mx.value, ws.value, (chunk_symbols, group_chunks, max_len, coder, table_log))
 

@@ -11,6 +11,7 @@ struct dfx_plan_s {
     uint64_t n;
     uint32_t K, G, max_len;
     uint32_t coder, table_log;  // exponent coder; tANS table log (coder 1)
+    uint32_t decode_flags;      // DFX_DECODE_*
     dfx::Layout L;
     uint64_t max_bytes;
     uint64_t ws_bytes;
@@ -33,7 +34,7 @@ struct dfx_plan_s {
 namespace {
 
 struct Params {
-    uint32_t K, G, L, coder, R;
+    uint32_t K, G, L, coder, R, flags;
 };
 
 // Defaults and checks of dfx_params.  Only the fields of the chosen coder are checked:
@@ -44,6 +45,8 @@ int resolve_params(const dfx_params* p, Params* r) {
     r->L = (p && p->max_len) ? p->max_len : 24u;
     r->coder = p ? p->coder : DFX_CODER_HUFFMAN;
     r->R = (p && p->table_log) ? p->table_log : dfx::kTansMaxLog;
+    r->flags = p ? p->decode_flags : 0u;
+    if (r->flags & ~(uint32_t)DFX_DECODE_EARLY_READ) return DFX_ERR_ARG;
     if (r->K < 8 || r->K % 8 != 0) return DFX_ERR_ARG;  // chunks are made of 8-element blocks
     if (r->coder == DFX_CODER_HUFFMAN) {
         if (r->L < 8 || r->L > dfx::kMaxLenLimit) return DFX_ERR_ARG;
@@ -143,6 +146,7 @@ int dfx_plan(dfx_plan_t* plan, uint64_t n, const dfx_params* params, size_t* max
     p->max_len = q.L;
     p->coder = q.coder;
     p->table_log = q.R;
+    p->decode_flags = q.flags;
     p->L = dfx::make_layout(n, K, G, q.coder);
     p->max_bytes = p->L.off_stream + dfx::stream_bytes(max_stream_bits(q, n, p->L.n_chunk));
     p->ws_bytes = dfx::workspace_bytes_for(p->L.n_group, q.coder);
@@ -435,6 +439,7 @@ int make_decode_args(const dfx_plan_s* plan, const void* d_comp, size_t comp_byt
     a->g_end = (uint32_t)plan->L.n_group;
     a->out_first = 0;
     a->inject = g_inject;
+    a->early = (plan->decode_flags & DFX_DECODE_EARLY_READ) ? 1u : 0u;
     return DFX_OK;
 }
 

@@ -329,20 +329,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
             }
             __syncwarp();
         };
-        // the m bytes of block k of round j of this lane's chunk
-        auto m_of = [&](uint32_t j, uint32_t k) -> uint2 {
+        // the m bytes of this lane's chunk in round j: block k at m_base(j) + 32 k (uint2)
+        auto m_base = [&](uint32_t j) -> const uint2* {
             const uint32_t grp = j / 8, c = 4u * (j % 8) + q;
-            return __ldg(reinterpret_cast<const uint2*>(mplane + row * ga.cols + grp * 32u * a.K + (32u * k + c) * 8u));
+            return reinterpret_cast<const uint2*>(mplane + row * ga.cols + grp * 32u * a.K) + c;
         };
+        // this lane's 16-byte chunks in an A stage, for the first and second block of a stage
+        const uint32_t a_off0 = sA + sw128_offset(kGemmTileRows, R, 0, q);
+        const uint32_t a_off1 = sA + sw128_offset(kGemmTileRows, R, 0, 4u + q);
 
         load_group(0);
         stage_round(0, 0);
         uint32_t sphase = 0;  // parity of each round buffer's next phase
-        uint2 m0 = make_uint2(0, 0), m1 = make_uint2(0, 0);
-        if (live) {
-            m0 = m_of(0, 0);
-            m1 = m_of(0, 1);
-        }
+        // the m bytes of the next kMAhead blocks (ring: block k in mq[k % kMAhead]); at a
+        // round's end the ring runs on into the next round's first blocks
+        constexpr uint32_t kMAhead = 4;
+        uint2 mq[kMAhead];
+        const uint2* mp = m_base(0);
+#pragma unroll
+        for (uint32_t k = 0; k < kMAhead; k++) mq[k] = live ? __ldg(mp + 32u * k) : make_uint2(0, 0);
         uint32_t i = 0;  // stage
         for (uint32_t j = 0; j < rounds; j++) {
             const uint32_t b = j & 1u, jj = j % 8, c = 4u * jj + q;
@@ -368,31 +373,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
             const unsigned long long p0 = g_start + c_start;  // the chunk's first stream bit
             // decode the round: every lane runs the same steps; a lane without a row stores
             // nothing and its reader reads the slot's buffer (or word 0 of the stream)
+            const uint2* mnext = j + 1 < rounds ? m_base(j + 1) : mp;  // the next round's m bytes
             auto run = [&](auto& br) {
-                for (uint32_t bp = 0; bp < spr; bp++, i++) {
-                    const uint32_t st = i % kStages, u = i / kStages;
-                    if (u >= 1 && !mbar_wait(&bar_free[st], (u - 1) & 1u)) err |= DFX_STATUS_TIMEOUT;
+                // two stages (four blocks) per step: the m ring index is then fixed in each
+                // unrolled block (bpr is a multiple of 4)
+                for (uint32_t bq = 0; bq < bpr; bq += 4) {
 #pragma unroll
-                    for (uint32_t h = 0; h < 2; h++) {
-                        const uint32_t k = 2u * bp + h;
-                        const uint2 m = h ? m1 : m0;
-                        // the m bytes two blocks on (the next round's first two at a round's end)
-                        if (live) {
-                            const uint2 mn = k + 2 < bpr ? m_of(j, k + 2) : (j + 1 < rounds ? m_of(j + 1, k + 2 - bpr) : m);
-                            if (h) m1 = mn;
-                            else m0 = mn;
+                    for (uint32_t hs = 0; hs < 2; hs++, i++) {
+                        const uint32_t st = i % kStages, u = i / kStages;
+                        if (u >= 1 && !mbar_wait(&bar_free[st], (u - 1) & 1u)) err |= DFX_STATUS_TIMEOUT;
+#pragma unroll
+                        for (uint32_t h = 0; h < 2; h++) {
+                            const uint32_t kr = 2u * hs + h, k = bq + kr;
+                            const uint2 m = mq[kr];
+                            // the m bytes kMAhead blocks on (in the next round at a round's end)
+                            if (live)
+                                mq[kr] = k + kMAhead < bpr ? __ldg(mp + 32u * (k + kMAhead))
+                                                           : __ldg(mnext + 32u * (k + kMAhead - bpr));
+                            const uint4 o = decode_block(br, T, m, err);
+                            if (live) {
+                                st_shared_v4((h ? a_off1 : a_off0) + st * kAStageBytes, o);
+                                if (ga.w_out)
+                                    *reinterpret_cast<uint4*>(ga.w_out + row * ga.cols + ga.cols / ga.gpr * (j / 8) +
+                                                              (32u * k + c) * 8u) = o;
+                            }
                         }
-                        const uint4 o = decode_block(br, T, m, err);
-                        if (live) {
-                            st_shared_v4(sA + st * kAStageBytes + sw128_offset(kGemmTileRows, R, 0, 4u * h + q), o);
-                            if (ga.w_out)
-                                *reinterpret_cast<uint4*>(ga.w_out + row * ga.cols + ga.cols / ga.gpr * (j / 8) +
-                                                          (32u * k + c) * 8u) = o;
-                        }
+                        fence_proxy_async();  // A is read by the tensor cores
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bar_full[st]);
                     }
-                    fence_proxy_async();  // A is read by the tensor cores
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar_full[st]);
                 }
                 if (live && br.consumed() != c_bits) err |= DFX_STATUS_STREAM;
             };
@@ -408,6 +417,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
                 br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, live ? (uint32_t)(p0 & 31u) : 0u);
                 run(br);
             }
+            mp = mnext;
         }
 
         // ------------------------------------------------------------ epilogue

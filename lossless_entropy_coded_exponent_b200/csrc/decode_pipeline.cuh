@@ -421,6 +421,19 @@ __device__ void decode_tail_group(const DecodeArgs& a, const typename C::Tables&
     if (!ok) err |= DFX_STATUS_STREAM;
 }
 
+// The decode kernels are launched as programmatic dependents of the work before them in
+// the stream: a CTA may be scheduled while the previous kernel is still finishing (back-to-
+// back decodes then lose no time between launches).  It waits for that work to complete,
+// memory included, before it reads anything in global memory, or, when the plan says the
+// preceding kernel does not write the container (DFX_DECODE_EARLY_READ), only before its
+// first output write: its header checks, table build and first copies then overlap the
+// preceding kernel's last groups.
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void enter_dependent(const DecodeArgs& a) {
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    if (!a.early) wait_prior_grid();
+}
+
 // One tensor's decode by `ctas` CTAs of which this is number `cta`: the body of both
 // kernels below.
 template <class C, int K>
@@ -459,6 +472,7 @@ __device__ __forceinline__ void decode_tensor(const DecodeArgs& a, uint32_t cta,
     GroupState<K> gs;
     if (gw < full_end) group_prologue<C, K>(a, T, wb, gw, step, full_end, lane, gs);
     C::build(T, table, scratch);
+    if (a.early) wait_prior_grid();  // before the first output write
     if (gw < full_end) decode_full_groups<C, K>(a, T, table, wb, gs, step, full_end, lane, err);
     // the ragged last group, by the warp whose sequence it would continue
     if (n_full < a.n_group && n_full >= a.g_begin && n_full < a.g_end && gw == a.g_begin + (n_full - a.g_begin) % step)
@@ -466,18 +480,9 @@ __device__ __forceinline__ void decode_tensor(const DecodeArgs& a, uint32_t cta,
     if (err) atomicOr(a.status, err);
 }
 
-// Launched as a programmatic dependent of the work before it in the stream: a CTA may be
-// scheduled while the previous kernel is still finishing (back-to-back decodes then lose
-// no time between launches), and waits for that work to complete, memory included,
-// before it reads or writes anything in global memory.
-__device__ __forceinline__ void wait_prior_grid() {
-    asm volatile("griddepcontrol.wait;\n" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-}
-
 template <class C, int K>
 __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeArgs a) {
-    wait_prior_grid();
+    enter_dependent(a);
     decode_tensor<C, K>(a, blockIdx.x, gridDim.x);
 }
 
@@ -485,9 +490,9 @@ __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode(DecodeAr
 // share of one tensor, so it builds that tensor's tables once.
 template <class C, int K>
 __global__ void __launch_bounds__(DecodeShape<K>::kThreads, 1) k_decode_batch(const __grid_constant__ BatchArgs b) {
-    wait_prior_grid();
     uint32_t i = 0;
     while (i + 1 < b.count && blockIdx.x >= b.cta_begin[i + 1]) i++;
+    enter_dependent(b.t[i]);
     decode_tensor<C, K>(b.t[i], blockIdx.x - b.cta_begin[i], b.cta_begin[i + 1] - b.cta_begin[i]);
 }
 
@@ -520,7 +525,7 @@ cudaError_t allow_smem(F* kernel, size_t bytes, bool* done) {
     return e;
 }
 
-// Launch with programmatic stream serialisation (the kernel starts with wait_prior_grid).
+// Launch with programmatic stream serialisation (the kernel starts with enter_dependent).
 template <class Kern, class Arg>
 cudaError_t launch_programmatic(Kern* kernel, int grid, int threads, size_t smem, cudaStream_t s, const Arg& arg) {
     cudaLaunchConfig_t cfg = {};

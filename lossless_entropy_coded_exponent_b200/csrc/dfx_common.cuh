@@ -67,6 +67,7 @@ struct DecodeArgs {
     uint32_t g_begin, g_end;  // groups to decode (all: 0, n_group)
     uint64_t out_first;       // element index stored at out[0] (g_begin * G * K)
     uint32_t inject;          // test hook flags (dfx_debug_inject), normally 0
+    uint32_t early;           // 1: read the container before the preceding kernel completes
 };
 
 struct EncodeArgs {

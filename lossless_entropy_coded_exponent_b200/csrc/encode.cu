@@ -50,7 +50,7 @@ __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long lon
 
 // ---------------------------------------------------------------- 1. histogram
 //
-// One CTA of 16 warps per SM.  The input's 16-byte units (8 exponents each) are cut into
+// One CTA of 32 warps per SM.  The input's 16-byte units (8 exponents each) are cut into
 // chunks of 128 units (2 KiB); each warp takes a contiguous run of chunks and streams them
 // into its shared-memory buffers with the bulk-copy engine, kHistBufs chunks in flight,
 // so the bytes in flight do not depend on registers.  The exponents of a weight tensor
@@ -59,12 +59,13 @@ __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long lon
 // sample.  From then on a lane counts the values in that window in registers, four 8-bit
 // counters per 32-bit word (one shift and one add per value and word; a shift by 32 or
 // more gives 0, so a value lands in at most one word), and folds them into 32-bit counts
-// every kHistFold chunks (32 values per lane per chunk: no counter passes 255); values
-// outside the window take a shared-memory atomic.
+// every kHistFold chunks (32 values per lane per chunk: no counter passes 255).  Values
+// outside the window are rare: the warp checks once per 8 values whether any lane has
+// one, and only then takes shared-memory atomics for them.
 
-constexpr int kHistWarps = 16;
+constexpr int kHistWarps = 32;
 constexpr uint32_t kHistChunkUnits = 128;  // 16-byte units per chunk (2 KiB)
-constexpr uint32_t kHistBufs = 4;          // chunks in flight per warp
+constexpr uint32_t kHistBufs = 2;          // chunks in flight per warp
 constexpr uint32_t kHistFold = 7;          // chunks between folds (7 x 32 < 256)
 
 struct HistWarpBuffers {
@@ -174,15 +175,23 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
         }
 #pragma unroll
         for (uint32_t j = 0; j < kHistChunkUnits / 32; j++) {
-            if (lane + 32 * j >= nu) break;
+            const bool valid = lane + 32 * j < nu;  // (a partial chunk's lanes past its end count nothing)
             const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+            uint32_t outside = 0;
 #pragma unroll
             for (int q = 0; q < 8; q++) {
-                const uint32_t e = (w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu;
-                const uint32_t d = e - b;
-                c0w += shl_clamped(8u * d);
-                c1w += shl_clamped(8u * d - 32u);
-                if (d >= 8u) atomicAdd(&h[e], 1u);
+                const uint32_t d = ((w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu) - b;
+                const uint32_t s8 = valid ? 8u * d : 64u;
+                c0w += shl_clamped(s8);
+                c1w += shl_clamped(s8 - 32u);
+                outside |= d;
+            }
+            if (__any_sync(kFull, valid && outside >= 8u) && valid && outside >= 8u) {
+#pragma unroll
+                for (int q = 0; q < 8; q++) {
+                    const uint32_t e = (w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu;
+                    if (e - b >= 8u) atomicAdd(&h[e], 1u);
+                }
             }
         }
         if (++since == kHistFold) {
@@ -542,15 +551,15 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
 // Chunk lengths, the scan of the group lengths and the pack in one kernel, reading the
 // input once.  A CTA of 8 warps takes the next 8 groups from a ticket counter (so the
 // CTAs holding earlier groups are always running and the scan below always makes
-// progress); a warp loads its group into registers (lane i: the 16-byte blocks i, i + 32,
-// ... of the group), sums its chunk's code lengths, and finds the group's start bit by a
+// progress); a warp reads its group (lane i: the 16-byte blocks i, i + 32, ... of the
+// group), sums its chunk's code lengths, and finds the group's start bit by a
 // decoupled look-back over the group words of the workspace.  A group publishes its bit
 // count as soon as it is known (flag kGroupCount) and, once it has its own start, writes
 // the next group's gbase entry (its inclusive end) and then sets kGroupEnd; a warp adds
 // up its predecessors' counts, 32 at a time, back to the nearest group whose end is
-// published.  Then it packs its codes from the same registers (into the warp's shared
-// copy of its words, as k_pack does) and writes the sign+mantissa bytes.  The ragged last
-// group reads its elements from global memory.
+// published.  Then it packs its codes into the warp's shared copy of its words, reading
+// its input again (now from L2) one block ahead, writes the words out and writes the
+// sign+mantissa bytes.
 
 constexpr int kFusedWarps = 8;
 constexpr uint32_t kGroupCount = 1u << 30;  // the group's bit count (bits 0-29) is published
@@ -612,7 +621,7 @@ __device__ uint64_t lookback(const EncodeArgs& a, uint32_t g, unsigned lane, uin
 }
 
 template <int K>
-__global__ void __launch_bounds__(kFusedWarps * 32) k_pack_fused(EncodeArgs a) {
+__global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a) {
     __shared__ uint32_t cl_sh[256];  // code << 8 | length
     __shared__ uint32_t slice[kFusedWarps][kPackSliceWords];
     __shared__ uint32_t cta_ticket;
@@ -626,16 +635,14 @@ __global__ void __launch_bounds__(kFusedWarps * 32) k_pack_fused(EncodeArgs a) {
     const bool ragged = (uint64_t)(g + 1) * 32u * K > a.n;
     uint32_t err = 0;
 
-    // the lane's chunk: its code bits
+    // the lane's chunk: its code bits (the input is read again, from L2, by the pack)
     constexpr uint32_t NB = K / 8;
-    uint4 v[NB];
     uint32_t bits = 0;
     if (!ragged) {
-#pragma unroll
-        for (uint32_t k = 0; k < NB; k++) v[k] = __ldg(reinterpret_cast<const uint4*>(a.in + block_element(g, K, k, lane)));
-#pragma unroll
+#pragma unroll 4
         for (uint32_t k = 0; k < NB; k++) {
-            const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.in + block_element(g, K, k, lane)));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int q = 0; q < 4; q++) bits += (cl_sh[(w[q] >> 7) & 0xFFu] & 0xFFu) + (cl_sh[(w[q] >> 23) & 0xFFu] & 0xFFu);
         }
@@ -668,28 +675,13 @@ __global__ void __launch_bounds__(kFusedWarps * 32) k_pack_fused(EncodeArgs a) {
     uint32_t* stream = reinterpret_cast<uint32_t*>(a.out + a.off_stream);
     const uint64_t wf = gb0 >> 5, wl = (gb0 + group_bits + 31) >> 5;  // the group's words [wf, wl)
     const uint32_t count = (uint32_t)(wl - wf);
-    if (!ragged && count <= kPackSliceWords) {
+    if (count <= kPackSliceWords) {
         uint32_t* sm = slice[warp];
         for (uint32_t i = lane; i < count; i += 32) sm[i] = 0u;
         __syncwarp();
-        SharedWriter bw = make_writer(SharedSink{sm, wf}, start);
-        uint8_t* mpl = a.out + a.off_m;
-#pragma unroll
-        for (uint32_t k = 0; k < NB; k++) {
-            const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-            uint32_t mb[2] = {0u, 0u};
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                const uint32_t h = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-                const uint32_t partner = (w[j >> 1] >> (16 * ((j & 1) ^ 1))) & 0xFFFFu;  // element j ^ 1
-                const uint32_t ce = cl_sh[(h >> 7) & 0xFFu];
-                bw.put(ce >> 8, ce & 0xFFu);
-                mb[j >> 2] |= (((h & 0x7Fu) << 1) | (partner >> 15)) << (8 * (j & 3));
-            }
-            *reinterpret_cast<uint2*>(mpl + block_element(g, K, k, lane)) = make_uint2(mb[0], mb[1]);
-        }
-        bw.finish();
+        pack_chunk<K>(a, cl_sh, c, lane, start, SharedSink{sm, wf});
         __syncwarp();
+        // the group's first and last words may hold bits of its neighbours: OR-ed in
         for (uint32_t i = lane; i < count; i += 32) {
             const uint32_t wv = sm[i];
             if (i == 0 || i + 1 == count) {
@@ -697,16 +689,6 @@ __global__ void __launch_bounds__(kFusedWarps * 32) k_pack_fused(EncodeArgs a) {
             } else {
                 stream[wf + i] = wv;
             }
-        }
-    } else if (count <= kPackSliceWords) {
-        uint32_t* sm = slice[warp];
-        for (uint32_t i = lane; i < count; i += 32) sm[i] = 0u;
-        __syncwarp();
-        pack_chunk<K>(a, cl_sh, c, lane, start, SharedSink{sm, wf});
-        __syncwarp();
-        for (uint32_t i = lane; i < count; i += 32) {
-            const uint32_t wv = sm[i];
-            if (wv) atomicOr(stream + wf + i, wv);
         }
     } else {
         pack_chunk<K>(a, cl_sh, c, lane, start, GlobalSink{stream});

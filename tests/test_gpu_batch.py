@@ -138,3 +138,29 @@ def test_back_to_back_launches_of_one_plan():
             dfx.dfx_decode_range(plan, c, c.numel(), 200, 100, part)
             assert torch.equal(part, x[4096 * 200: 4096 * 300]), rep
         assert dfx.dfx_device_status(plan) == 0
+
+
+@pytest.mark.parametrize("K", [128, 64])
+def test_early_read_back_to_back_decodes(K):
+    """DFX_DECODE_EARLY_READ: containers written once, then decoded one after another into
+    one reused buffer and into separate buffers, launches back to back (each CTA reads its
+    container while the previous decode finishes and writes only after it)."""
+    ws = [inputs.llama3_8b_layer_tensor(i) for i in (0, 2, 3, 1)]  # 4096^2, 1024x4096, 1024x4096, 4096^2
+    comps = [torch.from_numpy(oracle.encode(w, K=K)).cuda() for w in ws]
+    xs = [to_dev(w) for w in ws]
+    plans = [dfx.dfx_plan(w.size, chunk_symbols=K, decode_flags=dfx.DFX_DECODE_EARLY_READ) for w in ws]
+    try:
+        big = torch.full((max(w.size for w in ws),), -1, dtype=torch.int16, device="cuda")
+        outs = [torch.full_like(x, -1) for x in xs]
+        for _ in range(3):
+            for p, c, o in zip(plans, comps, outs):
+                dfx.dfx_decode(p, c, c.numel(), o)
+            for p, c, x in zip(plans, comps, xs):
+                dfx.dfx_decode(p, c, c.numel(), big)
+        torch.cuda.synchronize()
+        assert all(dfx.dfx_device_status(p) == 0 for p in plans)
+        assert all(torch.equal(o, x) for o, x in zip(outs, xs))
+        assert torch.equal(big[: xs[-1].numel()], xs[-1])
+    finally:
+        for p in plans:
+            p.free()

@@ -81,6 +81,9 @@ def test_host_argument_errors_precede_cuda(lib):
     with pytest.raises(dfx.DfxError) as e:
         dfx.dfx_container_layout(10, 0, chunk_symbols=60)  # not a multiple of 8
     assert e.value.code == dfx.DFX_ERR_ARG
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_plan(1000, decode_flags=0x2)  # an unknown decode flag
+    assert e.value.code == dfx.DFX_ERR_ARG
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
