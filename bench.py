@@ -546,7 +546,7 @@ def run_tans_compare(args, dev, stream, xs, huff_sizes, huff_launch_us, n, tenso
 
     T = min(tensors, len(xs))
     K = args.chunk_symbols
-    plan = dfx.dfx_plan(n, chunk_symbols=K, coder=dfx.DFX_CODER_TANS)
+    plan = dfx.dfx_plan(n, chunk_symbols=K, coder=dfx.DFX_CODER_TANS, decode_flags=dfx.DFX_DECODE_EARLY_READ)
     try:
         scratch = torch.empty(plan.max_compressed_bytes, dtype=torch.uint8, device=dev)
         ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
@@ -564,20 +564,18 @@ def run_tans_compare(args, dev, stream, xs, huff_sizes, huff_launch_us, n, tenso
                 sizes.append(size)
         del scratch, ws
         out = torch.empty(n, dtype=torch.int16, device=dev)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps * T + 1)]
-        with torch.cuda.stream(stream):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        with torch.cuda.stream(stream):  # as the main measurement: events at step boundaries only
             for _ in range(3):
                 for i in range(T):
                     dfx.dfx_decode(plan, comps[i], sizes[i], out, stream=stream)
             ev[0].record(stream)
-            k = 1
-            for _ in range(reps):
+            for k in range(1, reps + 1):
                 for i in range(T):
                     dfx.dfx_decode(plan, comps[i], sizes[i], out, stream=stream)
-                    ev[k].record(stream)
-                    k += 1
+                ev[k].record(stream)
         stream.synchronize()
-        launch_us = [1e3 * ev[j].elapsed_time(ev[j + 1]) for j in range(len(ev) - 1)]
+        launch_us = [1e3 * ev[j].elapsed_time(ev[j + 1]) / T for j in range(len(ev) - 1)]
         exact = dfx.dfx_device_status(plan, stream=stream) == 0
         with torch.cuda.stream(stream):
             for i in range(T):

@@ -138,7 +138,8 @@ typedef struct {
  * builds its tables and starts copying its first group during that time, and waits for
  * the preceding kernel only before its first output write.  Without it (the default)
  * the CTA waits before it reads anything, which is always safe.  Applies to dfx_decode,
- * dfx_decode_range, dfx_decode_batch and dfx_decode_host; dfx_decode_gemm ignores it. */
+ * dfx_decode_range, dfx_decode_batch, dfx_decode_host and dfx_decode_gemm (which, with
+ * the flag, reads X and writes Y and W only after the wait). */
 #define DFX_DECODE_EARLY_READ 0x1u
 
 /* Byte offsets of the container sections for given n, params and stream length. */
@@ -252,7 +253,7 @@ int dfx_decode_host(dfx_plan_t plan, const void *h_comp, size_t comp_bytes, void
  * Y is the exact product rounded by FP32 accumulation in an order of the hardware's
  * choosing.  A corrupt container sets the plan's status word as dfx_decode does (Y
  * is then not valid).  Asynchronous; one kernel launch of one CTA per SM, each
- * decoding a tile of at most 120 rows once and feeding it to the tensor cores. */
+ * decoding a tile of at most 100 rows once and feeding it to the tensor cores. */
 int dfx_decode_gemm(dfx_plan_t plan, const void *d_comp, size_t comp_bytes, uint64_t rows, uint64_t cols,
                     const void *d_x, uint32_t tokens, float *d_y, void *d_w_out, cudaStream_t stream);
 

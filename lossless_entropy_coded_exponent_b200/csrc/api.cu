@@ -201,8 +201,10 @@ int dfx_encode(dfx_plan_t plan, const void* d_bf16, void* d_out, size_t out_capa
     a.ws_code = (uint32_t*)(ws + dfx::kWsCode);
     a.ws_len = ws + dfx::kWsLen;
     a.ws_group_bits = (uint32_t*)(ws + dfx::kWsGroupBits);
+    a.ws_edge = (unsigned long long*)(ws + dfx::ws_edge_offset(plan->L.n_group));
     a.ws_tans = (uint32_t*)(ws + dfx::ws_tans_offset(plan->L.n_group));
     a.status = plan->d_status;
+    a.max_bytes = plan->max_bytes;
     if (dfx::launch_encode(a, plan->max_bytes, stream) != cudaSuccess) {
         cudaGetLastError();
         return DFX_ERR_CUDA;

@@ -11,20 +11,24 @@
 // number of groups (32 chunks of K codes), so every group lies inside one row.  X is
 // tokens x cols BF16 (row-major), tokens <= 32; Y is tokens x rows FP32 (row-major).
 //
-// One CTA (one per SM) takes a tile of at most 120 rows of W (the MMA's M = 128):
-//   * every thread first helps build the Huffman tables in shared memory (the canonical
-//     per-length limits and the 14-bit pair table of huffman_tables.cuh);
-//   * 15 decoding warps hold up to 8 rows each, tile row R in warp R mod 15; four lanes
-//     share a row.  A group's 32 chunks are decoded in 8 rounds of 4: in round j lane q of
-//     a row decodes chunk 4 (j mod 8) + q from its first code to its last, 8 codes (one
+// One CTA of 26 warps (one per SM) takes a tile of at most 100 rows of W (the MMA's
+// M = 128 covers them):
+//   * every thread first helps build the Huffman tables in shared memory: the canonical
+//     per-length limits and a pair table on the next 13 stream bits (huffman_tables.cuh;
+//     32 KiB, half the decode kernel's);
+//   * 25 decoding warps hold up to 4 rows each, tile row R in warp R mod 25 (a warp without
+//     a row sits out); eight lanes share a row, so a tile of 97 rows (14336 rows on 148
+//     SMs) leaves 3 of 100 lane groups idle.  A group's 32 chunks are decoded in 4 rounds
+//     of 8: in round j lane q of
+//     a row decodes chunk 8 (j mod 4) + q from its first code to its last, 8 codes (one
 //     block) at a time, with the decode kernel's reader, from a shared-memory copy of the
 //     round's stream slice that the bulk-copy engine brought in during the previous round;
 //   * the sum over K of X W^T does not depend on the order of K, so the kernel takes K in
-//     the order it decodes it: two consecutive blocks of the four chunks of a round, 64
-//     weights per row, make one stage of A, 128 rows x 128 bytes (one K atom of the
-//     canonical K-major layout with the 128-byte swizzle: in each 8-row group, row r's
-//     16-byte chunk c sits at chunk c ^ (r mod 8)); the MMA warp gathers the same 64
-//     columns of X into the stage's B tile;
+//     the order it decodes it: one block of the eight chunks of a round, 64 weights per
+//     row, makes one stage of A, 128 rows x 128 bytes (one K atom of the canonical K-major
+//     layout with the 128-byte swizzle: in each 8-row group, row r's 16-byte chunk c sits
+//     at chunk c ^ (r mod 8)); the MMA warp gathers the same 64 columns of X into the
+//     stage's B tile;
 //   * the MMA warp waits for a stage's A (every decoding warp arrives on its barrier),
 //     issues 4 tcgen05.mma (M = 128, N = tokens rounded up to 16, K = 16) accumulating in
 //     tensor memory and commits them to the stage's "free" barrier, which the decoding
@@ -37,6 +41,7 @@
 // outside its own shared memory.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "decode_pipeline.cuh"
 #include "huffman_reader.cuh"
@@ -45,18 +50,22 @@
 namespace dfx {
 namespace {
 
-constexpr int kGemmDecodeWarps = 15;  // + the MMA warp: 16 warps, up to 128 registers each
-constexpr int kGemmRowSlots = 8;      // rows per decoding warp, four lanes each
-static_assert(kGemmMaxRows == kGemmDecodeWarps * kGemmRowSlots, "rows per tile at most");
+constexpr int kGemmLutBits = 13;      // pair table index bits
+constexpr int kGemmDecodeWarps = 25;  // + the MMA warp: 26 warps of up to 72 registers
+constexpr int kGemmLanesPerRow = 8;
+constexpr int kGemmRowSlots = 32 / kGemmLanesPerRow;  // rows per decoding warp
+static_assert(kGemmMaxRows <= kGemmDecodeWarps * kGemmRowSlots, "rows per tile at most");
 constexpr int kGemmTileRows = 128;    // MMA M (tile rows past the tile's own are never stored)
 static_assert(kGemmMaxRows <= kGemmTileRows, "the rows of a tile fit the MMA's M = 128");
 constexpr int kGemmThreads = (kGemmDecodeWarps + 1) * 32;
+constexpr uint32_t kRoundsPerGroup = 32 / kGemmLanesPerRow;
 constexpr uint32_t kAtomBytes = 128;                           // one swizzle row: 64 BF16
 constexpr uint32_t kAStageBytes = kGemmTileRows * kAtomBytes;  // 16 KiB: 128 rows x 64 K
-constexpr uint32_t kStages = 4;
+constexpr uint32_t kStages = 3;
 constexpr uint32_t kTmemCols = 32;                             // FP32 accumulator columns
-constexpr uint32_t kSliceBytes = 256;                          // a row's stream slice for one round
+constexpr uint32_t kSliceBytes = 416;                          // a row's stream slice for one round
 constexpr uint32_t kSliceWords = kSliceBytes / 4;
+static_assert(kSliceBytes % 16 == 0, "bulk copies move 16-byte units");
 
 // ---------------------------------------------------------------- tcgen05 helpers
 
@@ -156,9 +165,10 @@ __host__ __device__ constexpr uint32_t gemm_b_stage_bytes() {
 template <int NT>
 constexpr size_t gemm_dyn_smem_bytes() {
     // 1 KiB of alignment slack, the A and B stages, the pair table, the warps' buffers
-    return 1024 + kStages * (size_t)(kAStageBytes + gemm_b_stage_bytes<NT>()) + (sizeof(uint32_t) << kLutBits) +
+    return 1024 + kStages * (size_t)(kAStageBytes + gemm_b_stage_bytes<NT>()) + (sizeof(uint32_t) << kGemmLutBits) +
            kGemmDecodeWarps * sizeof(GemmWarp);
 }
+static_assert(gemm_dyn_smem_bytes<2>() + 1536 <= 227 * 1024, "shared memory");
 
 template <int NT>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_constant__ GemmArgs ga) {
@@ -177,15 +187,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
     const uint32_t sB = sA + kStages * kAStageBytes;  // kStages B stages
     uint8_t* after_b = dyn_smem + pad + kStages * (kAStageBytes + kBStage);
     uint32_t* lut = reinterpret_cast<uint32_t*>(after_b);
-    GemmWarp* warps = reinterpret_cast<GemmWarp*>(after_b + (sizeof(uint32_t) << kLutBits));
+    GemmWarp* warps = reinterpret_cast<GemmWarp*>(after_b + (sizeof(uint32_t) << kGemmLutBits));
 
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lo = (uint32_t)((uint64_t)blockIdx.x * ga.rows / gridDim.x);
     const uint32_t hi = (uint32_t)((uint64_t)(blockIdx.x + 1) * ga.rows / gridDim.x);
     const uint32_t rows_t = hi - lo;  // <= 120 (the host sizes the grid)
+    const uint32_t busy = min(rows_t, (uint32_t)kGemmDecodeWarps);  // decoding warps with rows
 
+    // launched as a programmatic dependent: without DFX_DECODE_EARLY_READ wait for the
+    // preceding kernel here; with it, only before reading X and before writing Y or W
+    enter_dependent(a);
     if (!build_canonical(a, T)) return;
-    build_pair_table(T, lut);
+    build_pair_table<kGemmLutBits>(T, lut);
 
     if (warp == kGemmDecodeWarps) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_addr(&tmem_slot)),
@@ -194,7 +208,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
         if (lane == 0) {
             for (uint32_t i = 0; i < kStages; i++) {
-                mbar_init_count(&bar_full[i], kGemmDecodeWarps);
+                mbar_init_count(&bar_full[i], busy);
                 mbar_init_count(&bar_free[i], 1);
             }
             mbar_init_count(&bar_done, 1);
@@ -214,44 +228,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
 
-    const uint32_t bpr = a.K / 8;            // blocks per chunk: per round
-    const uint32_t spr = bpr / 2;            // stages per round
-    const uint32_t rounds = ga.gpr * 8;      // rounds per row
-    const uint32_t n_stages = rounds * spr;  // stages per tile
+    const uint32_t bpr = a.K / 8;                       // blocks per chunk: stages per round
+    const uint32_t rounds = ga.gpr * kRoundsPerGroup;  // rounds per row
+    const uint32_t n_stages = rounds * bpr;             // stages per tile
     uint32_t err = 0;
 
     if (warp == kGemmDecodeWarps) {
         // ------------------------------------------------------------ MMA warp: B tiles, MMAs
+        // Stage i's B tile is X's 64 columns that hold block k of chunks 8 jj .. 8 jj + 7 of
+        // group grp (round j = kRoundsPerGroup grp + jj = i / bpr, k = i mod bpr), all tokens
+        // (rows past `tokens` zero): the warp loads the next stage's 16-byte pieces while the
+        // decoding warps fill the current stage's A, and stores them swizzled once the MMAs
+        // that last read the buffer have completed.
         constexpr uint32_t idesc = idesc_bf16_f32(N);
-        constexpr uint32_t NX = N * 8 / 32;  // 16-byte B chunks per lane per stage
+        constexpr uint32_t NX = N * 8 / 32;
         uint4 xv[NX];
-        // B chunk q of stage i: token q / 8, column chunk c = q mod 8, which holds block
-        // 2 bp + c / 4 of chunk 4 jj + c mod 4 of group grp (round j = 8 grp + jj = i / spr,
-        // bp = i mod spr)
         auto load_x = [&](uint32_t i) {
-            const uint32_t j = i / spr, bp = i % spr, grp = j / 8, jj = j % 8;
+            const uint32_t j = i / bpr, k = i % bpr, grp = j / kRoundsPerGroup, jj = j % kRoundsPerGroup;
 #pragma unroll
             for (uint32_t u = 0; u < NX; u++) {
                 const uint32_t q = lane + 32u * u, t = q / 8, c = q % 8;
-                const uint32_t pos = grp * 32u * a.K + (32u * (2u * bp + c / 4) + 4u * jj + c % 4) * 8u;
+                const uint32_t pos = grp * 32u * a.K + (32u * k + kGemmLanesPerRow * jj + c) * 8u;
                 xv[u] = t < ga.tokens ? __ldg(reinterpret_cast<const uint4*>(ga.x + (uint64_t)t * ga.cols + pos))
                                       : make_uint4(0, 0, 0, 0);
             }
         };
+        if (a.early) wait_prior_grid();
         load_x(0);
+        uint32_t st = 0, ph = 0;
         for (uint32_t i = 0; i < n_stages; i++) {
-            const uint32_t st = i % kStages, u = i / kStages;
-            // the stage's previous MMAs have read it
-            if (u >= 1 && !mbar_wait(&bar_free[st], (u - 1) & 1u)) err |= DFX_STATUS_TIMEOUT;
+            if (i >= kStages && !mbar_wait(&bar_free[st], ph ^ 1u)) err |= DFX_STATUS_TIMEOUT;
 #pragma unroll
             for (uint32_t v = 0; v < NX; v++) {
                 const uint32_t q = lane + 32u * v;
                 st_shared_v4(sB + st * kBStage + sw128_offset(N, q / 8, 0, q % 8), xv[v]);
             }
             if (i + 1 < n_stages) load_x(i + 1);
-            fence_proxy_async();  // B is read by the tensor cores
+            fence_proxy_async();
             __syncwarp();
-            if (!mbar_wait(&bar_full[st], u & 1u)) err |= DFX_STATUS_TIMEOUT;
+            if (!mbar_wait(&bar_full[st], ph)) err |= DFX_STATUS_TIMEOUT;
             tc_fence_after();
             if (lane == 0) {
 #pragma unroll
@@ -262,8 +277,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
                 if (i + 1 == n_stages) mma_commit(&bar_done);
             }
             __syncwarp();
+            if (++st == kStages) {
+                st = 0;
+                ph ^= 1u;
+            }
         }
-    } else {
+    } else if (warp < busy) {
         // ------------------------------------------------------------ decoding warps
         GemmWarp& W = warps[warp];
         const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
@@ -271,7 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
         const uint8_t* mplane = a.comp + a.off_m;
         const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.comp + kOffGbase);
         const uint16_t* clen = reinterpret_cast<const uint16_t*>(a.comp + a.off_clen);
-        const uint32_t slot = lane >> 2, q = lane & 3;
+        const uint32_t slot = lane / kGemmLanesPerRow, q = lane % kGemmLanesPerRow;
         const uint32_t R = warp + kGemmDecodeWarps * slot;  // this lane's tile row
         const bool live = R < rows_t;
         const uint64_t row = lo + R;
@@ -306,23 +325,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
             }
             __syncwarp();
         };
-        // lanes 0-7: copy round j's slice of row slot `lane` into buffer b (or arrive
-        // without a copy when the row is empty or its slice does not fit)
+        // lanes 0 .. kGemmRowSlots - 1: copy round j's slice of row slot `lane` into buffer
+        // b (or arrive without a copy when the row is empty or its slice does not fit)
         auto stage_round = [&](uint32_t j, uint32_t b) {
             if (lane < kGemmRowSlots) {
-                const uint32_t r = lane, jj = j % 8;
+                const uint32_t r = lane, c0 = kGemmLanesPerRow * (j % kRoundsPerGroup);
                 uint32_t bytes = 0;
                 if (warp + kGemmDecodeWarps * r < rows_t) {
-                    const unsigned long long s0 = W.gb0[r] + (jj ? W.incl[r][4 * jj - 1] : 0u);
-                    const unsigned long long s1 = W.gb0[r] + W.incl[r][4 * jj + 3];
+                    const unsigned long long s0 = W.gb0[r] + (c0 ? W.incl[r][c0 - 1] : 0u);
+                    const unsigned long long s1 = W.gb0[r] + W.incl[r][c0 + kGemmLanesPerRow - 1];
                     const uint32_t beg = ((uint32_t)(s0 >> 5) * 4u) & ~15u;
                     const uint32_t end = min((((uint32_t)(s1 >> 5) + 4u) * 4u + 15u) & ~15u, T.n_words * 4u);
                     W.base[b][r] = beg / 4u;
                     if (end > beg && end - beg <= kSliceBytes) bytes = end - beg;
                 }
-                const uint32_t mask = __ballot_sync(0xFFu, bytes != 0);
+                const uint32_t mask = __ballot_sync((1u << kGemmRowSlots) - 1u, bytes != 0);
                 if (lane == 0) W.staged[b] = mask;
-                __syncwarp(0xFFu);
+                __syncwarp((1u << kGemmRowSlots) - 1u);
                 fence_proxy_async();  // the buffer's previous contents were read (generic proxy)
                 if (bytes) bulk_copy(W.slice[b][r], a.comp + a.off_stream + 4ull * W.base[b][r], bytes, &W.bar[b]);
                 else mbar_arrive(&W.bar[b]);
@@ -331,26 +350,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
         };
         // the m bytes of this lane's chunk in round j: block k at m_base(j) + 32 k (uint2)
         auto m_base = [&](uint32_t j) -> const uint2* {
-            const uint32_t grp = j / 8, c = 4u * (j % 8) + q;
+            const uint32_t grp = j / kRoundsPerGroup, c = kGemmLanesPerRow * (j % kRoundsPerGroup) + q;
             return reinterpret_cast<const uint2*>(mplane + row * ga.cols + grp * 32u * a.K) + c;
         };
-        // this lane's 16-byte chunks in an A stage, for the first and second block of a stage
-        const uint32_t a_off0 = sA + sw128_offset(kGemmTileRows, R, 0, q);
-        const uint32_t a_off1 = sA + sw128_offset(kGemmTileRows, R, 0, 4u + q);
+        const uint32_t a_off = sA + sw128_offset(kGemmTileRows, R, 0, q);  // this lane's 16 bytes of an A stage
 
+        if (a.early && ga.w_out) wait_prior_grid();
         load_group(0);
         stage_round(0, 0);
         uint32_t sphase = 0;  // parity of each round buffer's next phase
-        // the m bytes of the next kMAhead blocks (ring: block k in mq[k % kMAhead]); at a
-        // round's end the ring runs on into the next round's first blocks
-        constexpr uint32_t kMAhead = 4;
-        uint2 mq[kMAhead];
+        // the m bytes of the next two blocks (block k in mq[k % 2]); at a round's end the ring
+        // runs on into the next round's first blocks
+        uint2 mq[2];
         const uint2* mp = m_base(0);
-#pragma unroll
-        for (uint32_t k = 0; k < kMAhead; k++) mq[k] = live ? __ldg(mp + 32u * k) : make_uint2(0, 0);
-        uint32_t i = 0;  // stage
+        mq[0] = live ? __ldg(mp) : make_uint2(0, 0);
+        mq[1] = live ? __ldg(mp + 32) : make_uint2(0, 0);
+        uint32_t st = 0, ph = 0;  // stage buffer of the current stage and the parity of its use
+        bool reuse = false;       // the stage buffers have been used once (their frees are awaited)
         for (uint32_t j = 0; j < rounds; j++) {
-            const uint32_t b = j & 1u, jj = j % 8, c = 4u * jj + q;
+            const uint32_t b = j & 1u, c = kGemmLanesPerRow * (j % kRoundsPerGroup) + q;
             // this lane's chunk: start (relative to the group) and bits, read before the
             // next group's index replaces them
             uint32_t c_start = 0, c_bits = 0;
@@ -364,56 +382,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
             __syncwarp();
             // the next round's slice (a new group's index first)
             if (j + 1 < rounds) {
-                if ((j + 1) % 8 == 0) load_group((j + 1) / 8);
+                if ((j + 1) % kRoundsPerGroup == 0) load_group((j + 1) / kRoundsPerGroup);
                 stage_round(j + 1, b ^ 1u);
             }
             if (!mbar_wait(&W.bar[b], (sphase >> b) & 1u)) err |= DFX_STATUS_TIMEOUT;
             sphase ^= 1u << b;
             const bool staged = (W.staged[b] >> slot) & 1u;
             const unsigned long long p0 = g_start + c_start;  // the chunk's first stream bit
-            // decode the round: every lane runs the same steps; a lane without a row stores
-            // nothing and its reader reads the slot's buffer (or word 0 of the stream)
             const uint2* mnext = j + 1 < rounds ? m_base(j + 1) : mp;  // the next round's m bytes
+            // decode the round: every lane runs the same steps; a lane without a row stores
+            // nothing and its reader reads the slot's zeroed buffer (or word 0 of the stream)
             auto run = [&](auto& br) {
-                // two stages (four blocks) per step: the m ring index is then fixed in each
-                // unrolled block (bpr is a multiple of 4)
-                for (uint32_t bq = 0; bq < bpr; bq += 4) {
+                for (uint32_t k0 = 0; k0 < bpr; k0 += 2) {  // bpr is even
 #pragma unroll
-                    for (uint32_t hs = 0; hs < 2; hs++, i++) {
-                        const uint32_t st = i % kStages, u = i / kStages;
-                        if (u >= 1 && !mbar_wait(&bar_free[st], (u - 1) & 1u)) err |= DFX_STATUS_TIMEOUT;
-#pragma unroll
-                        for (uint32_t h = 0; h < 2; h++) {
-                            const uint32_t kr = 2u * hs + h, k = bq + kr;
-                            const uint2 m = mq[kr];
-                            // the m bytes kMAhead blocks on (in the next round at a round's end)
-                            if (live)
-                                mq[kr] = k + kMAhead < bpr ? __ldg(mp + 32u * (k + kMAhead))
-                                                           : __ldg(mnext + 32u * (k + kMAhead - bpr));
-                            const uint4 o = decode_block(br, T, m, err);
-                            if (live) {
-                                st_shared_v4((h ? a_off1 : a_off0) + st * kAStageBytes, o);
-                                if (ga.w_out)
-                                    *reinterpret_cast<uint4*>(ga.w_out + row * ga.cols + ga.cols / ga.gpr * (j / 8) +
-                                                              (32u * k + c) * 8u) = o;
-                            }
+                    for (uint32_t h = 0; h < 2; h++) {
+                        const uint32_t k = k0 + h;
+                        const uint2 m = mq[h];
+                        // the m bytes two blocks on (in the next round at a round's end)
+                        if (live) mq[h] = k + 2 < bpr ? __ldg(mp + 32u * (k + 2)) : __ldg(mnext + 32u * (k + 2 - bpr));
+                        const uint4 o = decode_block(br, T, m, err);
+                        if (reuse && !mbar_wait(&bar_free[st], ph ^ 1u)) err |= DFX_STATUS_TIMEOUT;
+                        if (live) {
+                            st_shared_v4(a_off + st * kAStageBytes, o);
+                            if (ga.w_out)
+                                *reinterpret_cast<uint4*>(ga.w_out + row * ga.cols + ga.cols / ga.gpr * (j / kRoundsPerGroup) +
+                                                          (32u * k + c) * 8u) = o;
                         }
                         fence_proxy_async();  // A is read by the tensor cores
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&bar_full[st]);
+                        if (++st == kStages) {
+                            st = 0;
+                            ph ^= 1u;
+                            reuse = true;
+                        }
                     }
                 }
                 if (live && br.consumed() != c_bits) err |= DFX_STATUS_STREAM;
             };
             if (__all_sync(kFull, staged || !live)) {
-                BitReader<SlotWords> br;
+                BitReader<SlotWords, kGemmLutBits> br;
                 const uint32_t rel = live ? (uint32_t)(p0 - 32ull * W.base[b][slot]) : 0u;
                 br.init(lut, SlotWords{smem_addr(W.slice[b][slot])}, rel);
                 run(br);
             } else {
                 // a slice that did not fit: the whole warp reads this round from global memory
                 const uint32_t first = live ? (uint32_t)(p0 >> 5) : 0u;
-                BitReader<ClampedGlobalWords> br;
+                BitReader<ClampedGlobalWords, kGemmLutBits> br;
                 br.init(lut, ClampedGlobalWords{sw + first, maxw - first}, live ? (uint32_t)(p0 & 31u) : 0u);
                 run(br);
             }
@@ -422,6 +437,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
 
         // ------------------------------------------------------------ epilogue
         if (warp < 4) {
+            if (a.early) wait_prior_grid();
             if (!mbar_wait(&bar_done, 0)) err |= DFX_STATUS_TIMEOUT;
             tc_fence_after();
             const uint32_t r = 32u * warp + lane;  // tile row = tensor-memory lane
@@ -452,8 +468,7 @@ cudaError_t launch_gemm_nt(const GemmArgs& g, int grid, cudaStream_t s) {
     static bool attr_set[64] = {};
     const cudaError_t e = allow_smem(k_decode_gemm<NT>, gemm_dyn_smem_bytes<NT>(), attr_set);
     if (e != cudaSuccess) return e;
-    k_decode_gemm<NT><<<grid, kGemmThreads, gemm_dyn_smem_bytes<NT>(), s>>>(g);
-    return cudaGetLastError();
+    return launch_programmatic(k_decode_gemm<NT>, grid, kGemmThreads, gemm_dyn_smem_bytes<NT>(), s, g);
 }
 
 }  // namespace
@@ -462,6 +477,7 @@ cudaError_t launch_gemm_nt(const GemmArgs& g, int grid, cudaStream_t s) {
 cudaError_t launch_decode_gemm(const DecodeArgs& d, const uint16_t* x, float* y, uint16_t* w_out, uint32_t rows,
                                uint32_t cols, uint32_t tokens, int grid, cudaStream_t s) {
     GemmArgs g;
+    memset(&g, 0, sizeof(g));
     g.d = d;
     g.x = x;
     g.y = y;

@@ -21,7 +21,7 @@ constexpr unsigned kFull = 0xffffffffu;  // all lanes of a warp
 
 __host__ __device__ inline uint32_t gbase_offset(uint32_t coder) { return coder == DFX_CODER_TANS ? kOffGbaseTans : kOffGbase; }
 
-__host__ __device__ inline uint64_t align16(uint64_t x) { return (x + 15u) & ~uint64_t(15); }
+__host__ __device__ constexpr uint64_t align16(uint64_t x) { return (x + 15u) & ~uint64_t(15); }
 
 struct Layout {
     uint64_t n, n_chunk, n_group;
@@ -82,8 +82,10 @@ struct EncodeArgs {
     uint32_t* ws_code;              // [256]
     uint8_t* ws_len;                // [256]
     uint32_t* ws_group_bits;        // [n_group]
+    unsigned long long* ws_edge;    // coder 0: [n_group + 1] arrivals and bits at each group boundary
     uint32_t* ws_tans;              // coder 1: [kWsTansWords] encode tables
     uint32_t* status;
+    uint64_t max_bytes;             // the container's capacity (bytes past its end are zeroed)
 };
 
 // Several tensors decoded by one launch: tensor i gets CTAs [cta_begin[i], cta_begin[i+1]).
@@ -98,14 +100,20 @@ struct BatchArgs {
 constexpr uint64_t kWsCounts = 0;
 constexpr uint64_t kWsCode = 2048;
 constexpr uint64_t kWsLen = 3072;
+constexpr uint64_t kWsTicket = 3328;     // coder 0: the pack's CTA ticket counter
+constexpr uint64_t kWsTotalBits = 3336;  // coder 0: the stream's bit count, from the code book
 constexpr uint64_t kWsGroupBits = 4096;
+// coder 0: per group boundary b = 0 .. n_group (the start of group b), the bits that groups
+// b - 1 and b put in the stream word the boundary falls in (low half) and how many of the
+// two have done so (high half)
+__host__ __device__ constexpr uint64_t ws_edge_offset(uint64_t n_group) { return align16(kWsGroupBits + 4 * n_group); }
 // coder 1: per symbol (threshold << 16 | nb_hi, cs << 16 | f) and the slot of every
 // (symbol, state number) pair, after the group sums
 constexpr uint64_t kWsTansWords = 2 * 256 + (1u << kTansMaxLog);
 inline uint64_t ws_tans_offset(uint64_t n_group) { return (kWsGroupBits + 4 * n_group + 255) & ~uint64_t(255); }
 inline uint64_t workspace_bytes_for(uint64_t n_group, uint32_t coder = DFX_CODER_HUFFMAN) {
-    const uint64_t base = ws_tans_offset(n_group);
-    return coder == DFX_CODER_TANS ? base + 4 * kWsTansWords : base;
+    return coder == DFX_CODER_TANS ? ws_tans_offset(n_group) + 4 * kWsTansWords
+                                   : ws_edge_offset(n_group) + 8 * (n_group + 1);
 }
 
 // Launchers (encode.cu, encode_tans.cu / decode.cu, decode_tans.cu); `coder` selects the
@@ -126,7 +134,7 @@ int decode_blocks_per_sm_tans(uint32_t K);
 // Y = X W^T from W's container (decode_gemm.cu): at most kGemmMaxTokens tokens, at most
 // kGemmMaxRows rows of W per CTA
 constexpr uint32_t kGemmMaxTokens = 32;
-constexpr uint32_t kGemmMaxRows = 120;
+constexpr uint32_t kGemmMaxRows = 100;
 cudaError_t launch_decode_gemm(const DecodeArgs& d, const uint16_t* x, float* y, uint16_t* w_out, uint32_t rows,
                                uint32_t cols, uint32_t tokens, int grid, cudaStream_t s);
 

@@ -1,21 +1,23 @@
 // encode.cu -- GPU encoder for DFX1 containers (sm_100a).
 //
 // Passes, all stream-ordered on the caller's stream:
-//   0. zero the container's index region and everything after the m plane;
+//   0. zero the container's index region and the workspace words the pack counts in;
 //   1. k_histogram      exponent histogram: input streamed by the bulk-copy engine, counts
-//                       of the 8 most frequent neighbouring values in registers;
+//                       of the 16 most frequent neighbouring values in registers;
 //   2. k_build_codebook one CTA: package-merge code lengths (limit max_len), canonical codes,
-//                       len[256] and the constant header fields;
-//   3. k_pack_fused     one warp per group, groups in ticket order: the group's input
-//                       into registers once (a group's elements come in 8-element
-//                       blocks, block b belongs to chunk b mod 32, so lane i reads
-//                       blocks i, i+32, ...: 16-byte loads, 512 contiguous bytes per warp
-//                       instruction), per chunk its code bits (clen), the group's start
-//                       bit by a decoupled look-back over the groups before it (gbase,
-//                       total_bits, total_bytes), codes packed MSB-first into 32-bit
-//                       words in the same block order, and the mantissa+sign bytes
-//                       (mantissa * 2 + the sign of the pair partner, element x ^ 1) in
-//                       element order.
+//                       len[256], the constant header fields and the stream's bit count;
+//   3. k_pack_fused     one warp per group, groups in ticket order: the group's input read
+//                       once (a group's elements come in 8-element blocks, block b belongs
+//                       to chunk b mod 32, so lane i reads blocks i, i+32, ...: 16-byte
+//                       loads, 512 contiguous bytes per warp instruction), per block its 8
+//                       codes joined into one word and its mantissa+sign bytes (mantissa * 2
+//                       + the sign of the pair partner, element x ^ 1) written in element
+//                       order, per chunk its code bits (clen), the group's start bit by a
+//                       decoupled look-back over the groups before it (gbase, total_bits,
+//                       total_bytes), and the joined codes packed MSB-first into 32-bit
+//                       words; every stream word is written once (the word two groups share
+//                       by the second of them to finish), and the bytes past the container
+//                       are zeroed on the side.
 // The tANS coder shares pass 1 and k_group_scan (a one-CTA scan of per-group sums); its
 // passes 2, 3 and 5 are in encode_tans.cu.
 // The method: frequent exponent values get short codes ("DFloat11: lossless LLM
@@ -55,18 +57,20 @@ __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long lon
 // into its shared-memory buffers with the bulk-copy engine, kHistBufs chunks in flight,
 // so the bytes in flight do not depend on registers.  The exponents of a weight tensor
 // crowd into a few neighbouring values: each CTA counts its warps' first chunks into a
-// shared histogram and picks the 8 consecutive exponents [b, b + 8) with the most of that
-// sample.  From then on a lane counts the values in that window in registers, four 8-bit
-// counters per 32-bit word (one shift and one add per value and word; a shift by 32 or
-// more gives 0, so a value lands in at most one word), and folds them into 32-bit counts
-// every kHistFold chunks (32 values per lane per chunk: no counter passes 255).  Values
-// outside the window are rare: the warp checks once per 8 values whether any lane has
-// one, and only then takes shared-memory atomics for them.
-
+// shared histogram and picks the 16 consecutive exponents [b, b + 16) with the most of
+// that sample.  From then on a lane counts the values in that window in registers:
+// 4-bit counters, eight per 32-bit word (value b + d adds 1 << 4d to the first word for
+// d < 8 and 1 << 4(d - 8) to the second for 8 <= d < 16; a shift by 32 or more gives 0,
+// so a value lands in at most one word, and one three-input add takes the two values of
+// a 32-bit input word).  After every unit (at most 8 per counter) the nibbles are spread
+// into 8-bit counters, after kHistFold chunks those into 16-bit counters, and these into
+// the shared histogram at the end.  Values outside the window are rare: the warp checks
+// once per unit whether any lane met one, and only then takes shared-memory atomics.
 constexpr int kHistWarps = 32;
 constexpr uint32_t kHistChunkUnits = 128;  // 16-byte units per chunk (2 KiB)
 constexpr uint32_t kHistBufs = 2;          // chunks in flight per warp
-constexpr uint32_t kHistFold = 7;          // chunks between folds (7 x 32 < 256)
+constexpr uint32_t kHistFold = 7;          // chunks between byte folds (7 x 32 < 256)
+constexpr uint32_t kHistHalfFolds = 256;   // byte folds between half-word flushes (256 x 224 < 65536)
 
 struct HistWarpBuffers {
     uint4 chunk[kHistBufs][kHistChunkUnits];
@@ -81,13 +85,29 @@ __device__ __forceinline__ uint32_t shl_clamped(uint32_t s) {
     return r;
 }
 
-__device__ __forceinline__ void fold8(uint32_t& c0, uint32_t& c1, uint32_t (&r)[8]) {
+// Spread two words of 4-bit counters (values b .. b + 15) into four words of 8-bit counters:
+// c8[0] takes values b + {0, 2, 4, 6}, c8[1] b + {1, 3, 5, 7}, c8[2] and c8[3] the same for
+// b + 8 ..
+__device__ __forceinline__ void fold_nibbles(uint32_t& n0, uint32_t& n1, uint32_t (&c8)[4]) {
+    c8[0] += n0 & 0x0F0F0F0Fu;
+    c8[1] += (n0 >> 4) & 0x0F0F0F0Fu;
+    c8[2] += n1 & 0x0F0F0F0Fu;
+    c8[3] += (n1 >> 4) & 0x0F0F0F0Fu;
+    n0 = n1 = 0u;
+}
+// Spread the 8-bit counters into 16-bit ones: c16[2 w + h] holds byte h and byte h + 2 of
+// c8[w] (values b + {0, 4}, {2, 6}, {1, 5}, {3, 7}, {8, 12}, ...).
+__device__ __forceinline__ void fold_bytes(uint32_t (&c8)[4], uint32_t (&c16)[8]) {
 #pragma unroll
-    for (int k = 0; k < 4; k++) {
-        r[k] += (c0 >> (8 * k)) & 0xFFu;
-        r[k + 4] += (c1 >> (8 * k)) & 0xFFu;
+    for (int w = 0; w < 4; w++) {
+        c16[2 * w] += c8[w] & 0x00FF00FFu;
+        c16[2 * w + 1] += (c8[w] >> 8) & 0x00FF00FFu;
+        c8[w] = 0u;
     }
-    c0 = c1 = 0u;
+}
+// The value b + d that half h (0: low, 1: high) of c16[i] counts.
+__host__ __device__ constexpr uint32_t c16_value(int i, int h) {
+    return 8u * ((i >> 2) & 1) + 2u * (i & 1) + ((i >> 1) & 1) + 4u * h;
 }
 
 __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t* __restrict__ in, uint64_t n,
@@ -138,9 +158,9 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
     __syncthreads();
     if (threadIdx.x < 32) {  // the window with the largest sample mass: lane l tries b = l + 32 j
         uint32_t best = 0, best_b = 0;
-        for (uint32_t b = threadIdx.x; b <= 248; b += 32) {
+        for (uint32_t b = threadIdx.x; b <= 240; b += 32) {
             uint32_t m = 0;
-            for (uint32_t k = 0; k < 8; k++) m += h[b + k];
+            for (uint32_t k = 0; k < 16; k++) m += h[b + k];
             if (m > best) {
                 best = m;
                 best_b = b;
@@ -157,9 +177,9 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
         if (threadIdx.x == 0) window = best_b;
     }
     __syncthreads();
-    const uint32_t b = window;
-    uint32_t c0w = 0u, c1w = 0u, r[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-    uint32_t since = 0;
+    const uint32_t b = window, b4 = 4u * window, b4h = 4u * window + 32u;
+    uint32_t n0 = 0u, n1 = 0u, c8[4] = {0u, 0u, 0u, 0u}, c16[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    uint32_t since = 0, folds = 0;
     for (uint32_t k = 1; k < nc; k++) {
         const uint32_t slot = k % kHistBufs;
         if (!mbar_wait(&wb.bar[slot], (k / kHistBufs) & 1u)) err |= DFX_STATUS_TIMEOUT;
@@ -173,36 +193,56 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
             fence_proxy_async();
             issue(k + kHistBufs);
         }
+        if (nu == kHistChunkUnits) {
 #pragma unroll
-        for (uint32_t j = 0; j < kHistChunkUnits / 32; j++) {
-            const bool valid = lane + 32 * j < nu;  // (a partial chunk's lanes past its end count nothing)
-            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-            uint32_t outside = 0;
+            for (uint32_t j = 0; j < kHistChunkUnits / 32; j++) {
+                const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+                uint32_t outside = 0;
 #pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const uint32_t d = ((w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu) - b;
-                const uint32_t s8 = valid ? 8u * d : 64u;
-                c0w += shl_clamped(s8);
-                c1w += shl_clamped(s8 - 32u);
-                outside |= d;
-            }
-            if (__any_sync(kFull, valid && outside >= 8u) && valid && outside >= 8u) {
+                for (int q = 0; q < 4; q++) {
+                    // 4 e of the word's two values (exponent bits 7-14 and 23-30)
+                    const uint32_t e0 = (w[q] >> 5) & 0x3FCu, e1 = (w[q] >> 21) & 0x3FCu;
+                    const uint32_t s0 = e0 - b4, s1 = e1 - b4;
+                    n0 += shl_clamped(s0) + shl_clamped(s1);
+                    n1 += shl_clamped(e0 - b4h) + shl_clamped(e1 - b4h);
+                    outside |= s0 | s1;
+                }
+                fold_nibbles(n0, n1, c8);
+                if (__any_sync(kFull, outside >= 64u) && outside >= 64u) {
 #pragma unroll
-                for (int q = 0; q < 8; q++) {
-                    const uint32_t e = (w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu;
-                    if (e - b >= 8u) atomicAdd(&h[e], 1u);
+                    for (int q = 0; q < 8; q++) {
+                        const uint32_t e = (w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu;
+                        if (e - b >= 16u) atomicAdd(&h[e], 1u);
+                    }
                 }
             }
-        }
-        if (++since == kHistFold) {
-            fold8(c0w, c1w, r);
-            since = 0;
+            if (++since == kHistFold) {
+                fold_bytes(c8, c16);
+                since = 0;
+                if (++folds == kHistHalfFolds) {
+#pragma unroll
+                    for (int i = 0; i < 8; i++) {
+                        if (c16[i] & 0xFFFFu) atomicAdd(&h[b + c16_value(i, 0)], c16[i] & 0xFFFFu);
+                        if (c16[i] >> 16) atomicAdd(&h[b + c16_value(i, 1)], c16[i] >> 16);
+                        c16[i] = 0u;
+                    }
+                    folds = 0;
+                }
+            }
+        } else {  // the last chunk of the input, partial: shared-memory atomics
+            for (uint32_t j = 0; j < kHistChunkUnits / 32; j++) {
+                if (lane + 32 * j >= nu) continue;
+                const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+                for (int q = 0; q < 8; q++) atomicAdd(&h[(w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu], 1u);
+            }
         }
     }
-    fold8(c0w, c1w, r);
+    fold_bytes(c8, c16);
 #pragma unroll
-    for (int k = 0; k < 8; k++)
-        if (r[k]) atomicAdd(&h[b + k], r[k]);
+    for (int i = 0; i < 8; i++) {
+        if (c16[i] & 0xFFFFu) atomicAdd(&h[b + c16_value(i, 0)], c16[i] & 0xFFFFu);
+        if (c16[i] >> 16) atomicAdd(&h[b + c16_value(i, 1)], c16[i] >> 16);
+    }
     if (blockIdx.x == 0 && threadIdx.x < (n & 7)) atomicAdd(&h[(in[units * 8 + threadIdx.x] >> 7) & 0xFFu], 1u);
     if (err) atomicOr(status, err);
     __syncthreads();
@@ -339,6 +379,13 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     a.ws_code[t] = code;
     a.ws_len[t] = (uint8_t)l;
     a.out[kOffLen + t] = (uint8_t)l;
+    // the stream's bit count, for the pack's zeroing of the bytes past the container
+    __shared__ unsigned long long total_bits;
+    if (t == 0) total_bits = 0;
+    __syncthreads();
+    if (l) atomicAdd(&total_bits, c * l);
+    __syncthreads();
+    if (t == 0) *reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTotalBits) = total_bits;
 
     if (t == 0) {
         uint8_t* h = a.out;
@@ -410,20 +457,13 @@ __global__ void __launch_bounds__(kScanThreads) k_group_scan(EncodeArgs a) {
 
 // ---------------------------------------------------------------- bit writers
 
-constexpr uint32_t kPackSliceWords = 1024;  // a group's stream words staged per warp (4 KiB)
-
-// Where a chunk's packed words go: the stream in global memory, or the warp's shared
-// copy of its group's words.  The first word of a chunk and its last, partial word may
-// hold bits of the neighbouring chunks and are OR-ed in; the words between belong to the
-// chunk alone.
+// Where a chunk's packed words go when pack_chunk writes them straight to the stream in
+// global memory: the first word of a chunk and its last, partial word may hold bits of
+// the neighbouring chunks and are OR-ed in; the words between belong to the chunk alone.
 struct GlobalSink {
     uint32_t* stream;
     __device__ __forceinline__ void shared_word(uint64_t wi, uint32_t v) const { atomicOr(stream + wi, v); }
     __device__ __forceinline__ void own_word(uint64_t wi, uint32_t v) const { stream[wi] = v; }
-};
-struct SharedSink {
-    uint32_t* words;  // the group's first stream word is words[0] (see SharedWriter)
-    uint64_t base;
 };
 
 template <class Sink>
@@ -461,30 +501,6 @@ struct BitWriter {
     }
 };
 
-// A chunk's writer into the warp's shared copy of its group's words, without branches:
-// the codes go into a 64-bit accumulator and every completed word is OR-ed in (the copy
-// starts zeroed, and a chunk's first and last words may hold bits of its neighbours).
-struct SharedWriter {
-    uint32_t* words;  // the group's first stream word is words[0]
-    uint64_t base;
-    uint64_t wi;      // stream index of the word being completed
-    uint64_t acc;     // the low `nbits` bits are the pending bits
-    uint32_t nbits;
-
-    __device__ __forceinline__ void put(uint32_t code, uint32_t l) {
-        acc = (acc << l) | code;
-        nbits += l;
-        if (nbits >= 32) {
-            nbits -= 32;
-            atomicOr(words + (wi - base), (uint32_t)(acc >> nbits));
-            wi++;
-        }
-    }
-    __device__ __forceinline__ void finish() {
-        if (nbits) atomicOr(words + (wi - base), (uint32_t)(acc << (32 - nbits)));
-    }
-};
-
 __device__ __forceinline__ BitWriter<GlobalSink> make_writer(GlobalSink sink, uint64_t start) {
     BitWriter<GlobalSink> bw;
     bw.sink = sink;
@@ -494,10 +510,30 @@ __device__ __forceinline__ BitWriter<GlobalSink> make_writer(GlobalSink sink, ui
     bw.first = true;
     return bw;
 }
-__device__ __forceinline__ SharedWriter make_writer(SharedSink sink, uint64_t start) {
-    // the bits of the previous chunk in the first word count as already placed zeros
-    return SharedWriter{sink.words, sink.base, start >> 5, 0ull, (uint32_t)(start & 31)};
-}
+
+// A chunk's writer into the warp's shared copy of its group's words: the codes go into a
+// 64-bit accumulator and every completed word is OR-ed in (the copy starts zeroed, and a
+// chunk's first and last words may hold bits of its neighbours).  A put takes at most 32
+// bits, so the accumulator never holds more than 63.
+struct SliceWriter {
+    uint32_t* words;          // the group's first stream word is words[0]
+    uint32_t wo;              // offset of the word being completed
+    unsigned long long acc;   // the low `nbits` bits are the pending bits
+    uint32_t nbits;
+
+    __device__ __forceinline__ void put(uint32_t code, uint32_t l) {
+        acc = (acc << l) | code;
+        nbits += l;
+        if (nbits >= 32) {
+            nbits -= 32;
+            atomicOr(words + wo, (uint32_t)(acc >> nbits));
+            wo++;
+        }
+    }
+    __device__ __forceinline__ void finish() {
+        if (nbits) atomicOr(words + wo, (uint32_t)(acc << (32 - nbits)));
+    }
+};
 
 // Pack chunk c (lane `lane` of group c / 32), whose codes start at stream bit `start`,
 // and write its elements' mantissa+sign bytes.  cl_sh[e] = code << 8 | length.
@@ -522,16 +558,22 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
             const uint4 v = v_next;
             if (k + 1 < full) v_next = __ldg(reinterpret_cast<const uint4*>(a.in + block_element(g, K, k + 1, lane)));
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t mb[2] = {0u, 0u};
+            uint32_t mw[4];
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                const uint32_t h = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-                const uint32_t partner = (w[j >> 1] >> (16 * ((j & 1) ^ 1))) & 0xFFFFu;  // element j ^ 1
-                const uint32_t e = (h >> 7) & 0xFFu;
-                bw.put(cl_sh[e] >> 8, cl_sh[e] & 0xFFu);
-                mb[j >> 2] |= (((h & 0x7Fu) << 1) | (partner >> 15)) << (8 * (j & 3));
+            for (int j = 0; j < 4; j++) {
+                // the pair (2j, 2j + 1): its two codes, as one put when they fit 32 bits
+                const uint32_t c0 = cl_sh[(w[j] >> 7) & 0xFFu], c1 = cl_sh[(w[j] >> 23) & 0xFFu];
+                const uint32_t l0 = c0 & 0xFFu, l1 = c1 & 0xFFu;
+                if (l0 + l1 <= 32u) {
+                    bw.put(((c0 >> 8) << l1) | (c1 >> 8), l0 + l1);
+                } else {
+                    bw.put(c0 >> 8, l0);
+                    bw.put(c1 >> 8, l1);
+                }
+                // their m bytes in bytes 0 and 2: each mantissa above the other's sign
+                mw[j] = ((w[j] & 0x007F007Fu) << 1) | (w[j] >> 31) | ((w[j] << 1) & 0x00010000u);
             }
-            *reinterpret_cast<uint2*>(mpl + x0) = make_uint2(mb[0], mb[1]);
+            *reinterpret_cast<uint2*>(mpl + x0) = make_uint2(__byte_perm(mw[0], mw[1], 0x6420), __byte_perm(mw[2], mw[3], 0x6420));
         } else {  // the partial block, if any
             for (uint64_t x = x0; x < a.n; x++) {
                 const uint32_t h = a.in[x];
@@ -552,20 +594,36 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
 // input once.  A CTA of 8 warps takes the next 8 groups from a ticket counter (so the
 // CTAs holding earlier groups are always running and the scan below always makes
 // progress); a warp reads its group (lane i: the 16-byte blocks i, i + 32, ... of the
-// group), sums its chunk's code lengths, and finds the group's start bit by a
+// group) and, per block, looks up its 8 codes, joins them two by two and then into one
+// 64-bit word (kept in shared memory with its length), writes the block's sign+mantissa
+// bytes and adds the length to its chunk's count.  It finds the group's start bit by a
 // decoupled look-back over the group words of the workspace.  A group publishes its bit
 // count as soon as it is known (flag kGroupCount) and, once it has its own start, writes
 // the next group's gbase entry (its inclusive end) and then sets kGroupEnd; a warp adds
 // up its predecessors' counts, 32 at a time, back to the nearest group whose end is
-// published.  Then it packs its codes into the warp's shared copy of its words, reading
-// its input again (now from L2) one block ahead, writes the words out and writes the
-// sign+mantissa bytes.
+// published.  Then it puts its blocks' joined codes into the warp's shared copy of its
+// words, one or two puts per block, and writes the words out.  A block whose codes do
+// not fit 64 bits (or a pair of them 32) is looked up again, code by code, at the put;
+// the last, partial group and a group whose words do not fit the shared copy are packed
+// straight into the stream (pack_chunk).
 
 constexpr int kFusedWarps = 8;
+constexpr uint32_t kPackSliceWords = 512;  // a group's stream words staged per warp (2 KiB)
+constexpr uint8_t kSlowBlock = 255;        // a block whose codes are not joined (lengths are <= 192)
+
+template <int K>
+struct PackWarp {
+    unsigned long long code[K / 8][32];  // block k of lane i: its codes joined, in the low len bits
+    uint8_t len[K / 8][32];              // their length, or kSlowBlock
+    uint32_t slice[kPackSliceWords];     // the group's stream words
+};
+template <int K>
+constexpr size_t pack_smem_bytes() {
+    return kFusedWarps * sizeof(PackWarp<K>);
+}
 constexpr uint32_t kGroupCount = 1u << 30;  // the group's bit count (bits 0-29) is published
 constexpr uint32_t kGroupEnd = 1u << 31;    // and its end bit is in gbase[g + 1]
 constexpr uint32_t kLookbackPolls = 1u << 20;
-constexpr uint64_t kWsTicket = 3328;        // the pass's CTA ticket counter in the workspace
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
     uint32_t v;
@@ -579,6 +637,16 @@ __device__ __forceinline__ unsigned long long ld_relaxed64(const unsigned long l
 }
 __device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_volatile(const uint32_t* p) { return *reinterpret_cast<const volatile uint32_t*>(p); }
+
+// The stream word at the start of group b holds bits of groups b - 1 and b.  Each adds its
+// bits (disjoint from the other's, so the sum is their union) and one arrival to the
+// boundary's workspace word in one atomic; the group that arrives second writes the word.
+__device__ __forceinline__ void boundary_word(const EncodeArgs& a, uint32_t b, uint32_t* word, uint32_t bits) {
+    const unsigned long long old = atomicAdd(a.ws_edge + b, (1ull << 32) | bits);
+    if ((old >> 32) == 1u) *word = (uint32_t)old | bits;
 }
 
 // The exclusive start bit of group g: predecessors' published counts back to the nearest
@@ -623,28 +691,63 @@ __device__ uint64_t lookback(const EncodeArgs& a, uint32_t g, unsigned lane, uin
 template <int K>
 __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a) {
     __shared__ uint32_t cl_sh[256];  // code << 8 | length
-    __shared__ uint32_t slice[kFusedWarps][kPackSliceWords];
     __shared__ uint32_t cta_ticket;
+    extern __shared__ __align__(16) uint8_t pack_smem[];
     cl_sh[threadIdx.x] = (a.ws_code[threadIdx.x] << 8) | a.ws_len[threadIdx.x];
     if (threadIdx.x == 0) cta_ticket = atomicAdd(reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTicket), 1u);
     __syncthreads();
+    {
+        // this CTA's share of the bytes past the container (the stream's length is known
+        // from the code book), zeroed while the pack proceeds
+        const unsigned long long total =
+            *reinterpret_cast<const unsigned long long*>(reinterpret_cast<const uint8_t*>(a.ws_counts) + kWsTotalBits);
+        const uint64_t z0 = a.off_stream + 4 * ((total + 31) / 32), z16 = align16(z0);
+        if (z16 <= a.max_bytes) {
+            if (blockIdx.x == 0 && threadIdx.x < (z16 - z0) / 4) reinterpret_cast<uint32_t*>(a.out + z0)[threadIdx.x] = 0u;
+            const uint64_t units = (a.max_bytes - z16) / 16;
+            uint4* zp = reinterpret_cast<uint4*>(a.out + z16);
+            for (uint64_t u = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units; u += (uint64_t)gridDim.x * blockDim.x)
+                zp[u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t g = cta_ticket * kFusedWarps + warp;
     if (g >= a.n_group) return;
+    PackWarp<K>& pw = reinterpret_cast<PackWarp<K>*>(pack_smem)[warp];
     const uint64_t c = (uint64_t)g * 32 + lane;
     const bool ragged = (uint64_t)(g + 1) * 32u * K > a.n;
     uint32_t err = 0;
 
-    // the lane's chunk: its code bits (the input is read again, from L2, by the pack)
+    // the lane's chunk: its blocks' joined codes, their m bytes and the chunk's code bits
     constexpr uint32_t NB = K / 8;
     uint32_t bits = 0;
     if (!ragged) {
+        uint8_t* mpl = a.out + a.off_m;
 #pragma unroll 4
         for (uint32_t k = 0; k < NB; k++) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.in + block_element(g, K, k, lane)));
+            const uint64_t x0 = block_element(g, K, k, lane);
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.in + x0));
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t p[4], pl[4], mw[4];
 #pragma unroll
-            for (int q = 0; q < 4; q++) bits += (cl_sh[(w[q] >> 7) & 0xFFu] & 0xFFu) + (cl_sh[(w[q] >> 23) & 0xFFu] & 0xFFu);
+            for (int q = 0; q < 4; q++) {
+                const uint32_t c0 = cl_sh[(w[q] >> 7) & 0xFFu], c1 = cl_sh[(w[q] >> 23) & 0xFFu];
+                const uint32_t l1 = c1 & 0xFFu;
+                pl[q] = (c0 & 0xFFu) + l1;
+                p[q] = ((c0 >> 8) << l1) | (c1 >> 8);  // exact when pl[q] <= 32
+                // the m bytes in bytes 0 and 2: each mantissa above the other's sign
+                mw[q] = ((w[q] & 0x007F007Fu) << 1) | (w[q] >> 31) | ((w[q] << 1) & 0x00010000u);
+            }
+            const uint32_t L = pl[0] + pl[1] + pl[2] + pl[3];
+            const bool slow = max(max(pl[0], pl[1]), max(pl[2], pl[3])) > 32u || L > 64u;
+            unsigned long long x = p[0];
+            x = (x << pl[1]) | p[1];
+            x = (x << pl[2]) | p[2];
+            x = (x << pl[3]) | p[3];
+            pw.code[k][lane] = x;
+            pw.len[k][lane] = slow ? kSlowBlock : (uint8_t)L;
+            bits += L;
+            *reinterpret_cast<uint2*>(mpl + x0) = make_uint2(__byte_perm(mw[0], mw[1], 0x6420), __byte_perm(mw[2], mw[3], 0x6420));
         }
     } else {
         for (uint32_t k = 0; k < NB; k++) {
@@ -675,39 +778,86 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
     uint32_t* stream = reinterpret_cast<uint32_t*>(a.out + a.off_stream);
     const uint64_t wf = gb0 >> 5, wl = (gb0 + group_bits + 31) >> 5;  // the group's words [wf, wl)
     const uint32_t count = (uint32_t)(wl - wf);
-    if (count <= kPackSliceWords) {
-        uint32_t* sm = slice[warp];
+    // a word shared with the previous or the next group (a whole group holds at least 32 K
+    // bits, so only the last group can end in the word it starts in, and it has no next)
+    const bool shared_first = (gb0 & 31u) != 0;
+    const bool shared_last = ((gb0 + group_bits) & 31u) != 0 && g + 1 < a.n_group;
+    if (!ragged && count <= kPackSliceWords) {
+        uint32_t* sm = pw.slice;
         for (uint32_t i = lane; i < count; i += 32) sm[i] = 0u;
         __syncwarp();
-        pack_chunk<K>(a, cl_sh, c, lane, start, SharedSink{sm, wf});
-        __syncwarp();
-        // the group's first and last words may hold bits of its neighbours: OR-ed in
-        for (uint32_t i = lane; i < count; i += 32) {
-            const uint32_t wv = sm[i];
-            if (i == 0 || i + 1 == count) {
-                if (wv) atomicOr(stream + wf + i, wv);
-            } else {
-                stream[wf + i] = wv;
+        // the bits of the previous chunk in the first word count as already placed zeros
+        SliceWriter bw{sm, (uint32_t)((start >> 5) - wf), 0ull, (uint32_t)(start & 31)};
+        for (uint32_t k = 0; k < NB; k++) {
+            const uint32_t L = pw.len[k][lane];
+            const unsigned long long x = pw.code[k][lane];
+            if (L <= 32u) {
+                bw.put((uint32_t)x, L);
+            } else if (L != kSlowBlock) {
+                bw.put((uint32_t)(x >> 32), L - 32u);
+                bw.put((uint32_t)x, 32u);
+            } else {  // code by code
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.in + block_element(g, K, k, lane)));
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 8; q++) {
+                    const uint32_t cl = cl_sh[(w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu];
+                    bw.put(cl >> 8, cl & 0xFFu);
+                }
             }
         }
+        bw.finish();
+        __syncwarp();
+        for (uint32_t i = lane; i < count; i += 32) {
+            if ((i == 0 && shared_first) || (i + 1 == count && shared_last)) continue;
+            stream[wf + i] = sm[i];
+        }
+        if (lane == 0 && shared_first) boundary_word(a, g, stream + wf, sm[0]);
+        if (lane == 0 && shared_last) boundary_word(a, g + 1, stream + wl - 1, sm[count - 1]);
     } else {
+        // straight into the stream: the group's words start at zero, the codes are OR-ed in
+        for (uint32_t i = lane; i < count; i += 32) stream[wf + i] = 0u;
+        __syncwarp();
+        __threadfence();
         pack_chunk<K>(a, cl_sh, c, lane, start, GlobalSink{stream});
+        __syncwarp();
+        __threadfence();
+        if (lane == 0 && shared_first) boundary_word(a, g, stream + wf, ld_volatile(stream + wf));
+        if (lane == 0 && shared_last) boundary_word(a, g + 1, stream + wl - 1, ld_volatile(stream + wl - 1));
     }
     if (err) atomicOr(a.status, err);
+}
+
+template <int K>
+cudaError_t launch_pack(const EncodeArgs& a, unsigned ctas, int dev, cudaStream_t s) {
+    static bool attr_set[64] = {};
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(k_pack_fused<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pack_smem_bytes<K>());
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    k_pack_fused<K><<<ctas, kFusedWarps * 32, pack_smem_bytes<K>(), s>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t s) {
     cudaError_t err;
-    // index region (header .. clen padding) and everything after the m plane start at zero
+    // the index region (header .. clen padding) starts at zero; so does everything after the
+    // m plane, except that the Huffman pack writes every stream word and zeroes the bytes past
+    // the stream itself
+    const bool packs = a.coder != DFX_CODER_TANS && a.n_group > 0;
     if ((err = cudaMemsetAsync(a.out, 0, a.off_m, s)) != cudaSuccess) return err;
-    if ((err = cudaMemsetAsync(a.out + a.off_m + a.n, 0, max_bytes - (a.off_m + a.n), s)) != cudaSuccess) return err;
+    const uint64_t zero_end = packs ? a.off_stream : max_bytes;
+    if (zero_end > a.off_m + a.n &&
+        (err = cudaMemsetAsync(a.out + a.off_m + a.n, 0, zero_end - (a.off_m + a.n), s)) != cudaSuccess)
+        return err;
     if ((err = cudaMemsetAsync(a.ws_counts, 0, 256 * sizeof(unsigned long long), s)) != cudaSuccess) return err;
-    // the fused pass's CTA ticket and group words start at zero
-    if (a.coder != DFX_CODER_TANS &&
-        (err = cudaMemsetAsync(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTicket, 0,
-                               kWsGroupBits - kWsTicket + 4ull * a.n_group, s)) != cudaSuccess)
+    // the fused pass's CTA ticket, group words and boundary words start at zero
+    if (packs && (err = cudaMemsetAsync(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTicket, 0,
+                                        ws_edge_offset(a.n_group) + 8 * (a.n_group + 1) - kWsTicket, s)) != cudaSuccess)
         return err;
 
     int dev = 0, sms = 148;
@@ -742,12 +892,11 @@ cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t 
     }
     const unsigned ctas = (a.n_group + kFusedWarps - 1) / kFusedWarps;
     switch (a.K) {
-        case 32: k_pack_fused<32><<<ctas, kFusedWarps * 32, 0, s>>>(a); break;
-        case 64: k_pack_fused<64><<<ctas, kFusedWarps * 32, 0, s>>>(a); break;
-        case 128: k_pack_fused<128><<<ctas, kFusedWarps * 32, 0, s>>>(a); break;
+        case 32: return launch_pack<32>(a, ctas, dev, s);
+        case 64: return launch_pack<64>(a, ctas, dev, s);
+        case 128: return launch_pack<128>(a, ctas, dev, s);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace dfx

@@ -34,7 +34,7 @@
 namespace {
 
 constexpr uint64_t kStaticMaxGroups = 262144;
-constexpr uint64_t kStaticWorkspace = dfx::kWsGroupBits + 4 * kStaticMaxGroups;
+constexpr uint64_t kStaticWorkspace = dfx::ws_edge_offset(kStaticMaxGroups) + 8 * (kStaticMaxGroups + 1);
 constexpr uint64_t kStaticStatus = kStaticWorkspace;          // one u32, unused by encode kernels
 constexpr uint64_t kStaticBytes = kStaticWorkspace + 256;
 
@@ -90,8 +90,10 @@ extern "C" int dfx_encode_static(const void* d_bf16, uint64_t n, const dfx_param
     a.ws_code = (uint32_t*)(scratch + dfx::kWsCode);
     a.ws_len = scratch + dfx::kWsLen;
     a.ws_group_bits = (uint32_t*)(scratch + dfx::kWsGroupBits);
+    a.ws_edge = (unsigned long long*)(scratch + dfx::ws_edge_offset(lay.n_group));
     a.ws_tans = nullptr;
     a.status = (uint32_t*)(scratch + kStaticStatus);
+    a.max_bytes = max_bytes;
     if (dfx::launch_encode(a, max_bytes, stream) != cudaSuccess) {
         cudaGetLastError();
         return DFX_ERR_CUDA;

@@ -23,16 +23,16 @@ namespace {
 // its words along and load one new word.  No reload follows more than 32 consumed bits
 // (two table pairs take at most 28, a single code at most 24), so p moves at most one
 // word between reloads, and about one lane in three loads a word per round.  Every
-// pair the table resolves consumes at most kLutBits = 14 bits, so after the first pair
+// pair the table resolves consumes at most LB (<= 14) bits, so after the first pair
 // of a round at least 18 valid bits remain for the second.  Pairs the table cannot
 // resolve (the second code does not fit the index bits, or the first code is longer)
 // take a rare branch: it reloads after the first code and, when both codes are at most
-// kLutBits long, reads the second from the table entry at the new position; otherwise
+// LB long, reads the second from the table entry at the new position; otherwise
 // it decodes code by code with the canonical limits.
 //
 // Word sources: the global stream (with or without a bound clamp) or a warp's
 // shared-memory copy of a stream slice (decode_pipeline.cuh).
-template <class Words>
+template <class Words, int LB = kLutBits>  // LB: index bits of the pair table
 struct BitReader {
     const uint32_t* lut;  // pair table in shared memory
     Words words;
@@ -58,10 +58,10 @@ struct BitReader {
     }
     // One code, the general way (peek must be current): returns its symbol.
     __device__ __forceinline__ uint32_t one(const HuffTables& T, uint32_t& err) {
-        const uint32_t e = lut[peek >> (32 - kLutBits)];
+        const uint32_t e = lut[peek >> (32 - LB)];
         uint32_t len, sym;
         if ((e & 0x001F0000u) == 0) {
-            uint32_t ent = decode_long(peek, T);
+            uint32_t ent = decode_long<LB>(peek, T);
             if (ent >> 16) {
                 err |= DFX_STATUS_STREAM;
                 ent &= 0xFFFFu;
@@ -80,7 +80,7 @@ struct BitReader {
     template <int j>
     __device__ __forceinline__ uint32_t pair(uint32_t mw, const HuffTables& T, uint32_t& err) {
         constexpr uint32_t sel = j == 0 ? 0x5140u : 0x5342u;  // [mw.2j, sym0, mw.2j+1, sym1]
-        const uint32_t e = lut[peek >> (32 - kLutBits)];
+        const uint32_t e = lut[peek >> (32 - LB)];
         const uint32_t len = e >> 26;           // bit 5 is set when the entry is not a pair
         peek = __funnelshift_l(0u, peek, len);  // shifts by len & 31
         p += len;
@@ -90,7 +90,7 @@ struct BitReader {
             reload();
             // usually both codes fit the table on their own: the second one is the first
             // code of the entry at the new position, and peek keeps at least 18 valid bits
-            const uint32_t e2 = lut[peek >> (32 - kLutBits)];
+            const uint32_t e2 = lut[peek >> (32 - LB)];
             if ((e & 0x001F0000u) && (e2 & 0x001F0000u)) {
                 const uint32_t l1 = (e2 >> 16) & 31u;
                 p += l1;
@@ -108,8 +108,8 @@ struct BitReader {
 };
 
 // Decode the 8 codes of one block and merge them with the block's m bytes: 8 BF16.
-template <class Words>
-__device__ __forceinline__ uint4 decode_block(BitReader<Words>& br, const HuffTables& T, uint2 m, uint32_t& err) {
+template <class Words, int LB>
+__device__ __forceinline__ uint4 decode_block(BitReader<Words, LB>& br, const HuffTables& T, uint2 m, uint32_t& err) {
     uint4 o;
     br.reload();
     o.x = br.template pair<0>(m.x, T, err);

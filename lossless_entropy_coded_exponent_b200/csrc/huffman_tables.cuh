@@ -14,11 +14,12 @@
 namespace dfx {
 namespace {
 
-constexpr int kLutBits = 14;
+constexpr int kLutBits = 14;  // the decode kernel's pair table: 2^14 entries (64 KiB)
 
-// Pair table entry (u32), indexed by the next kLutBits stream bits:
+// Pair table entry (u32), indexed by the next LB stream bits (LB = kLutBits for the decode
+// kernel; the table has 2^LB entries):
 //   bits 0-7   first symbol        bits 8-15  second symbol
-//   bits 16-20 length of the first code (0: the first code is longer than kLutBits)
+//   bits 16-20 length of the first code (0: the first code is longer than LB)
 //   bits 26-30 bits the fast path consumes: both codes' lengths when both fit in the
 //              index bits, else the first code's length (0 for a long first code)
 //   bit  31    set when the entry does not hold two complete codes
@@ -140,22 +141,23 @@ __device__ __forceinline__ void fill_run(uint32_t* p, uint32_t cnt, uint32_t v, 
     }
 }
 
-// The pair table `lut` (1 << kLutBits entries) from the canonical tables.  The entries
-// whose index bits start with the code c0 of a first symbol s0 of length l0 <= kLutBits
-// are [c0, c0 + 1) << (kLutBits - l0); one warp per first symbol marks that run "first
+// The pair table `lut` (1 << LB entries) from the canonical tables.  The entries whose
+// index bits start with the code c0 of a first symbol s0 of length l0 <= LB are
+// [c0, c0 + 1) << (LB - l0); one warp per first symbol marks that run "first
 // code only" and then overwrites, for every second symbol whose code c1 fits the
-// remaining r = kLutBits - l0 bits, the sub-run that continues with c1.  Entries no short
+// remaining r = LB - l0 bits, the sub-run that continues with c1.  Entries no short
 // code starts keep the "long first code" mark.  Every thread of the block calls it.
+template <int LB = kLutBits>
 __device__ void build_pair_table(const HuffTables& T, uint32_t* lut) {
     const int t = threadIdx.x;
     const unsigned warp = t >> 5, lane = t & 31;
-    for (int i = t; i < (1 << kLutBits) / 4; i += blockDim.x)
+    for (int i = t; i < (1 << LB) / 4; i += blockDim.x)
         reinterpret_cast<uint4*>(lut)[i] = make_uint4(kNotPair, kNotPair, kNotPair, kNotPair);
     __syncthreads();
-    const uint32_t n_short = T.index[kLutBits + 1];  // symbols with codes of at most kLutBits bits
+    const uint32_t n_short = T.index[LB + 1];  // symbols with codes of at most LB bits
     for (uint32_t i0 = warp; i0 < n_short; i0 += blockDim.x >> 5) {
         const uint32_t l0 = T.slen[i0], s0 = T.sorted[i0];
-        const uint32_t r = kLutBits - l0;
+        const uint32_t r = LB - l0;
         const uint32_t lo = (T.first[l0] + i0 - T.index[l0]) << r;
         fill_run(lut + lo, 1u << r, kNotPair | s0 | (l0 << 16) | (l0 << 26), lane);
         __syncwarp();
@@ -174,9 +176,10 @@ __device__ void build_pair_table(const HuffTables& T, uint32_t* lut) {
 // A code longer than kLutBits: find its length from the canonical limits.  Returns
 // (len << 8) | symbol; bit 16 flags a bit pattern that is no code (Kraft-complete
 // tables make that impossible for a well-formed stream).
+template <int LB = kLutBits>
 __device__ __noinline__ uint32_t decode_long(uint32_t peek, const HuffTables& T) {
     const uint32_t v = peek >> (32 - kMaxLenLimit);
-    int l = kLutBits + 1;
+    int l = LB + 1;
     while (l <= (int)kMaxLenLimit && v >= T.limit[l]) l++;
     if (l > (int)kMaxLenLimit) return (1u << 16) | (kMaxLenLimit << 8);
     return ((uint32_t)l << 8) | T.sorted[T.index[l] + (v >> (kMaxLenLimit - l)) - T.first[l]];
