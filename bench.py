@@ -683,7 +683,9 @@ def run_decode_into_gemm(args, dev, tokens=16, slice_rows=3584):
     rows, cols = 14336, 4096
     n_slices = rows // slice_rows
     side = torch.cuda.Stream(device=dev)
-    plan = dfx.dfx_plan(rows * cols, chunk_symbols=args.chunk_symbols)
+    # weights written once and decoded for every product: the decodes may read their
+    # container while the kernel before them finishes (both decoding paths alike)
+    plan = dfx.dfx_plan(rows * cols, chunk_symbols=args.chunk_symbols, decode_flags=dfx.DFX_DECODE_EARLY_READ)
     try:
         assert dfx.group_elements(plan) == cols, "one group per row needs chunk_symbols = 128"
         w = inputs.llama3_8b_layer_tensor_cuda(4, device=dev)  # gate_proj

@@ -25,14 +25,16 @@
 //     round's stream slice that the bulk-copy engine brought in during the previous round;
 //   * the sum over K of X W^T does not depend on the order of K, so the kernel takes K in
 //     the order it decodes it: one block of the eight chunks of a round, 64 weights per
-//     row, makes one stage of A, 128 rows x 128 bytes (one K atom of the canonical K-major
-//     layout with the 128-byte swizzle: in each 8-row group, row r's 16-byte chunk c sits
-//     at chunk c ^ (r mod 8)); the MMA warp gathers the same 64 columns of X into the
-//     stage's B tile;
+//     row, makes one K atom of A, 128 rows x 128 bytes (the canonical K-major layout with
+//     the 128-byte swizzle: in each 8-row group, row r's 16-byte chunk c sits at chunk
+//     c ^ (r mod 8)); two consecutive blocks make one pipeline stage.  The MMA warp copies
+//     the same columns of X into the stage's B tile with 16-byte asynchronous copies
+//     (cp.async), one stage ahead;
 //   * the MMA warp waits for a stage's A (every decoding warp arrives on its barrier),
-//     issues 4 tcgen05.mma (M = 128, N = tokens rounded up to 16, K = 16) accumulating in
+//     issues 8 tcgen05.mma (M = 128, N = tokens rounded up to 16, K = 16) accumulating in
 //     tensor memory and commits them to the stage's "free" barrier, which the decoding
-//     warps wait on before they write the stage again, kStages stages later;
+//     warps (and the next B copy) wait on before they write the stage again, kStages
+//     stages later;
 //   * after the last stage, decoding warps 0-3 read the accumulator (tensor-memory lanes
 //     32 w .. 32 w + 31 are tile rows) and write Y.
 // Every wait is bounded: a wait that runs out sets DFX_STATUS_TIMEOUT and the kernel
@@ -60,8 +62,10 @@ static_assert(kGemmMaxRows <= kGemmTileRows, "the rows of a tile fit the MMA's M
 constexpr int kGemmThreads = (kGemmDecodeWarps + 1) * 32;
 constexpr uint32_t kRoundsPerGroup = 32 / kGemmLanesPerRow;
 constexpr uint32_t kAtomBytes = 128;                           // one swizzle row: 64 BF16
-constexpr uint32_t kAStageBytes = kGemmTileRows * kAtomBytes;  // 16 KiB: 128 rows x 64 K
-constexpr uint32_t kStages = 3;
+constexpr uint32_t kStageAtoms = 2;                            // K atoms (blocks of the round) per stage
+constexpr uint32_t kAAtomBytes = kGemmTileRows * kAtomBytes;    // 16 KiB: 128 rows x 64 K
+constexpr uint32_t kAStageBytes = kStageAtoms * kAAtomBytes;    // 32 KiB
+constexpr uint32_t kStages = 2;
 constexpr uint32_t kTmemCols = 32;                             // FP32 accumulator columns
 constexpr uint32_t kSliceBytes = 416;                          // a row's stream slice for one round
 constexpr uint32_t kSliceWords = kSliceBytes / 4;
@@ -114,6 +118,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 }
+// 16 bytes from global src to shared dst without a register stage; zeros when !valid
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(valid ? 16u : 0u)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+// waits until at most the newest committed group of this thread's copies is in flight
+__device__ __forceinline__ void cp_async_wait_prior() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
@@ -160,7 +172,7 @@ struct GemmWarp {
 
 template <int NT>  // N = 16 NT accumulator columns (tokens rounded up to 16)
 __host__ __device__ constexpr uint32_t gemm_b_stage_bytes() {
-    return 16u * NT * kAtomBytes;
+    return kStageAtoms * 16u * NT * kAtomBytes;
 }
 template <int NT>
 constexpr size_t gemm_dyn_smem_bytes() {
@@ -199,8 +211,112 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
     // preceding kernel here; with it, only before reading X and before writing Y or W
     enter_dependent(a);
     if (!build_canonical(a, T)) return;
-    build_pair_table<kGemmLutBits>(T, lut);
+    const uint32_t bpr = a.K / 8;                       // blocks per chunk: stages per round
+    const uint32_t rounds = ga.gpr * kRoundsPerGroup;  // rounds per row
+    const uint32_t spr = bpr / kStageAtoms;              // stages per round (bpr is even)
+    const uint32_t n_stages = rounds * spr;             // stages per tile
+    uint32_t err = 0;
 
+    // the MMA warp's state
+    constexpr uint32_t idesc = idesc_bf16_f32(N);
+    constexpr uint32_t NX = kStageAtoms * N * 8 / 32;  // 16-byte pieces per lane and stage
+    // B of stage i into stage buffer sb with 16-byte asynchronous copies (tokens past
+    // `tokens` read as zeros).  Piece q: atom q / 8N, token t, 16-byte column chunk c; the
+    // atom holds block k0 + atom of chunks 8 jj .. 8 jj + 7 of group grp (round j = i / spr)
+    auto copy_x = [&](uint32_t i, uint32_t sb) {
+        const uint32_t j = i / spr, k0 = kStageAtoms * (i % spr), grp = j / kRoundsPerGroup, jj = j % kRoundsPerGroup;
+#pragma unroll
+        for (uint32_t u = 0; u < NX; u++) {
+            const uint32_t q = lane + 32u * u, at = q / (8u * N), t = (q % (8u * N)) / 8, c = q % 8;
+            const uint32_t pos = grp * 32u * a.K + (32u * (k0 + at) + kGemmLanesPerRow * jj + c) * 8u;
+            const bool valid = t < ga.tokens;
+            cp_async16_zfill(sB + sb * kBStage + at * (N * kAtomBytes) + sw128_offset(N, t, 0, c),
+                             ga.x + (valid ? (uint64_t)t * ga.cols + pos : 0u), valid);
+        }
+    };
+
+    // the decoding warps' state (warp < busy)
+    GemmWarp& W = warps[warp < kGemmDecodeWarps ? warp : 0];
+    const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
+    const uint32_t maxw = T.n_words - 1;
+    const uint8_t* mplane = a.comp + a.off_m;
+    const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.comp + kOffGbase);
+    const uint16_t* clen = reinterpret_cast<const uint16_t*>(a.comp + a.off_clen);
+    const uint32_t slot = lane / kGemmLanesPerRow, q = lane % kGemmLanesPerRow;
+    const uint32_t R = warp + kGemmDecodeWarps * slot;  // this lane's tile row
+    const bool live = R < rows_t;
+    const uint64_t row = lo + R;
+
+    // group grp's index for every row of the warp (lane = chunk)
+    auto load_group = [&](uint32_t grp) {
+        unsigned long long g0[kGemmRowSlots], g1[kGemmRowSlots];
+        uint32_t cl[kGemmRowSlots];
+#pragma unroll
+        for (int r = 0; r < kGemmRowSlots; r++) {
+            if (warp + kGemmDecodeWarps * r < rows_t) {
+                const uint64_t g = (uint64_t)(lo + warp + kGemmDecodeWarps * r) * ga.gpr + grp;
+                g0[r] = __ldg(gbase + g);
+                g1[r] = __ldg(gbase + g + 1);
+                cl[r] = __ldg(clen + g * 32 + lane);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kGemmRowSlots; r++) {
+            if (warp + kGemmDecodeWarps * r >= rows_t) continue;  // the same for every lane
+            uint32_t incl = cl[r];
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const uint32_t yv = __shfl_up_sync(kFull, incl, d);
+                if (lane >= (unsigned)d) incl += yv;
+            }
+            const uint32_t sum = __shfl_sync(kFull, incl, 31);
+            const bool ok = g1[r] >= g0[r] && g1[r] <= T.total_bits && g1[r] - g0[r] == (unsigned long long)sum;
+            if (!ok) err |= DFX_STATUS_INDEX;
+            W.incl[r][lane] = ok ? incl : 0u;
+            if (lane == 0) W.gb0[r] = ok ? g0[r] : 0ull;
+        }
+        __syncwarp();
+    };
+    // lanes 0 .. kGemmRowSlots - 1: copy round j's slice of row slot `lane` into buffer
+    // b (or arrive without a copy when the row is empty or its slice does not fit)
+    auto stage_round = [&](uint32_t j, uint32_t b) {
+        if (lane < kGemmRowSlots) {
+            const uint32_t r = lane, c0 = kGemmLanesPerRow * (j % kRoundsPerGroup);
+            uint32_t bytes = 0;
+            if (warp + kGemmDecodeWarps * r < rows_t) {
+                const unsigned long long s0 = W.gb0[r] + (c0 ? W.incl[r][c0 - 1] : 0u);
+                const unsigned long long s1 = W.gb0[r] + W.incl[r][c0 + kGemmLanesPerRow - 1];
+                const uint32_t beg = ((uint32_t)(s0 >> 5) * 4u) & ~15u;
+                const uint32_t end = min((((uint32_t)(s1 >> 5) + 4u) * 4u + 15u) & ~15u, T.n_words * 4u);
+                W.base[b][r] = beg / 4u;
+                if (end > beg && end - beg <= kSliceBytes) bytes = end - beg;
+            }
+            const uint32_t mask = __ballot_sync((1u << kGemmRowSlots) - 1u, bytes != 0);
+            if (lane == 0) W.staged[b] = mask;
+            __syncwarp((1u << kGemmRowSlots) - 1u);
+            fence_proxy_async();  // the buffer's previous contents were read (generic proxy)
+            if (bytes) bulk_copy(W.slice[b][r], a.comp + a.off_stream + 4ull * W.base[b][r], bytes, &W.bar[b]);
+            else mbar_arrive(&W.bar[b]);
+        }
+        __syncwarp();
+    };
+    // the m bytes of this lane's chunk in round j: block k at m_base(j) + 32 k (uint2)
+    auto m_base = [&](uint32_t j) -> const uint2* {
+        const uint32_t grp = j / kRoundsPerGroup, c = kGemmLanesPerRow * (j % kRoundsPerGroup) + q;
+        return reinterpret_cast<const uint2*>(mplane + row * ga.cols + grp * 32u * a.K) + c;
+    };
+    const uint32_t a_off = sA + sw128_offset(kGemmTileRows, R, 0, q);  // this lane's 16 bytes of an A stage
+
+    uint32_t sphase = 0;  // parity of each round buffer's next phase
+    // the m bytes of the next two blocks (block k in mq[k % 2]); at a round's end the ring
+    // runs on into the next round's first blocks
+    uint2 mq[2] = {make_uint2(0, 0), make_uint2(0, 0)};
+    const uint2* mp = nullptr;
+
+    // Start-up: the MMA warp allocates the accumulator, sets up the stage barriers and
+    // loads the first B stage; each decoding warp loads its rows' first group index and
+    // starts its first round's copies and m loads; all of them in flight while every
+    // thread then builds the pair table.
     if (warp == kGemmDecodeWarps) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_addr(&tmem_slot)),
                      "r"(kTmemCols)
@@ -214,24 +330,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
             mbar_init_count(&bar_done, 1);
             fence_mbar_init();
         }
+        if (a.early) wait_prior_grid();
+        copy_x(0, 0);
+        cp_async_commit();
     } else {
         // slices start zeroed: a lane without a row decodes zeros from its never-staged slot
-        uint4* z = reinterpret_cast<uint4*>(&warps[warp].slice[0][0][0]);
-        for (uint32_t k = lane; k < sizeof(warps[warp].slice) / 16; k += 32) z[k] = make_uint4(0, 0, 0, 0);
+        uint4* z = reinterpret_cast<uint4*>(&W.slice[0][0][0]);
+        for (uint32_t k = lane; k < sizeof(W.slice) / 16; k += 32) z[k] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async();  // before the bulk copies into the same buffers
         if (lane == 0) {
-            for (int b = 0; b < 2; b++) mbar_init_count(&warps[warp].bar[b], kGemmRowSlots);
+            for (int b = 0; b < 2; b++) mbar_init_count(&W.bar[b], kGemmRowSlots);
             fence_mbar_init();
         }
+        __syncwarp();
+        if (warp < busy) {
+            if (a.early && ga.w_out) wait_prior_grid();
+            load_group(0);
+            stage_round(0, 0);
+            mp = m_base(0);
+            mq[0] = live ? __ldg(mp) : make_uint2(0, 0);
+            mq[1] = live ? __ldg(mp + 32) : make_uint2(0, 0);
+        }
     }
+    build_pair_table<kGemmLutBits>(T, lut);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
-
-    const uint32_t bpr = a.K / 8;                       // blocks per chunk: stages per round
-    const uint32_t rounds = ga.gpr * kRoundsPerGroup;  // rounds per row
-    const uint32_t n_stages = rounds * bpr;             // stages per tile
-    uint32_t err = 0;
 
     if (warp == kGemmDecodeWarps) {
         // ------------------------------------------------------------ MMA warp: B tiles, MMAs
@@ -240,39 +365,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
         // (rows past `tokens` zero): the warp loads the next stage's 16-byte pieces while the
         // decoding warps fill the current stage's A, and stores them swizzled once the MMAs
         // that last read the buffer have completed.
-        constexpr uint32_t idesc = idesc_bf16_f32(N);
-        constexpr uint32_t NX = N * 8 / 32;
-        uint4 xv[NX];
-        auto load_x = [&](uint32_t i) {
-            const uint32_t j = i / bpr, k = i % bpr, grp = j / kRoundsPerGroup, jj = j % kRoundsPerGroup;
-#pragma unroll
-            for (uint32_t u = 0; u < NX; u++) {
-                const uint32_t q = lane + 32u * u, t = q / 8, c = q % 8;
-                const uint32_t pos = grp * 32u * a.K + (32u * k + kGemmLanesPerRow * jj + c) * 8u;
-                xv[u] = t < ga.tokens ? __ldg(reinterpret_cast<const uint4*>(ga.x + (uint64_t)t * ga.cols + pos))
-                                      : make_uint4(0, 0, 0, 0);
-            }
-        };
-        if (a.early) wait_prior_grid();
-        load_x(0);
         uint32_t st = 0, ph = 0;
         for (uint32_t i = 0; i < n_stages; i++) {
-            if (i >= kStages && !mbar_wait(&bar_free[st], ph ^ 1u)) err |= DFX_STATUS_TIMEOUT;
-#pragma unroll
-            for (uint32_t v = 0; v < NX; v++) {
-                const uint32_t q = lane + 32u * v;
-                st_shared_v4(sB + st * kBStage + sw128_offset(N, q / 8, 0, q % 8), xv[v]);
+            // the next stage's B, into the buffer the MMAs of stage i + 1 - kStages read
+            if (i + 1 < n_stages) {
+                const uint32_t nb = st + 1 == kStages ? 0u : st + 1;
+                if (i + 1 >= kStages && !mbar_wait(&bar_free[nb], ((i + 1 - kStages) / kStages) & 1u))
+                    err |= DFX_STATUS_TIMEOUT;
+                copy_x(i + 1, nb);
             }
-            if (i + 1 < n_stages) load_x(i + 1);
-            fence_proxy_async();
+            cp_async_commit();
+            cp_async_wait_prior();  // every group but the newest: stage i's B has landed
+            fence_proxy_async();    // B is read by the tensor cores
             __syncwarp();
             if (!mbar_wait(&bar_full[st], ph)) err |= DFX_STATUS_TIMEOUT;
             tc_fence_after();
             if (lane == 0) {
 #pragma unroll
-                for (uint32_t kk = 0; kk < 4; kk++)
-                    mma_bf16(tmem, smem_desc_sw128(sA + st * kAStageBytes + kk * 32u),
-                             smem_desc_sw128(sB + st * kBStage + kk * 32u), idesc, (i | kk) != 0);
+                for (uint32_t at = 0; at < kStageAtoms; at++)
+#pragma unroll
+                    for (uint32_t kk = 0; kk < 4; kk++)
+                        mma_bf16(tmem, smem_desc_sw128(sA + st * kAStageBytes + at * kAAtomBytes + kk * 32u),
+                                 smem_desc_sw128(sB + st * kBStage + at * (N * kAtomBytes) + kk * 32u), idesc,
+                                 (i | at | kk) != 0);
                 mma_commit(&bar_free[st]);
                 if (i + 1 == n_stages) mma_commit(&bar_done);
             }
@@ -284,87 +399,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
         }
     } else if (warp < busy) {
         // ------------------------------------------------------------ decoding warps
-        GemmWarp& W = warps[warp];
-        const uint32_t* sw = reinterpret_cast<const uint32_t*>(a.comp + a.off_stream);
-        const uint32_t maxw = T.n_words - 1;
-        const uint8_t* mplane = a.comp + a.off_m;
-        const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.comp + kOffGbase);
-        const uint16_t* clen = reinterpret_cast<const uint16_t*>(a.comp + a.off_clen);
-        const uint32_t slot = lane / kGemmLanesPerRow, q = lane % kGemmLanesPerRow;
-        const uint32_t R = warp + kGemmDecodeWarps * slot;  // this lane's tile row
-        const bool live = R < rows_t;
-        const uint64_t row = lo + R;
-
-        // group grp's index for every row of the warp (lane = chunk)
-        auto load_group = [&](uint32_t grp) {
-            unsigned long long g0[kGemmRowSlots], g1[kGemmRowSlots];
-            uint32_t cl[kGemmRowSlots];
-#pragma unroll
-            for (int r = 0; r < kGemmRowSlots; r++) {
-                if (warp + kGemmDecodeWarps * r < rows_t) {
-                    const uint64_t g = (uint64_t)(lo + warp + kGemmDecodeWarps * r) * ga.gpr + grp;
-                    g0[r] = __ldg(gbase + g);
-                    g1[r] = __ldg(gbase + g + 1);
-                    cl[r] = __ldg(clen + g * 32 + lane);
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < kGemmRowSlots; r++) {
-                if (warp + kGemmDecodeWarps * r >= rows_t) continue;  // the same for every lane
-                uint32_t incl = cl[r];
-#pragma unroll
-                for (int d = 1; d < 32; d <<= 1) {
-                    const uint32_t yv = __shfl_up_sync(kFull, incl, d);
-                    if (lane >= (unsigned)d) incl += yv;
-                }
-                const uint32_t sum = __shfl_sync(kFull, incl, 31);
-                const bool ok = g1[r] >= g0[r] && g1[r] <= T.total_bits && g1[r] - g0[r] == (unsigned long long)sum;
-                if (!ok) err |= DFX_STATUS_INDEX;
-                W.incl[r][lane] = ok ? incl : 0u;
-                if (lane == 0) W.gb0[r] = ok ? g0[r] : 0ull;
-            }
-            __syncwarp();
-        };
-        // lanes 0 .. kGemmRowSlots - 1: copy round j's slice of row slot `lane` into buffer
-        // b (or arrive without a copy when the row is empty or its slice does not fit)
-        auto stage_round = [&](uint32_t j, uint32_t b) {
-            if (lane < kGemmRowSlots) {
-                const uint32_t r = lane, c0 = kGemmLanesPerRow * (j % kRoundsPerGroup);
-                uint32_t bytes = 0;
-                if (warp + kGemmDecodeWarps * r < rows_t) {
-                    const unsigned long long s0 = W.gb0[r] + (c0 ? W.incl[r][c0 - 1] : 0u);
-                    const unsigned long long s1 = W.gb0[r] + W.incl[r][c0 + kGemmLanesPerRow - 1];
-                    const uint32_t beg = ((uint32_t)(s0 >> 5) * 4u) & ~15u;
-                    const uint32_t end = min((((uint32_t)(s1 >> 5) + 4u) * 4u + 15u) & ~15u, T.n_words * 4u);
-                    W.base[b][r] = beg / 4u;
-                    if (end > beg && end - beg <= kSliceBytes) bytes = end - beg;
-                }
-                const uint32_t mask = __ballot_sync((1u << kGemmRowSlots) - 1u, bytes != 0);
-                if (lane == 0) W.staged[b] = mask;
-                __syncwarp((1u << kGemmRowSlots) - 1u);
-                fence_proxy_async();  // the buffer's previous contents were read (generic proxy)
-                if (bytes) bulk_copy(W.slice[b][r], a.comp + a.off_stream + 4ull * W.base[b][r], bytes, &W.bar[b]);
-                else mbar_arrive(&W.bar[b]);
-            }
-            __syncwarp();
-        };
-        // the m bytes of this lane's chunk in round j: block k at m_base(j) + 32 k (uint2)
-        auto m_base = [&](uint32_t j) -> const uint2* {
-            const uint32_t grp = j / kRoundsPerGroup, c = kGemmLanesPerRow * (j % kRoundsPerGroup) + q;
-            return reinterpret_cast<const uint2*>(mplane + row * ga.cols + grp * 32u * a.K) + c;
-        };
-        const uint32_t a_off = sA + sw128_offset(kGemmTileRows, R, 0, q);  // this lane's 16 bytes of an A stage
-
-        if (a.early && ga.w_out) wait_prior_grid();
-        load_group(0);
-        stage_round(0, 0);
-        uint32_t sphase = 0;  // parity of each round buffer's next phase
-        // the m bytes of the next two blocks (block k in mq[k % 2]); at a round's end the ring
-        // runs on into the next round's first blocks
-        uint2 mq[2];
-        const uint2* mp = m_base(0);
-        mq[0] = live ? __ldg(mp) : make_uint2(0, 0);
-        mq[1] = live ? __ldg(mp + 32) : make_uint2(0, 0);
         uint32_t st = 0, ph = 0;  // stage buffer of the current stage and the parity of its use
         bool reuse = false;       // the stage buffers have been used once (their frees are awaited)
         for (uint32_t j = 0; j < rounds; j++) {
@@ -401,20 +435,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_decode_gemm(const __grid_co
                         // the m bytes two blocks on (in the next round at a round's end)
                         if (live) mq[h] = k + 2 < bpr ? __ldg(mp + 32u * (k + 2)) : __ldg(mnext + 32u * (k + 2 - bpr));
                         const uint4 o = decode_block(br, T, m, err);
-                        if (reuse && !mbar_wait(&bar_free[st], ph ^ 1u)) err |= DFX_STATUS_TIMEOUT;
+                        if (h == 0 && reuse && !mbar_wait(&bar_free[st], ph ^ 1u)) err |= DFX_STATUS_TIMEOUT;
                         if (live) {
-                            st_shared_v4(a_off + st * kAStageBytes, o);
+                            st_shared_v4(a_off + st * kAStageBytes + h * kAAtomBytes, o);
                             if (ga.w_out)
                                 *reinterpret_cast<uint4*>(ga.w_out + row * ga.cols + ga.cols / ga.gpr * (j / kRoundsPerGroup) +
                                                           (32u * k + c) * 8u) = o;
                         }
-                        fence_proxy_async();  // A is read by the tensor cores
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&bar_full[st]);
-                        if (++st == kStages) {
-                            st = 0;
-                            ph ^= 1u;
-                            reuse = true;
+                        if (h + 1 == kStageAtoms) {  // the stage is complete
+                            fence_proxy_async();  // A is read by the tensor cores
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&bar_full[st]);
+                            if (++st == kStages) {
+                                st = 0;
+                                ph ^= 1u;
+                                reuse = true;
+                            }
                         }
                     }
                 }
