@@ -75,6 +75,15 @@ def lib() -> ctypes.CDLL:
                                        u8p, ctypes.c_uint64, u64p]
         L.dfxo_tans_encode_chunk.argtypes = [u32p, ctypes.c_uint32, u8p, ctypes.c_uint32, u8p, u64p]
         L.dfxo_tans_encode_chunk.restype = ctypes.c_int
+        L.dfxo_tans_encode_chunk_ways.argtypes = [u32p, ctypes.c_uint32, ctypes.c_uint32, u8p, ctypes.c_uint32, u8p,
+                                                  u64p]
+        L.dfxo_tans_encode_chunk_ways.restype = ctypes.c_int
+        L.dfxo_encode_tans2.argtypes = [u16p, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint32,
+                                        u8p, ctypes.c_uint64, u64p]
+        L.dfxo_encode_tans2.restype = ctypes.c_int
+        L.dfxo_tans2_max_container_bytes.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
+                                                     ctypes.c_uint32]
+        L.dfxo_tans2_max_container_bytes.restype = ctypes.c_uint64
         L.dfxo_tans_container_bytes.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint64]
         L.dfxo_tans_container_bytes.restype = ctypes.c_uint64
         L.dfxo_tans_max_container_bytes.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
@@ -186,16 +195,17 @@ def tans_tables(freq, table_log: int = 12):
     return sym, k
 
 
-def tans_encode_chunk(freq, symbols, table_log: int = 12) -> str:
-    """Rule T4 for one chunk with a given frequency table: its bits as a '0'/'1' string."""
+def tans_encode_chunk(freq, symbols, table_log: int = 12, states: int = 1) -> str:
+    """Rule T4 (states = 1) or T6 (states = 2) for one chunk with a given frequency
+    table: its bits as a '0'/'1' string."""
     f = np.zeros(256, dtype=np.uint32)
     src = np.asarray(freq, dtype=np.uint32)
     f[: src.size] = src
     syms = np.ascontiguousarray(symbols, dtype=np.uint8)
-    out = np.zeros((table_log * (syms.size + 1) + 7) // 8 + 8, dtype=np.uint8)
+    out = np.zeros((table_log * (syms.size + states) + 7) // 8 + 8, dtype=np.uint8)
     bits = np.zeros(1, dtype=np.uint64)
-    rc = lib().dfxo_tans_encode_chunk(_ptr(f, ctypes.c_uint32), table_log, _ptr(syms, ctypes.c_uint8), syms.size,
-                                      _ptr(out, ctypes.c_uint8), _ptr(bits, ctypes.c_uint64))
+    rc = lib().dfxo_tans_encode_chunk_ways(_ptr(f, ctypes.c_uint32), table_log, states, _ptr(syms, ctypes.c_uint8),
+                                           syms.size, _ptr(out, ctypes.c_uint8), _ptr(bits, ctypes.c_uint64))
     if rc:
         raise OracleError(rc, "tans_encode_chunk")
     nbits = int(bits[0])
@@ -212,14 +222,22 @@ def tans_max_container_bytes(n: int, K: int, G: int, table_log: int = 12) -> int
     return int(lib().dfxo_tans_max_container_bytes(n, K, G, table_log))
 
 
-def encode_tans(w: np.ndarray, K: int = 128, G: int = 32, table_log: int = 12) -> np.ndarray:
-    """Whole-tensor encode with the tANS exponent coder (coder 1)."""
+def tans2_max_container_bytes(n: int, K: int, G: int, table_log: int = 12) -> int:
+    return int(lib().dfxo_tans2_max_container_bytes(n, K, G, table_log))
+
+
+def encode_tans(w: np.ndarray, K: int = 128, G: int = 32, table_log: int = 12, states: int = 1) -> np.ndarray:
+    """Whole-tensor encode with the tANS exponent coder: coder 1 (one state per
+    chunk, rules T1-T5) or, with states = 2, coder 2 (rule T6 added)."""
+    if states not in (1, 2):
+        raise ValueError("states must be 1 or 2")
     w = np.ascontiguousarray(w, dtype=np.uint16).reshape(-1)
-    cap = tans_max_container_bytes(w.size, K, G, table_log)
+    cap = (tans_max_container_bytes if states == 1 else tans2_max_container_bytes)(w.size, K, G, table_log)
     out = np.empty(cap, dtype=np.uint8)
     used = np.zeros(1, dtype=np.uint64)
-    rc = lib().dfxo_encode_tans(_ptr(w, ctypes.c_uint16), w.size, K, G, table_log,
-                                _ptr(out, ctypes.c_uint8), cap, _ptr(used, ctypes.c_uint64))
+    fn = lib().dfxo_encode_tans if states == 1 else lib().dfxo_encode_tans2
+    rc = fn(_ptr(w, ctypes.c_uint16), w.size, K, G, table_log, _ptr(out, ctypes.c_uint8), cap,
+            _ptr(used, ctypes.c_uint64))
     if rc:
         raise OracleError(rc, "encode_tans")
     return out[: int(used[0])].copy()

@@ -38,7 +38,8 @@
  *      against the walk, merge the two bytes back.
  * No step is blocked, fused or reordered beyond that list.
  * A second exponent coder (coder 1, tANS) replaces steps 3-5 and 8 with the
- * rules T1-T5 stated at the end of this file; everything else is shared.
+ * rules T1-T5 stated at the end of this file, and coder 2 adds rule T6 (two
+ * interleaved tANS states per chunk) to them; everything else is shared.
  *
  * The container layout (all integers little-endian, every section starts at a
  * 16-byte boundary, every padding byte is zero):
@@ -79,6 +80,7 @@
 #define DFXO_GBASE_OFFSET 320u
 #define DFXO_CODER_HUFFMAN 0u
 #define DFXO_CODER_TANS 1u
+#define DFXO_CODER_TANS2 2u /* tANS with two interleaved states per chunk (rule T6) */
 #define DFXO_FREQ_OFFSET 64u
 #define DFXO_TANS_GBASE_OFFSET 576u
 
@@ -275,7 +277,8 @@ static uint64_t chunk_element(uint64_t g, uint32_t lane, uint32_t pos, uint32_t 
 }
 /* The sections after the code section are the same for both coders; only the
  * code section's size (len[256] for coder 0, freq[256] for coder 1) moves them. */
-static uint64_t gbase_of(uint32_t coder) { return coder == DFXO_CODER_TANS ? DFXO_TANS_GBASE_OFFSET : DFXO_GBASE_OFFSET; }
+static int is_tans(uint32_t coder) { return coder == DFXO_CODER_TANS || coder == DFXO_CODER_TANS2; }
+static uint64_t gbase_of(uint32_t coder) { return is_tans(coder) ? DFXO_TANS_GBASE_OFFSET : DFXO_GBASE_OFFSET; }
 static uint64_t off_clen_of(uint64_t ng, uint32_t coder) { return align16(gbase_of(coder) + 8 * (ng + 1)); }
 static uint64_t off_m_of(uint64_t nc, uint64_t ng, uint32_t coder) { return align16(off_clen_of(ng, coder) + 2 * nc); }
 static uint64_t off_stream_of(uint64_t n, uint64_t nc, uint64_t ng, uint32_t coder) {
@@ -386,7 +389,7 @@ uint64_t dfxo_max_container_bytes(uint64_t n, uint32_t K, uint32_t G) {
 static int decode_tans(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, uint64_t *n_out);
 
 int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, uint64_t *n_out) {
-    if (bytes >= DFXO_HEADER_BYTES && memcmp(c, "DFX1", 4) == 0 && get_u32(c + 60) == DFXO_CODER_TANS)
+    if (bytes >= DFXO_HEADER_BYTES && memcmp(c, "DFX1", 4) == 0 && is_tans(get_u32(c + 60)))
         return decode_tans(c, bytes, w, n_cap, n_out);
     if (bytes < DFXO_GBASE_OFFSET + 8) return DFXO_ERR_CORRUPT;
     if (memcmp(c, "DFX1", 4) != 0) return DFXO_ERR_CORRUPT;
@@ -513,10 +516,20 @@ int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, u
  *   T5. decoding a chunk: x = its first R bits; for each symbol, slot x holds
  *       symbol s with number k; with nb = R - floor(log2 k), x becomes
  *       k * 2^nb + (the next nb bits) - M.  After the last symbol x is 0.
- * The container is the DFX1 layout with u32 coder = 1 at offset 60, the table
- * log in the max_len word (offset 56), u16 freq[256] at offset 64 and the
- * group start bits at offset 576; the chunks, groups and blocks are those of
- * coder 0.                                                               */
+ *   T6. (coder 2) two interleaved states: a chunk's symbols at even positions
+ *       (0, 2, ...) are coded by state A, those at odd positions by state B,
+ *       each by T4 on its own, both starting from X = M, the chunk still
+ *       taken from its last symbol to its first; the chunk's bits are A's
+ *       final X - M (R bits), B's final X - M (R bits), then every symbol's
+ *       field in symbol order.  Decoding (T5 per state) reads A's and B's start
+ *       states, then decodes symbol i with the state of i's parity; both
+ *       states end at 0.  A lane's two table lookups per symbol pair are then
+ *       independent, which halves the decoder's chain of dependent loads; the
+ *       price is R more bits per chunk.
+ * The container is the DFX1 layout with u32 coder = 1 (2 for T6) at offset 60,
+ * the table log in the max_len word (offset 56), u16 freq[256] at offset 64
+ * and the group start bits at offset 576; the chunks, groups and blocks are
+ * those of coder 0.                                                      */
 
 static int tans_params_ok(uint64_t n, uint32_t K, uint32_t G, uint32_t R) {
     if (n >= ((uint64_t)1 << 32)) return 0;
@@ -578,27 +591,31 @@ int dfxo_tans_tables(const uint32_t f[256], uint32_t R, uint8_t *slot_sym, uint3
     return DFXO_OK;
 }
 
-/* T4 for one chunk of cnt symbols e[]: its bit length; when stream is not
- * NULL the bits are also written from stream bit `pos` on.  enc[cs[s] + k -
- * f[s]] is the slot of s numbered k; v and nb hold cnt fields. */
+/* T4 (ways = 1) or T6 (ways = 2) for one chunk of cnt symbols e[]: its bit
+ * length; when stream is not NULL the bits are also written from stream bit
+ * `pos` on.  enc[cs[s] + k - f[s]] is the slot of s numbered k; v and nb hold
+ * cnt fields.  Symbol i is coded by state i mod ways. */
 static uint64_t tans_chunk(const uint32_t f[256], const uint32_t cs[256], const uint32_t *enc, uint32_t R,
-                           const uint8_t *e, uint32_t cnt, uint8_t *stream, uint64_t pos, uint32_t *v, uint8_t *nb) {
+                           uint32_t ways, const uint8_t *e, uint32_t cnt, uint8_t *stream, uint64_t pos, uint32_t *v,
+                           uint8_t *nb) {
     if (cnt == 0) return 0;
     const uint32_t M = 1u << R;
-    uint32_t X = M;
-    uint64_t bits = R;
+    uint32_t X[2] = {M, M};
+    uint64_t bits = (uint64_t)R * ways;
     for (uint32_t i = cnt; i-- > 0;) {
-        const uint32_t s = e[i];
+        const uint32_t s = e[i], st = i % ways;
         uint32_t b = 0;
-        while ((X >> b) >= 2 * f[s]) b++;
-        v[i] = X & ((1u << b) - 1u);
+        while ((X[st] >> b) >= 2 * f[s]) b++;
+        v[i] = X[st] & ((1u << b) - 1u);
         nb[i] = (uint8_t)b;
         bits += b;
-        X = M + enc[cs[s] + (X >> b) - f[s]];
+        X[st] = M + enc[cs[s] + (X[st] >> b) - f[s]];
     }
     if (stream) {
-        put_bits(stream, pos, X - M, R);
-        pos += R;
+        for (uint32_t st = 0; st < ways; st++) {
+            put_bits(stream, pos, X[st] - M, R);
+            pos += R;
+        }
         for (uint32_t i = 0; i < cnt; i++) {
             put_bits(stream, pos, v[i], nb[i]);
             pos += nb[i];
@@ -607,12 +624,13 @@ static uint64_t tans_chunk(const uint32_t f[256], const uint32_t cs[256], const 
     return bits;
 }
 
-/* T4 for one chunk of cnt symbols with a given frequency table f (summing to M):
- * writes the chunk's bits MSB-first from bit 0 of `out` (zeroed by the caller, at least
- * R * (cnt + 1) bits long) and returns their number. */
-int dfxo_tans_encode_chunk(const uint32_t f[256], uint32_t R, const uint8_t *syms, uint32_t cnt, uint8_t *out,
-                           uint64_t *bits) {
-    if (R < 4 || R > 12) return DFXO_ERR_ARG;
+/* T4 (ways = 1) or T6 (ways = 2) for one chunk of cnt symbols with a given
+ * frequency table f (summing to M): writes the chunk's bits MSB-first from bit 0
+ * of `out` (zeroed by the caller, at least R * (cnt + ways) bits long) and
+ * returns their number. */
+int dfxo_tans_encode_chunk_ways(const uint32_t f[256], uint32_t R, uint32_t ways, const uint8_t *syms, uint32_t cnt,
+                                uint8_t *out, uint64_t *bits) {
+    if (R < 4 || R > 12 || ways < 1 || ways > 2) return DFXO_ERR_ARG;
     const uint32_t M = 1u << R;
     uint32_t cs[256], run = 0;
     for (int s = 0; s < 256; s++) {
@@ -628,7 +646,7 @@ int dfxo_tans_encode_chunk(const uint32_t f[256], uint32_t R, const uint8_t *sym
     int rc = DFXO_ERR_ARG;
     if (slot_sym && slot_k && enc && v && nb && dfxo_tans_tables(f, R, slot_sym, slot_k) == DFXO_OK) {
         for (uint32_t j = 0; j < M; j++) enc[cs[slot_sym[j]] + slot_k[j] - f[slot_sym[j]]] = j;
-        *bits = tans_chunk(f, cs, enc, R, syms, cnt, out, 0, v, nb);
+        *bits = tans_chunk(f, cs, enc, R, ways, syms, cnt, out, 0, v, nb);
         rc = DFXO_OK;
     }
     free(slot_sym);
@@ -639,6 +657,11 @@ int dfxo_tans_encode_chunk(const uint32_t f[256], uint32_t R, const uint8_t *sym
     return rc;
 }
 
+int dfxo_tans_encode_chunk(const uint32_t f[256], uint32_t R, const uint8_t *syms, uint32_t cnt, uint8_t *out,
+                           uint64_t *bits) {
+    return dfxo_tans_encode_chunk_ways(f, R, 1, syms, cnt, out, bits);
+}
+
 uint64_t dfxo_tans_container_bytes(uint64_t n, uint32_t K, uint32_t G, uint64_t total_bits) {
     return container_bytes_of(n, K, G, total_bits, DFXO_CODER_TANS);
 }
@@ -647,6 +670,12 @@ uint64_t dfxo_tans_max_container_bytes(uint64_t n, uint32_t K, uint32_t G, uint3
     /* a field is at most R bits (k >= 1), plus R bits of state per chunk */
     uint64_t nc = n_groups(n, K, G) * G;
     return container_bytes_of(n, K, G, (uint64_t)R * (n + nc), DFXO_CODER_TANS);
+}
+
+uint64_t dfxo_tans2_max_container_bytes(uint64_t n, uint32_t K, uint32_t G, uint32_t R) {
+    /* T6: two states per chunk */
+    uint64_t nc = n_groups(n, K, G) * G;
+    return container_bytes_of(n, K, G, (uint64_t)R * (n + 2 * nc), DFXO_CODER_TANS2);
 }
 
 /* The symbols of chunk `lane` of group g, in chunk order; returns how many. */
@@ -661,9 +690,10 @@ static uint32_t chunk_symbols(const uint16_t *w, uint64_t n, uint64_t g, uint32_
     return cnt;
 }
 
-int dfxo_encode_tans(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t R, uint8_t *out, uint64_t cap,
-                     uint64_t *out_bytes) {
+static int encode_tans_ways(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t R, uint32_t ways,
+                            uint8_t *out, uint64_t cap, uint64_t *out_bytes) {
     if (!tans_params_ok(n, K, G, R)) return DFXO_ERR_ARG;
+    const uint32_t coder = ways == 2 ? DFXO_CODER_TANS2 : DFXO_CODER_TANS;
     const uint32_t M = 1u << R;
     uint64_t counts[256];
     uint32_t f[256], cs[256];
@@ -694,9 +724,9 @@ int dfxo_encode_tans(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint
     for (uint64_t g = 0; g < ng; g++)
         for (uint32_t lane = 0; lane < G; lane++) {
             uint32_t cnt = chunk_symbols(w, n, g, lane, K, G, e);
-            total_bits += tans_chunk(f, cs, enc, R, e, cnt, NULL, 0, v, nb);
+            total_bits += tans_chunk(f, cs, enc, R, ways, e, cnt, NULL, 0, v, nb);
         }
-    uint64_t total = container_bytes_of(n, K, G, total_bits, DFXO_CODER_TANS);
+    uint64_t total = container_bytes_of(n, K, G, total_bits, coder);
     if (out_bytes) *out_bytes = total;
     if (cap < total) {
         rc = DFXO_ERR_CAPACITY;
@@ -713,21 +743,21 @@ int dfxo_encode_tans(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint
     put_u32(out + 36, G);
     put_u32(out + 40, (uint32_t)nc);
     put_u32(out + 44, (uint32_t)ng);
-    put_u64(out + 48, off_m_of(nc, ng, DFXO_CODER_TANS));
+    put_u64(out + 48, off_m_of(nc, ng, coder));
     put_u32(out + 56, R);
-    put_u32(out + 60, DFXO_CODER_TANS);
+    put_u32(out + 60, coder);
     for (int s = 0; s < 256; s++) put_u16(out + DFXO_FREQ_OFFSET + 2 * s, (uint16_t)f[s]);
     {
         uint8_t *gbase = out + DFXO_TANS_GBASE_OFFSET;
-        uint8_t *clen = out + off_clen_of(ng, DFXO_CODER_TANS);
-        uint8_t *mplane = out + off_m_of(nc, ng, DFXO_CODER_TANS);
-        uint8_t *stream = out + off_stream_of(n, nc, ng, DFXO_CODER_TANS);
+        uint8_t *clen = out + off_clen_of(ng, coder);
+        uint8_t *mplane = out + off_m_of(nc, ng, coder);
+        uint8_t *stream = out + off_stream_of(n, nc, ng, coder);
         uint64_t pos = 0;
         for (uint64_t g = 0; g < ng; g++) {
             put_u64(gbase + 8 * g, pos);
             for (uint32_t lane = 0; lane < G; lane++) {
                 uint32_t cnt = chunk_symbols(w, n, g, lane, K, G, e);
-                uint64_t bits = tans_chunk(f, cs, enc, R, e, cnt, stream, pos, v, nb);
+                uint64_t bits = tans_chunk(f, cs, enc, R, ways, e, cnt, stream, pos, v, nb);
                 put_u16(clen + 2 * (g * G + lane), (uint16_t)bits);
                 pos += bits;
             }
@@ -746,19 +776,30 @@ done:
     return rc;
 }
 
-/* T5, with every header field, the frequency table, the index and the
- * padding checked. */
+int dfxo_encode_tans(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t R, uint8_t *out, uint64_t cap,
+                     uint64_t *out_bytes) {
+    return encode_tans_ways(w, n, K, G, R, 1, out, cap, out_bytes);
+}
+
+int dfxo_encode_tans2(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t R, uint8_t *out, uint64_t cap,
+                      uint64_t *out_bytes) {
+    return encode_tans_ways(w, n, K, G, R, 2, out, cap, out_bytes);
+}
+
+/* T5 (T6 for coder 2), with every header field, the frequency table, the index
+ * and the padding checked. */
 static int decode_tans(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, uint64_t *n_out) {
     if (bytes < DFXO_TANS_GBASE_OFFSET + 8) return DFXO_ERR_CORRUPT;
     if (get_u16(c + 4) != 1 || get_u16(c + 6) != DFXO_HEADER_BYTES) return DFXO_ERR_CORRUPT;
+    const uint32_t coder = get_u32(c + 60), ways = coder == DFXO_CODER_TANS2 ? 2u : 1u;
     uint64_t n = get_u64(c + 8), total_bits = get_u64(c + 16), total = get_u64(c + 24);
     uint32_t K = get_u32(c + 32), G = get_u32(c + 36), R = get_u32(c + 56);
     if (!tans_params_ok(n, K, G, R)) return DFXO_ERR_CORRUPT;
     uint64_t ng = n_groups(n, K, G), nc = ng * G;
     if (get_u32(c + 40) != nc || get_u32(c + 44) != ng) return DFXO_ERR_CORRUPT;
-    if (get_u64(c + 48) != off_m_of(nc, ng, DFXO_CODER_TANS)) return DFXO_ERR_CORRUPT;
-    if (total_bits > (uint64_t)R * (n + nc)) return DFXO_ERR_CORRUPT;
-    if (total != container_bytes_of(n, K, G, total_bits, DFXO_CODER_TANS) || total > bytes) return DFXO_ERR_CORRUPT;
+    if (get_u64(c + 48) != off_m_of(nc, ng, coder)) return DFXO_ERR_CORRUPT;
+    if (total_bits > (uint64_t)R * (n + ways * nc)) return DFXO_ERR_CORRUPT;
+    if (total != container_bytes_of(n, K, G, total_bits, coder) || total > bytes) return DFXO_ERR_CORRUPT;
     if (n_out) *n_out = n;
     if (n > n_cap) return DFXO_ERR_CAPACITY;
 
@@ -777,14 +818,14 @@ static int decode_tans(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n
     if (n > 0) dfxo_tans_tables(f, R, slot_sym, slot_k);
 
     const uint8_t *gbase = c + DFXO_TANS_GBASE_OFFSET;
-    const uint8_t *clen = c + off_clen_of(ng, DFXO_CODER_TANS);
-    const uint8_t *mplane = c + off_m_of(nc, ng, DFXO_CODER_TANS);
-    const uint8_t *stream = c + off_stream_of(n, nc, ng, DFXO_CODER_TANS);
-    for (uint64_t b = DFXO_TANS_GBASE_OFFSET + 8 * (ng + 1); b < off_clen_of(ng, DFXO_CODER_TANS); b++)
+    const uint8_t *clen = c + off_clen_of(ng, coder);
+    const uint8_t *mplane = c + off_m_of(nc, ng, coder);
+    const uint8_t *stream = c + off_stream_of(n, nc, ng, coder);
+    for (uint64_t b = DFXO_TANS_GBASE_OFFSET + 8 * (ng + 1); b < off_clen_of(ng, coder); b++)
         if (c[b]) goto done;
-    for (uint64_t b = off_clen_of(ng, DFXO_CODER_TANS) + 2 * nc; b < off_m_of(nc, ng, DFXO_CODER_TANS); b++)
+    for (uint64_t b = off_clen_of(ng, coder) + 2 * nc; b < off_m_of(nc, ng, coder); b++)
         if (c[b]) goto done;
-    for (uint64_t b = off_m_of(nc, ng, DFXO_CODER_TANS) + n; b < off_stream_of(n, nc, ng, DFXO_CODER_TANS); b++)
+    for (uint64_t b = off_m_of(nc, ng, coder) + n; b < off_stream_of(n, nc, ng, coder); b++)
         if (c[b]) goto done;
     if (get_u64(gbase) != 0 || get_u64(gbase + 8 * ng) != total_bits) goto done;
 
@@ -793,27 +834,28 @@ static int decode_tans(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n
         if (get_u64(gbase + 8 * g) != pos) goto done;
         for (uint32_t lane = 0; lane < G; lane++) {
             uint64_t chunk_start = pos;
-            uint32_t x = 0;
+            uint32_t x[2] = {0, 0};
             for (uint32_t k = 0; k < K; k++) {
                 uint64_t xe = chunk_element(g, lane, k, K, G);
                 if (xe >= n) break;
-                if (k == 0) { /* the chunk's first R bits: the decoder's start state */
-                    for (uint32_t b = 0; b < R; b++) {
-                        if (pos >= total_bits) goto done;
-                        x = (x << 1) | get_bit(stream, pos++);
-                    }
-                }
-                uint32_t s = slot_sym[x], kk = slot_k[x], nbits = R, t = kk;
+                if (k == 0) /* the chunk's first R bits (per state): the decoder's start states */
+                    for (uint32_t st = 0; st < ways; st++)
+                        for (uint32_t b = 0; b < R; b++) {
+                            if (pos >= total_bits) goto done;
+                            x[st] = (x[st] << 1) | get_bit(stream, pos++);
+                        }
+                uint32_t *xs = &x[k % ways]; /* T6: symbol k's state */
+                uint32_t s = slot_sym[*xs], kk = slot_k[*xs], nbits = R, t = kk;
                 while (t >>= 1) nbits--;
                 uint32_t val = 0;
                 for (uint32_t b = 0; b < nbits; b++) {
                     if (pos >= total_bits) goto done;
                     val = (val << 1) | get_bit(stream, pos++);
                 }
-                x = (kk << nbits) + val - M;
+                *xs = (kk << nbits) + val - M;
                 w[xe] = dfxo_merge((uint8_t)s, mplane[xe], mplane[dfxo_partner(xe, n)]);
             }
-            if (x != 0) goto done; /* every chunk ends in the encoder's start state */
+            if (x[0] != 0 || x[1] != 0) goto done; /* every state ends in the encoder's start state */
             if (get_u16(clen + 2 * (g * G + lane)) != pos - chunk_start) goto done;
         }
     }
