@@ -409,6 +409,7 @@ def run_ours(args, world, rank, local):
     # ---- the other exponent coder (tANS) on the same tensors and launch configuration
     if not args.no_tans and rank == 0:
         line["tans"] = run_tans_compare(args, dev, stream, xs, sizes, 1e3 * mean_launch_ms, n)
+        line["tans2"] = run_tans_compare(args, dev, stream, xs, sizes, 1e3 * mean_launch_ms, n, states=2)
     # ---- the smaller configurations, with and without an L2 flush
     if not args.no_config_table and rank == 0:
         line["config_table"] = run_config_table(args, dev, stream)
@@ -534,11 +535,12 @@ def run_oracle_table():
     return res
 
 
-def run_tans_compare(args, dev, stream, xs, huff_sizes, huff_launch_us, n, tensors=4, reps=10):
-    """The tANS exponent coder (4096 states) on the first `tensors` tensors of the workload,
-    with the same chunk size and launch configuration: bits/weight, encode time and decode
-    time per launch (CUDA events, launches back to back into the reused output buffer),
-    next to the Huffman coder's numbers on the same tensors."""
+def run_tans_compare(args, dev, stream, xs, huff_sizes, huff_launch_us, n, tensors=4, reps=10, states=1):
+    """The tANS exponent coder (4096 states; one state per chunk, or with states = 2 two
+    interleaved states) on the first `tensors` tensors of the workload, with the same
+    chunk size and launch configuration: bits/weight, encode time and decode time per
+    launch (CUDA events, launches back to back into the reused output buffer), next to
+    the Huffman coder's numbers on the same tensors."""
     import numpy as np
     import torch
 
@@ -546,7 +548,8 @@ def run_tans_compare(args, dev, stream, xs, huff_sizes, huff_launch_us, n, tenso
 
     T = min(tensors, len(xs))
     K = args.chunk_symbols
-    plan = dfx.dfx_plan(n, chunk_symbols=K, coder=dfx.DFX_CODER_TANS, decode_flags=dfx.DFX_DECODE_EARLY_READ)
+    coder = dfx.DFX_CODER_TANS2 if states == 2 else dfx.DFX_CODER_TANS
+    plan = dfx.dfx_plan(n, chunk_symbols=K, coder=coder, decode_flags=dfx.DFX_DECODE_EARLY_READ)
     try:
         scratch = torch.empty(plan.max_compressed_bytes, dtype=torch.uint8, device=dev)
         ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
@@ -588,14 +591,15 @@ def run_tans_compare(args, dev, stream, xs, huff_sizes, huff_launch_us, n, tenso
         algo = float(sum(sizes)) / T + 2.0 * n
         achieved = algo / (mean_us * 1e-6) / 1e9
         peak, peak_kind = measured_hbm_peak()
-        return {"coder": "tANS, 4096 states", "tensors": T, "chunk_symbols": K,
+        return {"coder": "tANS, 4096 states" + (", two interleaved states per chunk" if states == 2 else ""),
+                "tensors": T, "chunk_symbols": K,
                 "bits_per_weight": 8.0 * sum(sizes) / (n * T),
                 "huffman_bits_per_weight": 8.0 * sum(huff_sizes[:T]) / (n * T),
                 "decode_mean_launch_us": mean_us, "huffman_mean_launch_us": huff_launch_us,
                 "decode_bf16_gbs": 2.0 * n / (mean_us * 1e-6) / 1e9,
                 "decode_algorithmic_gbs": achieved, "decode_frac_of_measured": achieved / peak, "peak_kind": peak_kind,
                 "encode_median_ms_per_tensor": statistics.median(enc_ms), "bit_exact": bool(exact),
-                "kernel": f"k_decode<TansCoder, {K}>",
+                "kernel": f"k_decode<TansCoder<{states}>, {K}>",
                 "note": f"{reps} x {T} launches back to back after 3 x {T} warm-up; the Huffman figures are "
                         "the main measurement's (same shape, K and grid)"}
     finally:

@@ -38,6 +38,12 @@
  *     X, and X becomes M + the slot of state X >> nb) and stored as the final state
  *     minus M (table_log bits) followed by the fields in symbol order (a chunk of the
  *     last group with no element has no bits);
+ *   - or (coder 2, DFX_CODER_TANS2) the same tANS code with two interleaved states
+ *     per chunk: the symbols at even positions of a chunk are coded by state A, those
+ *     at odd positions by state B, each as above from state M on its own, and the
+ *     chunk is stored as A's final state minus M, B's final state minus M, then every
+ *     symbol's field in symbol order (a decoder's two table lookups per symbol pair
+ *     are independent; a chunk costs table_log bits more);
  *   - the m bytes are stored raw, in element order;
  *   - the exponent codes are cut into chunks of K codes, 32 chunks to a group:
  *     a group covers 32*K consecutive elements in 8-element blocks, block b of
@@ -118,13 +124,14 @@ typedef struct dfx_plan_s *dfx_plan_t; /* opaque, host-owned */
 /* Exponent coders. */
 #define DFX_CODER_HUFFMAN 0u /* canonical length-limited Huffman (the default) */
 #define DFX_CODER_TANS 1u    /* tabled asymmetric numeral systems */
+#define DFX_CODER_TANS2 2u   /* tANS with two interleaved states per chunk */
 
 typedef struct {
     uint32_t chunk_symbols; /* K: a multiple of 8; 32, 64 or 128 on the GPU path (0 -> 128) */
     uint32_t group_chunks;  /* G: 32 on the GPU path (0 -> 32) */
     uint32_t max_len;       /* coder 0: code-length limit, 8..24 (0 -> 24) */
-    uint32_t coder;         /* DFX_CODER_HUFFMAN or DFX_CODER_TANS */
-    uint32_t table_log;     /* coder 1: log2 of the state table, 4..12 (0 -> 12); dfx_encode
+    uint32_t coder;         /* DFX_CODER_HUFFMAN, DFX_CODER_TANS or DFX_CODER_TANS2 */
+    uint32_t table_log;     /* coders 1, 2: log2 of the state table, 4..12 (0 -> 12); dfx_encode
                                needs 8..12 (room for all 256 exponent values), every value
                                decodes */
     uint32_t decode_flags;  /* 0 or DFX_DECODE_EARLY_READ */

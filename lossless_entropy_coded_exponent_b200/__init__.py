@@ -31,6 +31,7 @@ DFX_STATUS_TIMEOUT = 0x10
 DFX_INJECT_SKIP_SLICE_COPY = 0x1
 DFX_CODER_HUFFMAN = 0
 DFX_CODER_TANS = 1
+DFX_CODER_TANS2 = 2  # tANS with two interleaved states per chunk
 DFX_DECODE_EARLY_READ = 0x1
 
 # The exported C symbols, in include/dfx.h order.

@@ -38,7 +38,7 @@ struct Params {
 };
 
 // Defaults and checks of dfx_params.  Only the fields of the chosen coder are checked:
-// max_len for coder 0, table_log for coder 1.
+// max_len for coder 0, table_log for coders 1 and 2.
 int resolve_params(const dfx_params* p, Params* r) {
     r->K = (p && p->chunk_symbols) ? p->chunk_symbols : 128u;
     r->G = (p && p->group_chunks) ? p->group_chunks : 32u;
@@ -52,9 +52,10 @@ int resolve_params(const dfx_params* p, Params* r) {
         if (r->L < 8 || r->L > dfx::kMaxLenLimit) return DFX_ERR_ARG;
         if ((uint64_t)r->K * r->L > 65535u) return DFX_ERR_ARG;  // a chunk's bit length must fit u16
         r->R = 0;
-    } else if (r->coder == DFX_CODER_TANS) {
+    } else if (dfx::is_tans(r->coder)) {
         if (r->R < dfx::kTansMinLog || r->R > dfx::kTansMaxLog) return DFX_ERR_ARG;
-        if ((uint64_t)(r->K + 1) * r->R > 65535u) return DFX_ERR_ARG;  // fields and state fit u16
+        // fields and states fit u16
+        if ((uint64_t)(r->K + dfx::tans_states(r->coder)) * r->R > 65535u) return DFX_ERR_ARG;
         r->L = 0;
     } else {
         return DFX_ERR_ARG;
@@ -63,9 +64,9 @@ int resolve_params(const dfx_params* p, Params* r) {
 }
 
 // Longest stream a coder may produce: at most 8 bits per exponent for an optimal prefix
-// code, at most table_log bits per exponent and per chunk for tANS.
+// code, at most table_log bits per exponent and per chunk state for tANS.
 uint64_t max_stream_bits(const Params& q, uint64_t n, uint64_t n_chunk) {
-    return q.coder == DFX_CODER_TANS ? (uint64_t)q.R * (n + n_chunk) : 8 * n;
+    return dfx::is_tans(q.coder) ? (uint64_t)q.R * (n + dfx::tans_states(q.coder) * n_chunk) : 8 * n;
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -117,7 +118,7 @@ int dfx_container_layout(uint64_t n, const dfx_params* params, uint64_t total_bi
     out->n = n;
     out->n_chunk = lay.n_chunk;
     out->n_group = lay.n_group;
-    out->off_len = q.coder == DFX_CODER_TANS ? dfx::kOffFreq : dfx::kOffLen;
+    out->off_len = dfx::is_tans(q.coder) ? dfx::kOffFreq : dfx::kOffLen;
     out->off_gbase = lay.off_gbase;
     out->off_clen = lay.off_clen;
     out->off_m = lay.off_m;
@@ -178,7 +179,7 @@ int dfx_encode(dfx_plan_t plan, const void* d_bf16, void* d_out, size_t out_capa
     if (!aligned16(d_bf16) || !aligned16(d_out) || !aligned16(d_workspace)) return DFX_ERR_ARG;
     if (out_capacity < plan->max_bytes || workspace_bytes < plan->ws_bytes) return DFX_ERR_CAPACITY;
     // all 256 exponent values must fit a tANS table
-    if (plan->coder == DFX_CODER_TANS && plan->table_log < 8) return DFX_ERR_UNSUPPORTED;
+    if (dfx::is_tans(plan->coder) && plan->table_log < 8) return DFX_ERR_UNSUPPORTED;
     int rc = check_device(plan);
     if (rc) return rc;
     dfx::EncodeArgs a;

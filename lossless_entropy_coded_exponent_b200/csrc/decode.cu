@@ -82,15 +82,15 @@ cudaError_t launch_decode_batch_huffman(const BatchArgs& b, uint32_t K, cudaStre
 }
 
 int decode_blocks_per_sm(uint32_t K, uint32_t coder) {
-    return coder == DFX_CODER_TANS ? decode_blocks_per_sm_tans(K) : decode_blocks_per_sm_huffman(K);
+    return is_tans(coder) ? decode_blocks_per_sm_tans(K, tans_states(coder)) : decode_blocks_per_sm_huffman(K);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, uint32_t coder, int grid, cudaStream_t s) {
-    return coder == DFX_CODER_TANS ? launch_decode_tans(a, grid, s) : launch_decode_huffman(a, grid, s);
+    return is_tans(coder) ? launch_decode_tans(a, tans_states(coder), grid, s) : launch_decode_huffman(a, grid, s);
 }
 
 cudaError_t launch_decode_batch(const BatchArgs& b, uint32_t K, uint32_t coder, cudaStream_t s) {
-    return coder == DFX_CODER_TANS ? launch_decode_batch_tans(b, K, s) : launch_decode_batch_huffman(b, K, s);
+    return is_tans(coder) ? launch_decode_batch_tans(b, K, tans_states(coder), s) : launch_decode_batch_huffman(b, K, s);
 }
 
 }  // namespace dfx

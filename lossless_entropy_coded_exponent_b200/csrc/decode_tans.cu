@@ -1,5 +1,6 @@
-// decode_tans.cu -- the DFX1 decode kernel for sm_100a with the tANS exponent coder
-// (coder 1): compressed container -> BF16 in HBM.
+// decode_tans.cu -- the DFX1 decode kernels for sm_100a with the tANS exponent coder,
+// one state per chunk (coder 1) or two interleaved states (coder 2): compressed container
+// -> BF16 in HBM.
 //
 // The memory pipeline and group loop are those of the Huffman decoder
 // (decode_pipeline.cuh); this file holds what is particular to tabled asymmetric numeral
@@ -16,6 +17,9 @@
 //     amount from the entry's low 5 bits) and one add, with no per-symbol branch;
 //   * a lane's state is kept as 4 x (its table index), the byte offset of its next
 //     entry; its first R bits are the chunk's start state and the chunk ends in state 0;
+//     with two states (coder 2) the chunk starts with state A's R bits, then B's, A
+//     decodes the even positions and B the odd ones, so the two table loads of a symbol
+//     pair do not wait on each other and only the field extraction stays in order;
 //   * two symbols per peek reload (a field is at most R <= 12 bits), merged with their m
 //     bytes by two byte permutes and one rotate into two BF16.
 #include <cuda_runtime.h>
@@ -38,9 +42,10 @@ struct TansTables {
 };
 
 
-// Checks the header and loads the frequency table and its prefix sums into T.  Every
-// thread of the block calls it; false means the container was rejected and its status
-// bits are set.
+// Checks the header (coder 1 or 2, as `states` says) and loads the frequency table and
+// its prefix sums into T.  Every thread of the block calls it; false means the container
+// was rejected and its status bits are set.
+template <uint32_t States>
 __device__ bool tans_prepare(const DecodeArgs& a, TansTables& T) {
     const int t = threadIdx.x;
     const unsigned warp = t >> 5, lane = t & 31;
@@ -63,9 +68,9 @@ __device__ bool tans_prepare(const DecodeArgs& a, TansTables& T) {
         if (n != a.n || *reinterpret_cast<const uint32_t*>(h + 32) != a.K || *reinterpret_cast<const uint32_t*>(h + 36) != a.G ||
             *reinterpret_cast<const uint32_t*>(h + 40) != a.n_chunk || *reinterpret_cast<const uint32_t*>(h + 44) != a.n_group ||
             *reinterpret_cast<const unsigned long long*>(h + 48) != a.off_m ||
-            *reinterpret_cast<const uint32_t*>(h + 60) != DFX_CODER_TANS)
+            *reinterpret_cast<const uint32_t*>(h + 60) != (States == 2 ? DFX_CODER_TANS2 : DFX_CODER_TANS))
             bad = DFX_STATUS_HEADER;
-        if (R < kTansMinLog || R > kTansMaxLog || total_bits > (unsigned long long)R * (a.n + a.n_chunk))
+        if (R < kTansMinLog || R > kTansMaxLog || total_bits > (unsigned long long)R * (a.n + States * a.n_chunk))
             bad = DFX_STATUS_HEADER;
         if (total_bytes != a.off_stream + stream_bytes(total_bits) || total_bytes > a.comp_bytes) bad = DFX_STATUS_HEADER;
         // the group index must start at bit 0 and end at total_bits
@@ -119,13 +124,14 @@ __device__ void tans_build(const TansTables& T, uint32_t* table, uint8_t* scratc
 // The bit position p, the 32-bit peek and the two cached words are kept as in the
 // Huffman reader; reloads come once per two symbols (at most 2R <= 24 bits), so p moves
 // at most one word between them.
-template <class Words>
+template <class Words, uint32_t States>
 struct TansReader {
     const uint8_t* tbl;  // decoding table (shared memory)
     Words words;
     uint32_t p, p0, peek;
     uint32_t cw, cur, nxt;  // cur = word cw, nxt = word cw + 1
-    uint32_t x4;            // the state times 4: byte offset of its table entry
+    uint32_t x4[States];    // the states times 4: byte offsets of their table entries
+    uint32_t next;          // the state of the next single symbol (the tail's one())
 
     __device__ __forceinline__ void reload() {
         const uint32_t wi = p >> 5;
@@ -144,47 +150,61 @@ struct TansReader {
         cur = words.load(cw);
         nxt = words.load(cw + 1);
         reload();
-        x4 = (peek >> (32 - R)) << 2;  // the chunk's first R bits: its start state
-        p += R;
+        // the chunk's first R bits per state: the start states (2R <= 24 bits of the peek)
+#pragma unroll
+        for (uint32_t s = 0; s < States; s++) x4[s] = ((peek << (s * R)) >> (32 - R)) << 2;
+        p += States * R;
+        next = 0;
     }
-    // One decoding step: the entry of the current state; the state becomes base + the
-    // next nb bits.  The caller advances p.
-    __device__ __forceinline__ uint32_t step() {
-        const uint32_t e = *reinterpret_cast<const uint32_t*>(tbl + x4);
+    // One decoding step of state x: its entry; the state becomes base + the next nb bits.
+    // The caller advances p.
+    __device__ __forceinline__ uint32_t step(uint32_t& x) {
+        const uint32_t e = *reinterpret_cast<const uint32_t*>(tbl + x);
         const uint32_t v = __funnelshift_l(peek, 0u, e);  // peek >> (32 - nb); 0 when nb = 0
         peek = __funnelshift_l(0u, peek, e);               // peek << nb
-        x4 = (e >> 16) + (v << 2);
+        x = (e >> 16) + (v << 2);
         return e;
     }
     // Two symbols (peek current), merged with their m bytes (bytes 2j and 2j+1 of mw).
+    // With two states the pair's first symbol is A's and its second B's.
     template <int j>
     __device__ __forceinline__ uint32_t pair(uint32_t mw) {
         constexpr uint32_t sel = j == 0 ? 0x5140u : 0x5342u;  // [mw.2j, sym0, mw.2j+1, sym1]
-        const uint32_t e0 = step();
-        const uint32_t e1 = step();
+        const uint32_t e0 = step(x4[0]);
+        const uint32_t e1 = step(x4[States - 1]);
         p += (e0 + e1) & 63u;  // nb0 + nb1 (each below 32, in the entries' low bits)
         return bf16_pair(__byte_perm(mw, __byte_perm(e0, e1, 0x0051u), sel));
     }
     // One symbol (peek current); reloads after it.
     __device__ __forceinline__ uint32_t one() {
-        const uint32_t e = step();
+        uint32_t e;
+        if (States == 2 && next) e = step(x4[States - 1]);
+        else e = step(x4[0]);
+        next ^= States - 1;
         p += e & 31u;
         reload();
         return (e >> 8) & 0xFFu;
     }
-    __device__ __forceinline__ bool done(uint32_t clen) const { return p - p0 == clen && x4 == 0; }
+    __device__ __forceinline__ bool done(uint32_t clen) const {
+        bool zero = true;
+#pragma unroll
+        for (uint32_t s = 0; s < States; s++) zero = zero && x4[s] == 0;
+        return p - p0 == clen && zero;
+    }
 };
 
+template <uint32_t States>
 struct TansCoder {
     using Tables = TansTables;
     template <class Words>
-    using Reader = TansReader<Words>;
+    using Reader = TansReader<Words, States>;
     static constexpr uint32_t kGbaseOffset = kOffGbaseTans;
     static constexpr size_t kTableBytes = 4u * kTansSlotsMax;
     static constexpr size_t kScratchBytes = (kTansScratchBytes + 15) & ~size_t(15);
-    // fields of at most 12 bits and a 12-bit state: a chunk spans at most 3K/8 + 2 words
-    __host__ __device__ static constexpr uint32_t chunk_words(uint32_t K) { return (3u * K) / 8u + 2u; }
-    __device__ static bool prepare(const DecodeArgs& a, Tables& T) { return tans_prepare(a, T); }
+    // fields of at most 12 bits and 12-bit states: a chunk spans at most 3K/8 + 2 words
+    // (3K/8 + 3 with two states)
+    __host__ __device__ static constexpr uint32_t chunk_words(uint32_t K) { return (3u * K) / 8u + 1u + States; }
+    __device__ static bool prepare(const DecodeArgs& a, Tables& T) { return tans_prepare<States>(a, T); }
     __device__ static void build(const Tables& T, uint32_t* table, uint8_t* scratch) { tans_build(T, table, scratch); }
     template <class Words>
     __device__ static void init(Reader<Words>& br, const Tables& T, const uint32_t* table, const Words& w, uint32_t start) {
@@ -215,22 +235,24 @@ struct TansCoder {
     }
 };
 
-static_assert(dyn_smem_bytes<TansCoder, 64>() + sizeof(TansTables) + 1024 <= 227 * 1024 &&
-                  dyn_smem_bytes<TansCoder, 128>() + sizeof(TansTables) + 1024 <= 227 * 1024,
+static_assert(dyn_smem_bytes<TansCoder<2>, 64>() + sizeof(TansTables) + 1024 <= 227 * 1024 &&
+                  dyn_smem_bytes<TansCoder<2>, 128>() + sizeof(TansTables) + 1024 <= 227 * 1024,
               "shared memory");
 static_assert(DecodeShape<128>::kThreads == 1024 && DecodeShape<128>::kWarps <= 32,
               "the state-number rounds hold one slot per thread and one count per warp");
 
 }  // namespace
 
-int decode_blocks_per_sm_tans(uint32_t K) { return blocks_per_sm_coder<TansCoder>(K); }
-
-cudaError_t launch_decode_tans(const DecodeArgs& a, int grid, cudaStream_t s) {
-    return launch_coder<TansCoder>(a, grid, s);
+int decode_blocks_per_sm_tans(uint32_t K, uint32_t states) {
+    return states == 2 ? blocks_per_sm_coder<TansCoder<2>>(K) : blocks_per_sm_coder<TansCoder<1>>(K);
 }
 
-cudaError_t launch_decode_batch_tans(const BatchArgs& b, uint32_t K, cudaStream_t s) {
-    return launch_batch_coder<TansCoder>(b, K, s);
+cudaError_t launch_decode_tans(const DecodeArgs& a, uint32_t states, int grid, cudaStream_t s) {
+    return states == 2 ? launch_coder<TansCoder<2>>(a, grid, s) : launch_coder<TansCoder<1>>(a, grid, s);
+}
+
+cudaError_t launch_decode_batch_tans(const BatchArgs& b, uint32_t K, uint32_t states, cudaStream_t s) {
+    return states == 2 ? launch_batch_coder<TansCoder<2>>(b, K, s) : launch_batch_coder<TansCoder<1>>(b, K, s);
 }
 
 }  // namespace dfx

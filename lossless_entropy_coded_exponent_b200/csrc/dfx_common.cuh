@@ -19,7 +19,10 @@ constexpr uint32_t kTansMinLog = 4, kTansMaxLog = 12;  // tANS table sizes 2^4 .
 constexpr uint32_t kWarp = 32;
 constexpr unsigned kFull = 0xffffffffu;  // all lanes of a warp
 
-__host__ __device__ inline uint32_t gbase_offset(uint32_t coder) { return coder == DFX_CODER_TANS ? kOffGbaseTans : kOffGbase; }
+// coders 1 and 2 are the tANS code with one or two states per chunk: same container layout
+__host__ __device__ constexpr bool is_tans(uint32_t coder) { return coder == DFX_CODER_TANS || coder == DFX_CODER_TANS2; }
+__host__ __device__ constexpr uint32_t tans_states(uint32_t coder) { return coder == DFX_CODER_TANS2 ? 2u : 1u; }
+__host__ __device__ inline uint32_t gbase_offset(uint32_t coder) { return is_tans(coder) ? kOffGbaseTans : kOffGbase; }
 
 __host__ __device__ constexpr uint64_t align16(uint64_t x) { return (x + 15u) & ~uint64_t(15); }
 
@@ -112,7 +115,7 @@ __host__ __device__ constexpr uint64_t ws_edge_offset(uint64_t n_group) { return
 constexpr uint64_t kWsTansWords = 2 * 256 + (1u << kTansMaxLog);
 inline uint64_t ws_tans_offset(uint64_t n_group) { return (kWsGroupBits + 4 * n_group + 255) & ~uint64_t(255); }
 inline uint64_t workspace_bytes_for(uint64_t n_group, uint32_t coder = DFX_CODER_HUFFMAN) {
-    return coder == DFX_CODER_TANS ? ws_tans_offset(n_group) + 4 * kWsTansWords
+    return is_tans(coder) ? ws_tans_offset(n_group) + 4 * kWsTansWords
                                    : ws_edge_offset(n_group) + 8 * (n_group + 1);
 }
 
@@ -128,9 +131,9 @@ bool decode_supports(uint32_t K, uint32_t G);
 cudaError_t launch_decode_huffman(const DecodeArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_decode_batch_huffman(const BatchArgs& b, uint32_t K, cudaStream_t s);
 int decode_blocks_per_sm_huffman(uint32_t K);
-cudaError_t launch_decode_tans(const DecodeArgs& a, int grid, cudaStream_t s);
-cudaError_t launch_decode_batch_tans(const BatchArgs& b, uint32_t K, cudaStream_t s);
-int decode_blocks_per_sm_tans(uint32_t K);
+cudaError_t launch_decode_tans(const DecodeArgs& a, uint32_t states, int grid, cudaStream_t s);
+cudaError_t launch_decode_batch_tans(const BatchArgs& b, uint32_t K, uint32_t states, cudaStream_t s);
+int decode_blocks_per_sm_tans(uint32_t K, uint32_t states);
 // Y = X W^T from W's container (decode_gemm.cu): at most kGemmMaxTokens tokens, at most
 // kGemmMaxRows rows of W per CTA
 constexpr uint32_t kGemmMaxTokens = 32;

@@ -848,7 +848,7 @@ cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t 
     // the index region (header .. clen padding) starts at zero; so does everything after the
     // m plane, except that the Huffman pack writes every stream word and zeroes the bytes past
     // the stream itself
-    const bool packs = a.coder != DFX_CODER_TANS && a.n_group > 0;
+    const bool packs = !is_tans(a.coder) && a.n_group > 0;
     if ((err = cudaMemsetAsync(a.out, 0, a.off_m, s)) != cudaSuccess) return err;
     const uint64_t zero_end = packs ? a.off_stream : max_bytes;
     if (zero_end > a.off_m + a.n &&
@@ -878,7 +878,7 @@ cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t 
         k_histogram<<<hist_blocks, kHistWarps * 32, kHistSmem, s>>>(a.in, a.n, a.ws_counts, a.status);
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if (a.coder == DFX_CODER_TANS) {  // the tANS passes around the same group scan
+    if (is_tans(a.coder)) {  // the tANS passes around the same group scan
         if ((err = launch_encode_tans(a, 0, s)) != cudaSuccess) return err;
         k_group_scan<<<1, kScanThreads, 0, s>>>(a);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;

@@ -49,7 +49,7 @@ extern "C" int dfx_encode_static(const void* d_bf16, uint64_t n, const dfx_param
     const uint32_t G = (params && params->group_chunks) ? params->group_chunks : 32u;
     const uint32_t L = (params && params->max_len) ? params->max_len : 24u;
     if (L < 8 || L > dfx::kMaxLenLimit || K < 8 || K % 8 != 0) return DFX_ERR_ARG;
-    if (params && params->coder == DFX_CODER_TANS) return DFX_ERR_UNSUPPORTED;
+    if (params && dfx::is_tans(params->coder)) return DFX_ERR_UNSUPPORTED;
     if (params && params->coder != DFX_CODER_HUFFMAN) return DFX_ERR_ARG;
     if (!dfx::decode_supports(K, G)) return DFX_ERR_UNSUPPORTED;
     if (!d_out || (!d_bf16 && n)) return DFX_ERR_ARG;

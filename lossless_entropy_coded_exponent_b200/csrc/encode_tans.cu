@@ -1,4 +1,6 @@
-// encode_tans.cu -- GPU encoder passes of the tANS exponent coder (coder 1), sm_100a.
+// encode_tans.cu -- GPU encoder passes of the tANS exponent coder, one state per chunk
+// (coder 1) or two interleaved states (coder 2: even positions on state A, odd on B),
+// sm_100a.
 //
 // After the exponent histogram (encode.cu), on the caller's stream:
 //   phase 0  k_tans_tables      one CTA: the frequencies (counts * M / n rounded half up,
@@ -13,7 +15,8 @@
 //   phase 1  k_tans_pack        per group (one warp): every lane runs its chunk's encoder
 //                               again and writes the fields backward from the chunk's end,
 //                               the last one emitted (the chunk's first symbol) right after
-//                               the final state, which goes first; the mantissa+sign bytes.
+//                               the final state(s), which go first (A's, then B's); the
+//                               mantissa+sign bytes.
 // The encoding step for symbol s in state X (M <= X < 2M): nb = the bits with
 // f <= X >> nb < 2f, which for h = floor(log2 f) is R - h, one less when X < f << (R - h);
 // emit the low nb bits of X; X becomes M + the slot of s numbered X >> nb.  The rules are
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(kTablesThreads) k_tans_tables(EncodeArgs a) {
         *reinterpret_cast<uint32_t*>(h + 44) = a.n_group;
         *reinterpret_cast<unsigned long long*>(h + 48) = a.off_m;
         *reinterpret_cast<uint32_t*>(h + 56) = R;
-        *reinterpret_cast<uint32_t*>(h + 60) = DFX_CODER_TANS;
+        *reinterpret_cast<uint32_t*>(h + 60) = a.coder;
     }
 }
 
@@ -153,14 +156,15 @@ __device__ __forceinline__ uint32_t enc_step(const EncTables& E, uint32_t X, uin
 }
 
 // Runs the encoder over chunk `lane` of group g from its last element to its first,
-// starting in state M; put(v, nb) receives the fields in that order.  With WriteM the
-// chunk's mantissa+sign bytes are written too.  Returns the final state (M when the
-// chunk is empty, which has no bits).
-template <int K, bool WriteM, class Put>
-__device__ __forceinline__ uint32_t encode_chunk(const EncodeArgs& a, const EncTables& E, uint64_t g, unsigned lane,
-                                                 Put& put) {
+// starting in state M (each state, with two: the element at chunk position i on state
+// i mod 2); put(v, nb) receives the fields in that order.  With WriteM the chunk's
+// mantissa+sign bytes are written too.  Returns the final states (M when the chunk is
+// empty, which has no bits).
+template <int K, uint32_t States, bool WriteM, class Put>
+__device__ __forceinline__ uint2 encode_chunk(const EncodeArgs& a, const EncTables& E, uint64_t g, unsigned lane,
+                                              Put& put) {
     const uint32_t M = 1u << a.table_log;
-    uint32_t X = M;
+    uint32_t X[2] = {M, M};
     uint8_t* mpl = a.out + a.off_m;
     // the chunk's whole blocks (a prefix of its K/8 blocks) and a partial one after them
     uint32_t full = K / 8;
@@ -172,7 +176,8 @@ __device__ __forceinline__ uint32_t encode_chunk(const EncodeArgs& a, const EncT
         const uint64_t x0 = block_element(g, K, full, lane);
         for (uint64_t x = a.n; x-- > x0;) {  // nothing when x0 >= n
             const uint32_t h = a.in[x];
-            X = enc_step(E, X, (h >> 7) & 0xFFu, put);
+            uint32_t& Xs = X[States == 2 ? (uint32_t)(x - x0) & 1u : 0u];  // blocks before hold 8 k elements
+            Xs = enc_step(E, Xs, (h >> 7) & 0xFFu, put);
             if (WriteM) {
                 const uint32_t partner = a.in[(x ^ 1u) < a.n ? (x ^ 1u) : x];
                 mpl[x] = (uint8_t)(((h & 0x7Fu) << 1) | (partner >> 15));
@@ -188,7 +193,8 @@ __device__ __forceinline__ uint32_t encode_chunk(const EncodeArgs& a, const EncT
 #pragma unroll
         for (int j = 7; j >= 0; j--) {
             const uint32_t h = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-            X = enc_step(E, X, (h >> 7) & 0xFFu, put);
+            uint32_t& Xs = X[States == 2 ? (uint32_t)j & 1u : 0u];
+            Xs = enc_step(E, Xs, (h >> 7) & 0xFFu, put);
         }
         if (WriteM) {
             uint32_t mb[2] = {0u, 0u};
@@ -201,7 +207,7 @@ __device__ __forceinline__ uint32_t encode_chunk(const EncodeArgs& a, const EncT
             *reinterpret_cast<uint2*>(mpl + block_element(g, K, k, lane)) = make_uint2(mb[0], mb[1]);
         }
     }
-    return X;
+    return make_uint2(X[0], X[1]);
 }
 
 // ---------------------------------------------------------------- chunk bit lengths
@@ -213,7 +219,7 @@ struct CountBits {
     __device__ __forceinline__ void operator()(uint32_t, uint32_t nb) { bits += nb; }
 };
 
-template <int K>
+template <int K, uint32_t States>
 __global__ void __launch_bounds__(kTansChunkThreads) k_tans_chunk_bits(EncodeArgs a) {
     __shared__ EncTables E;
     load_enc_tables(a, E);
@@ -223,9 +229,9 @@ __global__ void __launch_bounds__(kTansChunkThreads) k_tans_chunk_bits(EncodeArg
     if (c < a.n_chunk) {
         const uint64_t g = c / 32;
         CountBits cb{0u};
-        encode_chunk<K, false>(a, E, g, lane, cb);
+        encode_chunk<K, States, false>(a, E, g, lane, cb);
         const bool empty = block_element(g, K, 0, lane) >= a.n;
-        bits = empty ? 0u : cb.bits + a.table_log;
+        bits = empty ? 0u : cb.bits + States * a.table_log;
         reinterpret_cast<uint16_t*>(a.out + a.off_clen)[c] = (uint16_t)bits;
     }
     const uint32_t incl = warp_incl_scan_u32(bits, lane);
@@ -267,7 +273,7 @@ struct BackWriter {
     }
 };
 
-template <int K>
+template <int K, uint32_t States>
 __global__ void __launch_bounds__(kTansPackThreads) k_tans_pack(EncodeArgs a) {
     __shared__ EncTables E;
     __shared__ uint32_t slice[kTansPackThreads / 32][kTansPackSliceWords];
@@ -294,8 +300,10 @@ __global__ void __launch_bounds__(kTansPackThreads) k_tans_pack(EncodeArgs a) {
     if (cl) {  // a chunk with elements (an empty one has no bits and no m bytes)
         BackWriter bw{staged ? sm : stream, staged ? wf : 0ull, (end - 1) >> 5, 0ull, 0u};
         bw.r = (uint32_t)(end - 32ull * bw.wi);
-        const uint32_t X = encode_chunk<K, true>(a, E, g, lane, bw);
-        bw(X - (1u << a.table_log), a.table_log);  // the state: the chunk's first bits
+        const uint2 X = encode_chunk<K, States, true>(a, E, g, lane, bw);
+        // the states: the chunk's first bits, A's before B's
+        if (States == 2) bw(X.y - (1u << a.table_log), a.table_log);
+        bw(X.x - (1u << a.table_log), a.table_log);
         bw.finish();
     }
     if (staged) {
@@ -311,6 +319,26 @@ __global__ void __launch_bounds__(kTansPackThreads) k_tans_pack(EncodeArgs a) {
     }
 }
 
+template <uint32_t States>
+cudaError_t launch_tans_passes(const EncodeArgs& a, int phase, unsigned blocks, cudaStream_t s) {
+    if (phase == 0) {
+        switch (a.K) {
+            case 32: k_tans_chunk_bits<32, States><<<blocks, kTansChunkThreads, 0, s>>>(a); break;
+            case 64: k_tans_chunk_bits<64, States><<<blocks, kTansChunkThreads, 0, s>>>(a); break;
+            case 128: k_tans_chunk_bits<128, States><<<blocks, kTansChunkThreads, 0, s>>>(a); break;
+            default: return cudaErrorInvalidValue;
+        }
+    } else {
+        switch (a.K) {
+            case 32: k_tans_pack<32, States><<<blocks, kTansPackThreads, 0, s>>>(a); break;
+            case 64: k_tans_pack<64, States><<<blocks, kTansPackThreads, 0, s>>>(a); break;
+            case 128: k_tans_pack<128, States><<<blocks, kTansPackThreads, 0, s>>>(a); break;
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_encode_tans(const EncodeArgs& a, int phase, cudaStream_t s) {
@@ -320,21 +348,9 @@ cudaError_t launch_encode_tans(const EncodeArgs& a, int phase, cudaStream_t s) {
         k_tans_tables<<<1, kTablesThreads, 0, s>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess || a.n_chunk == 0) return e;
-        switch (a.K) {
-            case 32: k_tans_chunk_bits<32><<<blocks, kTansChunkThreads, 0, s>>>(a); break;
-            case 64: k_tans_chunk_bits<64><<<blocks, kTansChunkThreads, 0, s>>>(a); break;
-            case 128: k_tans_chunk_bits<128><<<blocks, kTansChunkThreads, 0, s>>>(a); break;
-            default: return cudaErrorInvalidValue;
-        }
-    } else {
-        switch (a.K) {
-            case 32: k_tans_pack<32><<<blocks, kTansPackThreads, 0, s>>>(a); break;
-            case 64: k_tans_pack<64><<<blocks, kTansPackThreads, 0, s>>>(a); break;
-            case 128: k_tans_pack<128><<<blocks, kTansPackThreads, 0, s>>>(a); break;
-            default: return cudaErrorInvalidValue;
-        }
     }
-    return cudaGetLastError();
+    return tans_states(a.coder) == 2 ? launch_tans_passes<2>(a, phase, blocks, s)
+                                     : launch_tans_passes<1>(a, phase, blocks, s);
 }
 
 }  // namespace dfx

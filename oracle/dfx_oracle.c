@@ -531,11 +531,11 @@ int dfxo_decode(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n_cap, u
  * and the group start bits at offset 576; the chunks, groups and blocks are
  * those of coder 0.                                                      */
 
-static int tans_params_ok(uint64_t n, uint32_t K, uint32_t G, uint32_t R) {
+static int tans_params_ok(uint64_t n, uint32_t K, uint32_t G, uint32_t R, uint32_t ways) {
     if (n >= ((uint64_t)1 << 32)) return 0;
     if (R < 4 || R > 12) return 0;
     if (K < 8 || K % 8 != 0 || G < 1) return 0;
-    if ((uint64_t)(K + 1) * R > 65535u) return 0; /* a chunk length must fit in u16 */
+    if ((uint64_t)(K + ways) * R > 65535u) return 0; /* a chunk length must fit in u16 */
     return 1;
 }
 
@@ -692,7 +692,7 @@ static uint32_t chunk_symbols(const uint16_t *w, uint64_t n, uint64_t g, uint32_
 
 static int encode_tans_ways(const uint16_t *w, uint64_t n, uint32_t K, uint32_t G, uint32_t R, uint32_t ways,
                             uint8_t *out, uint64_t cap, uint64_t *out_bytes) {
-    if (!tans_params_ok(n, K, G, R)) return DFXO_ERR_ARG;
+    if (!tans_params_ok(n, K, G, R, ways)) return DFXO_ERR_ARG;
     const uint32_t coder = ways == 2 ? DFXO_CODER_TANS2 : DFXO_CODER_TANS;
     const uint32_t M = 1u << R;
     uint64_t counts[256];
@@ -794,7 +794,7 @@ static int decode_tans(const uint8_t *c, uint64_t bytes, uint16_t *w, uint64_t n
     const uint32_t coder = get_u32(c + 60), ways = coder == DFXO_CODER_TANS2 ? 2u : 1u;
     uint64_t n = get_u64(c + 8), total_bits = get_u64(c + 16), total = get_u64(c + 24);
     uint32_t K = get_u32(c + 32), G = get_u32(c + 36), R = get_u32(c + 56);
-    if (!tans_params_ok(n, K, G, R)) return DFXO_ERR_CORRUPT;
+    if (!tans_params_ok(n, K, G, R, ways)) return DFXO_ERR_CORRUPT;
     uint64_t ng = n_groups(n, K, G), nc = ng * G;
     if (get_u32(c + 40) != nc || get_u32(c + 44) != ng) return DFXO_ERR_CORRUPT;
     if (get_u64(c + 48) != off_m_of(nc, ng, coder)) return DFXO_ERR_CORRUPT;

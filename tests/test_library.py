@@ -145,7 +145,12 @@ def test_tans_argument_errors_precede_cuda(lib):
             dfx.dfx_plan(1000, coder=dfx.DFX_CODER_TANS, **kw)
         assert e.value.code == dfx.DFX_ERR_ARG, kw
     with pytest.raises(dfx.DfxError) as e:
-        dfx.dfx_plan(1000, coder=2)
+        dfx.dfx_plan(1000, coder=3)
+    assert e.value.code == dfx.DFX_ERR_ARG
+    # a chunk's length (fields and states) must fit u16: one state more with coder 2
+    dfx.dfx_container_layout(10, 0, chunk_symbols=6552, coder=dfx.DFX_CODER_TANS, table_log=10)  # 6553 x 10
+    with pytest.raises(dfx.DfxError) as e:
+        dfx.dfx_container_layout(10, 0, chunk_symbols=6552, coder=dfx.DFX_CODER_TANS2, table_log=10)  # 6554 x 10
     assert e.value.code == dfx.DFX_ERR_ARG
     # the tANS coder ignores max_len, the Huffman coder table_log
     with pytest.raises(dfx.DfxError) as e:
@@ -153,9 +158,10 @@ def test_tans_argument_errors_precede_cuda(lib):
     assert e.value.code == dfx.DFX_ERR_ARG
     dfx.dfx_container_layout(10, 0, chunk_symbols=4000, max_len=99, coder=dfx.DFX_CODER_TANS)
     dfx.dfx_container_layout(10, 0, table_log=99)
-    with pytest.raises(dfx.DfxError) as e:
-        dfx.dfx_encode_static(None, 10, None, 0, coder=dfx.DFX_CODER_TANS)
-    assert e.value.code == dfx.DFX_ERR_UNSUPPORTED
+    for coder in (dfx.DFX_CODER_TANS, dfx.DFX_CODER_TANS2):
+        with pytest.raises(dfx.DfxError) as e:
+            dfx.dfx_encode_static(None, 10, None, 0, coder=coder)
+        assert e.value.code == dfx.DFX_ERR_UNSUPPORTED
 
 
 def header_struct_fields(name):
