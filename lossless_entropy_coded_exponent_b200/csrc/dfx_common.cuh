@@ -84,7 +84,7 @@ struct EncodeArgs {
     unsigned long long* ws_counts;  // [256]
     uint32_t* ws_code;              // [256]
     uint8_t* ws_len;                // [256]
-    uint32_t* ws_group_bits;        // [n_group]
+    uint32_t* ws_group_bits;        // coder 0: [n_group] u64 look-back words; tANS: [n_group] u32 group sums
     unsigned long long* ws_edge;    // coder 0: [n_group + 1] arrivals and bits at each group boundary
     uint32_t* ws_tans;              // coder 1: [kWsTansWords] encode tables
     uint32_t* status;
@@ -109,7 +109,7 @@ constexpr uint64_t kWsGroupBits = 4096;
 // coder 0: per group boundary b = 0 .. n_group (the start of group b), the bits that groups
 // b - 1 and b put in the stream word the boundary falls in (low half) and how many of the
 // two have done so (high half)
-__host__ __device__ constexpr uint64_t ws_edge_offset(uint64_t n_group) { return align16(kWsGroupBits + 4 * n_group); }
+__host__ __device__ constexpr uint64_t ws_edge_offset(uint64_t n_group) { return align16(kWsGroupBits + 8 * n_group); }
 // coder 1: per symbol (threshold << 16 | nb_hi, cs << 16 | f) and the slot of every
 // (symbol, state number) pair, after the group sums
 constexpr uint64_t kWsTansWords = 2 * 256 + (1u << kTansMaxLog);

@@ -60,9 +60,11 @@ __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long lon
 // shared histogram and picks the 16 consecutive exponents [b, b + 16) with the most of
 // that sample.  From then on a lane counts the values in that window in registers:
 // 4-bit counters, eight per 32-bit word (value b + d adds 1 << 4d to the first word for
-// d < 8 and 1 << 4(d - 8) to the second for 8 <= d < 16; a shift by 32 or more gives 0,
-// so a value lands in at most one word, and one three-input add takes the two values of
-// a 32-bit input word).  After every unit (at most 8 per counter) the nibbles are spread
+// d < 8 and 1 << 4(d - 8) to the second for 8 <= d < 16).  The two values of a 32-bit
+// input word take one subtraction for both window offsets and one shared-memory load of
+// the increments of the pair (a 17 x 17 table, offset 16 standing for "outside"), which
+// keeps the integer pipe, the kernel's bound, free of the shifts.  After every unit (at
+// most 8 per counter) the nibbles are spread
 // into 8-bit counters, after kHistFold chunks those into 16-bit counters, and these into
 // the shared histogram at the end.  Values outside the window are rare: the warp checks
 // once per unit whether any lane met one, and only then takes shared-memory atomics.
@@ -77,13 +79,6 @@ struct HistWarpBuffers {
     unsigned long long bar[kHistBufs];
 };
 constexpr size_t kHistSmem = kHistWarps * sizeof(HistWarpBuffers);
-
-// 1 << s, 0 for s >= 32 (the PTX shift clamps its amount)
-__device__ __forceinline__ uint32_t shl_clamped(uint32_t s) {
-    uint32_t r;
-    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(1u), "r"(s));
-    return r;
-}
 
 // Spread two words of 4-bit counters (values b .. b + 15) into four words of 8-bit counters:
 // c8[0] takes values b + {0, 2, 4, 6}, c8[1] b + {1, 3, 5, 7}, c8[2] and c8[3] the same for
@@ -115,6 +110,7 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
                                                                   uint32_t* status) {
     __shared__ uint32_t h[256];
     __shared__ uint32_t window;
+    __shared__ uint2 pair_add[17 * 17];  // (d0, d1) -> the two counter words' increments
     extern __shared__ __align__(16) uint8_t hist_smem[];
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     HistWarpBuffers& wb = reinterpret_cast<HistWarpBuffers*>(hist_smem)[warp];
@@ -176,8 +172,22 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
         }
         if (threadIdx.x == 0) window = best_b;
     }
+    // one value at window offset d < 16 adds 1 << 4d to counter word 0 (d < 8) or
+    // 1 << 4 (d - 8) to word 1; offset 16 stands for any value outside the window
+    for (uint32_t i = threadIdx.x; i < 17 * 17; i += blockDim.x) {
+        uint2 v = make_uint2(0u, 0u);
+        for (uint32_t d : {i / 17, i % 17}) {
+            if (d < 8) v.x += 1u << (4 * d);
+            else if (d < 16) v.y += 1u << (4 * (d - 8));
+        }
+        pair_add[i] = v;
+    }
     __syncthreads();
-    const uint32_t b = window, b4 = 4u * window, b4h = 4u * window + 32u;
+    const uint32_t b = window;
+    // subtracting b from both exponent fields of a 32-bit word: bit 15 (the low value's
+    // sign, set first) takes the low field's borrow, so each field becomes (e - b) mod 256,
+    // which is 16 or more for every e outside [b, b + 16) since b <= 240
+    const uint32_t bb = (b << 7) | (b << 23);
     uint32_t n0 = 0u, n1 = 0u, c8[4] = {0u, 0u, 0u, 0u}, c16[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     uint32_t since = 0, folds = 0;
     for (uint32_t k = 1; k < nc; k++) {
@@ -200,15 +210,16 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
                 uint32_t outside = 0;
 #pragma unroll
                 for (int q = 0; q < 4; q++) {
-                    // 4 e of the word's two values (exponent bits 7-14 and 23-30)
-                    const uint32_t e0 = (w[q] >> 5) & 0x3FCu, e1 = (w[q] >> 21) & 0x3FCu;
-                    const uint32_t s0 = e0 - b4, s1 = e1 - b4;
-                    n0 += shl_clamped(s0) + shl_clamped(s1);
-                    n1 += shl_clamped(e0 - b4h) + shl_clamped(e1 - b4h);
-                    outside |= s0 | s1;
+                    // the word's two window offsets, 16 for a value outside the window
+                    const uint32_t y = (w[q] | 0x8000u) - bb;
+                    const uint32_t d0 = min((y >> 7) & 0xFFu, 16u), d1 = min((y >> 23) & 0xFFu, 16u);
+                    const uint2 t = pair_add[17u * d0 + d1];
+                    n0 += t.x;
+                    n1 += t.y;
+                    outside |= d0 | d1;
                 }
                 fold_nibbles(n0, n1, c8);
-                if (__any_sync(kFull, outside >= 64u) && outside >= 64u) {
+                if (__any_sync(kFull, outside >= 16u) && outside >= 16u) {
 #pragma unroll
                     for (int q = 0; q < 8; q++) {
                         const uint32_t e = (w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu;
@@ -598,10 +609,10 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
 // 64-bit word (kept in shared memory with its length), writes the block's sign+mantissa
 // bytes and adds the length to its chunk's count.  It finds the group's start bit by a
 // decoupled look-back over the group words of the workspace.  A group publishes its bit
-// count as soon as it is known (flag kGroupCount) and, once it has its own start, writes
-// the next group's gbase entry (its inclusive end) and then sets kGroupEnd; a warp adds
-// up its predecessors' counts, 32 at a time, back to the nearest group whose end is
-// published.  Then it puts its blocks' joined codes into the warp's shared copy of its
+// count as soon as it is known (flag kGroupCount) and, once it has its own start, its
+// inclusive end (flag kGroupEnd), each as one 64-bit word written by an atomic exchange; a
+// warp adds up its predecessors' counts, 32 at a time, back to the nearest group whose end
+// is published.  Then it puts its blocks' joined codes into the warp's shared copy of its
 // words, one or two puts per block, and writes the words out.  A block whose codes do
 // not fit 64 bits (or a pair of them 32) is looked up again, code by code, at the put;
 // the last, partial group and a group whose words do not fit the shared copy are packed
@@ -621,22 +632,18 @@ template <int K>
 constexpr size_t pack_smem_bytes() {
     return kFusedWarps * sizeof(PackWarp<K>);
 }
-constexpr uint32_t kGroupCount = 1u << 30;  // the group's bit count (bits 0-29) is published
-constexpr uint32_t kGroupEnd = 1u << 31;    // and its end bit is in gbase[g + 1]
+// A group's look-back word (u64, in the workspace): kGroupCount with its bit count, then
+// kGroupEnd | kGroupCount with its inclusive end bit.  Each is written whole by one atomic
+// exchange and read whole, so no other memory access needs ordering around it.
+constexpr unsigned long long kGroupCount = 1ull << 62;
+constexpr unsigned long long kGroupEnd = 1ull << 63;
+constexpr unsigned long long kGroupValue = kGroupCount - 1;
 constexpr uint32_t kLookbackPolls = 1u << 20;
 
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 __device__ __forceinline__ unsigned long long ld_relaxed64(const unsigned long long* p) {
     unsigned long long v;
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
-}
-__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ uint32_t ld_volatile(const uint32_t* p) { return *reinterpret_cast<const volatile uint32_t*>(p); }
@@ -650,18 +657,17 @@ __device__ __forceinline__ void boundary_word(const EncodeArgs& a, uint32_t b, u
 }
 
 // The exclusive start bit of group g: predecessors' published counts back to the nearest
-// published end.  Every wait is bounded (a flag that never comes sets DFX_STATUS_TIMEOUT
+// published end.  Every wait is bounded (a word that never comes sets DFX_STATUS_TIMEOUT
 // and counts as 0).
 __device__ uint64_t lookback(const EncodeArgs& a, uint32_t g, unsigned lane, uint32_t& err) {
-    const uint32_t* gw = a.ws_group_bits;
-    const unsigned long long* gbase = reinterpret_cast<const unsigned long long*>(a.out + kOffGbase);
+    const unsigned long long* gw = reinterpret_cast<const unsigned long long*>(a.ws_group_bits);
     uint64_t excl = 0;
     int64_t pos = (int64_t)g - 1;
     while (pos >= 0) {
         const int64_t i = pos - (int64_t)lane;
-        uint32_t v = kGroupCount | kGroupEnd;  // before group 0: an end at bit 0
+        unsigned long long v = kGroupCount | kGroupEnd;  // before group 0: an end at bit 0
         for (uint32_t it = 0;; it++) {
-            if (i >= 0) v = ld_acquire(gw + i);
+            if (i >= 0) v = ld_relaxed64(gw + i);
             if (__all_sync(kFull, (v & kGroupCount) != 0)) break;
             if (it == kLookbackPolls) {
                 err |= DFX_STATUS_TIMEOUT;
@@ -671,14 +677,10 @@ __device__ uint64_t lookback(const EncodeArgs& a, uint32_t g, unsigned lane, uin
             __nanosleep(32);
         }
         const uint32_t ends = __ballot_sync(kFull, (v & kGroupEnd) != 0);
-        uint64_t c = 0;
-        if (ends) {
-            const unsigned first = __ffs(ends) - 1;  // the nearest predecessor with its end published
-            if (lane < first) c = v & (kGroupCount - 1);
-            if (lane == first && i >= 0) c = ld_relaxed64(gbase + i + 1);  // ordered after the flag's acquire
-        } else {
-            c = v & (kGroupCount - 1);
-        }
+        // the nearest predecessor with its end published gives that end, the ones after it
+        // their counts
+        const unsigned first = ends ? __ffs(ends) - 1 : 32u;
+        uint64_t c = lane <= first ? (v & kGroupValue) : 0ull;
 #pragma unroll
         for (int d = 16; d >= 1; d >>= 1) c += __shfl_xor_sync(kFull, c, d);
         excl += c;
@@ -761,12 +763,13 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
     const uint32_t group_bits = __shfl_sync(kFull, incl, 31);
 
     // the group's start bit
-    if (lane == 0) st_release(a.ws_group_bits + g, kGroupCount | group_bits);
+    unsigned long long* gw = reinterpret_cast<unsigned long long*>(a.ws_group_bits);
+    if (lane == 0) atomicExch(gw + g, kGroupCount | group_bits);
     const uint64_t gb0 = lookback(a, g, lane, err);
     if (lane == 0) {
         unsigned long long* gbase = reinterpret_cast<unsigned long long*>(a.out + kOffGbase);
         gbase[g + 1] = gb0 + group_bits;
-        st_release(a.ws_group_bits + g, kGroupEnd | kGroupCount | group_bits);
+        atomicExch(gw + g, kGroupEnd | kGroupCount | (gb0 + group_bits));
         if (g + 1 == a.n_group) {
             *reinterpret_cast<unsigned long long*>(a.out + 16) = gb0 + group_bits;
             *reinterpret_cast<unsigned long long*>(a.out + 24) = a.off_stream + stream_bytes(gb0 + group_bits);
