@@ -41,6 +41,25 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, unsigned lane) {
     return v;
 }
 
+// Programmatic dependent launch within the encode: the code book and the pack are launched
+// while the kernel before them runs and wait for its completion (and memory) here.
+__device__ __forceinline__ void wait_for_previous_kernel() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void allow_next_kernel() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+template <class Kern, class... Args>
+cudaError_t launch_dependent(Kern* kernel, unsigned grid, unsigned threads, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long long v, unsigned lane) {
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -112,6 +131,7 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
     __shared__ uint32_t window;
     __shared__ uint2 pair_add[17 * 17];  // (d0, d1) -> the two counter words' increments
     extern __shared__ __align__(16) uint8_t hist_smem[];
+    allow_next_kernel();  // the code book may be scheduled; it waits for this kernel to end
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     HistWarpBuffers& wb = reinterpret_cast<HistWarpBuffers*>(hist_smem)[warp];
     for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0;
@@ -287,6 +307,8 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     __shared__ uint32_t nlen[kMaxLenLimit + 1];
     __shared__ uint32_t firstc[kMaxLenLimit + 1];
 
+    allow_next_kernel();
+    wait_for_previous_kernel();  // the histogram's counts
     const int t = threadIdx.x;
     const int L = (int)a.max_len;
     const unsigned long long c = a.ws_counts[t];
@@ -695,6 +717,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
     __shared__ uint32_t cl_sh[256];  // code << 8 | length
     __shared__ uint32_t cta_ticket;
     extern __shared__ __align__(16) uint8_t pack_smem[];
+    wait_for_previous_kernel();  // the code book
     cl_sh[threadIdx.x] = (a.ws_code[threadIdx.x] << 8) | a.ws_len[threadIdx.x];
     if (threadIdx.x == 0) cta_ticket = atomicAdd(reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTicket), 1u);
     __syncthreads();
@@ -840,8 +863,7 @@ cudaError_t launch_pack(const EncodeArgs& a, unsigned ctas, int dev, cudaStream_
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    k_pack_fused<K><<<ctas, kFusedWarps * 32, pack_smem_bytes<K>(), s>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(k_pack_fused<K>, ctas, kFusedWarps * 32, pack_smem_bytes<K>(), s, a);
 }
 
 }  // namespace
@@ -887,8 +909,7 @@ cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t 
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         return launch_encode_tans(a, 1, s);
     }
-    k_build_codebook<<<1, 256, 0, s>>>(a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if ((err = launch_dependent(k_build_codebook, 1, 256, 0, s, a)) != cudaSuccess) return err;
     if (a.n_group == 0) {  // an empty tensor: the group scan writes the header totals
         k_group_scan<<<1, kScanThreads, 0, s>>>(a);
         return cudaGetLastError();
