@@ -295,6 +295,24 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
 // last list, q_j = number of leaves in the selected prefix of list j, and the
 // length of the leaf of sorted rank i is the number of lists with i < q_j.
 
+// The number of the first n (<= 256) entries of the ascending array v that are below w
+// (or, with Le, not above it), in two dependent rounds of shared loads instead of a binary
+// search's eight: 16 block ends first, then the 16 entries of the one block that straddles w.
+template <bool Le>
+__device__ __forceinline__ int count_sorted(const unsigned long long* v, int n, unsigned long long w) {
+    auto in = [&](unsigned long long x) { return Le ? x <= w : x < w; };
+    int blocks = 0;  // whole 16-entry blocks below w (their last entry is)
+#pragma unroll
+    for (int i = 0; i < 16; i++) blocks += (16 * i + 15 < n && in(v[16 * i + 15])) ? 1 : 0;
+    int r = 16 * blocks;
+#pragma unroll
+    for (int k = 0; k < 16; k++) {
+        const int i = 16 * blocks + k;
+        r += (i < n && in(v[i])) ? 1 : 0;
+    }
+    return r;
+}
+
 __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     __shared__ unsigned long long cnt[256];
     __shared__ unsigned long long leafw[256];
@@ -306,6 +324,7 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     __shared__ uint8_t lens[256];
     __shared__ uint32_t nlen[kMaxLenLimit + 1];
     __shared__ uint32_t firstc[kMaxLenLimit + 1];
+    __shared__ uint8_t wlen[8][kMaxLenLimit + 1];  // symbols of each length per 32-symbol slice
 
     allow_next_kernel();
     wait_for_previous_kernel();  // the histogram's counts
@@ -315,6 +334,7 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     cnt[t] = c;
     lens[t] = 0;
     if (t <= (int)kMaxLenLimit) nlen[t] = 0;
+    if (t < 8 * (int)(kMaxLenLimit + 1)) (&wlen[0][0])[t] = 0;
     const bool used = c > 0;
     const int m = __syncthreads_count(used);
 
@@ -327,6 +347,7 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     } else if (m >= 2) {
         if (used) {
             int r = 0;
+#pragma unroll 16
             for (int s = 0; s < 256; s++) {
                 const unsigned long long cs = cnt[s];
                 r += (cs > 0) && (cs < c || (cs == c && s < t));
@@ -346,41 +367,30 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
             __syncthreads();
             if (t < m) {
                 const unsigned long long w = leafw[t];
-                int lo = 0, hi = np;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (pkw[mid] < w) lo = mid + 1;
-                    else hi = mid;
-                }
+                const int lo = count_sorted<false>(pkw, np, w);  // packages lighter than the leaf
                 cur[t + lo] = w;
                 leafpos[j][t] = (uint16_t)(t + lo);
             }
             if (t < np) {
                 const unsigned long long w = pkw[t];
-                int lo = 0, hi = m;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (leafw[mid] <= w) lo = mid + 1;
-                    else hi = mid;
-                }
-                cur[t + lo] = w;
+                cur[t + count_sorted<true>(leafw, m, w)] = w;  // after the leaves not heavier
             }
             size = m + np;
             __syncthreads();
         }
-        if (t == 0) {
+        if (t < 32) {  // one warp: the leaves among the first s items of each list, last list first
             int s = 2 * m - 2;
             for (int j = L - 1; j >= 1; j--) {
-                int lo = 0, hi = m;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (leafpos[j][mid] < s) lo = mid + 1;
-                    else hi = mid;
+                int lo = 0;
+#pragma unroll
+                for (int k = 0; k < 8; k++) {
+                    const int i = t + 32 * k;
+                    lo += __popc(__ballot_sync(kFull, i < m && leafpos[j][i] < s));
                 }
-                qsel[j] = lo;
+                if (t == 0) qsel[j] = lo;
                 s = 2 * (s - lo);
             }
-            qsel[0] = s;
+            if (t == 0) qsel[0] = s;
         }
         __syncthreads();
         if (t < m) {
@@ -394,6 +404,11 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     // canonical codes: first code per length, then rank among equal lengths by symbol
     const uint32_t l = lens[t];
     if (l) atomicAdd(&nlen[l], 1u);
+    // rank of the symbol among those of its length: lower lanes of its warp now, the
+    // counts of lower warps after the barrier
+    const unsigned lane = t & 31, warp = t >> 5;
+    const unsigned peers = __match_any_sync(kFull, l), below = peers & ((1u << lane) - 1u);
+    if (l && below == 0) wlen[warp][l] = (uint8_t)__popc(peers);
     __syncthreads();
     if (t == 0) {
         uint32_t code = 0;
@@ -405,8 +420,8 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     __syncthreads();
     uint32_t code = 0;
     if (l) {
-        uint32_t r = 0;
-        for (int s = 0; s < t; s++) r += (lens[s] == l);
+        uint32_t r = __popc(below);
+        for (unsigned w = 0; w < warp; w++) r += wlen[w][l];
         code = firstc[l] + r;
     }
     a.ws_code[t] = code;
