@@ -763,6 +763,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
     uint32_t bits = 0;
     if (!ragged) {
         uint8_t* mpl = a.out + a.off_m;
+        if (lane == 0) prefetch_l2(a.in + (uint64_t)g * 32u * K, 64u * K);  // the whole group, while its first blocks load
 #pragma unroll 4
         for (uint32_t k = 0; k < NB; k++) {
             const uint64_t x0 = block_element(g, K, k, lane);
