@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
     if (blockIdx.x == 0 && threadIdx.x < (n & 7)) atomicAdd(&h[(in[units * 8 + threadIdx.x] >> 7) & 0xFFu], 1u);
     if (err) atomicOr(status, err);
     __syncthreads();
+    wait_for_previous_kernel();  // the counts are zeroed by the kernel before this one
     for (int k = threadIdx.x; k < 256; k += blockDim.x)
         if (h[k]) atomicAdd(&counts[k], (unsigned long long)h[k]);
 }
@@ -870,6 +871,24 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
     if (err) atomicOr(a.status, err);
 }
 
+// The zeroing a Huffman encode needs before its passes: the container's index region
+// [0, off_m) and the padding [off_m + n, off_stream), the workspace's histogram counts
+// [0, 2048) and [kWsTicket, ws_end) (the pack's ticket, look-back and boundary words).
+// Every region but the padding is a whole number of 8-byte words.
+__global__ void __launch_bounds__(256) k_zero_regions(EncodeArgs a, uint64_t ws_end) {
+    allow_next_kernel();  // the histogram waits for this kernel only before its final counts
+    const uint64_t w_out = a.off_m / 8, w_cnt = 2048 / 8, w_ws = (ws_end - kWsTicket) / 8;
+    unsigned long long* out = reinterpret_cast<unsigned long long*>(a.out);
+    unsigned long long* ws = reinterpret_cast<unsigned long long*>(a.ws_counts);
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < w_out + w_cnt + w_ws; i += stride) {
+        if (i < w_out) out[i] = 0ull;
+        else if (i < w_out + w_cnt) ws[i - w_out] = 0ull;
+        else ws[kWsTicket / 8 + (i - w_out - w_cnt)] = 0ull;
+    }
+    if (blockIdx.x == 0 && a.off_m + a.n + threadIdx.x < a.off_stream) a.out[a.off_m + a.n + threadIdx.x] = 0;
+}
+
 template <int K>
 cudaError_t launch_pack(const EncodeArgs& a, unsigned ctas, int dev, cudaStream_t s) {
     static bool attr_set[64] = {};
@@ -890,16 +909,21 @@ cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t 
     // m plane, except that the Huffman pack writes every stream word and zeroes the bytes past
     // the stream itself
     const bool packs = !is_tans(a.coder) && a.n_group > 0;
-    if ((err = cudaMemsetAsync(a.out, 0, a.off_m, s)) != cudaSuccess) return err;
-    const uint64_t zero_end = packs ? a.off_stream : max_bytes;
-    if (zero_end > a.off_m + a.n &&
-        (err = cudaMemsetAsync(a.out + a.off_m + a.n, 0, zero_end - (a.off_m + a.n), s)) != cudaSuccess)
-        return err;
-    if ((err = cudaMemsetAsync(a.ws_counts, 0, 256 * sizeof(unsigned long long), s)) != cudaSuccess) return err;
-    // the fused pass's CTA ticket, group words and boundary words start at zero
-    if (packs && (err = cudaMemsetAsync(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTicket, 0,
-                                        ws_edge_offset(a.n_group) + 8 * (a.n_group + 1) - kWsTicket, s)) != cudaSuccess)
-        return err;
+    if (packs) {
+        // one kernel: the index region, the m plane's padding, the histogram counts and the
+        // pack's ticket, look-back and boundary words
+        const uint64_t ws_end = ws_edge_offset(a.n_group) + 8 * (a.n_group + 1);
+        const uint64_t words = (a.off_m + 2048 + ws_end - kWsTicket) / 8;
+        const unsigned blocks = (unsigned)((words + 4095) / 4096 < 148 ? (words + 4095) / 4096 : 148);
+        k_zero_regions<<<blocks, 256, 0, s>>>(a, ws_end);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    } else {
+        if ((err = cudaMemsetAsync(a.out, 0, a.off_m, s)) != cudaSuccess) return err;
+        if (max_bytes > a.off_m + a.n &&
+            (err = cudaMemsetAsync(a.out + a.off_m + a.n, 0, max_bytes - (a.off_m + a.n), s)) != cudaSuccess)
+            return err;
+        if ((err = cudaMemsetAsync(a.ws_counts, 0, 256 * sizeof(unsigned long long), s)) != cudaSuccess) return err;
+    }
 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -916,9 +940,10 @@ cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t 
         const uint64_t chunks = (a.n / 8 + kHistChunkUnits - 1) / kHistChunkUnits;
         const uint64_t ctas = (chunks + kHistWarps - 1) / kHistWarps;
         const unsigned hist_blocks = (unsigned)(ctas == 0 ? 1 : (ctas < (uint64_t)sms ? ctas : (uint64_t)sms));
-        k_histogram<<<hist_blocks, kHistWarps * 32, kHistSmem, s>>>(a.in, a.n, a.ws_counts, a.status);
+        if ((err = launch_dependent(k_histogram, hist_blocks, kHistWarps * 32, kHistSmem, s, a.in, a.n, a.ws_counts,
+                                    a.status)) != cudaSuccess)
+            return err;
     }
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (is_tans(a.coder)) {  // the tANS passes around the same group scan
         if ((err = launch_encode_tans(a, 0, s)) != cudaSuccess) return err;
         k_group_scan<<<1, kScanThreads, 0, s>>>(a);
