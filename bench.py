@@ -388,7 +388,11 @@ def run_ours(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": algo_bytes_per_launch,
-                         "mean_launch_us": 1e3 * mean_launch_ms, "kernel": f"k_decode<HuffmanCoder, {K}>"},
+                         "mean_launch_us": 1e3 * mean_launch_ms, "kernel": f"k_decode<HuffmanCoder, {K}>",
+                         # per-step means: the first steps against the last show the effect of the
+                         # power cap over the timed region
+                         "launch_us_by_step": {"first": 1e3 * launch_ms[0], "last": 1e3 * launch_ms[-1],
+                                               "min": 1e3 * min(launch_ms), "max": 1e3 * max(launch_ms)}},
             "gpu_launches": args.steps * T,
             "clocks": clocks.summary(),
             "encode": {"unit": "GB/s", "value": 2.0 * n / (statistics.median(enc_ms) * 1e-3) / 1e9,
