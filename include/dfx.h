@@ -180,7 +180,8 @@ int dfx_plan(dfx_plan_t *plan, uint64_t n, const dfx_params *params,
  * container at d_out (device, 16-byte aligned, out_capacity >=
  * max_compressed_bytes).  d_workspace: device scratch of workspace_bytes
  * (16-byte aligned), contents on entry ignored.  The bytes of d_out past the
- * container's end, up to max_compressed_bytes, are zeroed.
+ * container's end (up to max_compressed_bytes) are not part of the result: the
+ * Huffman coder leaves them as they were, the tANS coders zero them.
  * h_compressed_bytes: NULL keeps the call asynchronous; otherwise the call
  * synchronises the stream and stores the container size.  The size is also
  * in the header at byte offset 24 (u64). */

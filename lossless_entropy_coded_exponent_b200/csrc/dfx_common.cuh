@@ -88,7 +88,7 @@ struct EncodeArgs {
     unsigned long long* ws_edge;    // coder 0: [n_group + 1] arrivals and bits at each group boundary
     uint32_t* ws_tans;              // coder 1: [kWsTansWords] encode tables
     uint32_t* status;
-    uint64_t max_bytes;             // the container's capacity (bytes past its end are zeroed)
+    uint64_t max_bytes;             // the container's capacity (tANS: zeroed past the m plane)
 };
 
 // Several tensors decoded by one launch: tensor i gets CTAs [cta_begin[i], cta_begin[i+1]).

@@ -16,8 +16,8 @@
 //                       decoupled look-back over the groups before it (gbase, total_bits,
 //                       total_bytes), and the joined codes packed MSB-first into 32-bit
 //                       words; every stream word is written once (the word two groups share
-//                       by the second of them to finish), and the bytes past the container
-//                       are zeroed on the side.
+//                       by the second of them to finish), then the container's zero
+//                       padding; the bytes past the container are not written.
 // The tANS coder shares pass 1 and k_group_scan (a one-CTA scan of per-group sums); its
 // passes 2, 3 and 5 are in encode_tans.cu.
 // The method: frequent exponent values get short codes ("DFloat11: lossless LLM
@@ -80,10 +80,11 @@ __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long lon
 // that sample.  From then on a lane counts the values in that window in registers:
 // 4-bit counters, eight per 32-bit word (value b + d adds 1 << 4d to the first word for
 // d < 8 and 1 << 4(d - 8) to the second for 8 <= d < 16).  The two values of a 32-bit
-// input word take one subtraction for both window offsets and one shared-memory load of
-// the increments of the pair (a 17 x 17 table, offset 16 standing for "outside"), which
-// keeps the integer pipe, the kernel's bound, free of the shifts.  After every unit (at
-// most 8 per counter) the nibbles are spread
+// input word take one shared-memory load of the increments of the pair (a 17 x 17 table,
+// offset 16 standing for "outside") instead of shifts.  The loop is bound by the integer
+// (ALU) pipe, so its field extractions are multiplications by powers of two, which run on
+// the FMA pipe: x * 2^k is x << k and the high word of x * 2^(32 - k) is x >> k.  After
+// every unit (at most 8 per counter) the nibbles are spread
 // into 8-bit counters, after kHistFold chunks those into 16-bit counters, and these into
 // the shared histogram at the end.  Values outside the window are rare: the warp checks
 // once per unit whether any lane met one, and only then takes shared-memory atomics.
@@ -102,11 +103,12 @@ constexpr size_t kHistSmem = kHistWarps * sizeof(HistWarpBuffers);
 // Spread two words of 4-bit counters (values b .. b + 15) into four words of 8-bit counters:
 // c8[0] takes values b + {0, 2, 4, 6}, c8[1] b + {1, 3, 5, 7}, c8[2] and c8[3] the same for
 // b + 8 ..
-__device__ __forceinline__ void fold_nibbles(uint32_t& n0, uint32_t& n1, uint32_t (&c8)[4]) {
+// x16 = 2^28: the high nibbles move down by the high word of a multiplication.
+__device__ __forceinline__ void fold_nibbles(uint32_t& n0, uint32_t& n1, uint32_t (&c8)[4], uint32_t x16) {
     c8[0] += n0 & 0x0F0F0F0Fu;
-    c8[1] += (n0 >> 4) & 0x0F0F0F0Fu;
+    c8[1] = __umulhi(n0 & 0xF0F0F0F0u, x16) + c8[1];
     c8[2] += n1 & 0x0F0F0F0Fu;
-    c8[3] += (n1 >> 4) & 0x0F0F0F0Fu;
+    c8[3] = __umulhi(n1 & 0xF0F0F0F0u, x16) + c8[3];
     n0 = n1 = 0u;
 }
 // Spread the 8-bit counters into 16-bit ones: c16[2 w + h] holds byte h and byte h + 2 of
@@ -129,6 +131,7 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
                                                                   uint32_t* status) {
     __shared__ uint32_t h[256];
     __shared__ uint32_t window;
+    __shared__ uint32_t pow2[4];         // 2^17, 2, 2^8, 2^28, read back so they stay multiplications
     __shared__ uint2 pair_add[17 * 17];  // (d0, d1) -> the two counter words' increments
     extern __shared__ __align__(16) uint8_t hist_smem[];
     allow_next_kernel();  // the code book may be scheduled; it waits for this kernel to end
@@ -202,12 +205,20 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
         }
         pair_add[i] = v;
     }
+    if (threadIdx.x == 0) {
+        pow2[0] = 1u << 17;
+        pow2[1] = 2u;
+        pow2[2] = 1u << 8;
+        pow2[3] = 1u << 28;
+    }
     __syncthreads();
     const uint32_t b = window;
-    // subtracting b from both exponent fields of a 32-bit word: bit 15 (the low value's
-    // sign, set first) takes the low field's borrow, so each field becomes (e - b) mod 256,
-    // which is 16 or more for every e outside [b, b + 16) since b <= 240
-    const uint32_t bb = (b << 7) | (b << 23);
+    // a word's two window offsets (e - b) mod 256, which is 16 or more for every e outside
+    // [b, b + 16) since b <= 240: the low exponent field (bits 7..14) is moved to the top
+    // byte by * 2^17, the high one (bits 23..30) by * 2, b is subtracted from the top byte
+    // alone (cb has no lower bits) and the top byte taken by the high word of * 2^8
+    const uint32_t x17 = pow2[0], x1 = pow2[1], x8 = pow2[2], x28 = pow2[3];
+    const uint32_t cb = 0u - (b << 24);
     uint32_t n0 = 0u, n1 = 0u, c8[4] = {0u, 0u, 0u, 0u}, c16[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     uint32_t since = 0, folds = 0;
     for (uint32_t k = 1; k < nc; k++) {
@@ -230,15 +241,13 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
                 uint32_t outside = 0;
 #pragma unroll
                 for (int q = 0; q < 4; q++) {
-                    // the word's two window offsets, 16 for a value outside the window
-                    const uint32_t y = (w[q] | 0x8000u) - bb;
-                    const uint32_t d0 = min((y >> 7) & 0xFFu, 16u), d1 = min((y >> 23) & 0xFFu, 16u);
-                    const uint2 t = pair_add[17u * d0 + d1];
+                    const uint32_t d0 = __umulhi(w[q] * x17 + cb, x8), d1 = __umulhi(w[q] * x1 + cb, x8);
+                    const uint2 t = pair_add[17u * min(d0, 16u) + min(d1, 16u)];  // 16: outside
                     n0 += t.x;
                     n1 += t.y;
                     outside |= d0 | d1;
                 }
-                fold_nibbles(n0, n1, c8);
+                fold_nibbles(n0, n1, c8, x28);
                 if (__any_sync(kFull, outside >= 16u) && outside >= 16u) {
 #pragma unroll
                     for (int q = 0; q < 8; q++) {
@@ -295,49 +304,70 @@ __global__ void __launch_bounds__(kHistWarps * 32, 1) k_histogram(const uint16_t
 // which expand to the first 2 p_j items of list j-1.  So walking back from the
 // last list, q_j = number of leaves in the selected prefix of list j, and the
 // length of the leaf of sorted rank i is the number of lists with i < q_j.
+//
+// The kernel is one CTA and a chain of short dependent steps, so it is written for
+// latency: the used symbols are compacted first (the sort compares m counts, not 256);
+// a package's weight is summed from list j-1 where it is needed, so a level takes one
+// barrier; with m <= 128 the leaves' ranks and the packages' ranks are computed by
+// different warps; and a rank search probes 8 x 8 entries when the list has at most 64.
 
-// The number of the first n (<= 256) entries of the ascending array v that are below w
-// (or, with Le, not above it), in two dependent rounds of shared loads instead of a binary
-// search's eight: 16 block ends first, then the 16 entries of the one block that straddles w.
-template <bool Le>
-__device__ __forceinline__ int count_sorted(const unsigned long long* v, int n, unsigned long long w) {
+// The number of the first n (<= 256) entries of the ascending sequence v(0), v(1), ...
+// that are below w (or, with Le, not above it), in two dependent rounds of probes instead
+// of a binary search's eight: the last entries of B blocks of B first, then the B entries
+// of the one block that straddles w (B * B >= n).
+template <int B, bool Le, class V>
+__device__ __forceinline__ int count_sorted_in(V v, int n, unsigned long long w) {
     auto in = [&](unsigned long long x) { return Le ? x <= w : x < w; };
-    int blocks = 0;  // whole 16-entry blocks below w (their last entry is)
+    int blocks = 0;  // whole B-entry blocks below w (their last entry is)
 #pragma unroll
-    for (int i = 0; i < 16; i++) blocks += (16 * i + 15 < n && in(v[16 * i + 15])) ? 1 : 0;
-    int r = 16 * blocks;
+    for (int i = 0; i < B; i++) blocks += (B * i + B - 1 < n && in(v(B * i + B - 1))) ? 1 : 0;
+    int r = B * blocks;
 #pragma unroll
-    for (int k = 0; k < 16; k++) {
-        const int i = 16 * blocks + k;
-        r += (i < n && in(v[i])) ? 1 : 0;
+    for (int k = 0; k < B; k++) {
+        const int i = B * blocks + k;
+        r += (i < n && in(v(i))) ? 1 : 0;
     }
     return r;
 }
+template <bool Le, class V>
+__device__ __forceinline__ int count_sorted(V v, int n, unsigned long long w) {
+    return n <= 64 ? count_sorted_in<8, Le>(v, n, w) : count_sorted_in<16, Le>(v, n, w);
+}
 
 __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
-    __shared__ unsigned long long cnt[256];
+    __shared__ unsigned long long ucnt[256];  // the used symbols' counts, in symbol order
     __shared__ unsigned long long leafw[256];
     __shared__ uint8_t leafsym[256];
     __shared__ unsigned long long lw[2][512];
-    __shared__ unsigned long long pkw[256];
     __shared__ uint16_t leafpos[kMaxLenLimit][256];
     __shared__ int qsel[kMaxLenLimit];
     __shared__ uint8_t lens[256];
     __shared__ uint32_t nlen[kMaxLenLimit + 1];
     __shared__ uint32_t firstc[kMaxLenLimit + 1];
     __shared__ uint8_t wlen[8][kMaxLenLimit + 1];  // symbols of each length per 32-symbol slice
+    __shared__ uint32_t wused[8];                  // used symbols per 32-symbol slice
 
     allow_next_kernel();
     wait_for_previous_kernel();  // the histogram's counts
     const int t = threadIdx.x;
+    const unsigned lane = t & 31, warp = t >> 5;
     const int L = (int)a.max_len;
     const unsigned long long c = a.ws_counts[t];
-    cnt[t] = c;
     lens[t] = 0;
     if (t <= (int)kMaxLenLimit) nlen[t] = 0;
     if (t < 8 * (int)(kMaxLenLimit + 1)) (&wlen[0][0])[t] = 0;
     const bool used = c > 0;
-    const int m = __syncthreads_count(used);
+    const unsigned used_bits = __ballot_sync(kFull, used);
+    if (lane == 0) wused[warp] = __popc(used_bits);
+    __syncthreads();
+    int m = 0, idx = __popc(used_bits & ((1u << lane) - 1u));  // idx: the symbol's place among the used
+#pragma unroll
+    for (int w = 0; w < 8; w++) {
+        m += wused[w];
+        idx += (w < (int)warp) ? wused[w] : 0;
+    }
+    if (used) ucnt[idx] = c;
+    __syncthreads();
 
     if (m == 1) {
         // one exponent value: it and a phantom partner both get 1-bit codes
@@ -346,45 +376,44 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
             lens[t == 0 ? 1 : 0] = 1;
         }
     } else if (m >= 2) {
-        if (used) {
+        if (used) {  // the rank by (count, symbol); the used symbols are in symbol order
             int r = 0;
-#pragma unroll 16
-            for (int s = 0; s < 256; s++) {
-                const unsigned long long cs = cnt[s];
-                r += (cs > 0) && (cs < c || (cs == c && s < t));
+#pragma unroll 4
+            for (int k = 0; k < m; k++) {
+                const unsigned long long ck = ucnt[k];
+                r += (ck < c || (ck == c && k < idx)) ? 1 : 0;
             }
             leafw[r] = c;
+            lw[0][r] = c;
             leafsym[r] = (uint8_t)t;
         }
         __syncthreads();
-        if (t < m) lw[0][t] = leafw[t];
+        // leaf t and package pk of each list; pk = t - 128 puts the packages on other warps
+        const int pk = m <= 128 ? t - 128 : t;
+        const unsigned long long leaf = t < m ? leafw[t] : 0ull;
         int size = m;
-        __syncthreads();
         for (int j = 1; j < L; j++) {
             const unsigned long long* prev = lw[(j - 1) & 1];
             unsigned long long* cur = lw[j & 1];
             const int np = size / 2;
-            if (t < np) pkw[t] = prev[2 * t] + prev[2 * t + 1];
-            __syncthreads();
             if (t < m) {
-                const unsigned long long w = leafw[t];
-                const int lo = count_sorted<false>(pkw, np, w);  // packages lighter than the leaf
-                cur[t + lo] = w;
+                const int lo = count_sorted<false>([&](int i) { return prev[2 * i] + prev[2 * i + 1]; }, np, leaf);
+                cur[t + lo] = leaf;  // after the packages lighter than the leaf
                 leafpos[j][t] = (uint16_t)(t + lo);
             }
-            if (t < np) {
-                const unsigned long long w = pkw[t];
-                cur[t + count_sorted<true>(leafw, m, w)] = w;  // after the leaves not heavier
+            if (pk >= 0 && pk < np) {
+                const unsigned long long w = prev[2 * pk] + prev[2 * pk + 1];
+                cur[pk + count_sorted<true>([&](int i) { return leafw[i]; }, m, w)] = w;  // after the leaves not heavier
             }
             size = m + np;
             __syncthreads();
         }
         if (t < 32) {  // one warp: the leaves among the first s items of each list, last list first
             int s = 2 * m - 2;
+            const int slices = (m + 31) / 32;
             for (int j = L - 1; j >= 1; j--) {
                 int lo = 0;
-#pragma unroll
-                for (int k = 0; k < 8; k++) {
+                for (int k = 0; k < slices; k++) {
                     const int i = t + 32 * k;
                     lo += __popc(__ballot_sync(kFull, i < m && leafpos[j][i] < s));
                 }
@@ -407,7 +436,6 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     if (l) atomicAdd(&nlen[l], 1u);
     // rank of the symbol among those of its length: lower lanes of its warp now, the
     // counts of lower warps after the barrier
-    const unsigned lane = t & 31, warp = t >> 5;
     const unsigned peers = __match_any_sync(kFull, l), below = peers & ((1u << lane) - 1u);
     if (l && below == 0) wlen[warp][l] = (uint8_t)__popc(peers);
     __syncthreads();
@@ -643,20 +671,29 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
 // input once.  A CTA of 8 warps takes the next 8 groups from a ticket counter (so the
 // CTAs holding earlier groups are always running and the scan below always makes
 // progress); a warp reads its group (lane i: the 16-byte blocks i, i + 32, ... of the
-// group) and, per block, looks up its 8 codes, joins them two by two and then into one
-// 64-bit word (kept in shared memory with its length), writes the block's sign+mantissa
-// bytes and adds the length to its chunk's count.  It finds the group's start bit by a
-// decoupled look-back over the group words of the workspace.  A group publishes its bit
-// count as soon as it is known (flag kGroupCount) and, once it has its own start, its
-// inclusive end (flag kGroupEnd), each as one 64-bit word written by an atomic exchange; a
-// warp adds up its predecessors' counts, 32 at a time, back to the nearest group whose end
-// is published.  Then it puts its blocks' joined codes into the warp's shared copy of its
-// words, one or two puts per block, and writes the words out.  A block whose codes do
-// not fit 64 bits (or a pair of them 32) is looked up again, code by code, at the put;
-// the last, partial group and a group whose words do not fit the shared copy are packed
-// straight into the stream (pack_chunk).
+// group) and, per block, looks up its 8 codes, joins them two by two, the pairs into two
+// 32-bit halves and those into one 64-bit word (kept in shared memory with its length),
+// writes the block's sign+mantissa bytes and adds the length to its chunk's count.  A
+// group publishes its bit count as soon as it is known (flag kGroupCount) and, once it has
+// its own start, its inclusive end (flag kGroupEnd), each as one 64-bit word written by an
+// atomic exchange.  Before it looks for its own start, a warp puts its blocks' joined
+// codes into the warp's shared copy of its words, counted from the group's bit 0 (one or
+// two puts per block), so that its predecessors' counts have arrived by the time it needs
+// them.  It finds the group's start bit by a decoupled look-back over the group words of
+// the workspace, adding up its predecessors' counts, 32 at a time, back to the nearest
+// group whose end is published; then it writes its words out, each shifted by the start
+// bit mod 32.  A block whose half does not fit 32 bits is looked up again, code by code,
+// at the put; the last, partial group and a group whose words do not fit the shared copy
+// are packed straight into the stream (pack_chunk) after the look-back.
 
 constexpr int kFusedWarps = 8;
+
+// x << n for any n (0 from 32 on, as the PTX shift defines it)
+__device__ __forceinline__ uint32_t shl32(uint32_t x, uint32_t n) {
+    uint32_t r;
+    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));
+    return r;
+}
 constexpr uint32_t kPackSliceWords = 512;  // a group's stream words staged per warp (2 KiB)
 constexpr uint8_t kSlowBlock = 255;        // a block whose codes are not joined (lengths are <= 192)
 
@@ -737,19 +774,13 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
     cl_sh[threadIdx.x] = (a.ws_code[threadIdx.x] << 8) | a.ws_len[threadIdx.x];
     if (threadIdx.x == 0) cta_ticket = atomicAdd(reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTicket), 1u);
     __syncthreads();
-    {
-        // this CTA's share of the bytes past the container (the stream's length is known
-        // from the code book), zeroed while the pack proceeds
+    if (blockIdx.x == 0) {
+        // the container's zero bytes after the last stream word (the stream's length is
+        // known from the code book): up to the 16-byte boundary, then 16 more
         const unsigned long long total =
             *reinterpret_cast<const unsigned long long*>(reinterpret_cast<const uint8_t*>(a.ws_counts) + kWsTotalBits);
-        const uint64_t z0 = a.off_stream + 4 * ((total + 31) / 32), z16 = align16(z0);
-        if (z16 <= a.max_bytes) {
-            if (blockIdx.x == 0 && threadIdx.x < (z16 - z0) / 4) reinterpret_cast<uint32_t*>(a.out + z0)[threadIdx.x] = 0u;
-            const uint64_t units = (a.max_bytes - z16) / 16;
-            uint4* zp = reinterpret_cast<uint4*>(a.out + z16);
-            for (uint64_t u = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units; u += (uint64_t)gridDim.x * blockDim.x)
-                zp[u] = make_uint4(0u, 0u, 0u, 0u);
-        }
+        const uint64_t z0 = a.off_stream + 4 * ((total + 31) / 32), z1 = a.off_stream + stream_bytes(total);
+        if (z1 <= a.max_bytes && threadIdx.x < (z1 - z0) / 4) reinterpret_cast<uint32_t*>(a.out + z0)[threadIdx.x] = 0u;
     }
     const unsigned warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t g = cta_ticket * kFusedWarps + warp;
@@ -780,12 +811,11 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
                 // the m bytes in bytes 0 and 2: each mantissa above the other's sign
                 mw[q] = ((w[q] & 0x007F007Fu) << 1) | (w[q] >> 31) | ((w[q] << 1) & 0x00010000u);
             }
-            const uint32_t L = pl[0] + pl[1] + pl[2] + pl[3];
-            const bool slow = max(max(pl[0], pl[1]), max(pl[2], pl[3])) > 32u || L > 64u;
-            unsigned long long x = p[0];
-            x = (x << pl[1]) | p[1];
-            x = (x << pl[2]) | p[2];
-            x = (x << pl[3]) | p[3];
+            // the pairs joined into two 32-bit halves, then one 64-bit shift
+            const uint32_t la = pl[0] + pl[1], lb = pl[2] + pl[3], L = la + lb;
+            const bool slow = max(la, lb) > 32u;
+            const uint32_t qa = shl32(p[0], pl[1]) | p[1], qb = shl32(p[2], pl[3]) | p[3];  // exact unless slow
+            const unsigned long long x = ((unsigned long long)qa << lb) | qb;
             pw.code[k][lane] = x;
             pw.len[k][lane] = slow ? kSlowBlock : (uint8_t)L;
             bits += L;
@@ -802,35 +832,19 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
     const uint32_t incl = warp_incl_scan(bits, lane);
     const uint32_t group_bits = __shfl_sync(kFull, incl, 31);
 
-    // the group's start bit
+    // publish the group's bit count, then assemble its words from the group's bit 0 while
+    // the predecessors' counts arrive; they are shifted into place once the start bit is known
     unsigned long long* gw = reinterpret_cast<unsigned long long*>(a.ws_group_bits);
     if (lane == 0) atomicExch(gw + g, kGroupCount | group_bits);
-    const uint64_t gb0 = lookback(a, g, lane, err);
-    if (lane == 0) {
-        unsigned long long* gbase = reinterpret_cast<unsigned long long*>(a.out + kOffGbase);
-        gbase[g + 1] = gb0 + group_bits;
-        atomicExch(gw + g, kGroupEnd | kGroupCount | (gb0 + group_bits));
-        if (g + 1 == a.n_group) {
-            *reinterpret_cast<unsigned long long*>(a.out + 16) = gb0 + group_bits;
-            *reinterpret_cast<unsigned long long*>(a.out + 24) = a.off_stream + stream_bytes(gb0 + group_bits);
-        }
-    }
-
-    // pack
-    const uint64_t start = gb0 + (incl - bits);
-    uint32_t* stream = reinterpret_cast<uint32_t*>(a.out + a.off_stream);
-    const uint64_t wf = gb0 >> 5, wl = (gb0 + group_bits + 31) >> 5;  // the group's words [wf, wl)
-    const uint32_t count = (uint32_t)(wl - wf);
-    // a word shared with the previous or the next group (a whole group holds at least 32 K
-    // bits, so only the last group can end in the word it starts in, and it has no next)
-    const bool shared_first = (gb0 & 31u) != 0;
-    const bool shared_last = ((gb0 + group_bits) & 31u) != 0 && g + 1 < a.n_group;
-    if (!ragged && count <= kPackSliceWords) {
-        uint32_t* sm = pw.slice;
-        for (uint32_t i = lane; i < count; i += 32) sm[i] = 0u;
+    uint32_t* sm = pw.slice;
+    const uint32_t staged_words = (group_bits + 31) / 32 + 1;  // the group's words, at any start bit
+    const bool staged = !ragged && staged_words <= kPackSliceWords;
+    if (staged) {
+        for (uint32_t i = lane; i < staged_words; i += 32) sm[i] = 0u;
         __syncwarp();
         // the bits of the previous chunk in the first word count as already placed zeros
-        SliceWriter bw{sm, (uint32_t)((start >> 5) - wf), 0ull, (uint32_t)(start & 31)};
+        const uint32_t rel = incl - bits;  // the chunk's first bit within the group
+        SliceWriter bw{sm, rel >> 5, 0ull, rel & 31u};
         for (uint32_t k = 0; k < NB; k++) {
             const uint32_t L = pw.len[k][lane];
             const unsigned long long x = pw.code[k][lane];
@@ -851,18 +865,45 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
         }
         bw.finish();
         __syncwarp();
+    }
+
+    // the group's start bit
+    const uint64_t gb0 = lookback(a, g, lane, err);
+    if (lane == 0) {
+        unsigned long long* gbase = reinterpret_cast<unsigned long long*>(a.out + kOffGbase);
+        gbase[g + 1] = gb0 + group_bits;
+        atomicExch(gw + g, kGroupEnd | kGroupCount | (gb0 + group_bits));
+        if (g + 1 == a.n_group) {
+            *reinterpret_cast<unsigned long long*>(a.out + 16) = gb0 + group_bits;
+            *reinterpret_cast<unsigned long long*>(a.out + 24) = a.off_stream + stream_bytes(gb0 + group_bits);
+        }
+    }
+
+    // the group's words
+    uint32_t* stream = reinterpret_cast<uint32_t*>(a.out + a.off_stream);
+    const uint64_t wf = gb0 >> 5, wl = (gb0 + group_bits + 31) >> 5;  // the group's words [wf, wl)
+    const uint32_t count = (uint32_t)(wl - wf);
+    // a word shared with the previous or the next group (a whole group holds at least 32 K
+    // bits, so only the last group can end in the word it starts in, and it has no next)
+    const bool shared_first = (gb0 & 31u) != 0;
+    const bool shared_last = ((gb0 + group_bits) & 31u) != 0 && g + 1 < a.n_group;
+    if (staged) {
+        // stream word wf + i holds the group's bits from 32 i - sh on (sh = gb0 mod 32): the
+        // low sh bits of staged word i - 1 above the high 32 - sh bits of staged word i
+        const uint32_t sh = (uint32_t)(gb0 & 31u);
         for (uint32_t i = lane; i < count; i += 32) {
             if ((i == 0 && shared_first) || (i + 1 == count && shared_last)) continue;
-            stream[wf + i] = sm[i];
+            stream[wf + i] = __funnelshift_r(sm[i], i ? sm[i - 1] : 0u, sh);
         }
-        if (lane == 0 && shared_first) boundary_word(a, g, stream + wf, sm[0]);
-        if (lane == 0 && shared_last) boundary_word(a, g + 1, stream + wl - 1, sm[count - 1]);
+        if (lane == 0 && shared_first) boundary_word(a, g, stream + wf, sm[0] >> sh);
+        if (lane == 0 && shared_last)
+            boundary_word(a, g + 1, stream + wl - 1, __funnelshift_r(sm[count - 1], count > 1 ? sm[count - 2] : 0u, sh));
     } else {
         // straight into the stream: the group's words start at zero, the codes are OR-ed in
         for (uint32_t i = lane; i < count; i += 32) stream[wf + i] = 0u;
         __syncwarp();
         __threadfence();
-        pack_chunk<K>(a, cl_sh, c, lane, start, GlobalSink{stream});
+        pack_chunk<K>(a, cl_sh, c, lane, gb0 + (incl - bits), GlobalSink{stream});
         __syncwarp();
         __threadfence();
         if (lane == 0 && shared_first) boundary_word(a, g, stream + wf, ld_volatile(stream + wf));
@@ -906,8 +947,8 @@ cudaError_t launch_pack(const EncodeArgs& a, unsigned ctas, int dev, cudaStream_
 cudaError_t launch_encode(const EncodeArgs& a, uint64_t max_bytes, cudaStream_t s) {
     cudaError_t err;
     // the index region (header .. clen padding) starts at zero; so does everything after the
-    // m plane, except that the Huffman pack writes every stream word and zeroes the bytes past
-    // the stream itself
+    // m plane for the tANS coders (their packs OR codes into the stream), while the Huffman
+    // pack writes every stream word and the container's zero padding itself
     const bool packs = !is_tans(a.coder) && a.n_group > 0;
     if (packs) {
         // one kernel: the index region, the m plane's padding, the histogram counts and the
