@@ -126,12 +126,29 @@ pynvml.nvmlInit()
 bus, index, period = sys.argv[1], int(sys.argv[2]), float(sys.argv[3])
 h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode()) if bus != "-" else pynvml.nvmlDeviceGetHandleByIndex(index)
 mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
-clk, reasons = [], 0
+clk, reasons, side = [], 0, []
+
+
+def probe():  # memory clock, GPU and HBM temperature, board power; None where NVML has no answer
+    out = []
+    for f in (lambda: pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_MEM),
+              lambda: pynvml.nvmlDeviceGetTemperature(h, pynvml.NVML_TEMPERATURE_GPU),
+              lambda: pynvml.nvmlDeviceGetFieldValues(h, [pynvml.NVML_FI_DEV_MEMORY_TEMP])[0].value.uiVal,
+              lambda: pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0):
+        try:
+            out.append(f())
+        except Exception:
+            out.append(None)
+    return out
+
+
 print("ready", flush=True)
 while not select.select([sys.stdin], [], [], period)[0]:
     clk.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
     reasons |= pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-print(json.dumps({"clk": clk, "max": mx, "reasons": reasons}), flush=True)
+    if len(clk) % 5 == 1:
+        side.append(probe())
+print(json.dumps({"clk": clk, "max": mx, "reasons": reasons, "side": side}), flush=True)
 """
 
 
@@ -145,7 +162,7 @@ class ClockSampler:
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
     def __init__(self, device_index: int, period_s: float = 0.01):
-        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.samples, self.reasons, self.max_mhz, self.side = [], set(), None, []
         self.period = period_s
         self.device_index = device_index
         self.error = None
@@ -181,7 +198,7 @@ class ClockSampler:
         try:
             out, _ = self._proc.communicate(input="", timeout=30)  # closes stdin: the child reports and exits
             d = json.loads(out.strip().splitlines()[-1])
-            self.samples, self.max_mhz = d["clk"], d["max"]
+            self.samples, self.max_mhz, self.side = d["clk"], d["max"], d.get("side", [])
             for bit, name in self.REASONS.items():
                 if d["reasons"] & bit:
                     self.reasons.add(name)
@@ -193,8 +210,17 @@ class ClockSampler:
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0,
                     "error": self.error or "no samples"}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        out = {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+               "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        # memory clock (median), GPU and HBM temperature and board power at the first and the
+        # last of the side samples (every fifth clock sample): a memory-bound kernel that slows
+        # down while the SM clock holds points at the memory side
+        for i, key in enumerate(("mem_mhz", "gpu_temp_c", "hbm_temp_c", "power_w")):
+            vals = [r[i] for r in self.side if r[i] is not None]
+            if not vals:
+                continue
+            out[key] = statistics.median(vals) if key == "mem_mhz" else {"first": vals[0], "last": vals[-1]}
+        return out
 
 
 def dist_setup(args):
