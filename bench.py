@@ -152,6 +152,15 @@ print(json.dumps({"clk": clk, "max": mx, "reasons": reasons, "side": side}), flu
 """
 
 
+def tenths(launch_ms):
+    """Mean microseconds per launch in each tenth of the timed steps, in order: how the
+    launch time moves over the run (the 1 kW part lowers its clock under the power cap)."""
+    k = len(launch_ms)
+    if k < 10:
+        return [round(1e3 * v, 1) for v in launch_ms]
+    return [round(1e3 * statistics.mean(launch_ms[k * i // 10:k * (i + 1) // 10]), 1) for i in range(10)]
+
+
 class ClockSampler:
     """Samples SM clock and clock-event reasons while running, through NVML in a child
     interpreter (so the launch loop of this one cannot starve it); stops when its stdin
@@ -418,7 +427,8 @@ def run_ours(args, world, rank, local):
                          # per-step means: the first steps against the last show the effect of the
                          # power cap over the timed region
                          "launch_us_by_step": {"first": 1e3 * launch_ms[0], "last": 1e3 * launch_ms[-1],
-                                               "min": 1e3 * min(launch_ms), "max": 1e3 * max(launch_ms)}},
+                                               "min": 1e3 * min(launch_ms), "max": 1e3 * max(launch_ms),
+                                               "by_tenth": tenths(launch_ms)}},
             "gpu_launches": args.steps * T,
             "clocks": clocks.summary(),
             "encode": {"unit": "GB/s", "value": 2.0 * n / (statistics.median(enc_ms) * 1e-3) / 1e9,
