@@ -156,6 +156,23 @@ def fibonacci_clamp_tensor(seed: int, n_symbols: int = 28, first_exponent: int =
     return ((sign << np.uint16(15)) | (e << np.uint16(7)) | mant).astype(np.uint16)
 
 
+def exponent_spread(n: int, n_values: int, seed: int, first_exponent: int = 40, decay: float = 0.95) -> np.ndarray:
+    """Exactly n_values distinct exponents, first_exponent .. first_exponent + n_values - 1:
+    each once, the other n - n_values drawn with probability proportional to decay^i, so the
+    code lengths spread out.  Sign and mantissa are random.  It sets the number of leaves
+    of the code book's package-merge."""
+    assert n_values <= n and first_exponent + n_values <= 255
+    rng = np.random.default_rng(seed)
+    p = decay ** np.arange(n_values, dtype=np.float64)
+    p /= p.sum()
+    e = np.concatenate([np.arange(n_values), rng.choice(n_values, size=n - n_values, p=p)]).astype(np.uint16)
+    e += np.uint16(first_exponent)
+    rng.shuffle(e)
+    sign = rng.integers(0, 2, size=n, dtype=np.uint16)
+    mant = rng.integers(0, 128, size=n, dtype=np.uint16)
+    return ((sign << np.uint16(15)) | (e << np.uint16(7)) | mant).astype(np.uint16)
+
+
 def edge_cases() -> dict[str, np.ndarray]:
     """The edge-case set: ragged lengths, one-symbol, incompressible, specials."""
     cases = {}

@@ -201,6 +201,19 @@ def test_tensor_helpers_round_trip():
     assert torch.equal(y.view(torch.int16), x.view(torch.int16))
 
 
+@pytest.mark.parametrize("n_values", [2, 33, 64, 65, 100, 128, 129, 200])
+def test_code_book_across_leaf_counts(n_values):
+    """The code book's package-merge changes strategy with the number m of used exponents
+    (probe rounds of 8 x 8 entries for lists of at most 64, 16 x 16 above; leaves and packages
+    ranked on different warps while m <= 128): containers equal the oracle's on both sides of
+    each switch, and decode back exactly."""
+    w = inputs.exponent_spread((1 << 20) + 77, n_values, seed=300 + n_values)
+    c = gpu_encode(w, 128)
+    assert np.array_equal(c, oracle.encode(w, K=128))
+    got, _ = gpu_decode(c, w.size, 128)
+    assert np.array_equal(got, w)
+
+
 HIST_CASES = {
     "small_gaussian": lambda: inputs.small_gaussian(),
     "layer70b_sample": lambda: inputs.layer70b_sample(1 << 22, 3),

@@ -231,6 +231,19 @@ def test_fibonacci_counts_force_the_clamp():
     assert cost == dp_length_limited_cost([int(c) for c in counts], 24)
 
 
+@pytest.mark.parametrize("n_values", [2, 65, 129, 200])
+def test_exponent_spread_sets_the_leaf_count(n_values):
+    """The generator behind the GPU code-book cases: exactly n_values distinct exponents, all
+    of them given a code by the oracle (a complete prefix code), and a lossless round trip."""
+    w = inputs.exponent_spread(20_000, n_values, seed=7)
+    e = ((w >> 7) & 0xFF).astype(np.int64)
+    assert np.unique(e).size == n_values
+    counts = np.bincount(e, minlength=256).astype(np.uint64)
+    lens = oracle.code_lengths(counts, 24)
+    assert int((lens > 0).sum()) == n_values and kraft24(lens) == 1 << 24
+    assert np.array_equal(oracle.decode(oracle.encode(w, K=128)), w)
+
+
 def test_dp_agrees_on_random_limited_cases():
     rng = np.random.default_rng(9)
     for _ in range(10):
