@@ -613,9 +613,9 @@ struct SliceWriter {
 };
 
 // Pack chunk c (lane `lane` of group c / 32), whose codes start at stream bit `start`,
-// and write its elements' mantissa+sign bytes.  cl_sh[e] = code << 8 | length.
+// and write its elements' mantissa+sign bytes.  cl2[e] = (code, length).
 template <int K, class Sink>
-__device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* cl_sh, uint64_t c, unsigned lane,
+__device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint2* cl2, uint64_t c, unsigned lane,
                                            uint64_t start, Sink sink) {
     auto bw = make_writer(sink, start);
     uint8_t* mpl = a.out + a.off_m;
@@ -639,13 +639,12 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
 #pragma unroll
             for (int j = 0; j < 4; j++) {
                 // the pair (2j, 2j + 1): its two codes, as one put when they fit 32 bits
-                const uint32_t c0 = cl_sh[(w[j] >> 7) & 0xFFu], c1 = cl_sh[(w[j] >> 23) & 0xFFu];
-                const uint32_t l0 = c0 & 0xFFu, l1 = c1 & 0xFFu;
-                if (l0 + l1 <= 32u) {
-                    bw.put(((c0 >> 8) << l1) | (c1 >> 8), l0 + l1);
+                const uint2 c0 = cl2[(w[j] >> 7) & 0xFFu], c1 = cl2[(w[j] >> 23) & 0xFFu];
+                if (c0.y + c1.y <= 32u) {
+                    bw.put((c0.x << c1.y) | c1.x, c0.y + c1.y);
                 } else {
-                    bw.put(c0 >> 8, l0);
-                    bw.put(c1 >> 8, l1);
+                    bw.put(c0.x, c0.y);
+                    bw.put(c1.x, c1.y);
                 }
                 // their m bytes in bytes 0 and 2: each mantissa above the other's sign
                 mw[j] = ((w[j] & 0x007F007Fu) << 1) | (w[j] >> 31) | ((w[j] << 1) & 0x00010000u);
@@ -656,7 +655,7 @@ __device__ __forceinline__ void pack_chunk(const EncodeArgs& a, const uint32_t* 
                 const uint32_t h = a.in[x];
                 const uint32_t partner = a.in[(x ^ 1u) < a.n ? (x ^ 1u) : x];
                 const uint32_t e = (h >> 7) & 0xFFu;
-                bw.put(cl_sh[e] >> 8, cl_sh[e] & 0xFFu);
+                bw.put(cl2[e].x, cl2[e].y);
                 mpl[x] = (uint8_t)(((h & 0x7Fu) << 1) | (partner >> 15));
             }
             break;
@@ -767,11 +766,11 @@ __device__ uint64_t lookback(const EncodeArgs& a, uint32_t g, unsigned lane, uin
 
 template <int K>
 __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a) {
-    __shared__ uint32_t cl_sh[256];  // code << 8 | length
+    __shared__ uint2 cl2[256];  // (code, length)
     __shared__ uint32_t cta_ticket;
     extern __shared__ __align__(16) uint8_t pack_smem[];
     wait_for_previous_kernel();  // the code book
-    cl_sh[threadIdx.x] = (a.ws_code[threadIdx.x] << 8) | a.ws_len[threadIdx.x];
+    cl2[threadIdx.x] = make_uint2(a.ws_code[threadIdx.x], a.ws_len[threadIdx.x]);
     if (threadIdx.x == 0) cta_ticket = atomicAdd(reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTicket), 1u);
     __syncthreads();
     if (blockIdx.x == 0) {
@@ -804,12 +803,11 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
             uint32_t p[4], pl[4], mw[4];
 #pragma unroll
             for (int q = 0; q < 4; q++) {
-                const uint32_t c0 = cl_sh[(w[q] >> 7) & 0xFFu], c1 = cl_sh[(w[q] >> 23) & 0xFFu];
-                const uint32_t l1 = c1 & 0xFFu;
-                pl[q] = (c0 & 0xFFu) + l1;
-                p[q] = ((c0 >> 8) << l1) | (c1 >> 8);  // exact when pl[q] <= 32
+                const uint2 c0 = cl2[(w[q] >> 7) & 0xFFu], c1 = cl2[(w[q] >> 23) & 0xFFu];
+                pl[q] = c0.y + c1.y;
+                p[q] = (c0.x << c1.y) | c1.x;  // exact when pl[q] <= 32
                 // the m bytes in bytes 0 and 2: each mantissa above the other's sign
-                mw[q] = ((w[q] & 0x007F007Fu) << 1) | (w[q] >> 31) | ((w[q] << 1) & 0x00010000u);
+                mw[q] = ((w[q] << 1) & 0x00FF00FEu) | (w[q] >> 31);
             }
             // the pairs joined into two 32-bit halves, then one 64-bit shift
             const uint32_t la = pl[0] + pl[1], lb = pl[2] + pl[3], L = la + lb;
@@ -824,7 +822,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
     } else {
         for (uint32_t k = 0; k < NB; k++) {
             const uint64_t x0 = block_element(g, K, k, lane);
-            for (uint64_t x = x0; x < x0 + 8 && x < a.n; x++) bits += cl_sh[(a.in[x] >> 7) & 0xFFu] & 0xFFu;
+            for (uint64_t x = x0; x < x0 + 8 && x < a.n; x++) bits += cl2[(a.in[x] >> 7) & 0xFFu].y;
             if (x0 + 8 > a.n) break;
         }
     }
@@ -858,8 +856,8 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int q = 0; q < 8; q++) {
-                    const uint32_t cl = cl_sh[(w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu];
-                    bw.put(cl >> 8, cl & 0xFFu);
+                    const uint2 cl = cl2[(w[q >> 1] >> (16 * (q & 1) + 7)) & 0xFFu];
+                    bw.put(cl.x, cl.y);
                 }
             }
         }
@@ -903,7 +901,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
         for (uint32_t i = lane; i < count; i += 32) stream[wf + i] = 0u;
         __syncwarp();
         __threadfence();
-        pack_chunk<K>(a, cl_sh, c, lane, gb0 + (incl - bits), GlobalSink{stream});
+        pack_chunk<K>(a, cl2, c, lane, gb0 + (incl - bits), GlobalSink{stream});
         __syncwarp();
         __threadfence();
         if (lane == 0 && shared_first) boundary_word(a, g, stream + wf, ld_volatile(stream + wf));
