@@ -769,6 +769,12 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 4) k_pack_fused(EncodeArgs a
     __shared__ uint2 cl2[256];  // (code, length)
     __shared__ uint32_t cta_ticket;
     extern __shared__ __align__(16) uint8_t pack_smem[];
+    {
+        // the input of the group this warp will most likely get (tickets follow the order in
+        // which the CTAs start), sent to L2 while the code book is still being built
+        const uint64_t gp = (uint64_t)blockIdx.x * kFusedWarps + (threadIdx.x >> 5);
+        if ((threadIdx.x & 31) == 0 && (gp + 1) * 32u * K <= a.n) prefetch_l2(a.in + gp * 32u * K, 64u * K);
+    }
     wait_for_previous_kernel();  // the code book
     cl2[threadIdx.x] = make_uint2(a.ws_code[threadIdx.x], a.ws_len[threadIdx.x]);
     if (threadIdx.x == 0) cta_ticket = atomicAdd(reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTicket), 1u);
