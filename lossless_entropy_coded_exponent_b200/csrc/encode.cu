@@ -72,7 +72,7 @@ __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long lon
 // ---------------------------------------------------------------- 1. histogram
 //
 // One CTA of 32 warps per SM.  The input's 16-byte units (8 exponents each) are cut into
-// chunks of 128 units (2 KiB); each warp takes a contiguous run of chunks and streams them
+// chunks of 192 units (3 KiB); each warp takes a contiguous run of chunks and streams them
 // into its shared-memory buffers with the bulk-copy engine, kHistBufs chunks in flight,
 // so the bytes in flight do not depend on registers.  The exponents of a weight tensor
 // crowd into a few neighbouring values: each CTA counts its warps' first chunks into a
@@ -89,9 +89,9 @@ __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long lon
 // the shared histogram at the end.  Values outside the window are rare: the warp checks
 // once per unit whether any lane met one, and only then takes shared-memory atomics.
 constexpr int kHistWarps = 32;
-constexpr uint32_t kHistChunkUnits = 128;  // 16-byte units per chunk (2 KiB)
+constexpr uint32_t kHistChunkUnits = 192;  // 16-byte units per chunk (3 KiB)
 constexpr uint32_t kHistBufs = 2;          // chunks in flight per warp
-constexpr uint32_t kHistFold = 7;          // chunks between byte folds (7 x 32 < 256)
+constexpr uint32_t kHistFold = 5;          // chunks between byte folds (5 x 48 < 256)
 constexpr uint32_t kHistHalfFolds = 256;   // byte folds between half-word flushes (256 x 224 < 65536)
 
 struct HistWarpBuffers {
