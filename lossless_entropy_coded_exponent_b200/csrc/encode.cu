@@ -456,13 +456,19 @@ __global__ void __launch_bounds__(256) k_build_codebook(EncodeArgs a) {
     a.ws_code[t] = code;
     a.ws_len[t] = (uint8_t)l;
     a.out[kOffLen + t] = (uint8_t)l;
-    // the stream's bit count, for the pack's zeroing of the bytes past the container
-    __shared__ unsigned long long total_bits;
-    if (t == 0) total_bits = 0;
+    // the stream's bit count (for the container's zero padding after the stream): a sum
+    // per warp, then over the warps
+    __shared__ unsigned long long wbits[8];
+    unsigned long long tb = l ? c * l : 0ull;
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) tb += __shfl_xor_sync(kFull, tb, d);
+    if (lane == 0) wbits[warp] = tb;
     __syncthreads();
-    if (l) atomicAdd(&total_bits, c * l);
-    __syncthreads();
-    if (t == 0) *reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTotalBits) = total_bits;
+    if (t == 0) {
+        unsigned long long total_bits = 0;
+        for (int w = 0; w < 8; w++) total_bits += wbits[w];
+        *reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(a.ws_counts) + kWsTotalBits) = total_bits;
+    }
 
     if (t == 0) {
         uint8_t* h = a.out;
