@@ -81,7 +81,7 @@ __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long lon
 // 4-bit counters, eight per 32-bit word (value b + d adds 1 << 4d to the first word for
 // d < 8 and 1 << 4(d - 8) to the second for 8 <= d < 16).  The two values of a 32-bit
 // input word take one shared-memory load of the increments of the pair (a 17 x 17 table,
-// offset 16 standing for "outside") instead of shifts.  The loop is bound by the integer
+// offset 16 standing for "outside") instead of shifts.  The loop leans on the integer
 // (ALU) pipe, so its field extractions are multiplications by powers of two, which run on
 // the FMA pipe: x * 2^k is x << k and the high word of x * 2^(32 - k) is x >> k.  After
 // every unit (at most 8 per counter) the nibbles are spread
@@ -92,7 +92,7 @@ constexpr int kHistWarps = 32;
 constexpr uint32_t kHistChunkUnits = 192;  // 16-byte units per chunk (3 KiB)
 constexpr uint32_t kHistBufs = 2;          // chunks in flight per warp
 constexpr uint32_t kHistFold = 5;          // chunks between byte folds (5 x 48 < 256)
-constexpr uint32_t kHistHalfFolds = 256;   // byte folds between half-word flushes (256 x 224 < 65536)
+constexpr uint32_t kHistHalfFolds = 256;   // byte folds between half-word flushes (256 x 240 < 65536)
 
 struct HistWarpBuffers {
     uint4 chunk[kHistBufs][kHistChunkUnits];
