@@ -40,3 +40,24 @@ def test_traffic_is_null_once_a_decode_source_changes(tmp_path, monkeypatch):
 def test_traffic_is_null_without_the_file(monkeypatch, tmp_path):
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.txt"))
     assert bench.ncu_traffic_per_launch(1000) is None
+
+
+def test_launch_times_by_tenth():
+    # 50 steps: five at 135 us then five at 145 us per tenth -> the tenths show the step
+    ms = [0.135] * 25 + [0.145] * 25
+    assert bench.tenths(ms) == [135.0] * 5 + [145.0] * 5
+    # fewer than ten steps: one entry per step
+    assert bench.tenths([0.1354, 0.1361]) == [135.4, 136.1]
+
+
+def test_clock_summary_reports_the_memory_side():
+    c = bench.ClockSampler(0)
+    c.samples, c.max_mhz = [1900, 1965, 1965], 1965
+    c.reasons = {"sw_power_cap"}
+    # side samples: memory clock, GPU temperature, HBM temperature (None: not reported), power
+    c.side = [[3996, 40, None, 600.0], [3996, 44, None, 650.0], [3996, 46, None, 700.5]]
+    s = c.summary()
+    assert s["sm_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
+    assert s["mem_mhz"] == 3996
+    assert s["gpu_temp_c"] == {"first": 40, "last": 46} and s["power_w"] == {"first": 600.0, "last": 700.5}
+    assert "hbm_temp_c" not in s  # no answer from NVML: the key is left out, not faked
